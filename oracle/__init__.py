@@ -1,0 +1,153 @@
+"""ctypes front of the fp64 C++ oracle of the MSA hot path.
+
+TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the bench's CPU
+baseline leg use this module; the product path never imports it.  It shares
+no code with the CUDA library.  See ``msa_oracle.cpp`` for the method and the
+passages each function follows.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import subprocess
+from typing import Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "msa_oracle.cpp")
+_LIB = os.path.join(_HERE, "libmsa_oracle.so")
+
+
+class Params(C.Structure):
+    _fields_ = [("h_q", C.c_int), ("h_kv", C.c_int), ("d", C.c_int), ("d_idx", C.c_int),
+                ("block_k", C.c_int), ("topk", C.c_int), ("causal", C.c_int),
+                ("force_local", C.c_int), ("scale", C.c_double), ("threads", C.c_int)]
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with g++ (plain -O2, OpenMP, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp%d" % os.getpid()
+        subprocess.check_call(["g++", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c++17",
+                               "-o", tmp, _SRC])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        _lib = C.CDLL(build())
+        P = C.POINTER(Params)
+        vp = C.c_void_p
+        _lib.msa_oracle_block_scores.argtypes = [P, vp, vp, C.c_int, C.c_int, C.c_longlong, vp, C.c_int, vp]
+        _lib.msa_oracle_index_topk.argtypes = [P, vp, vp, C.c_int, C.c_int, C.c_longlong, vp, C.c_int, vp]
+        _lib.msa_oracle_sparse_attn.argtypes = [P, vp, vp, vp, vp, C.c_int, C.c_int, C.c_longlong, vp,
+                                                C.c_int, vp, vp]
+        _lib.msa_oracle_dense_attn.argtypes = [P, vp, vp, vp, C.c_int, C.c_int, C.c_longlong, vp, C.c_int,
+                                               vp, vp]
+        _lib.msa_oracle_decode.argtypes = [P, vp, vp, vp, vp, vp, vp, C.c_int, vp, C.c_int, C.c_int, vp, vp]
+        for f in ("msa_oracle_block_scores", "msa_oracle_index_topk", "msa_oracle_sparse_attn",
+                  "msa_oracle_dense_attn", "msa_oracle_decode"):
+            getattr(_lib, f).restype = C.c_int
+    return _lib
+
+
+def params(h_q, h_kv, d, d_idx, block_k, topk, causal=1, force_local=1, scale=0.0, threads=0) -> Params:
+    return Params(h_q, h_kv, d, d_idx, block_k, topk, int(causal), int(force_local), float(scale),
+                  int(threads))
+
+
+def _u16(a) -> np.ndarray:
+    a = np.ascontiguousarray(a)
+    assert a.dtype == np.uint16, a.dtype
+    return a
+
+
+def _ptr(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(C.c_void_p)
+
+
+def _rows(rows: Optional[Sequence[int]], n: int):
+    if rows is None:
+        return None, n
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
+    return r, int(r.size)
+
+
+def block_scores(P: Params, q_idx, k_idx, q_pos0: int = 0, rows=None) -> np.ndarray:
+    """Eq. (6) pooled block scores M[rows, h_kv, nb] (-inf = not eligible)."""
+    q_idx, k_idx = _u16(q_idx), _u16(k_idx)
+    n_q, n_kv = q_idx.shape[0], k_idx.shape[0]
+    r, nr = _rows(rows, n_q)
+    nb = (n_kv + P.block_k - 1) // P.block_k
+    out = np.empty((nr, P.h_kv, nb), dtype=np.float64)
+    rc = lib().msa_oracle_block_scores(C.byref(P), _ptr(q_idx), _ptr(k_idx), n_q, n_kv, q_pos0,
+                                       _ptr(r), nr, _ptr(out))
+    if rc:
+        raise ValueError("oracle block_scores: bad arguments (%d)" % rc)
+    return out
+
+
+def index_topk(P: Params, q_idx, k_idx, q_pos0: int = 0, rows=None) -> np.ndarray:
+    """Index branch: block ids[rows, h_kv, topk], ascending, -1 padded."""
+    q_idx, k_idx = _u16(q_idx), _u16(k_idx)
+    n_q, n_kv = q_idx.shape[0], k_idx.shape[0]
+    r, nr = _rows(rows, n_q)
+    out = np.empty((nr, P.h_kv, P.topk), dtype=np.int32)
+    rc = lib().msa_oracle_index_topk(C.byref(P), _ptr(q_idx), _ptr(k_idx), n_q, n_kv, q_pos0,
+                                     _ptr(r), nr, _ptr(out))
+    if rc:
+        raise ValueError("oracle index_topk: bad arguments (%d)" % rc)
+    return out
+
+
+def sparse_attn(P: Params, q, k, v, ids, q_pos0: int = 0, rows=None, want_lse=False):
+    """Main branch, eq. (8), over the given ids (one id list per listed row)."""
+    q, k, v = _u16(q), _u16(k), _u16(v)
+    n_q, n_kv = q.shape[0], k.shape[0]
+    r, nr = _rows(rows, n_q)
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    assert ids.shape == (nr, P.h_kv, P.topk), ids.shape
+    o = np.empty((nr, P.h_q, P.d), dtype=np.float64)
+    lse = np.empty((nr, P.h_q), dtype=np.float64) if want_lse else None
+    rc = lib().msa_oracle_sparse_attn(C.byref(P), _ptr(q), _ptr(k), _ptr(v), _ptr(ids), n_q, n_kv,
+                                      q_pos0, _ptr(r), nr, _ptr(o), _ptr(lse))
+    if rc:
+        raise ValueError("oracle sparse_attn: bad arguments (%d)" % rc)
+    return (o, lse) if want_lse else o
+
+
+def dense_attn(P: Params, q, k, v, q_pos0: int = 0, rows=None, want_lse=False):
+    """Dense GQA attention, eq. (1) (no block logic)."""
+    q, k, v = _u16(q), _u16(k), _u16(v)
+    n_q, n_kv = q.shape[0], k.shape[0]
+    r, nr = _rows(rows, n_q)
+    o = np.empty((nr, P.h_q, P.d), dtype=np.float64)
+    lse = np.empty((nr, P.h_q), dtype=np.float64) if want_lse else None
+    rc = lib().msa_oracle_dense_attn(C.byref(P), _ptr(q), _ptr(k), _ptr(v), n_q, n_kv, q_pos0, _ptr(r),
+                                     nr, _ptr(o), _ptr(lse))
+    if rc:
+        raise ValueError("oracle dense_attn: bad arguments (%d)" % rc)
+    return (o, lse) if want_lse else o
+
+
+def decode(P: Params, q, q_idx, k_cache, v_cache, k_idx_cache, cu_kv, seqs=None, dense=False):
+    """One decode step per listed sequence: (ids[n_seq,h_kv,topk], o[n_seq,h_q,d])."""
+    q, q_idx = _u16(q), _u16(q_idx)
+    k_cache, v_cache, k_idx_cache = _u16(k_cache), _u16(v_cache), _u16(k_idx_cache)
+    cu = np.ascontiguousarray(cu_kv, dtype=np.int64)
+    batch = q.shape[0]
+    s, ns = _rows(seqs, batch)
+    ids = np.full((ns, P.h_kv, P.topk), -1, dtype=np.int32)
+    o = np.empty((ns, P.h_q, P.d), dtype=np.float64)
+    rc = lib().msa_oracle_decode(C.byref(P), _ptr(q), _ptr(q_idx), _ptr(k_cache), _ptr(v_cache),
+                                 _ptr(k_idx_cache), _ptr(cu), batch, _ptr(s), ns, int(dense), _ptr(ids),
+                                 _ptr(o))
+    if rc:
+        raise ValueError("oracle decode: bad arguments (%d)" % rc)
+    return ids, o
