@@ -1,0 +1,160 @@
+/*
+ * msa.h -- C ABI of the MiniMax Sparse Attention (MSA) hot path on NVIDIA
+ * B200 (sm_100a).  Library: libmsa.so (long_context_index_b200/).
+ *
+ * The method (titansim.online summary of "MiniMax Sparse Attention"):
+ *   * Index branch, eq. (6) (section 4.2): per GQA group r and query i,
+ *       S_ij = <Q_idx_i^(r), K_idx_j> / sqrt(d_idx),
+ *       M_ib = max_{j in block b, j <= i} S_ij          (causal block max-pool),
+ *     then the top-k blocks by M, the local block always included, form
+ *     I_i^(r).  Selection ranks raw scores; nothing is exponentiated
+ *     (section 4.4.1).  One index query per group and one index key shared by
+ *     all groups (m.163.com post, "Step 1 Index Attention":
+ *     Q_idx in R^{n x h x d}, K_idx in R^{n x 1 x d}).
+ *   * Main branch, eq. (8) (section 4.3): every query head h of group r runs
+ *     exact, causally masked softmax attention over K^(r), V^(r) gathered at
+ *     the selected blocks.  Dense attention is eq. (1) (section 2.2).
+ *
+ * Conventions shared by every entry point:
+ *   * Tensors are caller-owned DEVICE memory, contiguous, row-major with the
+ *     last dimension innermost, base addresses 16-byte aligned.  bf16 values
+ *     are passed as raw 16-bit patterns (void*).  The library never allocates
+ *     device memory: callers query msa_workspace_size() and pass a device
+ *     workspace of at least that many bytes (256-byte aligned).
+ *   * Head h of the main branch belongs to group r = h / (h_q / h_kv).
+ *   * Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).  They are stateless: concurrent calls on different
+ *     streams with different workspaces are safe.
+ *   * Return value: MSA_OK, or a negative MSA_ERR_* code.  Argument errors are
+ *     detected on the host before anything is launched.  Kernels bound every
+ *     wait instead of hanging; a wait that gave up is recorded in the status
+ *     word at the start of the call's workspace, which msa_device_status()
+ *     reads (MSA_ERR_TIMEOUT).
+ *   * block_ids: int32 [rows, h_kv, topk], ascending, padded with -1 when a
+ *     row has fewer than topk eligible blocks.
+ *   * Positions: query row i of a prefill sits at absolute position
+ *     q_pos0 + i (q_pos0 = 0 for a full prefill, n_kv - n_q for the final
+ *     chunk of a chunked prefill).  A decode query sits at position L_b - 1 of
+ *     its sequence, whose cache already holds that position.
+ *   * Supported shapes: d in {64, 128}; d_idx in {32, 64, 128};
+ *     block_k in {64, 128}; 1 <= topk <= 32; h_q % h_kv == 0 and the group
+ *     size h_q / h_kv divides 128; n_q, n_kv <= 2^24 (MSA_ERR_UNSUPPORTED
+ *     otherwise).
+ */
+#ifndef MSA_H_
+#define MSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MSA_API __attribute__((visibility("default")))
+#else
+#define MSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes. */
+#define MSA_OK 0
+#define MSA_ERR_INVALID (-1)     /* null pointer, negative or inconsistent size */
+#define MSA_ERR_UNSUPPORTED (-2) /* shape outside the supported set above */
+#define MSA_ERR_MISALIGNED (-3)  /* a base address is not 16-byte aligned */
+#define MSA_ERR_WORKSPACE (-4)   /* workspace smaller than msa_workspace_size() */
+#define MSA_ERR_CUDA (-5)        /* a CUDA call or launch failed */
+#define MSA_ERR_TIMEOUT (-6)     /* a kernel gave up a bounded wait */
+
+/* Operation ids for msa_workspace_size(). */
+#define MSA_OP_INDEX_TOPK 0
+#define MSA_OP_PREFILL 1
+#define MSA_OP_DECODE 2
+
+/* Problem parameters (the pages' notation: H_q, H_kv, d_h, d_idx, B_k, k). */
+typedef struct {
+  int h_q;         /* query heads of the main branch */
+  int h_kv;        /* KV heads = GQA groups = index queries per token */
+  int d;           /* head dimension d_h of Q, K, V */
+  int d_idx;       /* index dimension of Q_idx, K_idx */
+  int block_k;     /* KV block size B_k */
+  int topk;        /* selected blocks per (query, group), local block included */
+  int causal;      /* 1: key j visible from position p iff j <= p; 0: all keys */
+  int force_local; /* 1: the block holding the query position is always selected */
+  float scale;     /* main-branch softmax scale; <= 0 means 1/sqrt(d) */
+} msa_params;
+
+/*
+ * Workspace bytes needed by one call of `op` with these sizes (batch and
+ * max_kv are used by MSA_OP_DECODE only; n_q/n_kv by the prefill ops).
+ * Returns 0 for invalid arguments.  Host-only; never touches the GPU.
+ */
+MSA_API size_t msa_workspace_size(int op, const msa_params* p, int n_q, int n_kv, int batch, int max_kv);
+
+/*
+ * Index branch of a (chunked) prefill: eq. (6) scores, causal block
+ * max-pool and top-k with the local block (titansim.online section 4.2).
+ *   q_idx     bf16 [n_q, h_kv, d_idx]  index queries, one per group
+ *   k_idx     bf16 [n_kv, 1, d_idx]    index keys, shared by all groups
+ *   block_ids int32 [n_q, h_kv, topk]  output
+ * Ranking is by raw dot product (the 1/sqrt(d_idx) factor is positive and
+ * does not change order); ties go to the lower block index.  With integer-
+ * valued index inputs the scores are exact, and the ids are exactly those of
+ * the definition.  Requires q_pos0 >= 0 and q_pos0 + n_q <= n_kv.
+ */
+MSA_API int msa_index_topk(const msa_params* p, const void* q_idx, const void* k_idx, int n_q, int n_kv,
+                   int q_pos0, int32_t* block_ids, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Main branch of a (chunked) prefill, eq. (8) (titansim.online section 4.3):
+ *   q         bf16 [n_q, h_q, d]
+ *   k, v      bf16 [n_kv, h_kv, d]
+ *   block_ids int32 [n_q, h_kv, topk] from msa_index_topk, or NULL for the
+ *             dense run (every causal block: eq. (1))
+ *   o         bf16 [n_q, h_q, d] output (fp32 accumulation, rounded to
+ *             nearest even)
+ * Ids must be valid (each -1 or a block holding a visible key of the row).
+ */
+MSA_API int msa_sparse_attn_prefill(const msa_params* p, const void* q, const void* k, const void* v,
+                            const int32_t* block_ids, int n_q, int n_kv, int q_pos0, void* o, void* ws,
+                            size_t ws_bytes, void* stream);
+
+/*
+ * One batched decode step: for every sequence b the query at position
+ * L_b - 1 runs the index branch over its whole index-key cache, then the main
+ * branch over the selected blocks (split over KV blocks, then combined).
+ *   q            bf16 [batch, h_q, d]
+ *   q_idx        bf16 [batch, h_kv, d_idx]
+ *   k_cache,
+ *   v_cache      bf16 [sum L_b, h_kv, d]   sequences stored back to back
+ *   k_idx_cache  bf16 [sum L_b, 1, d_idx]
+ *   cu_kv        int64 [batch + 1] DEVICE prefix sums of L_b (cu_kv[0] = 0)
+ *   max_kv       host upper bound on every L_b (sizes the launch grid)
+ *   dense        1: attend to every causal block (the index branch is skipped
+ *                and block_ids is not written)
+ *   block_ids    int32 [batch, h_kv, topk] output (may be NULL when dense)
+ *   o            bf16 [batch, h_q, d] output
+ * Every L_b must be in [1, max_kv].
+ */
+MSA_API int msa_sparse_attn_decode(const msa_params* p, const void* q, const void* q_idx, const void* k_cache,
+                           const void* v_cache, const void* k_idx_cache, const int64_t* cu_kv, int batch,
+                           int max_kv, int dense, int32_t* block_ids, void* o, void* ws, size_t ws_bytes,
+                           void* stream);
+
+/*
+ * Device status recorded by the last call that used workspace `ws`: MSA_OK,
+ * or MSA_ERR_TIMEOUT when one of its kernels gave up a bounded wait.  Every
+ * call clears the status word (the first 4 bytes of its workspace) before
+ * launching.  Synchronises `stream` first; returns MSA_ERR_CUDA if that or the
+ * 4-byte read fails.
+ */
+MSA_API int msa_device_status(const void* ws, void* stream);
+
+/* Human-readable text of a status code (static storage). */
+MSA_API const char* msa_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MSA_H_ */

@@ -1,0 +1,209 @@
+"""MiniMax Sparse Attention (MSA) hot path for NVIDIA B200 (sm_100a).
+
+Thin ctypes binding of ``libmsa.so`` (C ABI in ``include/msa.h``).  This module
+only marshals arguments: every step of the path runs in the library's CUDA
+kernels.  Tensors are torch CUDA tensors (bf16, int32, int64); the binding
+passes their device pointers and the current CUDA stream.  There is no CPU
+fallback: if the library is missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from typing import Optional
+
+__all__ = ["MSAError", "Params", "lib", "workspace_size", "index_topk", "sparse_attn_prefill",
+           "sparse_attn_decode", "device_status", "status_string", "OP_INDEX_TOPK", "OP_PREFILL",
+           "OP_DECODE"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmsa.so")
+
+OP_INDEX_TOPK, OP_PREFILL, OP_DECODE = 0, 1, 2
+
+SYMBOLS = ("msa_workspace_size", "msa_index_topk", "msa_sparse_attn_prefill", "msa_sparse_attn_decode",
+           "msa_device_status", "msa_status_string")
+
+
+class MSAError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__("%s failed: %s (%d)" % (what, status_string(code) if _lib else "?", code))
+        self.code = code
+
+
+class Params(C.Structure):
+    """Mirror of ``msa_params`` (include/msa.h)."""
+    _fields_ = [("h_q", C.c_int), ("h_kv", C.c_int), ("d", C.c_int), ("d_idx", C.c_int),
+                ("block_k", C.c_int), ("topk", C.c_int), ("causal", C.c_int), ("force_local", C.c_int),
+                ("scale", C.c_float)]
+
+    @classmethod
+    def make(cls, h_q, h_kv, d, d_idx, block_k, topk, causal=True, force_local=True, scale=0.0):
+        return cls(h_q, h_kv, d, d_idx, block_k, topk, int(causal), int(force_local), float(scale))
+
+
+_lib = None
+
+# When True, every call synchronises its stream and raises MSAError if a
+# kernel recorded a timeout in the workspace status word (used by the tests).
+check_status = False
+
+
+def lib():
+    """Load libmsa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libmsa.so not built: run `python -m long_context_index_b200.build`")
+        L = C.CDLL(LIB_PATH)
+        P = C.POINTER(Params)
+        vp, i32, sz = C.c_void_p, C.c_int, C.c_size_t
+        L.msa_workspace_size.argtypes = [i32, P, i32, i32, i32, i32]
+        L.msa_workspace_size.restype = sz
+        L.msa_index_topk.argtypes = [P, vp, vp, i32, i32, i32, vp, vp, sz, vp]
+        L.msa_sparse_attn_prefill.argtypes = [P, vp, vp, vp, vp, i32, i32, i32, vp, vp, sz, vp]
+        L.msa_sparse_attn_decode.argtypes = [P, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, vp, vp, sz, vp]
+        L.msa_device_status.argtypes = [vp, vp]
+        L.msa_status_string.argtypes = [i32]
+        L.msa_status_string.restype = C.c_char_p
+        for f in ("msa_index_topk", "msa_sparse_attn_prefill", "msa_sparse_attn_decode", "msa_device_status"):
+            getattr(L, f).restype = i32
+        _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().msa_status_string(int(code)).decode()
+
+
+def workspace_size(op: int, p: Params, n_q: int = 0, n_kv: int = 0, batch: int = 0, max_kv: int = 0) -> int:
+    """Host-only query of the workspace bytes one call needs (0 = invalid)."""
+    return int(lib().msa_workspace_size(int(op), C.byref(p), int(n_q), int(n_kv), int(batch), int(max_kv)))
+
+
+# ---------------------------------------------------------------------------
+# torch-facing wrappers
+# ---------------------------------------------------------------------------
+
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _check(t, name, dtypes, shape=None):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError("%s must be a CUDA tensor" % name)
+    if t.dtype not in dtypes:
+        raise TypeError("%s has dtype %s, expected one of %s" % (name, t.dtype, dtypes))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError("%s has shape %s, expected %s" % (name, tuple(t.shape), tuple(shape)))
+
+
+def _stream(stream) -> int:
+    torch = _torch()
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _workspace(op, p, n_q=0, n_kv=0, batch=0, max_kv=0, ws=None, device=None):
+    torch = _torch()
+    need = workspace_size(op, p, n_q, n_kv, batch, max_kv)
+    if need == 0:
+        raise MSAError(-1, "msa_workspace_size")
+    if ws is None or ws.numel() < need:
+        ws = torch.empty(need, dtype=torch.uint8, device=device)
+    return ws
+
+
+def _bf16():
+    torch = _torch()
+    return (torch.bfloat16, torch.uint16, torch.int16)
+
+
+def index_topk(p: Params, q_idx, k_idx, q_pos0: int = 0, block_ids=None, ws=None, stream=None):
+    """Index branch of a prefill: block ids [n_q, h_kv, topk] (int32, ascending, -1 padded)."""
+    torch = _torch()
+    n_q, n_kv = q_idx.shape[0], k_idx.shape[0]
+    _check(q_idx, "q_idx", _bf16(), (n_q, p.h_kv, p.d_idx))
+    _check(k_idx, "k_idx", _bf16(), (n_kv, 1, p.d_idx))
+    if block_ids is None:
+        block_ids = torch.empty((n_q, p.h_kv, p.topk), dtype=torch.int32, device=q_idx.device)
+    _check(block_ids, "block_ids", (torch.int32,), (n_q, p.h_kv, p.topk))
+    ws = _workspace(OP_INDEX_TOPK, p, n_q, n_kv, ws=ws, device=q_idx.device)
+    rc = lib().msa_index_topk(C.byref(p), _ptr(q_idx), _ptr(k_idx), n_q, n_kv, int(q_pos0), _ptr(block_ids),
+                              _ptr(ws), ws.numel(), _stream(stream))
+    if rc:
+        raise MSAError(rc, "msa_index_topk")
+    _after(ws, stream, "msa_index_topk")
+    return block_ids
+
+
+def sparse_attn_prefill(p: Params, q, k, v, block_ids=None, q_pos0: int = 0, out=None, ws=None, stream=None):
+    """Main branch of a prefill: O [n_q, h_q, d] bf16.  block_ids=None runs dense."""
+    torch = _torch()
+    n_q, n_kv = q.shape[0], k.shape[0]
+    _check(q, "q", _bf16(), (n_q, p.h_q, p.d))
+    _check(k, "k", _bf16(), (n_kv, p.h_kv, p.d))
+    _check(v, "v", _bf16(), (n_kv, p.h_kv, p.d))
+    if block_ids is not None:
+        _check(block_ids, "block_ids", (torch.int32,), (n_q, p.h_kv, p.topk))
+    if out is None:
+        out = torch.empty((n_q, p.h_q, p.d), dtype=torch.bfloat16, device=q.device)
+    _check(out, "out", _bf16(), (n_q, p.h_q, p.d))
+    ws = _workspace(OP_PREFILL, p, n_q, n_kv, ws=ws, device=q.device)
+    rc = lib().msa_sparse_attn_prefill(C.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(block_ids), n_q, n_kv,
+                                       int(q_pos0), _ptr(out), _ptr(ws), ws.numel(), _stream(stream))
+    if rc:
+        raise MSAError(rc, "msa_sparse_attn_prefill")
+    _after(ws, stream, "msa_sparse_attn_prefill")
+    return out
+
+
+def sparse_attn_decode(p: Params, q, q_idx, k_cache, v_cache, k_idx_cache, cu_kv, max_kv: int, dense=False,
+                       block_ids=None, out=None, ws=None, stream=None):
+    """One decode step: (block_ids [B, h_kv, topk] or None when dense, O [B, h_q, d])."""
+    torch = _torch()
+    B = q.shape[0]
+    tot = k_cache.shape[0]
+    _check(q, "q", _bf16(), (B, p.h_q, p.d))
+    _check(k_cache, "k_cache", _bf16(), (tot, p.h_kv, p.d))
+    _check(v_cache, "v_cache", _bf16(), (tot, p.h_kv, p.d))
+    _check(cu_kv, "cu_kv", (torch.int64,), (B + 1,))
+    if not dense:
+        _check(q_idx, "q_idx", _bf16(), (B, p.h_kv, p.d_idx))
+        _check(k_idx_cache, "k_idx_cache", _bf16(), (tot, 1, p.d_idx))
+        if block_ids is None:
+            block_ids = torch.empty((B, p.h_kv, p.topk), dtype=torch.int32, device=q.device)
+        _check(block_ids, "block_ids", (torch.int32,), (B, p.h_kv, p.topk))
+    if out is None:
+        out = torch.empty((B, p.h_q, p.d), dtype=torch.bfloat16, device=q.device)
+    _check(out, "out", _bf16(), (B, p.h_q, p.d))
+    ws = _workspace(OP_DECODE, p, batch=B, max_kv=max_kv, ws=ws, device=q.device)
+    rc = lib().msa_sparse_attn_decode(C.byref(p), _ptr(q), _ptr(q_idx) if not dense else None,
+                                      _ptr(k_cache), _ptr(v_cache), _ptr(k_idx_cache) if not dense else None,
+                                      _ptr(cu_kv), B, int(max_kv), int(bool(dense)),
+                                      _ptr(block_ids) if not dense else None, _ptr(out), _ptr(ws), ws.numel(),
+                                      _stream(stream))
+    if rc:
+        raise MSAError(rc, "msa_sparse_attn_decode")
+    _after(ws, stream, "msa_sparse_attn_decode")
+    return block_ids, out
+
+
+def _after(ws, stream, what):
+    if check_status:
+        rc = device_status(ws, stream)
+        if rc:
+            raise MSAError(rc, what)
+
+
+def device_status(ws, stream=None) -> int:
+    """Status word of the last call that used workspace ``ws`` (synchronises)."""
+    return int(lib().msa_device_status(_ptr(ws), _stream(stream)))

@@ -1,0 +1,456 @@
+// attn_prefill.cu -- main branch of a (chunked) prefill on sm_100a.
+//
+// Computes, for every query row i and head h of group r = h / G (titansim.online
+// summary of "MiniMax Sparse Attention", eq. (8), section 4.3):
+//   O_i^(h) = softmax( Q_i^(h) K^(r)[I]^T / sqrt(d) ) V^(r)[I],
+// where I is the set of causally visible keys of the blocks selected for
+// (i, r) -- or of every causal block for the dense run (eq. (1)).
+//
+// Kernel design (query-outer, GQA-packed):
+//   * One CTA owns a 128-row tile = QT = 128/G consecutive queries x the G
+//     heads of one group.  All rows share each K/V block, so one 128-key block
+//     staged by TMA feeds a full M = 128 UMMA (the heads of a group share the
+//     block selection: "同一 GQA 分组内的所有 Query 头共享相同的检索结果",
+//     titansim.online section 1.2).
+//   * warp 0: TMA producer (Q tile once; K and V blocks through a 2-deep ring).
+//   * warp 1: UMMA issuer.  S_j = Q K_j^T (SS form) into one of two TMEM S
+//     buffers; O += P_j V_j with P_j read from TMEM (TS form) and V_j as an
+//     MN-major shared-memory operand.
+//   * warps 4..7: softmax + epilogue, one thread per TMEM lane (= row).  Online
+//     softmax in fp32 with base-2 exponentials; O is rescaled in TMEM only when
+//     the running max grows by more than 2^8 (otherwise P may exceed 1 by at
+//     most 256, which fp32 accumulation absorbs).  P is written back to TMEM as
+//     bf16 over the S buffer it came from.
+//   * The block list of a tile is either every causal block (dense) or the
+//     sorted union of the blocks its QT queries selected; a row masks every
+//     block its own query did not select, and keys after its position.
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "msa_internal.h"
+#include "ptx.cuh"
+
+namespace msa {
+namespace {
+
+constexpr int kThreads = 256;   // 8 warps
+constexpr int kSoftWarp0 = 4;   // softmax warps 4..7
+constexpr int kStages = 2;      // K/V ring depth
+constexpr float kRescaleLog2 = 8.0f;
+constexpr int kMaxList = 1024;  // max union size (QT * topk <= 1024)
+
+template <int D, int BK>
+struct AttnCfg {
+  static constexpr int kAtoms = D / 64;                    // 128-byte swizzle atoms along d
+  static constexpr int kQBytes = 128 * D * 2;
+  static constexpr int kKVBytes = BK * D * 2;
+  static constexpr int kSmemData = kQBytes + kStages * 2 * kKVBytes;
+  static constexpr int kSmemBytes = kSmemData + 2 * kMaxList * 4 + 4096 + 1024;
+  static constexpr int kTmemCols = (2 * BK + D) <= 256 ? 256 : 512;
+  static constexpr int kColS0 = 0;
+  static constexpr int kColS1 = BK;
+  static constexpr int kColO = 2 * BK;
+};
+
+struct AttnArgs {
+  const int32_t* block_ids;  // [n_q, h_kv, topk] or null (dense)
+  uint16_t* o;               // [n_q, h_q, d]
+  int* status;
+  int n_q, n_kv, q_pos0, h_q, h_kv, topk, causal;
+  int n_qtiles;
+  float scale_log2;          // softmax scale * log2(e)
+};
+
+template <int D, int BK, int G>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_qouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const AttnArgs args) {
+  using Cfg = AttnCfg<D, BK>;
+  constexpr int QT = 128 / G;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sq = smem;                                   // [atoms][128 rows][128 B]
+  uint8_t* skv = smem + Cfg::kQBytes;                   // [stage][K|V][atoms][BK rows][128 B]
+  int* s_list = reinterpret_cast<int*>(smem + Cfg::kSmemData);   // block list (sorted)
+  int* s_sel = s_list + kMaxList;                       // [QT][topk] selected ids of the tile's queries
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s_sel + kMaxList);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;                         // [kStages]
+  uint64_t* kv_empty = kv_full + kStages;               // [kStages]
+  uint64_t* s_full = kv_empty + kStages;                // [2]
+  uint64_t* s_free = s_full + 2;                        // [2]
+  uint64_t* p_full = s_free + 2;                        // [2]
+  uint64_t* o_done = p_full + 2;                        // one phase per PV
+  uint64_t* o_final = o_done + 1;                       // the last PV only
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_final + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  int* s_nblk = abort_flag + 1;
+
+  const int warp = warp_id();
+  const int lane = lane_id();
+  const int qtile = args.n_qtiles - 1 - static_cast<int>(blockIdx.x) / args.h_kv;  // heavy tiles first
+  const int r = static_cast<int>(blockIdx.x) % args.h_kv;
+  const int i0 = qtile * QT;
+  const int q_here = min(QT, args.n_q - i0);
+  const bool dense = args.block_ids == nullptr;
+
+  // ---------------------------------------------------------------- setup
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&s_free[b], 1);
+      mbar_init(&p_full[b], 4);
+    }
+    mbar_init(o_done, 1);
+    mbar_init(o_final, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  // Block list of the tile.
+  const int p_first = args.q_pos0 + i0;
+  const int p_last = p_first + q_here - 1;
+  const int nb_total = (args.n_kv + BK - 1) / BK;
+  if (dense) {
+    if (threadIdx.x == 0) *s_nblk = args.causal ? (p_last / BK + 1) : nb_total;
+  } else {
+    const int nsel = q_here * args.topk;
+    for (int t = threadIdx.x; t < QT * args.topk; t += kThreads) {
+      const int qi = t / args.topk;
+      const int v = t < nsel ? args.block_ids[(static_cast<size_t>(i0 + qi) * args.h_kv + r) * args.topk +
+                                              (t % args.topk)]
+                             : -1;
+      s_sel[t] = v;
+      s_list[t] = v < 0 ? 0x7fffffff : v;
+    }
+    __syncthreads();
+    // Bitonic sort of the (power-of-two padded) id list.
+    int n2 = 1;
+    while (n2 < QT * args.topk) n2 <<= 1;
+    for (int t = QT * args.topk + threadIdx.x; t < n2; t += kThreads) s_list[t] = 0x7fffffff;
+    __syncthreads();
+    for (int k = 2; k <= n2; k <<= 1) {
+      for (int j = k >> 1; j > 0; j >>= 1) {
+        for (int t = threadIdx.x; t < n2; t += kThreads) {
+          const int u = t ^ j;
+          if (u > t) {
+            const int a = s_list[t], b = s_list[u];
+            const bool up = (t & k) == 0;
+            if ((a > b) == up) {
+              s_list[t] = b;
+              s_list[u] = a;
+            }
+          }
+        }
+        __syncthreads();
+      }
+    }
+    if (threadIdx.x == 0) {
+      int n = 0;
+      for (int t = 0; t < n2; ++t) {
+        const int v = s_list[t];
+        if (v == 0x7fffffff) break;
+        if (n == 0 || s_list[n - 1] != v) s_list[n++] = v;
+      }
+      *s_nblk = n;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int nblk = *s_nblk;
+  const WaitCtx wc{abort_flag, args.status};
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA
+    if (lane == 0 && nblk > 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_arrive_expect_tx(q_full, Cfg::kQBytes);
+      for (int a = 0; a < Cfg::kAtoms; ++a) tma_load_3d(sq + a * 128 * 128, &tm_q, q_full, a * 64, r * G, i0);
+      for (int j = 0; j < nblk; ++j) {
+        const int s = j % kStages;
+        const int b = dense ? j : s_list[j];
+        if (!mbar_wait(&kv_empty[s], ((j / kStages) & 1) ^ 1, wc)) break;
+        mbar_arrive_expect_tx(&kv_full[s], 2 * Cfg::kKVBytes);
+        uint8_t* sk = skv + s * 2 * Cfg::kKVBytes;
+        uint8_t* sv = sk + Cfg::kKVBytes;
+        for (int a = 0; a < Cfg::kAtoms; ++a) {
+          tma_load_3d(sk + a * BK * 128, &tm_k, &kv_full[s], a * 64, r, b * BK);
+          tma_load_3d(sv + a * BK * 128, &tm_v, &kv_full[s], a * 64, r, b * BK);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- UMMA
+    if (lane == 0 && nblk > 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, BK, false, false);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
+      const uint32_t sq_addr = smem_u32(sq);
+      const uint32_t skv_addr = smem_u32(skv);
+      bool ok = mbar_wait(q_full, 0, wc);
+      auto issue_pv = [&](int j) -> bool {
+        const int s = j % kStages;
+        const int sb = j & 1;
+        if (!mbar_wait(&p_full[sb], (j >> 1) & 1, wc)) return false;
+        tc_fence_after();
+        const uint32_t sv_addr = skv_addr + s * 2 * Cfg::kKVBytes + Cfg::kKVBytes;
+        const uint32_t p_tmem = tmem + (sb ? Cfg::kColS1 : Cfg::kColS0);
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          // B = V block, MN-major: 16 keys per step = 2048 bytes; d atoms are BK*128 bytes apart.
+          const uint64_t bdesc = smem_desc(sv_addr + kk * 2048, BK * 128, 1024, kSwizzle128B);
+          umma_ts(tmem + Cfg::kColO, p_tmem + kk * 8, bdesc, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&kv_empty[s]);
+        umma_commit(&s_free[sb]);
+        umma_commit(o_done);
+        return true;
+      };
+      for (int j = 0; ok && j < nblk; ++j) {
+        const int s = j % kStages;
+        const int sb = j & 1;
+        if (!mbar_wait(&kv_full[s], (j / kStages) & 1, wc)) break;
+        if (!mbar_wait(&s_free[sb], ((j >> 1) & 1) ^ 1, wc)) break;
+        tc_fence_after();
+        const uint32_t sk_addr = skv_addr + s * 2 * Cfg::kKVBytes;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const int atom = ks / 4;
+          const uint32_t koff = (ks % 4) * 32;
+          const uint64_t adesc = smem_desc(sq_addr + atom * 128 * 128 + koff, 16, 1024, kSwizzle128B);
+          const uint64_t bdesc = smem_desc(sk_addr + atom * BK * 128 + koff, 16, 1024, kSwizzle128B);
+          umma_ss(tmem + (sb ? Cfg::kColS1 : Cfg::kColS0), adesc, bdesc, idesc_s, ks > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[sb]);
+        if (j > 0 && !issue_pv(j - 1)) {
+          ok = false;
+          break;
+        }
+      }
+      if (ok && issue_pv(nblk - 1)) umma_commit(o_final);
+    }
+  } else if (warp >= kSoftWarp0) {
+    // ---------------------------------------------------------------- softmax + epilogue
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const int qi = row / G;
+    const int hh = row % G;
+    const bool row_ok = qi < q_here;
+    const int p = args.q_pos0 + i0 + qi;
+    const int kv_lim = row_ok ? (args.causal ? min(p + 1, args.n_kv) : args.n_kv) : 0;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const float c = args.scale_log2;
+    float m_run = __int_as_float(0xff800000);  // running max of raw scores (-inf)
+    float l_run = 0.f;
+    const int* my_sel = s_sel + qi * args.topk;
+
+    for (int j = 0; j < nblk; ++j) {
+      const int sb = j & 1;
+      const int b = dense ? j : s_list[j];
+      // Is block b selected for this row's query?
+      bool row_sel = row_ok;
+      if (!dense && row_ok) {
+        row_sel = false;
+        for (int t = 0; t < args.topk; ++t) row_sel |= my_sel[t] == b;
+      }
+      const int kb0 = b * BK;
+      const int lim = row_sel ? min(BK, kv_lim - kb0) : 0;   // valid keys of this block for the row
+      if (!mbar_wait(&s_full[sb], (j >> 1) & 1, wc)) break;
+      tc_fence_after();
+      uint32_t sv[BK];
+      const uint32_t s_tmem = lane_base + (sb ? Cfg::kColS1 : Cfg::kColS0);
+#pragma unroll
+      for (int cch = 0; cch < BK / 32; ++cch)
+        tmem_ld32(s_tmem + cch * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[cch * 32]));
+      tmem_ld_wait();
+      float mx = __int_as_float(0xff800000);
+      if (lim >= BK) {
+#pragma unroll
+        for (int e = 0; e + 2 < BK; e += 3)
+          mx = max3f(mx, __uint_as_float(sv[e]), fmaxf(__uint_as_float(sv[e + 1]), __uint_as_float(sv[e + 2])));
+        if (BK % 3 != 0) {
+#pragma unroll
+          for (int e = (BK / 3) * 3; e < BK; ++e) mx = fmaxf(mx, __uint_as_float(sv[e]));
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < BK; ++e) {
+          const float v = e < lim ? __uint_as_float(sv[e]) : __int_as_float(0xff800000);
+          sv[e] = __float_as_uint(v);
+          mx = fmaxf(mx, v);
+        }
+      }
+      const float m_new = fmaxf(m_run, mx);
+      // Lazy rescale: only when the max grows by more than 2^kRescaleLog2.
+      const bool grow = m_run != __int_as_float(0xff800000) && (m_new - m_run) * c > kRescaleLog2;
+      float alpha = 1.f;
+      if (grow) {
+        alpha = ex2_approx((m_run - m_new) * c);
+        l_run *= alpha;
+        m_run = m_new;
+      } else if (m_run == __int_as_float(0xff800000)) {
+        m_run = m_new;   // first visible keys: O and l are still exactly zero
+      }
+      if (__any_sync(0xffffffffu, grow)) {
+        // O must hold every PV up to block j-1 before it is rescaled.  Here
+        // PV_{j-2} is complete (it was issued before S_j) and PV_j is not yet
+        // issued, so the PV barrier is at most one phase from phase j-1.
+        if (!mbar_wait(o_done, (j - 1) & 1, wc)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int cch = 0; cch < D / 32; ++cch) {
+          uint32_t ov[32];
+          tmem_ld32(lane_base + Cfg::kColO + cch * 32, ov);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+          tmem_st32(lane_base + Cfg::kColO + cch * 32, ov);
+        }
+        tmem_st_wait();
+      }
+      const float bias = m_run == __int_as_float(0xff800000) ? 0.f : m_run * c;
+      float lsum = 0.f;
+      uint32_t pk[BK / 2];
+#pragma unroll
+      for (int e = 0; e < BK; e += 2) {
+        const float p0 = ex2_approx(fmaf(__uint_as_float(sv[e]), c, -bias));
+        const float p1 = ex2_approx(fmaf(__uint_as_float(sv[e + 1]), c, -bias));
+        lsum += p0 + p1;
+        pk[e / 2] = pack_bf16x2(p0, p1);
+      }
+      l_run += lsum;
+#pragma unroll
+      for (int cch = 0; cch < BK / 64; ++cch)
+        tmem_st32(s_tmem + cch * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[cch * 32]));
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[sb]);
+    }
+
+    // Epilogue: O / l -> bf16.  (The PV barrier may run up to two phases
+    // ahead of this point, so the last PV signals a barrier of its own.)
+    bool ok = !*abort_flag && nblk > 0;
+    if (ok) ok = mbar_wait(o_final, 0, wc);
+    if (ok) {
+      tc_fence_after();
+      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      uint16_t* orow = args.o + (static_cast<size_t>(i0 + qi) * args.h_q + r * G + hh) * D;
+#pragma unroll
+      for (int cch = 0; cch < D / 32; ++cch) {
+        uint32_t ov[32];
+        tmem_ld32(lane_base + Cfg::kColO + cch * 32, ov);
+        tmem_ld_wait();
+        if (row_ok) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + cch * 32);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(ov[v4 * 8 + 0]) * inv, __uint_as_float(ov[v4 * 8 + 1]) * inv);
+            w.y = pack_bf16x2(__uint_as_float(ov[v4 * 8 + 2]) * inv, __uint_as_float(ov[v4 * 8 + 3]) * inv);
+            w.z = pack_bf16x2(__uint_as_float(ov[v4 * 8 + 4]) * inv, __uint_as_float(ov[v4 * 8 + 5]) * inv);
+            w.w = pack_bf16x2(__uint_as_float(ov[v4 * 8 + 6]) * inv, __uint_as_float(ov[v4 * 8 + 7]) * inv);
+            dst[v4] = w;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) __nanosleep(1000000);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Cfg::kTmemCols);
+  }
+}
+
+template <int D, int BK, int G>
+cudaError_t launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& a,
+                        cudaStream_t st) {
+  auto kern = attn_qouter_kernel<D, BK, G>;
+  const int smem = AttnCfg<D, BK>::kSmemBytes;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  kern<<<a.n_qtiles * a.h_kv, kThreads, smem, st>>>(tq, tk, tv, a);
+  return cudaGetLastError();
+}
+
+template <int D, int BK>
+cudaError_t launch_g(int G, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& a,
+                     cudaStream_t st) {
+  switch (G) {
+    case 1: return launch_attn<D, BK, 1>(tq, tk, tv, a, st);
+    case 2: return launch_attn<D, BK, 2>(tq, tk, tv, a, st);
+    case 4: return launch_attn<D, BK, 4>(tq, tk, tv, a, st);
+    case 8: return launch_attn<D, BK, 8>(tq, tk, tv, a, st);
+    case 16: return launch_attn<D, BK, 16>(tq, tk, tv, a, st);
+    case 32: return launch_attn<D, BK, 32>(tq, tk, tv, a, st);
+    case 64: return launch_attn<D, BK, 64>(tq, tk, tv, a, st);
+    default: return launch_attn<D, BK, 128>(tq, tk, tv, a, st);
+  }
+}
+
+}  // namespace
+
+size_t prefill_workspace_bytes(const msa_params&, int, int) { return 0; }
+
+int run_sparse_attn_prefill(const msa_params& p, const void* q, const void* k, const void* v,
+                            const int32_t* block_ids, int n_q, int n_kv, int q_pos0, void* o, void* /*ws*/,
+                            size_t /*ws_bytes*/, int* status, cudaStream_t stream) {
+  if (n_q == 0) return MSA_OK;
+  const int G = p.h_q / p.h_kv;
+  const int QT = 128 / G;
+  if (block_ids && QT * p.topk > kMaxList) return MSA_ERR_UNSUPPORTED;
+  CUtensorMap tq, tk, tv;
+  {
+    const uint64_t dims[3] = {static_cast<uint64_t>(p.d), static_cast<uint64_t>(p.h_q), static_cast<uint64_t>(n_q)};
+    const uint64_t strides[2] = {static_cast<uint64_t>(p.d) * 2, static_cast<uint64_t>(p.h_q) * p.d * 2};
+    const uint32_t box[3] = {64, static_cast<uint32_t>(G), static_cast<uint32_t>(QT)};
+    if (!encode_tma_bf16(&tq, 3, q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MSA_ERR_CUDA;
+  }
+  {
+    const uint64_t dims[3] = {static_cast<uint64_t>(p.d), static_cast<uint64_t>(p.h_kv),
+                              static_cast<uint64_t>(n_kv)};
+    const uint64_t strides[2] = {static_cast<uint64_t>(p.d) * 2, static_cast<uint64_t>(p.h_kv) * p.d * 2};
+    const uint32_t box[3] = {64, 1, static_cast<uint32_t>(p.block_k)};
+    if (!encode_tma_bf16(&tk, 3, k, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MSA_ERR_CUDA;
+    if (!encode_tma_bf16(&tv, 3, v, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MSA_ERR_CUDA;
+  }
+  AttnArgs a;
+  a.block_ids = block_ids;
+  a.o = static_cast<uint16_t*>(o);
+  a.status = status;
+  a.n_q = n_q;
+  a.n_kv = n_kv;
+  a.q_pos0 = q_pos0;
+  a.h_q = p.h_q;
+  a.h_kv = p.h_kv;
+  a.topk = p.topk;
+  a.causal = p.causal;
+  a.n_qtiles = (n_q + QT - 1) / QT;
+  const float scale = p.scale > 0.f ? p.scale : 1.0f / sqrtf(static_cast<float>(p.d));
+  a.scale_log2 = scale * 1.4426950408889634f;
+  cudaError_t e;
+  if (p.d == 64) {
+    e = p.block_k == 64 ? launch_g<64, 64>(G, tq, tk, tv, a, stream) : launch_g<64, 128>(G, tq, tk, tv, a, stream);
+  } else {
+    e = p.block_k == 64 ? launch_g<128, 64>(G, tq, tk, tv, a, stream) : launch_g<128, 128>(G, tq, tk, tv, a, stream);
+  }
+  return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
+}
+
+}  // namespace msa

@@ -1,0 +1,365 @@
+// index_prefill.cu -- index branch of a (chunked) prefill on sm_100a.
+//
+// Computes, per query row i and GQA group r (titansim.online summary of
+// "MiniMax Sparse Attention", eq. (6), section 4.2):
+//   S_ij = <Q_idx_i^(r), K_idx_j>                  (the 1/sqrt(d_idx) factor is
+//                                                   positive: order-preserving)
+//   M_ib = max over visible j in block b of S_ij   (causal block max-pool)
+//   I_i^(r) = local block + the best (topk - 1) other eligible blocks by M,
+//             ties to the lower block index, emitted ascending, -1 padded.
+// Selection compares raw scores and never exponentiates (section 4.4.1).
+//
+// Design (one CTA = 128 query rows x 2 groups):
+//   * warp 0, one lane: TMA producer.  Loads the two Q_idx tiles (A operands,
+//     resident for the CTA) and streams 128-key K_idx tiles (B operand, shared
+//     by both groups) through an NST-deep shared-memory ring.
+//   * warp 1, one lane: UMMA issuer.  Per key tile, two 128x128xd_idx
+//     tcgen05.mma (one per group) into one of two TMEM accumulator stages
+//     (2 stages x 2 groups x 128 fp32 columns = all 512 columns), so the MMA
+//     of tile t+1 overlaps the epilogue of tile t.
+//   * warps 4..11: epilogue.  Thread = (TMEM lane = query row, group).  Reads
+//     its row of S from TMEM, masks invisible keys, max-pools per block with
+//     3-input max, and keeps a register top-k list (insertion only when the
+//     candidate beats the current k-th score, so ties keep the earlier, lower
+//     block).  M is never written to memory.
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "msa_internal.h"
+#include "ptx.cuh"
+
+namespace msa {
+namespace {
+
+constexpr int kRows = 128;      // query rows per CTA (UMMA M)
+constexpr int kKeys = 128;      // keys per tile (UMMA N)
+constexpr int kThreads = 384;   // 12 warps
+constexpr int kEpiWarp0 = 4;    // first epilogue warp
+
+template <int DIDX>
+struct IdxCfg {
+  static constexpr int kSwB = DIDX * 2 >= 128 ? 128 : DIDX * 2;   // swizzle span (bytes)
+  static constexpr int kAtoms = DIDX * 2 / kSwB;                  // swizzle atoms along K
+  static constexpr uint32_t kSwz = kSwB == 128 ? kSwizzle128B : kSwizzle64B;
+  static constexpr int kTileBytes = kRows * DIDX * 2;             // one 128 x DIDX bf16 tile
+  static constexpr int kStages = DIDX == 128 ? 4 : (DIDX == 64 ? 6 : 8);
+  static constexpr int kSmemQ = 2 * kTileBytes;
+  static constexpr int kSmemK = kStages * kTileBytes;
+  static constexpr int kSmemBytes = kSmemQ + kSmemK + 1024 /*barriers etc.*/ + 1024 /*align*/;
+};
+
+struct IdxArgs {
+  int32_t* block_ids;
+  int* status;
+  int n_q, n_kv, q_pos0, h_kv, topk, causal, force_local;
+  int n_tiles, n_pairs;
+};
+
+// Sorted-descending register list of KMAX (score, block) pairs.  Slots
+// [0, KMAX - k_free) hold +inf sentinels that never move; the live part is
+// the last k_free slots.
+template <int KMAX>
+struct TopK {
+  float sc[KMAX];
+  int id[KMAX];
+
+  __device__ __forceinline__ void init(int k_free) {
+#pragma unroll
+    for (int i = 0; i < KMAX; ++i) {
+      const bool dead = i < KMAX - k_free;
+      sc[i] = dead ? __int_as_float(0x7f800000) : __int_as_float(0xff800000);
+      id[i] = -1;
+    }
+  }
+  __device__ __forceinline__ float threshold() const { return sc[KMAX - 1]; }
+
+  // Insert (x, b); caller guarantees x > threshold().  An equal score already
+  // in the list stays ahead of x (it has a lower block index).
+  __device__ __forceinline__ void insert(float x, int b) {
+#pragma unroll
+    for (int i = KMAX - 1; i > 0; --i) {
+      const bool down = x > sc[i - 1];          // element i-1 moves down to i
+      const bool here = !down && (x > sc[i]);   // x lands at i
+      sc[i] = down ? sc[i - 1] : (here ? x : sc[i]);
+      id[i] = down ? id[i - 1] : (here ? b : id[i]);
+    }
+    if (x > sc[0]) {
+      sc[0] = x;
+      id[0] = b;
+    }
+  }
+};
+
+template <int DIDX, int BK, int KMAX>
+__global__ void __launch_bounds__(kThreads, 1)
+    index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                              const IdxArgs args) {
+  using Cfg = IdxCfg<DIDX>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sq = smem;                       // [2 groups][atoms][128 rows][kSwB]
+  uint8_t* sk = smem + Cfg::kSmemQ;         // [stages][atoms][128 keys][kSwB]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sk + Cfg::kSmemK);
+  uint64_t* full = bars;                    // [kStages]
+  uint64_t* empty = bars + Cfg::kStages;    // [kStages]
+  uint64_t* acc_full = empty + Cfg::kStages;  // [2]
+  uint64_t* acc_empty = acc_full + 2;       // [2]
+  uint64_t* q_full = acc_empty + 2;         // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = warp_id();
+  const int lane = lane_id();
+  const int tile = args.n_tiles - 1 - static_cast<int>(blockIdx.x) / args.n_pairs;  // heavy tiles first
+  const int pair = static_cast<int>(blockIdx.x) % args.n_pairs;
+  const int i0 = tile * kRows;
+  const int rows_here = min(kRows, args.n_q - i0);
+  const int groups_here = min(2, args.h_kv - 2 * pair);
+
+  // Key range this CTA must score.  A row at position p needs keys < kv_lim(p)
+  // where kv_lim = p + 1 (causal) or n_kv; with force_local its own block is
+  // not scored, so it needs only keys below the start of that block.
+  const int p_last = args.q_pos0 + i0 + rows_here - 1;
+  int kv_end;
+  if (!args.causal) {
+    kv_end = args.n_kv;
+  } else if (args.force_local) {
+    kv_end = (p_last / BK) * BK;
+  } else {
+    kv_end = p_last + 1;
+  }
+  const int n_ktiles = (kv_end + kKeys - 1) / kKeys;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < Cfg::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 8);
+    }
+    mbar_init(q_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtx wc{abort_flag, args.status};
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA
+    if (lane == 0 && n_ktiles > 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      mbar_arrive_expect_tx(q_full, groups_here * Cfg::kTileBytes);
+      for (int g = 0; g < groups_here; ++g)
+        for (int a = 0; a < Cfg::kAtoms; ++a)
+          tma_load_3d(sq + (g * Cfg::kAtoms + a) * kRows * Cfg::kSwB, &tm_q, q_full, a * (Cfg::kSwB / 2),
+                      2 * pair + g, i0);
+      for (int t = 0; t < n_ktiles; ++t) {
+        const int s = t % Cfg::kStages;
+        const uint32_t ph = (t / Cfg::kStages) & 1;
+        if (!mbar_wait(&empty[s], ph ^ 1, wc)) break;
+        mbar_arrive_expect_tx(&full[s], Cfg::kTileBytes);
+        for (int a = 0; a < Cfg::kAtoms; ++a)
+          tma_load_2d(sk + (s * Cfg::kAtoms + a) * kKeys * Cfg::kSwB, &tm_k, &full[s], a * (Cfg::kSwB / 2),
+                      t * kKeys);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- UMMA
+    if (lane == 0 && n_ktiles > 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kRows, kKeys, false, false);
+      constexpr uint32_t sbo = 8 * Cfg::kSwB;   // 8-row core-matrix group stride
+      const uint32_t sq_addr = smem_u32(sq);
+      const uint32_t sk_addr = smem_u32(sk);
+      bool ok = mbar_wait(q_full, 0, wc);
+      for (int t = 0; ok && t < n_ktiles; ++t) {
+        const int s = t % Cfg::kStages;
+        const int acc = t & 1;
+        if (!mbar_wait(&acc_empty[acc], ((t >> 1) & 1) ^ 1, wc)) break;
+        if (!mbar_wait(&full[s], (t / Cfg::kStages) & 1, wc)) break;
+        tc_fence_after();
+        for (int g = 0; g < groups_here; ++g) {
+          const uint32_t d_tmem = tmem + acc * 256 + g * 128;
+#pragma unroll
+          for (int ks = 0; ks < DIDX / 16; ++ks) {
+            const int atom = ks / (Cfg::kSwB / 32);
+            const uint32_t koff = (ks % (Cfg::kSwB / 32)) * 32;
+            const uint64_t adesc =
+                smem_desc(sq_addr + (g * Cfg::kAtoms + atom) * kRows * Cfg::kSwB + koff, 16, sbo, Cfg::kSwz);
+            const uint64_t bdesc =
+                smem_desc(sk_addr + (s * Cfg::kAtoms + atom) * kKeys * Cfg::kSwB + koff, 16, sbo, Cfg::kSwz);
+            umma_ss(d_tmem, adesc, bdesc, idesc, ks > 0 ? 1u : 0u);
+          }
+        }
+        umma_commit(&empty[s]);       // smem stage free once these MMAs finish
+        umma_commit(&acc_full[acc]);  // accumulator ready for the epilogue
+      }
+    }
+  } else if (warp >= kEpiWarp0) {
+    // ---------------------------------------------------------------- epilogue
+    const int quarter = warp & 3;
+    const int g = (warp - kEpiWarp0) >> 2;   // group within the pair
+    const int row = quarter * 32 + lane;
+    const bool row_ok = row < rows_here && g < groups_here;
+    const int p = args.q_pos0 + i0 + row;
+    const int kv_lim = args.causal ? min(p + 1, args.n_kv) : args.n_kv;
+    const int b_loc = p / BK;
+    const int k_free = args.topk - (args.force_local ? 1 : 0);
+    TopK<KMAX> tk;
+    tk.init(k_free);
+    const uint32_t taddr_row = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + g * 128;
+
+    for (int t = 0; t < n_ktiles; ++t) {
+      const int acc = t & 1;
+      if (!mbar_wait(&acc_full[acc], (t >> 1) & 1, wc)) break;
+      tc_fence_after();
+      constexpr int kBlocksPerTile = kKeys / BK;
+      float bmax[kBlocksPerTile];
+#pragma unroll
+      for (int bb = 0; bb < kBlocksPerTile; ++bb) bmax[bb] = __int_as_float(0xff800000);
+      const int j0 = t * kKeys;
+      if (g < groups_here) {
+#pragma unroll
+        for (int c = 0; c < kKeys / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(taddr_row + acc * 256 + c * 32, v);
+          tmem_ld_wait();
+          const int jc = j0 + c * 32;
+          float m = __int_as_float(0xff800000);
+          if (jc + 32 <= kv_lim) {
+#pragma unroll
+            for (int e = 0; e < 30; e += 3)
+              m = max3f(m, fmaxf(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), __uint_as_float(v[e + 2]));
+            m = max3f(m, __uint_as_float(v[30]), __uint_as_float(v[31]));
+          } else if (jc < kv_lim) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (jc + e < kv_lim) m = fmaxf(m, __uint_as_float(v[e]));
+          }
+          bmax[(c * 32) / BK] = fmaxf(bmax[(c * 32) / BK], m);
+        }
+      }
+      // Release the accumulator stage to the MMA warp.
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      if (row_ok) {
+#pragma unroll
+        for (int bb = 0; bb < kBlocksPerTile; ++bb) {
+          const int b = (j0 / BK) + bb;
+          const bool eligible = static_cast<long long>(b) * BK < kv_lim && !(args.force_local && b == b_loc);
+          const float x = bmax[bb];
+          if (eligible && x > tk.threshold()) tk.insert(x, b);
+        }
+      }
+    }
+
+    if (row_ok) {
+      // Final set: live list entries plus the local block, ascending, -1 padded.
+      int ids[KMAX + 1];
+#pragma unroll
+      for (int i = 0; i < KMAX; ++i) ids[i] = tk.id[i] < 0 ? 0x7fffffff : tk.id[i];
+      ids[KMAX] = args.force_local ? b_loc : 0x7fffffff;
+      // Odd-even transposition sort on static indices (stays in registers).
+#pragma unroll
+      for (int pass = 0; pass < KMAX + 1; ++pass) {
+#pragma unroll
+        for (int i = pass & 1; i + 1 < KMAX + 1; i += 2) {
+          const int lo = min(ids[i], ids[i + 1]);
+          const int hi = max(ids[i], ids[i + 1]);
+          ids[i] = lo;
+          ids[i + 1] = hi;
+        }
+      }
+      int32_t* out = args.block_ids + (static_cast<size_t>(i0 + row) * args.h_kv + 2 * pair + g) * args.topk;
+#pragma unroll
+      for (int i = 0; i < KMAX + 1; ++i)
+        if (i < args.topk) out[i] = ids[i] == 0x7fffffff ? -1 : ids[i];
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) __nanosleep(1000000);  // let in-flight async copies/MMAs land
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int DIDX, int BK, int KMAX>
+cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const IdxArgs& a, cudaStream_t st) {
+  auto kern = index_topk_prefill_kernel<DIDX, BK, KMAX>;
+  const int smem = IdxCfg<DIDX>::kSmemBytes;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.n_tiles * a.n_pairs);
+  kern<<<grid, kThreads, smem, st>>>(tq, tk, a);
+  return cudaGetLastError();
+}
+
+template <int DIDX, int BK>
+cudaError_t launch_k(const CUtensorMap& tq, const CUtensorMap& tk, const IdxArgs& a, cudaStream_t st) {
+  if (a.topk <= 16) return launch_t<DIDX, BK, 16>(tq, tk, a, st);
+  return launch_t<DIDX, BK, 32>(tq, tk, a, st);
+}
+
+template <int DIDX>
+cudaError_t launch_b(int bk, const CUtensorMap& tq, const CUtensorMap& tk, const IdxArgs& a, cudaStream_t st) {
+  if (bk == 64) return launch_k<DIDX, 64>(tq, tk, a, st);
+  return launch_k<DIDX, 128>(tq, tk, a, st);
+}
+
+}  // namespace
+
+int run_index_topk_prefill(const msa_params& p, const void* q_idx, const void* k_idx, int n_q, int n_kv,
+                           int q_pos0, int32_t* block_ids, int* status, cudaStream_t stream) {
+  if (n_q == 0) return MSA_OK;
+  const int sw_elems = p.d_idx >= 64 ? 64 : p.d_idx;    // TMA box inner extent (elements)
+  const CUtensorMapSwizzle swz = p.d_idx >= 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  CUtensorMap tq, tk;
+  {
+    const uint64_t dims[3] = {static_cast<uint64_t>(p.d_idx), static_cast<uint64_t>(p.h_kv),
+                              static_cast<uint64_t>(n_q)};
+    const uint64_t strides[2] = {static_cast<uint64_t>(p.d_idx) * 2, static_cast<uint64_t>(p.h_kv) * p.d_idx * 2};
+    const uint32_t box[3] = {static_cast<uint32_t>(sw_elems), 1, 128};
+    if (!encode_tma_bf16(&tq, 3, q_idx, dims, strides, box, swz)) return MSA_ERR_CUDA;
+  }
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(p.d_idx), static_cast<uint64_t>(n_kv)};
+    const uint64_t strides[1] = {static_cast<uint64_t>(p.d_idx) * 2};
+    const uint32_t box[2] = {static_cast<uint32_t>(sw_elems), 128};
+    if (!encode_tma_bf16(&tk, 2, k_idx, dims, strides, box, swz)) return MSA_ERR_CUDA;
+  }
+  IdxArgs a;
+  a.block_ids = block_ids;
+  a.status = status;
+  a.n_q = n_q;
+  a.n_kv = n_kv;
+  a.q_pos0 = q_pos0;
+  a.h_kv = p.h_kv;
+  a.topk = p.topk;
+  a.causal = p.causal;
+  a.force_local = p.force_local;
+  a.n_tiles = (n_q + kRows - 1) / kRows;
+  a.n_pairs = (p.h_kv + 1) / 2;
+  cudaError_t e;
+  switch (p.d_idx) {
+    case 32: e = launch_b<32>(p.block_k, tq, tk, a, stream); break;
+    case 64: e = launch_b<64>(p.block_k, tq, tk, a, stream); break;
+    default: e = launch_b<128>(p.block_k, tq, tk, a, stream); break;
+  }
+  return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
+}
+
+}  // namespace msa

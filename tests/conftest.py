@@ -10,6 +10,8 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA GPU (B200, sm_100a)")
+    import long_context_index_b200 as msa
+    msa.check_status = True   # every library call in the tests checks the device status word
 
 
 def gpu_available() -> bool:

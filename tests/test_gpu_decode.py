@@ -1,0 +1,70 @@
+"""GPU parity of one batched decode step (msa_sparse_attn_decode) against the
+fp64 oracle: block ids bit for bit, O within 1e-2 abs + 1e-2 rel."""
+import numpy as np
+import pytest
+import torch
+
+import long_context_index_b200 as msa
+import oracle
+from synth import WORKLOADS, Workload, make_decode
+from tests.gpu_util import assert_close, dev, host_f64, params_pair
+
+pytestmark = pytest.mark.gpu
+
+
+def small(**kw):
+    base = dict(name="dcase", kind="decode", h_q=8, h_kv=2, d=64, d_idx=32, block_k=64, topk=4, seed=300,
+                batch=5, kv_min=300, kv_max=1500, needles=2)
+    base.update(kw)
+    return Workload(**base)
+
+
+def run_case(w, seqs=None, dense=False, force_local=1):
+    t = make_decode(w)
+    p, po = params_pair(w.h_q, w.h_kv, w.d, w.d_idx, w.block_k, w.topk, 1, force_local)
+    ids, o = msa.sparse_attn_decode(p, dev(t["q"]), dev(t["q_idx"]), dev(t["k_cache"]), dev(t["v_cache"]),
+                                    dev(t["k_idx_cache"]), dev(t["cu_kv"]), int(t["lens"].max()), dense=dense)
+    torch.cuda.synchronize()
+    B = t["q"].shape[0]
+    seqs = np.arange(B) if seqs is None else np.asarray(seqs)
+    ids_ref, o_ref = oracle.decode(po, t["q"], t["q_idx"], t["k_cache"], t["v_cache"], t["k_idx_cache"],
+                                   t["cu_kv"], seqs=seqs, dense=dense)
+    if not dense:
+        got_ids = ids.cpu().numpy()[seqs]
+        assert np.array_equal(got_ids, ids_ref), (np.argwhere(got_ids != ids_ref)[:4])
+        for b, r, pk in t["needles"]:
+            if b in set(seqs.tolist()):
+                assert pk // w.block_k in ids.cpu().numpy()[b, r]
+    assert_close(host_f64(o)[seqs], o_ref, what="decode O")
+
+
+def test_small_decode():
+    run_case(small())
+
+
+def test_small_decode_dense():
+    run_case(small(), dense=True)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(h_q=64, h_kv=4, d=128, d_idx=64, block_k=128, topk=16, batch=3, kv_min=5000, kv_max=20000),
+    dict(h_q=16, h_kv=4, d=128, d_idx=64, block_k=64, topk=6, batch=4, kv_min=1, kv_max=700),
+    dict(h_q=64, h_kv=2, d=64, d_idx=128, block_k=128, topk=32, batch=2, kv_min=9000, kv_max=9000),  # 2 head tiles
+    dict(batch=7, kv_min=64, kv_max=64),           # one full block per sequence
+    dict(batch=3, kv_min=1, kv_max=3),             # tiny caches
+    dict(topk=1, batch=3),                         # the local block alone
+])
+def test_shapes(kw):
+    run_case(small(seed=kw.get("batch", 1) * 31 + kw.get("kv_max", 0), **kw))
+
+
+def test_force_local_off():
+    run_case(small(seed=41), force_local=0)
+
+
+def test_decode_b64_64k_128k():
+    run_case(WORKLOADS["decode_b64_64k_128k"])
+
+
+def test_decode_b64_64k_128k_dense_sampled():
+    run_case(WORKLOADS["decode_b64_64k_128k"], dense=True, seqs=[0, 17, 63])
