@@ -1,0 +1,436 @@
+"""Benchmark of the MSA hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one pass of the whole hot path over synthetic inputs resident in
+HBM: the index branch and the main branch of a 128K-token causal prefill
+(64 query heads, 4 KV heads, d = 128, d_idx = 64, B_k = 128, k = 16), then one
+decode step of 64 sequences with KV lengths in [64K, 128K] (the same model
+shape).  Tokens per step = 131072 prefill + 64 decode tokens.
+
+Prints one JSON line (rank 0).  Under torchrun each rank runs its own
+independent problem (weak scaling, no data-path collective); the time is the
+max over ranks.  ``--impl reference`` times the fp64 CPU oracle on bounded
+samples of the same workload on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth import WORKLOADS, Workload, make_decode, make_prefill  # noqa: E402
+
+METRIC = "MSA prefill & decode tokens/s at 128K ctx; % of B200 tensor / HBM roofline"
+PREFILL = WORKLOADS["prefill_128k"]
+DECODE = WORKLOADS["decode_b64_64k_128k"]
+
+
+def cases(name):
+    """The bench workload, or a smaller instance of the same kernels for ncu
+    captures ("small": 32K prefill and 8 decode sequences)."""
+    if name == "small":
+        return WORKLOADS["prefill_32k"], Workload(**{**DECODE.__dict__, "batch": 8})
+    return PREFILL, DECODE
+
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 1024 * 1024
+
+# DRAM traffic per launch from the committed ncu captures, keyed by kernel,
+# with the digest of the kernel source it was measured on (stale -> null).
+TRAFFIC = {}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+def src_digest(name: str) -> str:
+    path = os.path.join(ROOT, "long_context_index_b200", "csrc", name)
+    return hashlib.sha1(open(path, "rb").read()).hexdigest()[:12]
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.lines = []
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", gpu_id, "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gpu_smi_id(torch, dev: int) -> str:
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(dev)
+
+
+# ---------------------------------------------------------------------------
+# our implementation
+# ---------------------------------------------------------------------------
+def to_dev(torch, a, pin=False):
+    t = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a)
+    if pin:
+        t = t.pin_memory()
+    return t
+
+
+def bf16(torch, t):
+    return t.view(torch.bfloat16) if t.dtype == torch.int16 else t
+
+
+def run_ours(args, rank, world, torch, dist):
+    import long_context_index_b200 as msa
+    from long_context_index_b200 import flops
+
+    PREFILL, DECODE = cases(args.case)
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+    seed_off = 1000 * rank   # each rank its own independent problem
+    wp = Workload(**{**PREFILL.__dict__, "seed": PREFILL.seed + seed_off})
+    wd = Workload(**{**DECODE.__dict__, "seed": DECODE.seed + seed_off})
+    tp = make_prefill(wp)
+    td = make_decode(wd)
+    pp = msa.Params.make(wp.h_q, wp.h_kv, wp.d, wp.d_idx, wp.block_k, wp.topk)
+    pd = msa.Params.make(wd.h_q, wd.h_kv, wd.d, wd.d_idx, wd.block_k, wd.topk)
+    n = wp.n_q
+    B = wd.batch
+    max_kv = int(td["lens"].max())
+
+    # Host (pinned) and device copies of every input.
+    host = {k: to_dev(torch, tp[k], pin=True) for k in ("q", "k", "v", "q_idx", "k_idx")}
+    hostd = {k: to_dev(torch, td[k], pin=True) for k in ("q", "q_idx", "cu_kv")}
+    d_in = {k: bf16(torch, v.to(dev)) for k, v in host.items()}
+    dd = {k: bf16(torch, to_dev(torch, td[k]).to(dev)) for k in ("q", "q_idx", "k_cache", "v_cache", "k_idx_cache",
+                                                                  "cu_kv")}
+    ids = torch.empty((n, wp.h_kv, wp.topk), dtype=torch.int32, device=dev)
+    o = torch.empty((n, wp.h_q, wp.d), dtype=torch.bfloat16, device=dev)
+    dids = torch.empty((B, wd.h_kv, wd.topk), dtype=torch.int32, device=dev)
+    do = torch.empty((B, wd.h_q, wd.d), dtype=torch.bfloat16, device=dev)
+    ws_i = torch.empty(msa.workspace_size(msa.OP_INDEX_TOPK, pp, n, n), dtype=torch.uint8, device=dev)
+    ws_p = torch.empty(max(256, msa.workspace_size(msa.OP_PREFILL, pp, n, n)), dtype=torch.uint8, device=dev)
+    ws_d = torch.empty(msa.workspace_size(msa.OP_DECODE, pd, batch=B, max_kv=max_kv), dtype=torch.uint8,
+                       device=dev)
+
+    def step():
+        msa.index_topk(pp, d_in["q_idx"], d_in["k_idx"], 0, block_ids=ids, ws=ws_i)
+        ev[1].record(stream)
+        msa.sparse_attn_prefill(pp, d_in["q"], d_in["k"], d_in["v"], ids, 0, out=o, ws=ws_p)
+        ev[2].record(stream)
+        msa.sparse_attn_decode(pd, dd["q"], dd["q_idx"], dd["k_cache"], dd["v_cache"], dd["k_idx_cache"],
+                               dd["cu_kv"], max_kv, block_ids=dids, out=do, ws=ws_d)
+
+    E = torch.cuda.Event
+    ev = [E(enable_timing=True) for _ in range(4)]
+    for _ in range(args.warmup):
+        ev[0].record(stream)
+        step()
+        ev[3].record(stream)
+    torch.cuda.synchronize()
+    for wsx in (ws_i, ws_p, ws_d):
+        rc = msa.device_status(wsx)
+        if rc:
+            raise RuntimeError("device status %d after warm-up" % rc)
+
+    # ---- timed region: K steps, per-call CUDA events on the launching stream
+    clk = ClockSampler(gpu_smi_id(torch, torch.cuda.current_device())) if rank == 0 else None
+    time.sleep(0.3 if clk else 0)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    evs = [[E(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for s in range(args.steps):
+        ev = evs[s]
+        ev[0].record(stream)
+        step()
+        ev[3].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = clk.stop() if clk else None
+    t_total = evs[0][0].elapsed_time(evs[-1][3])
+    t_idx = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    t_attn = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+    t_dec = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
+    for wsx in (ws_i, ws_p, ws_d):
+        rc = msa.device_status(wsx)
+        if rc:
+            raise RuntimeError("device status %d after the timed steps" % rc)
+    if world > 1:
+        tt = torch.tensor([t_total], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_total = float(tt.item())
+    ms_step = t_total / args.steps
+    tokens_step = n + B
+    value = tokens_step * world / (ms_step / 1e3)
+
+    # ---- useful work of this step (from the ids of the last step)
+    ids_h = ids.cpu().numpy()
+    dids_h = dids.cpu().numpy()
+    f_idx = flops.index_flops(n, n, 0, wp.h_kv, wp.d_idx)
+    sel = flops.selected_keys(ids_h, wp.block_k, n, 0)
+    f_main = flops.main_flops(sel, wp.h_q, wp.h_kv, wp.d)
+    b_dec = flops.decode_bytes(td["lens"], dids_h, wd.h_q, wd.h_kv, wd.d, wd.d_idx, wd.block_k)
+
+    # ---- dense run of the same kernels (every causal block), once, untimed above
+    t_dense_p = t_dense_d = None
+    if not args.no_dense:
+        e0, e1, e2 = E(enable_timing=True), E(enable_timing=True), E(enable_timing=True)
+        e0.record(stream)
+        msa.sparse_attn_prefill(pp, d_in["q"], d_in["k"], d_in["v"], None, 0, out=o, ws=ws_p)
+        e1.record(stream)
+        msa.sparse_attn_decode(pd, dd["q"], None, dd["k_cache"], dd["v_cache"], None, dd["cu_kv"], max_kv,
+                               dense=True, out=do, ws=ws_d)
+        e2.record(stream)
+        torch.cuda.synchronize()
+        t_dense_p, t_dense_d = e0.elapsed_time(e1), e1.elapsed_time(e2)
+
+    # ---- end to end through the public API with host buffers
+    out_h = torch.empty((n, wp.h_q, wp.d), dtype=torch.int16).pin_memory()
+    ids_hp = torch.empty((n, wp.h_kv, wp.topk), dtype=torch.int32).pin_memory()
+    dout_h = torch.empty((B, wd.h_q, wd.d), dtype=torch.int16).pin_memory()
+    dids_hp = torch.empty((B, wd.h_kv, wd.topk), dtype=torch.int32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in list(host.values()) + list(hostd.values()))
+    d2h = sum(t.numel() * t.element_size() for t in (out_h, ids_hp, dout_h, dids_hp))
+
+    def e2e_step():
+        for k_, t_ in host.items():
+            d_in[k_].view(torch.int16).copy_(t_, non_blocking=True)
+        for k_, t_ in hostd.items():
+            dd[k_].view(t_.dtype).copy_(t_, non_blocking=True)
+        msa.index_topk(pp, d_in["q_idx"], d_in["k_idx"], 0, block_ids=ids, ws=ws_i)
+        msa.sparse_attn_prefill(pp, d_in["q"], d_in["k"], d_in["v"], ids, 0, out=o, ws=ws_p)
+        msa.sparse_attn_decode(pd, dd["q"], dd["q_idx"], dd["k_cache"], dd["v_cache"], dd["k_idx_cache"],
+                               dd["cu_kv"], max_kv, block_ids=dids, out=do, ws=ws_d)
+        out_h.copy_(o.view(torch.int16), non_blocking=True)
+        ids_hp.copy_(ids, non_blocking=True)
+        dout_h.copy_(do.view(torch.int16), non_blocking=True)
+        dids_hp.copy_(dids, non_blocking=True)
+
+    e2e_value = None
+    if not args.no_e2e:
+        e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        a, b = E(enable_timing=True), E(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        t_e2e = a.elapsed_time(b)
+        if world > 1:
+            tt = torch.tensor([t_e2e], dtype=torch.float64, device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            t_e2e = float(tt.item())
+        e2e_value = tokens_step * world / (t_e2e / args.steps / 1e3)
+
+    peaks, peak_src = load_peaks()
+    kern = {
+        "index_topk_prefill": {"ms": t_idx, "bound": "tensor", "work": f_idx, "unit": "TFLOP/s",
+                               "achieved": f_idx / (t_idx / 1e3) / 1e12, "peak": peaks["bf16_tflops"]},
+        "attn_prefill": {"ms": t_attn, "bound": "tensor", "work": f_main, "unit": "TFLOP/s",
+                         "achieved": f_main / (t_attn / 1e3) / 1e12, "peak": peaks["bf16_tflops"]},
+        "decode_step": {"ms": t_dec, "bound": "hbm", "work": b_dec, "unit": "GB/s",
+                        "achieved": b_dec / (t_dec / 1e3) / 1e9, "peak": peaks["hbm_gbs"]},
+    }
+    for k_, v_ in kern.items():
+        v_["frac"] = v_["achieved"] / v_["peak"]
+    dom = max(kern, key=lambda k_: kern[k_]["ms"])
+    dk = kern[dom]
+    traffic = None
+    if dom in TRAFFIC and TRAFFIC[dom][1] == src_digest(TRAFFIC[dom][2]):
+        traffic = TRAFFIC[dom][0]
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded; integer index inputs with planted needles)",
+        "config": {"workload": "%s + %s" % (wp.name, wd.name if wd.batch == 64 else "decode_b%d" % wd.batch),
+                   "seq_len": n, "decode_batch": B,
+                   "h_q": wp.h_q, "h_kv": wp.h_kv, "d": wp.d, "d_idx": wp.d_idx, "block_k": wp.block_k,
+                   "topk": wp.topk, "tokens_per_step": tokens_step,
+                   "l2": "inputs larger than L2 (Q alone 2 GiB; decode caches 13 GB), no flush"},
+        "prefill": {"ms": t_idx + t_attn, "tokens_per_s": n * world / ((t_idx + t_attn) / 1e3),
+                    "index_ms": t_idx, "attn_ms": t_attn, "useful_tflop": (f_idx + f_main) / 1e12,
+                    "tensor_frac": (f_idx + f_main) / ((t_idx + t_attn) / 1e3) / 1e12 / peaks["bf16_tflops"]},
+        "decode": {"ms": t_dec, "tokens_per_s": B * world / (t_dec / 1e3), "bytes": b_dec,
+                   "hbm_frac": b_dec / (t_dec / 1e3) / 1e9 / peaks["hbm_gbs"]},
+        "dense": None if t_dense_p is None else {
+            "prefill_ms": t_dense_p, "decode_ms": t_dense_d,
+            "prefill_sparse_speedup": t_dense_p / (t_idx + t_attn), "decode_sparse_speedup": t_dense_d / t_dec},
+        "roofline": {"kernel": dom, "bound": dk["bound"], "achieved": dk["achieved"], "peak": dk["peak"],
+                     "unit": dk["unit"], "frac": dk["frac"], "traffic": traffic,
+                     "peak_source": peak_src + (" burst" if dk["bound"] == "tensor" else "")},
+        "kernels": {k_: {kk: vv for kk, vv in v_.items() if kk != "work"} for k_, v_ in kern.items()},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "note": "prefill inputs and outputs cross PCIe every step; decode KV caches stay resident"},
+        "gpu_launches": 6 * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.case == "full":
+        line["cpu_baseline"] = cpu_baseline(tp, td, wp, wd)
+    return line
+
+
+# ---------------------------------------------------------------------------
+# the fp64 oracle on the host cores (CPU baseline and the reference arm)
+# ---------------------------------------------------------------------------
+def oracle_sample(tp, td, wp, wd, rows, seqs, threads):
+    import oracle
+    po = oracle.params(wp.h_q, wp.h_kv, wp.d, wp.d_idx, wp.block_k, wp.topk, threads=threads)
+    t0 = time.perf_counter()
+    ids = oracle.index_topk(po, tp["q_idx"], tp["k_idx"], rows=rows)
+    oracle.sparse_attn(po, tp["q"], tp["k"], tp["v"], ids, rows=rows)
+    pd = oracle.params(wd.h_q, wd.h_kv, wd.d, wd.d_idx, wd.block_k, wd.topk, threads=threads)
+    oracle.decode(pd, td["q"], td["q_idx"], td["k_cache"], td["v_cache"], td["k_idx_cache"], td["cu_kv"], seqs=seqs)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(tp, td, wp, wd, rows_n=96, seqs_n=8):
+    threads = os.cpu_count() or 1
+    rows = np.linspace(0, wp.n_q - 1, rows_n).astype(np.int32)
+    seqs = np.arange(seqs_n, dtype=np.int32)
+    t = oracle_sample(tp, td, wp, wd, rows, seqs, threads)
+    return {"value": (rows_n + seqs_n) / t, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": "%d prefill rows evenly spaced over the 128K prefill (index + main branch) and %d decode "
+                      "sequences, fp64, %.1f s" % (rows_n, seqs_n, t)}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    tp = make_prefill(PREFILL)
+    td = make_decode(DECODE)
+    threads = os.cpu_count() or 1
+    rows_n, seqs_n = 24, 2
+    rng = np.random.default_rng(0)
+
+    def one():
+        rows = np.sort(rng.integers(0, PREFILL.n_q, rows_n)).astype(np.int32)
+        seqs = np.sort(rng.choice(DECODE.batch, seqs_n, replace=False)).astype(np.int32)
+        return oracle_sample(tp, td, PREFILL, DECODE, rows, seqs, threads)
+
+    for _ in range(args.warmup):
+        one()
+    times = [one() for _ in range(args.steps)]
+    t = sum(times) / len(times)
+    value = (rows_n + seqs_n) / t
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "prefill_128k + decode_b64_64k_128k", "seq_len": PREFILL.n_q,
+                   "decode_batch": DECODE.batch},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": "per step %d random rows of the 128K prefill (index + main branch) and %d "
+                                   "decode sequences" % (rows_n, seqs_n)},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--case", choices=["full", "small"], default="full")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
+    try:
+        line = run_ours(args, rank, world, torch, dist)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
