@@ -356,7 +356,7 @@ def oracle_sample(tp, td, wp, wd, rows, seqs, threads):
     return time.perf_counter() - t0
 
 
-def cpu_baseline(tp, td, wp, wd, rows_n=96, seqs_n=8):
+def cpu_baseline(tp, td, wp, wd, rows_n=2048, seqs_n=32):
     threads = os.cpu_count() or 1
     rows = np.linspace(0, wp.n_q - 1, rows_n).astype(np.int32)
     seqs = np.arange(seqs_n, dtype=np.int32)
