@@ -334,7 +334,8 @@ def run_ours(args, rank, world, torch, dist):
         "kernels": {k_: {kk: vv for kk, vv in v_.items() if kk != "work"} for k_, v_ in kern.items()},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "note": "prefill inputs and outputs cross PCIe every step; decode KV caches stay resident"},
-        "gpu_launches": 6 * args.steps,
+        # ours per step: index 1; sparse prefill 5 (count, scan, fill, KV-outer, merge); decode 4
+        "gpu_launches": 10 * args.steps,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.case == "full":

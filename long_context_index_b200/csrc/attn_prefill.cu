@@ -406,15 +406,16 @@ cudaError_t launch_g(int G, const CUtensorMap& tq, const CUtensorMap& tk, const 
 
 }  // namespace
 
-size_t prefill_workspace_bytes(const msa_params&, int, int) { return 0; }
+size_t prefill_workspace_bytes(const msa_params& p, int n_q, int n_kv) {
+  return sparse_prefill_workspace_bytes(p, n_q, n_kv);
+}
 
 int run_sparse_attn_prefill(const msa_params& p, const void* q, const void* k, const void* v,
-                            const int32_t* block_ids, int n_q, int n_kv, int q_pos0, void* o, void* /*ws*/,
-                            size_t /*ws_bytes*/, int* status, cudaStream_t stream) {
+                            const int32_t* block_ids, int n_q, int n_kv, int q_pos0, void* o, void* ws,
+                            size_t ws_bytes, int* status, cudaStream_t stream) {
   if (n_q == 0) return MSA_OK;
   const int G = p.h_q / p.h_kv;
   const int QT = 128 / G;
-  if (block_ids && QT * p.topk > kMaxList) return MSA_ERR_UNSUPPORTED;
   CUtensorMap tq, tk, tv;
   {
     const uint64_t dims[3] = {static_cast<uint64_t>(p.d), static_cast<uint64_t>(p.h_q), static_cast<uint64_t>(n_q)};
@@ -430,6 +431,8 @@ int run_sparse_attn_prefill(const msa_params& p, const void* q, const void* k, c
     if (!encode_tma_bf16(&tk, 3, k, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MSA_ERR_CUDA;
     if (!encode_tma_bf16(&tv, 3, v, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MSA_ERR_CUDA;
   }
+  if (block_ids)   // sparse: block-major schedule (attn_sparse.cu)
+    return run_sparse_attn_kvouter(p, q, tk, tv, block_ids, n_q, n_kv, q_pos0, o, ws, ws_bytes, status, stream);
   AttnArgs a;
   a.block_ids = block_ids;
   a.o = static_cast<uint16_t*>(o);

@@ -1,0 +1,655 @@
+// attn_sparse.cu -- block-major (KV-outer) main branch of a sparse prefill.
+//
+// Computes eq. (8) of the titansim.online summary of "MiniMax Sparse
+// Attention" (section 4.3) for every selected block, with the block as the
+// outer loop ("KV-Outer", section 4.4.2): the queries that selected a KV block
+// are gathered so one block load feeds full 128-row tensor-core tiles, and
+// the per-block results are merged afterwards (the pages' "two-stage merge",
+// with no atomics on the outputs).
+//
+//   1. sched_count / sched_scan / sched_fill: invert block_ids [n_q, h_kv, k]
+//      into one list per (group r, block b) of the (query, slot) pairs that
+//      selected it (counting sort; slot = position of b in the query's ids).
+//   2. attn_kvouter_kernel (persistent, warp-specialised, tcgen05):
+//      * warp 0 grabs the next (r, b) list with an atomic counter, loads
+//        K_b, V_b once by TMA, then streams chunks of 128/G queries of the
+//        list (each query's G head rows of group r are one 3-D TMA box), and
+//        publishes a descriptor per chunk in a 4-deep ring.
+//      * warp 1 issues S = Q K_b^T into one of two TMEM S buffers and
+//        O = P V_b (P read back from TMEM) into one of two TMEM O buffers.
+//      * warps 2..5 (softmax): one thread per row; the exact softmax of the
+//        row over the block's visible keys (causal only in the local block),
+//        in two passes over the TMEM row (max, then exp and bf16 pack in
+//        32-column chunks); P is written over S; (m, l) go to the epilogue.
+//      * warps 6..9 (epilogue): o = O / l in bf16 and lse2 = m c + log2 l to
+//        the partial buffers [slot][query][head].
+//   3. merge_partials_kernel: per (query, group), O = sum_s 2^(lse2_s - L) o_s
+//      over the valid slots, L = log2 sum 2^lse2_s; rounded to bf16.
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "msa_internal.h"
+#include "ptx.cuh"
+
+namespace msa {
+namespace {
+
+constexpr int kThreads = 320;   // 10 warps
+constexpr int kSoftW0 = 2;      // softmax warps 2..5 (one per TMEM lane quarter)
+constexpr int kEpiW0 = 6;       // epilogue warps 6..9
+constexpr int kQStages = 2;
+constexpr int kKVStages = 2;
+constexpr int kDesc = 4;        // descriptor ring depth
+constexpr int kSchedThreads = 256;
+
+template <int D, int BK>
+struct KvoCfg {
+  static constexpr int kAtoms = D / 64;
+  static constexpr int kQBytes = 128 * D * 2;
+  static constexpr int kKVBytes = BK * D * 2;          // one of K or V
+  static constexpr int kSmemData = kQStages * kQBytes + kKVStages * 2 * kKVBytes;
+  static constexpr int kSmemBytes = kSmemData + 8192 + 1024;
+  static constexpr int kColS = 0;        // S/P buffers: [0, BK), [BK, 2BK)
+  static constexpr int kColO = 2 * BK;   // O buffers: [2BK, 2BK + D), [2BK + D, 2BK + 2D)
+  static constexpr int kTmemCols = (2 * BK + 2 * D) <= 256 ? 256 : 512;
+};
+
+// One chunk of gathered queries of a (group, block) list.
+struct Desc {
+  int entry[128];   // (query << 5) | slot, for the first `count` rows' queries
+  int r, b, count, kvs;
+  int first_of_kv, last_of_kv, end;
+};
+
+struct KvoArgs {
+  const int* offs;       // [h_kv * nb + 1] list offsets
+  const int* entries;    // (query << 5) | slot, grouped by list
+  const int* lists;      // non-empty list ids (r * nb + b)
+  const int* n_lists;
+  int* work_counter;
+  uint16_t* part_o;      // [topk][n_q][h_q][d] bf16
+  float* part_lse;       // [topk][n_q][h_q]
+  int* status;
+  int n_q, n_kv, q_pos0, h_q, h_kv, topk, causal, nb;
+  float scale_log2;
+};
+
+template <int D, int BK, int G>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const KvoArgs args) {
+  using Cfg = KvoCfg<D, BK>;
+  constexpr int QPC = 128 / G;   // queries per chunk
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sq = smem;                                        // [stage][atoms][128][128 B]
+  uint8_t* skv = smem + kQStages * Cfg::kQBytes;             // [stage][K|V][atoms][BK][128 B]
+  Desc* desc = reinterpret_cast<Desc*>(smem + Cfg::kSmemData);
+  float2* ml = reinterpret_cast<float2*>(desc + kDesc);      // [kDesc][128] (m, l) per row
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ml + kDesc * 128);
+  uint64_t* q_full = bars;                                   // [kQStages]
+  uint64_t* q_empty = q_full + kQStages;
+  uint64_t* kv_full = q_empty + kQStages;                    // [kKVStages]
+  uint64_t* kv_empty = kv_full + kKVStages;
+  uint64_t* d_full = kv_empty + kKVStages;                   // [kDesc]
+  uint64_t* d_empty = d_full + kDesc;
+  uint64_t* s_full = d_empty + kDesc;                        // [2]
+  uint64_t* s_free = s_full + 2;
+  uint64_t* p_full = s_free + 2;
+  uint64_t* o_full = p_full + 2;
+  uint64_t* o_free = o_full + 2;
+  uint64_t* ml_full = o_free + 2;                            // [kDesc]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ml_full + kDesc);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = warp_id();
+  const int lane = lane_id();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kQStages; ++s) {
+      mbar_init(&q_full[s], 1);
+      mbar_init(&q_empty[s], 1);
+    }
+    for (int s = 0; s < kKVStages; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int s = 0; s < kDesc; ++s) {
+      mbar_init(&d_full[s], 1);
+      mbar_init(&d_empty[s], 9);   // MMA thread + 4 softmax warps + 4 epilogue warps
+      mbar_init(&ml_full[s], 4);   // 4 softmax warps
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_free[s], 1);
+      mbar_init(&p_full[s], 4);
+      mbar_init(&o_full[s], 1);
+      mbar_init(&o_free[s], 4);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtx wc{abort_flag, args.status};
+  const int n_lists = *args.n_lists;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      int t = 0;      // chunk counter
+      int kvc = 0;    // KV stage use counter
+      bool ok = true;
+      while (ok) {
+        const int li = atomicAdd(args.work_counter, 1);
+        if (li >= n_lists) break;
+        const int rb = args.lists[li];
+        const int r = rb / args.nb, b = rb % args.nb;
+        const int start = args.offs[rb], cnt = args.offs[rb + 1] - start;
+        const int kvs = kvc % kKVStages;
+        if (!mbar_wait(&kv_empty[kvs], ((kvc / kKVStages) & 1) ^ 1, wc)) break;
+        mbar_arrive_expect_tx(&kv_full[kvs], 2 * Cfg::kKVBytes);
+        uint8_t* sk = skv + kvs * 2 * Cfg::kKVBytes;
+        for (int a = 0; a < Cfg::kAtoms; ++a) {
+          tma_load_3d(sk + a * BK * 128, &tm_k, &kv_full[kvs], a * 64, r, b * BK);
+          tma_load_3d(sk + Cfg::kKVBytes + a * BK * 128, &tm_v, &kv_full[kvs], a * 64, r, b * BK);
+        }
+        ++kvc;
+        for (int c0 = 0; c0 < cnt; c0 += QPC) {
+          const int qs = t % kQStages, ds = t % kDesc;
+          if (!mbar_wait(&d_empty[ds], ((t / kDesc) & 1) ^ 1, wc)) { ok = false; break; }
+          if (!mbar_wait(&q_empty[qs], ((t / kQStages) & 1) ^ 1, wc)) { ok = false; break; }
+          Desc& dd = desc[ds];
+          const int n_here = min(QPC, cnt - c0);
+          dd.r = r;
+          dd.b = b;
+          dd.count = n_here;
+          dd.kvs = kvs;
+          dd.first_of_kv = c0 == 0;
+          dd.last_of_kv = c0 + QPC >= cnt;
+          dd.end = 0;
+          mbar_arrive_expect_tx(&q_full[qs], Cfg::kQBytes);
+          for (int qi = 0; qi < QPC; ++qi) {
+            const int e = qi < n_here ? args.entries[start + c0 + qi] : -1;
+            dd.entry[qi] = e;
+            const int q = e >= 0 ? (e >> 5) : args.n_q;   // past the end: TMA fills zeros
+            for (int a = 0; a < Cfg::kAtoms; ++a)
+              tma_load_3d(sq + qs * Cfg::kQBytes + a * 128 * 128 + qi * G * 128, &tm_q, &q_full[qs], a * 64,
+                          r * G, q);
+          }
+          mbar_arrive(&d_full[ds]);
+          ++t;
+        }
+      }
+      // End marker for the consumers.
+      if (ok && !*abort_flag) {
+        const int ds = t % kDesc;
+        if (mbar_wait(&d_empty[ds], ((t / kDesc) & 1) ^ 1, wc)) {
+          desc[ds].end = 1;
+          mbar_arrive(&d_full[ds]);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- UMMA
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, BK, false, false);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
+      const uint32_t sq_addr = smem_u32(sq);
+      const uint32_t skv_addr = smem_u32(skv);
+      int kvc = 0;
+      int prev_kvs = 0, prev_last = 0;
+      auto issue_pv = [&](int j, int kvs, int last) -> bool {
+        const int sb = j & 1;
+        if (!mbar_wait(&p_full[sb], (j >> 1) & 1, wc)) return false;
+        if (!mbar_wait(&o_free[sb], ((j >> 1) & 1) ^ 1, wc)) return false;
+        tc_fence_after();
+        const uint32_t sv_addr = skv_addr + kvs * 2 * Cfg::kKVBytes + Cfg::kKVBytes;
+        const uint32_t p_tmem = tmem + Cfg::kColS + sb * BK;
+        const uint32_t o_tmem = tmem + Cfg::kColO + sb * D;
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          const uint64_t bdesc = smem_desc(sv_addr + kk * 2048, BK * 128, 1024, kSwizzle128B);
+          umma_ts(o_tmem, p_tmem + kk * 8, bdesc, idesc_o, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&o_full[sb]);
+        umma_commit(&s_free[sb]);
+        if (last) umma_commit(&kv_empty[kvs]);
+        return true;
+      };
+      int t = 0;
+      bool ok = true;
+      while (ok) {
+        const int ds = t % kDesc;
+        if (!mbar_wait(&d_full[ds], (t / kDesc) & 1, wc)) { ok = false; break; }
+        const Desc& dd = desc[ds];
+        const int end = dd.end, kvs = dd.kvs, first = dd.first_of_kv, last = dd.last_of_kv;
+        mbar_arrive(&d_empty[ds]);
+        if (end) break;
+        const int qs = t % kQStages, sb = t & 1;
+        if (first) {
+          if (!mbar_wait(&kv_full[kvs], (kvc / kKVStages) & 1, wc)) { ok = false; break; }
+          ++kvc;
+        }
+        if (!mbar_wait(&q_full[qs], (t / kQStages) & 1, wc)) { ok = false; break; }
+        if (!mbar_wait(&s_free[sb], ((t >> 1) & 1) ^ 1, wc)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sk_addr = skv_addr + kvs * 2 * Cfg::kKVBytes;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const int atom = ks / 4;
+          const uint32_t koff = (ks % 4) * 32;
+          const uint64_t adesc =
+              smem_desc(sq_addr + qs * Cfg::kQBytes + atom * 128 * 128 + koff, 16, 1024, kSwizzle128B);
+          const uint64_t bdesc = smem_desc(sk_addr + atom * BK * 128 + koff, 16, 1024, kSwizzle128B);
+          umma_ss(tmem + Cfg::kColS + sb * BK, adesc, bdesc, idesc_s, ks > 0 ? 1u : 0u);
+        }
+        umma_commit(&q_empty[qs]);
+        umma_commit(&s_full[sb]);
+        if (t > 0 && !issue_pv(t - 1, prev_kvs, prev_last)) { ok = false; break; }
+        prev_kvs = kvs;
+        prev_last = last;
+        ++t;
+      }
+      if (ok && t > 0) issue_pv(t - 1, prev_kvs, prev_last);
+    }
+  } else if (warp >= kSoftW0 && warp < kEpiW0) {
+    // ---------------------------------------------------------------- softmax
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const int qi = row / G;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const float c = args.scale_log2;
+    for (int t = 0;; ++t) {
+      const int ds = t % kDesc;
+      if (!mbar_wait(&d_full[ds], (t / kDesc) & 1, wc)) break;
+      const Desc& dd = desc[ds];
+      if (dd.end) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&d_empty[ds]);
+        break;
+      }
+      const int e = qi < dd.count ? dd.entry[qi] : -1;
+      const int b = dd.b;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&d_empty[ds]);
+      int lim = 0;
+      if (e >= 0) {
+        const int p = args.q_pos0 + (e >> 5);
+        const int kv_lim = args.causal ? min(p + 1, args.n_kv) : args.n_kv;
+        lim = min(BK, kv_lim - b * BK);
+      }
+      const int sb = t & 1;
+      if (!mbar_wait(&s_full[sb], (t >> 1) & 1, wc)) break;
+      tc_fence_after();
+      const uint32_t s_tmem = lane_base + Cfg::kColS + sb * BK;
+      // Pass 1: row max over the visible keys.
+      float mx = __int_as_float(0xff800000);
+#pragma unroll
+      for (int cc = 0; cc < BK / 32; ++cc) {
+        uint32_t v[32];
+        tmem_ld32(s_tmem + cc * 32, v);
+        tmem_ld_wait();
+        if (lim >= (cc + 1) * 32) {
+#pragma unroll
+          for (int i = 0; i + 2 < 32; i += 3)
+            mx = max3f(mx, __uint_as_float(v[i]), fmaxf(__uint_as_float(v[i + 1]), __uint_as_float(v[i + 2])));
+          mx = max3f(mx, __uint_as_float(v[30]), __uint_as_float(v[31]));
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (cc * 32 + i < lim) mx = fmaxf(mx, __uint_as_float(v[i]));
+        }
+      }
+      // Pass 2: p = 2^((s - max) c), bf16 pairs written back over S.
+      const float bias = mx == __int_as_float(0xff800000) ? 0.f : mx * c;
+      float lsum = 0.f;
+#pragma unroll
+      for (int cc = 0; cc < BK / 32; ++cc) {
+        uint32_t v[32];
+        tmem_ld32(s_tmem + cc * 32, v);
+        tmem_ld_wait();
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const bool ok0 = cc * 32 + i < lim, ok1 = cc * 32 + i + 1 < lim;
+          const float p0 = ok0 ? ex2_approx(fmaf(__uint_as_float(v[i]), c, -bias)) : 0.f;
+          const float p1 = ok1 ? ex2_approx(fmaf(__uint_as_float(v[i + 1]), c, -bias)) : 0.f;
+          lsum += p0 + p1;
+          pk[i / 2] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(s_tmem + cc * 16, pk);
+      }
+      ml[ds * 128 + row] = make_float2(mx, lsum);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&p_full[sb]);
+        mbar_arrive(&ml_full[ds]);
+      }
+    }
+  } else if (warp >= kEpiW0) {
+    // ---------------------------------------------------------------- epilogue
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const int qi = row / G;
+    const int hh = row % G;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const float c = args.scale_log2;
+    for (int t = 0;; ++t) {
+      const int ds = t % kDesc;
+      if (!mbar_wait(&d_full[ds], (t / kDesc) & 1, wc)) break;
+      const Desc& dd = desc[ds];
+      if (dd.end) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&d_empty[ds]);
+        break;
+      }
+      const int e = qi < dd.count ? dd.entry[qi] : -1;
+      const int r = dd.r;
+      const int sb = t & 1;
+      if (!mbar_wait(&o_full[sb], (t >> 1) & 1, wc)) break;
+      if (!mbar_wait(&ml_full[ds], (t / kDesc) & 1, wc)) break;
+      tc_fence_after();
+      const float2 st = ml[ds * 128 + row];
+      const float inv = st.y > 0.f ? 1.f / st.y : 0.f;
+      const float lse2 = st.y > 0.f ? st.x * c + __log2f(st.y) : __int_as_float(0xff800000);
+      const int q = e >> 5, slot = e & 31;
+      const size_t prow = (static_cast<size_t>(slot) * args.n_q + q) * args.h_q + r * G + hh;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t ov[32];
+        tmem_ld32(lane_base + Cfg::kColO + sb * D + cc * 32, ov);
+        tmem_ld_wait();
+        if (e >= 0) {
+          uint4* dst = reinterpret_cast<uint4*>(args.part_o + prow * D + cc * 32);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(ov[v4 * 8 + 0]) * inv, __uint_as_float(ov[v4 * 8 + 1]) * inv);
+            w.y = pack_bf16x2(__uint_as_float(ov[v4 * 8 + 2]) * inv, __uint_as_float(ov[v4 * 8 + 3]) * inv);
+            w.z = pack_bf16x2(__uint_as_float(ov[v4 * 8 + 4]) * inv, __uint_as_float(ov[v4 * 8 + 5]) * inv);
+            w.w = pack_bf16x2(__uint_as_float(ov[v4 * 8 + 6]) * inv, __uint_as_float(ov[v4 * 8 + 7]) * inv);
+            dst[v4] = w;
+          }
+        }
+      }
+      if (e >= 0) args.part_lse[prow] = lse2;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&o_free[sb]);
+        mbar_arrive(&d_empty[ds]);   // also releases ml[ds]
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) __nanosleep(1000000);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Cfg::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// schedule: block_ids -> per-(group, block) lists of (query, slot)
+// ---------------------------------------------------------------------------
+__global__ void sched_count_kernel(const int32_t* ids, long long total, int h_kv, int topk, int nb, int* cnt) {
+  const long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (e >= total) return;
+  const int b = ids[e];
+  if (b < 0 || b >= nb) return;
+  const int r = static_cast<int>((e / topk) % h_kv);
+  atomicAdd(&cnt[r * nb + b], 1);
+}
+
+// One CTA: exclusive scan of cnt -> offs, and the compacted list of non-empty lists.
+__global__ void __launch_bounds__(1024) sched_scan_kernel(const int* cnt, int n, int* offs, int* lists,
+                                                          int* n_lists) {
+  __shared__ int s_a[1024], s_b[1024];
+  __shared__ int carry_a, carry_b;
+  if (threadIdx.x == 0) {
+    carry_a = 0;
+    carry_b = 0;
+  }
+  __syncthreads();
+  for (int base = 0; base < n; base += 1024) {
+    const int i = base + threadIdx.x;
+    const int v = i < n ? cnt[i] : 0;
+    const int nz = v > 0 ? 1 : 0;
+    s_a[threadIdx.x] = v;
+    s_b[threadIdx.x] = nz;
+    __syncthreads();
+    for (int off = 1; off < 1024; off <<= 1) {
+      const int ta = threadIdx.x >= off ? s_a[threadIdx.x - off] : 0;
+      const int tb = threadIdx.x >= off ? s_b[threadIdx.x - off] : 0;
+      __syncthreads();
+      s_a[threadIdx.x] += ta;
+      s_b[threadIdx.x] += tb;
+      __syncthreads();
+    }
+    if (i < n) {
+      offs[i] = carry_a + s_a[threadIdx.x] - v;
+      if (nz) lists[carry_b + s_b[threadIdx.x] - 1] = i;
+    }
+    __syncthreads();
+    if (threadIdx.x == 1023) {
+      carry_a += s_a[1023];
+      carry_b += s_b[1023];
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    offs[n] = carry_a;
+    *n_lists = carry_b;
+  }
+}
+
+__global__ void sched_fill_kernel(const int32_t* ids, long long total, int h_kv, int topk, int nb, const int* offs,
+                                  int* fill, int* entries) {
+  const long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (e >= total) return;
+  const int b = ids[e];
+  if (b < 0 || b >= nb) return;
+  const int slot = static_cast<int>(e % topk);
+  const int r = static_cast<int>((e / topk) % h_kv);
+  const int q = static_cast<int>(e / (static_cast<long long>(topk) * h_kv));
+  const int rb = r * nb + b;
+  const int pos = offs[rb] + atomicAdd(&fill[rb], 1);
+  entries[pos] = (q << 5) | slot;
+}
+
+// ---------------------------------------------------------------------------
+// merge: O[q, h] = sum over valid slots of 2^(lse2_s - L) o_s
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) merge_partials_kernel(const int32_t* ids, const uint16_t* part_o,
+                                                             const float* part_lse, uint16_t* o, int n_q, int h_q,
+                                                             int h_kv, int topk, int nb) {
+  // One CTA per (query, group); thread = (head within group, 8-column chunk).
+  const int qr = blockIdx.x;
+  const int q = qr / h_kv, r = qr % h_kv;
+  const int G = h_q / h_kv;
+  constexpr int kChunks = D / 8;
+  const int32_t* my_ids = ids + static_cast<size_t>(qr) * topk;
+  for (int w = threadIdx.x; w < G * kChunks; w += blockDim.x) {
+    const int hh = w / kChunks, ch = w % kChunks;
+    const int h = r * G + hh;
+    float L = __int_as_float(0xff800000);
+    for (int s = 0; s < topk; ++s) {
+      if (my_ids[s] < 0 || my_ids[s] >= nb) continue;   // the schedule skips these too
+      L = fmaxf(L, part_lse[(static_cast<size_t>(s) * n_q + q) * h_q + h]);
+    }
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    float den = 0.f;
+    if (L != __int_as_float(0xff800000)) {
+      for (int s = 0; s < topk; ++s) {
+        if (my_ids[s] < 0 || my_ids[s] >= nb) continue;
+        const size_t prow = (static_cast<size_t>(s) * n_q + q) * h_q + h;
+        const float ls = part_lse[prow];
+        if (ls == __int_as_float(0xff800000)) continue;
+        const float wgt = ex2_approx(ls - L);
+        den += wgt;
+        const uint4 v = *reinterpret_cast<const uint4*>(part_o + prow * D + ch * 8);
+        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          acc[2 * i] += wgt * __uint_as_float(u[i] << 16);
+          acc[2 * i + 1] += wgt * __uint_as_float(u[i] & 0xffff0000u);
+        }
+      }
+    }
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    uint4 out;
+    out.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+    out.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+    out.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
+    out.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
+    *reinterpret_cast<uint4*>(o + (static_cast<size_t>(q) * h_q + h) * D + ch * 8) = out;
+  }
+}
+
+template <int D, int BK, int G>
+cudaError_t launch_kvo(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const KvoArgs& a,
+                       int grid, cudaStream_t st) {
+  auto kern = attn_kvouter_kernel<D, BK, G>;
+  const int smem = KvoCfg<D, BK>::kSmemBytes;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, smem, st>>>(tq, tk, tv, a);
+  return cudaGetLastError();
+}
+
+template <int D, int BK>
+cudaError_t launch_kvo_g(int G, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                         const KvoArgs& a, int grid, cudaStream_t st) {
+  switch (G) {
+    case 1: return launch_kvo<D, BK, 1>(tq, tk, tv, a, grid, st);
+    case 2: return launch_kvo<D, BK, 2>(tq, tk, tv, a, grid, st);
+    case 4: return launch_kvo<D, BK, 4>(tq, tk, tv, a, grid, st);
+    case 8: return launch_kvo<D, BK, 8>(tq, tk, tv, a, grid, st);
+    case 16: return launch_kvo<D, BK, 16>(tq, tk, tv, a, grid, st);
+    case 32: return launch_kvo<D, BK, 32>(tq, tk, tv, a, grid, st);
+    case 64: return launch_kvo<D, BK, 64>(tq, tk, tv, a, grid, st);
+    default: return launch_kvo<D, BK, 128>(tq, tk, tv, a, grid, st);
+  }
+}
+
+struct SparseWs {
+  int *cnt, *fill, *offs, *lists, *n_lists, *work, *entries;
+  uint16_t* part_o;
+  float* part_lse;
+  size_t bytes;
+};
+
+SparseWs carve(const msa_params& p, int n_q, int n_kv, void* base) {
+  const int nb = (n_kv + p.block_k - 1) / p.block_k;
+  const size_t nl = static_cast<size_t>(p.h_kv) * nb;
+  const size_t nnz = static_cast<size_t>(n_q) * p.h_kv * p.topk;
+  uint8_t* w = static_cast<uint8_t*>(base);
+  size_t off = 0;
+  SparseWs s;
+  auto take = [&](size_t bytes) {
+    uint8_t* ptr = w ? w + off : nullptr;
+    off += align_up(bytes, 256);
+    return ptr;
+  };
+  // cnt, fill, work counter are contiguous so one memset clears them.
+  s.cnt = reinterpret_cast<int*>(take((2 * nl + 2) * 4));
+  s.fill = s.cnt ? s.cnt + nl : nullptr;
+  s.work = s.cnt ? s.cnt + 2 * nl : nullptr;
+  s.n_lists = s.cnt ? s.cnt + 2 * nl + 1 : nullptr;
+  s.offs = reinterpret_cast<int*>(take((nl + 1) * 4));
+  s.lists = reinterpret_cast<int*>(take(nl * 4));
+  s.entries = reinterpret_cast<int*>(take(nnz * 4));
+  s.part_lse = reinterpret_cast<float*>(take(static_cast<size_t>(p.topk) * n_q * p.h_q * 4));
+  s.part_o = reinterpret_cast<uint16_t*>(take(static_cast<size_t>(p.topk) * n_q * p.h_q * p.d * 2));
+  s.bytes = off;
+  return s;
+}
+
+}  // namespace
+
+size_t sparse_prefill_workspace_bytes(const msa_params& p, int n_q, int n_kv) {
+  return carve(p, n_q, n_kv, nullptr).bytes;
+}
+
+int run_sparse_attn_kvouter(const msa_params& p, const void* q, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const int32_t* block_ids, int n_q, int n_kv, int q_pos0, void* o, void* ws,
+                            size_t ws_bytes, int* status, cudaStream_t stream) {
+  SparseWs s = carve(p, n_q, n_kv, ws);
+  if (ws_bytes < s.bytes) return MSA_ERR_WORKSPACE;
+  const int G = p.h_q / p.h_kv;
+  CUtensorMap tq;   // one box = the G head rows of one query of one group
+  {
+    const uint64_t dims[3] = {static_cast<uint64_t>(p.d), static_cast<uint64_t>(p.h_q), static_cast<uint64_t>(n_q)};
+    const uint64_t strides[2] = {static_cast<uint64_t>(p.d) * 2, static_cast<uint64_t>(p.h_q) * p.d * 2};
+    const uint32_t box[3] = {64, static_cast<uint32_t>(G), 1};
+    if (!encode_tma_bf16(&tq, 3, q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MSA_ERR_CUDA;
+  }
+  const int nb = (n_kv + p.block_k - 1) / p.block_k;
+  const int nl = p.h_kv * nb;
+  const long long total = static_cast<long long>(n_q) * p.h_kv * p.topk;
+  if (cudaMemsetAsync(s.cnt, 0, (2 * static_cast<size_t>(nl) + 2) * 4, stream) != cudaSuccess) return MSA_ERR_CUDA;
+  const int gsz = static_cast<int>((total + kSchedThreads - 1) / kSchedThreads);
+  sched_count_kernel<<<gsz, kSchedThreads, 0, stream>>>(block_ids, total, p.h_kv, p.topk, nb, s.cnt);
+  sched_scan_kernel<<<1, 1024, 0, stream>>>(s.cnt, nl, s.offs, s.lists, s.n_lists);
+  sched_fill_kernel<<<gsz, kSchedThreads, 0, stream>>>(block_ids, total, p.h_kv, p.topk, nb, s.offs, s.fill,
+                                                       s.entries);
+  if (cudaGetLastError() != cudaSuccess) return MSA_ERR_CUDA;
+
+  KvoArgs a;
+  a.offs = s.offs;
+  a.entries = s.entries;
+  a.lists = s.lists;
+  a.n_lists = s.n_lists;
+  a.work_counter = s.work;
+  a.part_o = s.part_o;
+  a.part_lse = s.part_lse;
+  a.status = status;
+  a.n_q = n_q;
+  a.n_kv = n_kv;
+  a.q_pos0 = q_pos0;
+  a.h_q = p.h_q;
+  a.h_kv = p.h_kv;
+  a.topk = p.topk;
+  a.causal = p.causal;
+  a.nb = nb;
+  const float scale = p.scale > 0.f ? p.scale : 1.0f / sqrtf(static_cast<float>(p.d));
+  a.scale_log2 = scale * 1.4426950408889634f;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = sms;
+  cudaError_t e;
+  if (p.d == 64) {
+    e = p.block_k == 64 ? launch_kvo_g<64, 64>(G, tq, tk, tv, a, grid, stream)
+                        : launch_kvo_g<64, 128>(G, tq, tk, tv, a, grid, stream);
+  } else {
+    e = p.block_k == 64 ? launch_kvo_g<128, 64>(G, tq, tk, tv, a, grid, stream)
+                        : launch_kvo_g<128, 128>(G, tq, tk, tv, a, grid, stream);
+  }
+  if (e != cudaSuccess) return MSA_ERR_CUDA;
+  const int mgrid = n_q * p.h_kv;
+  if (p.d == 64)
+    merge_partials_kernel<64><<<mgrid, 256, 0, stream>>>(block_ids, s.part_o, s.part_lse, static_cast<uint16_t*>(o),
+                                                          n_q, p.h_q, p.h_kv, p.topk, nb);
+  else
+    merge_partials_kernel<128><<<mgrid, 256, 0, stream>>>(block_ids, s.part_o, s.part_lse,
+                                                           static_cast<uint16_t*>(o), n_q, p.h_q, p.h_kv, p.topk, nb);
+  return cudaGetLastError() == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
+}
+
+}  // namespace msa

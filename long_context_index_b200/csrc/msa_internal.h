@@ -31,6 +31,12 @@ int run_sparse_attn_prefill(const msa_params& p, const void* q, const void* k, c
                             const int32_t* block_ids, int n_q, int n_kv, int q_pos0, void* o, void* ws,
                             size_t ws_bytes, int* status, cudaStream_t stream);
 
+// Block-major sparse prefill (attn_sparse.cu).
+size_t sparse_prefill_workspace_bytes(const msa_params& p, int n_q, int n_kv);
+int run_sparse_attn_kvouter(const msa_params& p, const void* q, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const int32_t* block_ids, int n_q, int n_kv, int q_pos0, void* o, void* ws,
+                            size_t ws_bytes, int* status, cudaStream_t stream);
+
 // Decode step.
 size_t decode_workspace_bytes(const msa_params& p, int batch, int max_kv);
 int run_sparse_attn_decode(const msa_params& p, const void* q, const void* q_idx, const void* k_cache,
