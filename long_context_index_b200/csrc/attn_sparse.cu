@@ -8,8 +8,11 @@
 // with no atomics on the outputs).
 //
 //   1. sched_count / sched_scan / sched_fill: invert block_ids [n_q, h_kv, k]
-//      into one list per (group r, block b) of the (query, slot) pairs that
-//      selected it (counting sort; slot = position of b in the query's ids).
+//      into one list per (query wave, group r, block b) of the (query, slot)
+//      pairs that selected it (counting sort; slot = position of b in the
+//      query's ids).  Lists are handed out in (wave, group, block) order, so
+//      at any moment the CTAs gather the queries of one wave of kWave rows,
+//      whose Q rows (kWave x h_q x d x 2 bytes) stay resident in L2.
 //   2. attn_kvouter_kernel (persistent, warp-specialised, tcgen05):
 //      * warp 0 grabs the next (r, b) list with an atomic counter, loads
 //        K_b, V_b once by TMA, then streams chunks of 128/G queries of the
@@ -38,34 +41,45 @@ namespace {
 constexpr int kThreads = 320;   // 10 warps
 constexpr int kSoftW0 = 2;      // softmax warps 2..5 (one per TMEM lane quarter)
 constexpr int kEpiW0 = 6;       // epilogue warps 6..9
+// One K/V stage suffices because a CTA switches blocks only once per
+// (group, block) list (hundreds of chunks); the partial tile is staged in
+// two shared-memory buffers for the TMA stores.
 constexpr int kQStages = 2;
-constexpr int kKVStages = 2;
+constexpr int kKVStages = 1;
+constexpr int kOStages = 2;
 constexpr int kDesc = 4;        // descriptor ring depth
 constexpr int kSchedThreads = 256;
+constexpr int kStageEntries = 256;   // list entries staged in shared memory at a time
+constexpr int kWave = 4096;          // query rows per wave (L2-resident Q working set)
 
 template <int D, int BK>
 struct KvoCfg {
   static constexpr int kAtoms = D / 64;
   static constexpr int kQBytes = 128 * D * 2;
   static constexpr int kKVBytes = BK * D * 2;          // one of K or V
-  static constexpr int kSmemData = kQStages * kQBytes + kKVStages * 2 * kKVBytes;
+  static constexpr int kOBytes = 128 * D * 2;          // staged bf16 partial tile
+  static constexpr int kSmemData = kQStages * kQBytes + kKVStages * 2 * kKVBytes + kOStages * kOBytes;
   static constexpr int kSmemBytes = kSmemData + 8192 + 1024;
   static constexpr int kColS = 0;        // S/P buffers: [0, BK), [BK, 2BK)
   static constexpr int kColO = 2 * BK;   // O buffers: [2BK, 2BK + D), [2BK + D, 2BK + 2D)
   static constexpr int kTmemCols = (2 * BK + 2 * D) <= 256 ? 256 : 512;
 };
 
-// One chunk of gathered queries of a (group, block) list.
+// One chunk of gathered queries of a (group, block) list.  (Declared before
+// KvoCfg's users; the shared-memory budget check follows it.)
 struct Desc {
   int entry[128];   // (query << 5) | slot, for the first `count` rows' queries
   int r, b, count, kvs;
   int first_of_kv, last_of_kv, end;
 };
 
+static_assert(kDesc * (sizeof(Desc) + 128 * 8) + kStageEntries * 4 + 32 * 8 + 16 <= 8192,
+              "control block of attn_kvouter_kernel exceeds its shared-memory reservation");
+
 struct KvoArgs {
-  const int* offs;       // [h_kv * nb + 1] list offsets
+  const int* offs;       // [n_waves * h_kv * nb + 1] list offsets
   const int* entries;    // (query << 5) | slot, grouped by list
-  const int* lists;      // non-empty list ids (r * nb + b)
+  const int* lists;      // non-empty list ids ((wave * h_kv + r) * nb + b)
   const int* n_lists;
   int* work_counter;
   uint16_t* part_o;      // [topk][n_q][h_q][d] bf16
@@ -78,16 +92,19 @@ struct KvoArgs {
 template <int D, int BK, int G>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                        const __grid_constant__ CUtensorMap tm_v, const KvoArgs args) {
+                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_po,
+                        const KvoArgs args) {
   using Cfg = KvoCfg<D, BK>;
   constexpr int QPC = 128 / G;   // queries per chunk
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sq = smem;                                        // [stage][atoms][128][128 B]
   uint8_t* skv = smem + kQStages * Cfg::kQBytes;             // [stage][K|V][atoms][BK][128 B]
+  uint8_t* so = skv + kKVStages * 2 * Cfg::kKVBytes;         // [stage][atoms][128][128 B] partial tile
   Desc* desc = reinterpret_cast<Desc*>(smem + Cfg::kSmemData);
   float2* ml = reinterpret_cast<float2*>(desc + kDesc);      // [kDesc][128] (m, l) per row
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ml + kDesc * 128);
+  int* stage = reinterpret_cast<int*>(ml + kDesc * 128);     // [kStageEntries] staged list entries
+  uint64_t* bars = reinterpret_cast<uint64_t*>(stage + kStageEntries);
   uint64_t* q_full = bars;                                   // [kQStages]
   uint64_t* q_empty = q_full + kQStages;
   uint64_t* kv_full = q_empty + kQStages;                    // [kKVStages]
@@ -141,35 +158,63 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_lists = *args.n_lists;
 
   if (warp == 0) {
-    // ---------------------------------------------------------------- producer
+    // ---------------------------------------------------------------- producer (whole warp)
+    // The list's (query, slot) entries are staged in shared memory 256 at a
+    // time with coalesced loads, so no TMA issue waits on a dependent global
+    // load; each lane issues the TMA boxes of its own queries.
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      int t = 0;      // chunk counter
-      int kvc = 0;    // KV stage use counter
-      bool ok = true;
-      while (ok) {
-        const int li = atomicAdd(args.work_counter, 1);
-        if (li >= n_lists) break;
-        const int rb = args.lists[li];
-        const int r = rb / args.nb, b = rb % args.nb;
-        const int start = args.offs[rb], cnt = args.offs[rb + 1] - start;
-        const int kvs = kvc % kKVStages;
-        if (!mbar_wait(&kv_empty[kvs], ((kvc / kKVStages) & 1) ^ 1, wc)) break;
-        mbar_arrive_expect_tx(&kv_full[kvs], 2 * Cfg::kKVBytes);
-        uint8_t* sk = skv + kvs * 2 * Cfg::kKVBytes;
-        for (int a = 0; a < Cfg::kAtoms; ++a) {
-          tma_load_3d(sk + a * BK * 128, &tm_k, &kv_full[kvs], a * 64, r, b * BK);
-          tma_load_3d(sk + Cfg::kKVBytes + a * BK * 128, &tm_v, &kv_full[kvs], a * 64, r, b * BK);
+    }
+    int t = 0;      // chunk counter
+    int kvc = 0;    // KV stage use counter
+    bool ok = true;
+    while (ok) {
+      int li = 0;
+      if (lane == 0) li = atomicAdd(args.work_counter, 1);
+      li = __shfl_sync(0xffffffffu, li, 0);
+      if (li >= n_lists) break;
+      const int rb = args.lists[li];
+      const int r = (rb / args.nb) % args.h_kv, b = rb % args.nb;
+      const int start = args.offs[rb], cnt = args.offs[rb + 1] - start;
+      const int kvs = kvc % kKVStages;
+      if (lane == 0) {
+        ok = mbar_wait(&kv_empty[kvs], ((kvc / kKVStages) & 1) ^ 1, wc);
+        if (ok) {
+          mbar_arrive_expect_tx(&kv_full[kvs], 2 * Cfg::kKVBytes);
+          uint8_t* sk = skv + kvs * 2 * Cfg::kKVBytes;
+          for (int a = 0; a < Cfg::kAtoms; ++a) {
+            tma_load_3d(sk + a * BK * 128, &tm_k, &kv_full[kvs], a * 64, r, b * BK);
+            tma_load_3d(sk + Cfg::kKVBytes + a * BK * 128, &tm_v, &kv_full[kvs], a * 64, r, b * BK);
+          }
         }
-        ++kvc;
-        for (int c0 = 0; c0 < cnt; c0 += QPC) {
-          const int qs = t % kQStages, ds = t % kDesc;
-          if (!mbar_wait(&d_empty[ds], ((t / kDesc) & 1) ^ 1, wc)) { ok = false; break; }
-          if (!mbar_wait(&q_empty[qs], ((t / kQStages) & 1) ^ 1, wc)) { ok = false; break; }
-          Desc& dd = desc[ds];
-          const int n_here = min(QPC, cnt - c0);
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      ++kvc;
+      for (int c0 = 0; c0 < cnt; c0 += QPC) {
+        // Refill the staging buffer every kStage entries.
+        const int rel = c0 % kStageEntries;
+        if (rel == 0) {
+          __syncwarp();
+#pragma unroll
+          for (int u = 0; u < kStageEntries / 32; ++u) {
+            const int k = c0 + u * 32 + lane;
+            stage[u * 32 + lane] = k < cnt ? args.entries[start + k] : -1;
+          }
+          __syncwarp();
+        }
+        const int qs = t % kQStages, ds = t % kDesc;
+        if (lane == 0) {
+          ok = mbar_wait(&d_empty[ds], ((t / kDesc) & 1) ^ 1, wc) &&
+               mbar_wait(&q_empty[qs], ((t / kQStages) & 1) ^ 1, wc);
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        Desc& dd = desc[ds];
+        const int n_here = min(QPC, cnt - c0);
+        if (lane == 0) {
           dd.r = r;
           dd.b = b;
           dd.count = n_here;
@@ -178,25 +223,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           dd.last_of_kv = c0 + QPC >= cnt;
           dd.end = 0;
           mbar_arrive_expect_tx(&q_full[qs], Cfg::kQBytes);
-          for (int qi = 0; qi < QPC; ++qi) {
-            const int e = qi < n_here ? args.entries[start + c0 + qi] : -1;
-            dd.entry[qi] = e;
-            const int q = e >= 0 ? (e >> 5) : args.n_q;   // past the end: TMA fills zeros
-            for (int a = 0; a < Cfg::kAtoms; ++a)
-              tma_load_3d(sq + qs * Cfg::kQBytes + a * 128 * 128 + qi * G * 128, &tm_q, &q_full[qs], a * 64,
-                          r * G, q);
-          }
-          mbar_arrive(&d_full[ds]);
-          ++t;
         }
+        __syncwarp();
+        for (int qi = lane; qi < QPC; qi += 32) {
+          const int e = qi < n_here ? stage[rel + qi] : -1;
+          dd.entry[qi] = e;
+          const int q = e >= 0 ? (e >> 5) : args.n_q;   // past the end: TMA fills zeros
+          for (int a = 0; a < Cfg::kAtoms; ++a)
+            tma_load_3d(sq + qs * Cfg::kQBytes + a * 128 * 128 + qi * G * 128, &tm_q, &q_full[qs], a * 64,
+                        r * G, q);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&d_full[ds]);
+        ++t;
       }
-      // End marker for the consumers.
-      if (ok && !*abort_flag) {
-        const int ds = t % kDesc;
-        if (mbar_wait(&d_empty[ds], ((t / kDesc) & 1) ^ 1, wc)) {
-          desc[ds].end = 1;
-          mbar_arrive(&d_full[ds]);
-        }
+    }
+    // End marker for the consumers.
+    if (lane == 0 && ok && !*abort_flag) {
+      const int ds = t % kDesc;
+      if (mbar_wait(&d_empty[ds], ((t / kDesc) & 1) ^ 1, wc)) {
+        desc[ds].end = 1;
+        mbar_arrive(&d_full[ds]);
       }
     }
   } else if (warp == 1) {
@@ -228,6 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       int t = 0;
       bool ok = true;
+      bool pending = false;   // PV of chunk t-1 not yet issued
       while (ok) {
         const int ds = t % kDesc;
         if (!mbar_wait(&d_full[ds], (t / kDesc) & 1, wc)) { ok = false; break; }
@@ -255,12 +303,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         umma_commit(&q_empty[qs]);
         umma_commit(&s_full[sb]);
-        if (t > 0 && !issue_pv(t - 1, prev_kvs, prev_last)) { ok = false; break; }
-        prev_kvs = kvs;
-        prev_last = last;
+        if (pending && !issue_pv(t - 1, prev_kvs, prev_last)) { ok = false; break; }
+        if (last) {
+          // The last chunk of a list frees the K/V stage the producer waits on
+          // before it publishes the next list, so its PV cannot be deferred.
+          if (!issue_pv(t, kvs, last)) { ok = false; break; }
+          pending = false;
+        } else {
+          pending = true;
+          prev_kvs = kvs;
+          prev_last = last;
+        }
         ++t;
       }
-      if (ok && t > 0) issue_pv(t - 1, prev_kvs, prev_last);
+      if (ok && pending) issue_pv(t - 1, prev_kvs, prev_last);
     }
   } else if (warp >= kSoftW0 && warp < kEpiW0) {
     // ---------------------------------------------------------------- softmax
@@ -292,42 +348,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(&s_full[sb], (t >> 1) & 1, wc)) break;
       tc_fence_after();
       const uint32_t s_tmem = lane_base + Cfg::kColS + sb * BK;
-      // Pass 1: row max over the visible keys.
+      // The whole S row in registers: all TMEM loads in flight, one wait.
+      uint32_t sv[BK];
+#pragma unroll
+      for (int cc = 0; cc < BK / 32; ++cc)
+        tmem_ld32(s_tmem + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[cc * 32]));
+      tmem_ld_wait();
       float mx = __int_as_float(0xff800000);
+      if (lim >= BK) {
 #pragma unroll
-      for (int cc = 0; cc < BK / 32; ++cc) {
-        uint32_t v[32];
-        tmem_ld32(s_tmem + cc * 32, v);
-        tmem_ld_wait();
-        if (lim >= (cc + 1) * 32) {
+        for (int i = 0; i + 2 < BK; i += 3)
+          mx = max3f(mx, __uint_as_float(sv[i]), fmaxf(__uint_as_float(sv[i + 1]), __uint_as_float(sv[i + 2])));
 #pragma unroll
-          for (int i = 0; i + 2 < 32; i += 3)
-            mx = max3f(mx, __uint_as_float(v[i]), fmaxf(__uint_as_float(v[i + 1]), __uint_as_float(v[i + 2])));
-          mx = max3f(mx, __uint_as_float(v[30]), __uint_as_float(v[31]));
-        } else {
+        for (int i = (BK / 3) * 3; i < BK; ++i) mx = fmaxf(mx, __uint_as_float(sv[i]));
+      } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (cc * 32 + i < lim) mx = fmaxf(mx, __uint_as_float(v[i]));
+        for (int i = 0; i < BK; ++i) {
+          const float v = i < lim ? __uint_as_float(sv[i]) : __int_as_float(0xff800000);
+          sv[i] = __float_as_uint(v);
+          mx = fmaxf(mx, v);
         }
       }
-      // Pass 2: p = 2^((s - max) c), bf16 pairs written back over S.
+      // p = 2^((s - max) c) as bf16 pairs written back over S (masked keys give 0).
       const float bias = mx == __int_as_float(0xff800000) ? 0.f : mx * c;
       float lsum = 0.f;
 #pragma unroll
-      for (int cc = 0; cc < BK / 32; ++cc) {
-        uint32_t v[32];
-        tmem_ld32(s_tmem + cc * 32, v);
-        tmem_ld_wait();
-        uint32_t pk[16];
+      for (int h = 0; h < BK / 64; ++h) {
+        uint32_t pk[32];
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const bool ok0 = cc * 32 + i < lim, ok1 = cc * 32 + i + 1 < lim;
-          const float p0 = ok0 ? ex2_approx(fmaf(__uint_as_float(v[i]), c, -bias)) : 0.f;
-          const float p1 = ok1 ? ex2_approx(fmaf(__uint_as_float(v[i + 1]), c, -bias)) : 0.f;
+        for (int i = 0; i < 64; i += 2) {
+          const float p0 = ex2_approx(fmaf(__uint_as_float(sv[h * 64 + i]), c, -bias));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(sv[h * 64 + i + 1]), c, -bias));
           lsum += p0 + p1;
           pk[i / 2] = pack_bf16x2(p0, p1);
         }
-        tmem_st16(s_tmem + cc * 16, pk);
+        tmem_st32(s_tmem + h * 32, pk);
       }
       ml[ds * 128 + row] = make_float2(mx, lsum);
       tmem_st_wait();
@@ -365,33 +420,50 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float inv = st.y > 0.f ? 1.f / st.y : 0.f;
       const float lse2 = st.y > 0.f ? st.x * c + __log2f(st.y) : __int_as_float(0xff800000);
       const int q = e >> 5, slot = e & 31;
-      const size_t prow = (static_cast<size_t>(slot) * args.n_q + q) * args.h_q + r * G + hh;
+      const int n_here = dd.count;
+      uint32_t ov[D];
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t ov[32];
-        tmem_ld32(lane_base + Cfg::kColO + sb * D + cc * 32, ov);
-        tmem_ld_wait();
-        if (e >= 0) {
-          uint4* dst = reinterpret_cast<uint4*>(args.part_o + prow * D + cc * 32);
-#pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(ov[v4 * 8 + 0]) * inv, __uint_as_float(ov[v4 * 8 + 1]) * inv);
-            w.y = pack_bf16x2(__uint_as_float(ov[v4 * 8 + 2]) * inv, __uint_as_float(ov[v4 * 8 + 3]) * inv);
-            w.z = pack_bf16x2(__uint_as_float(ov[v4 * 8 + 4]) * inv, __uint_as_float(ov[v4 * 8 + 5]) * inv);
-            w.w = pack_bf16x2(__uint_as_float(ov[v4 * 8 + 6]) * inv, __uint_as_float(ov[v4 * 8 + 7]) * inv);
-            dst[v4] = w;
-          }
-        }
-      }
-      if (e >= 0) args.part_lse[prow] = lse2;
+      for (int cc = 0; cc < D / 32; ++cc)
+        tmem_ld32(lane_base + Cfg::kColO + sb * D + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&ov[cc * 32]));
+      tmem_ld_wait();
+      // The O buffer is free once its values are in registers.
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&o_free[sb]);
-        mbar_arrive(&d_empty[ds]);   // also releases ml[ds]
+      if (lane == 0) mbar_arrive(&o_free[sb]);
+      // Stage the bf16 row in the swizzled tile layout (the layout TMA uses),
+      // after the stores that last read this staging buffer have drained.
+      const int os = t % kOStages;
+      if (warp == kEpiW0 && lane == 0) bulk_wait_read_le1();
+      named_bar(1, 128);
+      const uint32_t so_addr = smem_u32(so + os * Cfg::kOBytes);
+#pragma unroll
+      for (int a = 0; a < D / 64; ++a) {
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const float* f = reinterpret_cast<const float*>(&ov[a * 64 + ch * 8]);
+          st_shared_v4(so_addr + a * 128 * 128 + row * 128 + ((ch ^ (row & 7)) << 4),
+                       pack_bf16x2(f[0] * inv, f[1] * inv), pack_bf16x2(f[2] * inv, f[3] * inv),
+                       pack_bf16x2(f[4] * inv, f[5] * inv), pack_bf16x2(f[6] * inv, f[7] * inv));
+        }
       }
+      if (e >= 0) args.part_lse[(static_cast<size_t>(slot) * args.n_q + q) * args.h_q + r * G + hh] = lse2;
+      fence_proxy_async_smem();
+      named_bar(1, 128);
+      // One thread issues, commits and later waits for the chunk's tile
+      // stores (bulk groups are tracked per thread).
+      if (warp == kEpiW0 && lane == 0) {
+        for (int qq = 0; qq < n_here; ++qq) {
+          const int eq = dd.entry[qq];
+          for (int a = 0; a < D / 64; ++a)
+            tma_store_3d(&tm_po, so + os * Cfg::kOBytes + a * 128 * 128 + qq * G * 128, a * 64, r * G,
+                         (eq & 31) * args.n_q + (eq >> 5));
+        }
+        bulk_commit();
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&d_empty[ds]);   // also releases ml[ds]
     }
+    if (warp == kEpiW0) bulk_wait0();
   }
 
   tc_fence_before();
@@ -412,7 +484,8 @@ __global__ void sched_count_kernel(const int32_t* ids, long long total, int h_kv
   const int b = ids[e];
   if (b < 0 || b >= nb) return;
   const int r = static_cast<int>((e / topk) % h_kv);
-  atomicAdd(&cnt[r * nb + b], 1);
+  const int wave = static_cast<int>(e / (static_cast<long long>(topk) * h_kv)) / kWave;
+  atomicAdd(&cnt[(wave * h_kv + r) * nb + b], 1);
 }
 
 // One CTA: exclusive scan of cnt -> offs, and the compacted list of non-empty lists.
@@ -466,7 +539,7 @@ __global__ void sched_fill_kernel(const int32_t* ids, long long total, int h_kv,
   const int slot = static_cast<int>(e % topk);
   const int r = static_cast<int>((e / topk) % h_kv);
   const int q = static_cast<int>(e / (static_cast<long long>(topk) * h_kv));
-  const int rb = r * nb + b;
+  const int rb = ((q / kWave) * h_kv + r) * nb + b;
   const int pos = offs[rb] + atomicAdd(&fill[rb], 1);
   entries[pos] = (q << 5) | slot;
 }
@@ -522,28 +595,26 @@ __global__ void __launch_bounds__(256) merge_partials_kernel(const int32_t* ids,
 }
 
 template <int D, int BK, int G>
-cudaError_t launch_kvo(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const KvoArgs& a,
-                       int grid, cudaStream_t st) {
+cudaError_t launch_kvo(const CUtensorMap* m, const KvoArgs& a, int grid, cudaStream_t st) {
   auto kern = attn_kvouter_kernel<D, BK, G>;
   const int smem = KvoCfg<D, BK>::kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, smem, st>>>(tq, tk, tv, a);
+  kern<<<grid, kThreads, smem, st>>>(m[0], m[1], m[2], m[3], a);
   return cudaGetLastError();
 }
 
 template <int D, int BK>
-cudaError_t launch_kvo_g(int G, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                         const KvoArgs& a, int grid, cudaStream_t st) {
+cudaError_t launch_kvo_g(int G, const CUtensorMap* m, const KvoArgs& a, int grid, cudaStream_t st) {
   switch (G) {
-    case 1: return launch_kvo<D, BK, 1>(tq, tk, tv, a, grid, st);
-    case 2: return launch_kvo<D, BK, 2>(tq, tk, tv, a, grid, st);
-    case 4: return launch_kvo<D, BK, 4>(tq, tk, tv, a, grid, st);
-    case 8: return launch_kvo<D, BK, 8>(tq, tk, tv, a, grid, st);
-    case 16: return launch_kvo<D, BK, 16>(tq, tk, tv, a, grid, st);
-    case 32: return launch_kvo<D, BK, 32>(tq, tk, tv, a, grid, st);
-    case 64: return launch_kvo<D, BK, 64>(tq, tk, tv, a, grid, st);
-    default: return launch_kvo<D, BK, 128>(tq, tk, tv, a, grid, st);
+    case 1: return launch_kvo<D, BK, 1>(m, a, grid, st);
+    case 2: return launch_kvo<D, BK, 2>(m, a, grid, st);
+    case 4: return launch_kvo<D, BK, 4>(m, a, grid, st);
+    case 8: return launch_kvo<D, BK, 8>(m, a, grid, st);
+    case 16: return launch_kvo<D, BK, 16>(m, a, grid, st);
+    case 32: return launch_kvo<D, BK, 32>(m, a, grid, st);
+    case 64: return launch_kvo<D, BK, 64>(m, a, grid, st);
+    default: return launch_kvo<D, BK, 128>(m, a, grid, st);
   }
 }
 
@@ -556,7 +627,8 @@ struct SparseWs {
 
 SparseWs carve(const msa_params& p, int n_q, int n_kv, void* base) {
   const int nb = (n_kv + p.block_k - 1) / p.block_k;
-  const size_t nl = static_cast<size_t>(p.h_kv) * nb;
+  const int n_waves = (n_q + kWave - 1) / kWave;
+  const size_t nl = static_cast<size_t>(n_waves) * p.h_kv * nb;
   const size_t nnz = static_cast<size_t>(n_q) * p.h_kv * p.topk;
   uint8_t* w = static_cast<uint8_t*>(base);
   size_t off = 0;
@@ -600,7 +672,7 @@ int run_sparse_attn_kvouter(const msa_params& p, const void* q, const CUtensorMa
     if (!encode_tma_bf16(&tq, 3, q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MSA_ERR_CUDA;
   }
   const int nb = (n_kv + p.block_k - 1) / p.block_k;
-  const int nl = p.h_kv * nb;
+  const int nl = ((n_q + kWave - 1) / kWave) * p.h_kv * nb;
   const long long total = static_cast<long long>(n_q) * p.h_kv * p.topk;
   if (cudaMemsetAsync(s.cnt, 0, (2 * static_cast<size_t>(nl) + 2) * 4, stream) != cudaSuccess) return MSA_ERR_CUDA;
   const int gsz = static_cast<int>((total + kSchedThreads - 1) / kSchedThreads);
@@ -633,13 +705,21 @@ int run_sparse_attn_kvouter(const msa_params& p, const void* q, const CUtensorMa
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = sms;
+  CUtensorMap maps[4] = {tq, tk, tv, tq};
+  {  // partial outputs [topk * n_q][h_q][d]: one box = the G head rows of one (slot, query)
+    const uint64_t dims[3] = {static_cast<uint64_t>(p.d), static_cast<uint64_t>(p.h_q),
+                              static_cast<uint64_t>(p.topk) * n_q};
+    const uint64_t strides[2] = {static_cast<uint64_t>(p.d) * 2, static_cast<uint64_t>(p.h_q) * p.d * 2};
+    const uint32_t box[3] = {64, static_cast<uint32_t>(G), 1};
+    if (!encode_tma_bf16(&maps[3], 3, s.part_o, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MSA_ERR_CUDA;
+  }
   cudaError_t e;
   if (p.d == 64) {
-    e = p.block_k == 64 ? launch_kvo_g<64, 64>(G, tq, tk, tv, a, grid, stream)
-                        : launch_kvo_g<64, 128>(G, tq, tk, tv, a, grid, stream);
+    e = p.block_k == 64 ? launch_kvo_g<64, 64>(G, maps, a, grid, stream)
+                        : launch_kvo_g<64, 128>(G, maps, a, grid, stream);
   } else {
-    e = p.block_k == 64 ? launch_kvo_g<128, 64>(G, tq, tk, tv, a, grid, stream)
-                        : launch_kvo_g<128, 128>(G, tq, tk, tv, a, grid, stream);
+    e = p.block_k == 64 ? launch_kvo_g<128, 64>(G, maps, a, grid, stream)
+                        : launch_kvo_g<128, 128>(G, maps, a, grid, stream);
   }
   if (e != cudaSuccess) return MSA_ERR_CUDA;
   const int mgrid = n_q * p.h_kv;
