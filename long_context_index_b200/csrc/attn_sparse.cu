@@ -20,14 +20,19 @@
 //        publishes a descriptor per chunk in a 4-deep ring.
 //      * warp 1 issues S = Q K_b^T into one of two TMEM S buffers and
 //        O = P V_b (P read back from TMEM) into one of two TMEM O buffers.
-//      * warps 2..5 (softmax): one thread per row; the exact softmax of the
-//        row over the block's visible keys (causal only in the local block),
-//        in two passes over the TMEM row (max, then exp and bf16 pack in
-//        32-column chunks); P is written over S; (m, l) go to the epilogue.
-//      * warps 6..9 (epilogue): o = O / l in bf16 and lse2 = m c + log2 l to
-//        the partial buffers [slot][query][head].
+//      * warps 2..9 (softmax): two threads per row, each owning 64 of the 128
+//        columns; the exact softmax of the row over the block's visible keys
+//        (causal only in the local block); the two halves exchange only their
+//        max through shared memory; P is written over S; (m, l_lo, l_hi) go
+//        to the epilogue.  (The exponentials are MUFU-bound: 16 per clock per
+//        SM, so one 128x128 tile costs as many cycles as its two MMAs; two
+//        warps per SM sub-partition keep the MUFU pipe fed.)
+//      * warps 10..13 (epilogue): o = O / l in bf16 staged in shared memory and
+//        written by TMA as one contiguous 128-row tile per chunk
+//        (chunk-major partials), lse2 = m c + log2 l beside it.
 //   3. merge_partials_kernel: per (query, group), O = sum_s 2^(lse2_s - L) o_s
-//      over the valid slots, L = log2 sum 2^lse2_s; rounded to bf16.
+//      over the valid slots, L = log2 sum 2^lse2_s; rounded to bf16.  The
+//      schedule records, per (query, group, slot), the partial row it wrote.
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -38,9 +43,9 @@
 namespace msa {
 namespace {
 
-constexpr int kThreads = 320;   // 10 warps
-constexpr int kSoftW0 = 2;      // softmax warps 2..5 (one per TMEM lane quarter)
-constexpr int kEpiW0 = 6;       // epilogue warps 6..9
+constexpr int kThreads = 448;   // 14 warps
+constexpr int kSoftW0 = 2;      // softmax warps 2..9: two per TMEM lane quarter, 64 columns each
+constexpr int kEpiW0 = 10;      // epilogue warps 10..13
 // One K/V stage suffices because a CTA switches blocks only once per
 // (group, block) list (hundreds of chunks); the partial tile is staged in
 // two shared-memory buffers for the TMA stores.
@@ -59,7 +64,7 @@ struct KvoCfg {
   static constexpr int kKVBytes = BK * D * 2;          // one of K or V
   static constexpr int kOBytes = 128 * D * 2;          // staged bf16 partial tile
   static constexpr int kSmemData = kQStages * kQBytes + kKVStages * 2 * kKVBytes + kOStages * kOBytes;
-  static constexpr int kSmemBytes = kSmemData + 8192 + 1024;
+  static constexpr int kSmemBytes = kSmemData + 12288 + 1024;
   static constexpr int kColS = 0;        // S/P buffers: [0, BK), [BK, 2BK)
   static constexpr int kColO = 2 * BK;   // O buffers: [2BK, 2BK + D), [2BK + D, 2BK + 2D)
   static constexpr int kTmemCols = (2 * BK + 2 * D) <= 256 ? 256 : 512;
@@ -70,20 +75,20 @@ struct KvoCfg {
 struct Desc {
   int entry[128];   // (query << 5) | slot, for the first `count` rows' queries
   int r, b, count, kvs;
-  int first_of_kv, last_of_kv, end;
+  int first_of_kv, last_of_kv, end, chunk;   // chunk: global chunk id (partial tile index)
 };
 
-static_assert(kDesc * (sizeof(Desc) + 128 * 8) + kStageEntries * 4 + 32 * 8 + 16 <= 8192,
+static_assert(kDesc * (sizeof(Desc) + 128 * 12) + 4 * 128 * 4 + kStageEntries * 4 + 32 * 8 + 16 <= 12288,
               "control block of attn_kvouter_kernel exceeds its shared-memory reservation");
 
 struct KvoArgs {
   const int* offs;       // [n_waves * h_kv * nb + 1] list offsets
+  const int* chunk_off;  // [n_waves * h_kv * nb] first global chunk id of each list
   const int* entries;    // (query << 5) | slot, grouped by list
   const int* lists;      // non-empty list ids ((wave * h_kv + r) * nb + b)
   const int* n_lists;
   int* work_counter;
-  uint16_t* part_o;      // [topk][n_q][h_q][d] bf16
-  float* part_lse;       // [topk][n_q][h_q]
+  float* part_lse;       // [chunks * 128] lse2 of each partial row
   int* status;
   int n_q, n_kv, q_pos0, h_q, h_kv, topk, causal, nb;
   float scale_log2;
@@ -102,8 +107,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* skv = smem + kQStages * Cfg::kQBytes;             // [stage][K|V][atoms][BK][128 B]
   uint8_t* so = skv + kKVStages * 2 * Cfg::kKVBytes;         // [stage][atoms][128][128 B] partial tile
   Desc* desc = reinterpret_cast<Desc*>(smem + Cfg::kSmemData);
-  float2* ml = reinterpret_cast<float2*>(desc + kDesc);      // [kDesc][128] (m, l) per row
-  int* stage = reinterpret_cast<int*>(ml + kDesc * 128);     // [kStageEntries] staged list entries
+  float2* ml = reinterpret_cast<float2*>(desc + kDesc);      // [kDesc][128] (m, l of columns 0..63)
+  float* lhi = reinterpret_cast<float*>(ml + kDesc * 128);   // [kDesc][128] l of columns 64..127
+  float* smx = lhi + kDesc * 128;                            // [2 parity][2 halves][128] row-max exchange
+  int* stage = reinterpret_cast<int*>(smx + 4 * 128);        // [kStageEntries] staged list entries
   uint64_t* bars = reinterpret_cast<uint64_t*>(stage + kStageEntries);
   uint64_t* q_full = bars;                                   // [kQStages]
   uint64_t* q_empty = q_full + kQStages;
@@ -133,13 +140,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < kDesc; ++s) {
       mbar_init(&d_full[s], 1);
-      mbar_init(&d_empty[s], 9);   // MMA thread + 4 softmax warps + 4 epilogue warps
-      mbar_init(&ml_full[s], 4);   // 4 softmax warps
+      mbar_init(&d_empty[s], 13);  // MMA thread + 8 softmax warps + 4 epilogue warps
+      mbar_init(&ml_full[s], 8);   // 8 softmax warps
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
       mbar_init(&s_free[s], 1);
-      mbar_init(&p_full[s], 4);
+      mbar_init(&p_full[s], 8);
       mbar_init(&o_full[s], 1);
       mbar_init(&o_free[s], 4);
     }
@@ -178,6 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int rb = args.lists[li];
       const int r = (rb / args.nb) % args.h_kv, b = rb % args.nb;
       const int start = args.offs[rb], cnt = args.offs[rb + 1] - start;
+      const int chunk0 = args.chunk_off[rb];
       const int kvs = kvc % kKVStages;
       if (lane == 0) {
         ok = mbar_wait(&kv_empty[kvs], ((kvc / kKVStages) & 1) ^ 1, wc);
@@ -222,6 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           dd.first_of_kv = c0 == 0;
           dd.last_of_kv = c0 + QPC >= cnt;
           dd.end = 0;
+          dd.chunk = chunk0 + c0 / QPC;
           mbar_arrive_expect_tx(&q_full[qs], Cfg::kQBytes);
         }
         __syncwarp();
@@ -320,7 +329,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= kSoftW0 && warp < kEpiW0) {
     // ---------------------------------------------------------------- softmax
+    constexpr int HC = BK / 2;                 // columns per thread
     const int quarter = warp & 3;
+    const int half = (warp - kSoftW0) / 4;     // 0: columns [0, HC), 1: [HC, BK)
     const int row = quarter * 32 + lane;
     const int qi = row / G;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
@@ -338,53 +349,67 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int b = dd.b;
       __syncwarp();
       if (lane == 0) mbar_arrive(&d_empty[ds]);
-      int lim = 0;
+      int lim = 0;   // visible keys of this block for the row, relative to this half
       if (e >= 0) {
         const int p = args.q_pos0 + (e >> 5);
         const int kv_lim = args.causal ? min(p + 1, args.n_kv) : args.n_kv;
-        lim = min(BK, kv_lim - b * BK);
+        lim = min(BK, kv_lim - b * BK) - half * HC;
       }
       const int sb = t & 1;
       if (!mbar_wait(&s_full[sb], (t >> 1) & 1, wc)) break;
       tc_fence_after();
       const uint32_t s_tmem = lane_base + Cfg::kColS + sb * BK;
-      // The whole S row in registers: all TMEM loads in flight, one wait.
-      uint32_t sv[BK];
+      uint32_t sv[HC];
 #pragma unroll
-      for (int cc = 0; cc < BK / 32; ++cc)
-        tmem_ld32(s_tmem + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[cc * 32]));
+      for (int cc = 0; cc < HC / 32; ++cc)
+        tmem_ld32(s_tmem + half * HC + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[cc * 32]));
       tmem_ld_wait();
-      float mx = __int_as_float(0xff800000);
-      if (lim >= BK) {
+      if (lim < HC) {
 #pragma unroll
-        for (int i = 0; i + 2 < BK; i += 3)
-          mx = max3f(mx, __uint_as_float(sv[i]), fmaxf(__uint_as_float(sv[i + 1]), __uint_as_float(sv[i + 2])));
-#pragma unroll
-        for (int i = (BK / 3) * 3; i < BK; ++i) mx = fmaxf(mx, __uint_as_float(sv[i]));
-      } else {
-#pragma unroll
-        for (int i = 0; i < BK; ++i) {
-          const float v = i < lim ? __uint_as_float(sv[i]) : __int_as_float(0xff800000);
-          sv[i] = __float_as_uint(v);
-          mx = fmaxf(mx, v);
-        }
+        for (int i = 0; i < HC; ++i)
+          if (i >= lim) sv[i] = 0xff800000u;   // -inf: masked key
       }
-      // p = 2^((s - max) c) as bf16 pairs written back over S (masked keys give 0).
+      float mq[4] = {__int_as_float(0xff800000), __int_as_float(0xff800000), __int_as_float(0xff800000),
+                     __int_as_float(0xff800000)};
+#pragma unroll
+      for (int i = 0; i < HC; i += 8) {
+        const int k = (i / 8) & 3;
+        mq[k] = max3f(mq[k], fmaxf(__uint_as_float(sv[i]), __uint_as_float(sv[i + 1])),
+                      max3f(__uint_as_float(sv[i + 2]), __uint_as_float(sv[i + 3]), __uint_as_float(sv[i + 4])));
+        mq[k] = max3f(mq[k], __uint_as_float(sv[i + 5]), fmaxf(__uint_as_float(sv[i + 6]), __uint_as_float(sv[i + 7])));
+      }
+      // Exchange the half-row maxima with the partner warp (same lane quarter).
+      // The slot alternates with the chunk parity: a warp rewrites slot
+      // (t & 1) only after the next barrier, which its partner reaches only
+      // after reading this chunk's value.
+      float* xs = smx + (t & 1) * 256;
+      xs[half * 128 + row] = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+      named_bar(2 + quarter, 64);
+      const float mx = fmaxf(xs[row], xs[128 + row]);
+      // Both halves' S values are in registers past this barrier, so P may
+      // overwrite any S column.
       const float bias = mx == __int_as_float(0xff800000) ? 0.f : mx * c;
-      float lsum = 0.f;
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[HC / 2];
 #pragma unroll
-      for (int h = 0; h < BK / 64; ++h) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 64; i += 2) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(sv[h * 64 + i]), c, -bias));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(sv[h * 64 + i + 1]), c, -bias));
-          lsum += p0 + p1;
-          pk[i / 2] = pack_bf16x2(p0, p1);
-        }
-        tmem_st32(s_tmem + h * 32, pk);
+      for (int i = 0; i < HC; i += 4) {
+        const float p0 = ex2_approx(fmaf(__uint_as_float(sv[i]), c, -bias));
+        const float p1 = ex2_approx(fmaf(__uint_as_float(sv[i + 1]), c, -bias));
+        const float p2 = ex2_approx(fmaf(__uint_as_float(sv[i + 2]), c, -bias));
+        const float p3 = ex2_approx(fmaf(__uint_as_float(sv[i + 3]), c, -bias));
+        ls[(i / 4) & 3] += (p0 + p1) + (p2 + p3);
+        pk[i / 2] = pack_bf16x2(p0, p1);
+        pk[i / 2 + 1] = pack_bf16x2(p2, p3);
       }
-      ml[ds * 128 + row] = make_float2(mx, lsum);
+#pragma unroll
+      for (int cc = 0; cc < HC / 64; ++cc)
+        tmem_st32(s_tmem + half * (HC / 2) + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[cc * 32]));
+      if (HC / 2 == 16) tmem_st16(s_tmem + half * (HC / 2), *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
+      const float lsum = (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      if (half == 0)
+        ml[ds * 128 + row] = make_float2(mx, lsum);
+      else
+        lhi[ds * 128 + row] = lsum;
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -417,47 +442,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(&ml_full[ds], (t / kDesc) & 1, wc)) break;
       tc_fence_after();
       const float2 st = ml[ds * 128 + row];
-      const float inv = st.y > 0.f ? 1.f / st.y : 0.f;
-      const float lse2 = st.y > 0.f ? st.x * c + __log2f(st.y) : __int_as_float(0xff800000);
-      const int q = e >> 5, slot = e & 31;
-      const int n_here = dd.count;
-      uint32_t ov[D];
-#pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc)
-        tmem_ld32(lane_base + Cfg::kColO + sb * D + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&ov[cc * 32]));
-      tmem_ld_wait();
-      // The O buffer is free once its values are in registers.
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&o_free[sb]);
+      const float lsum = st.y + lhi[ds * 128 + row];
+      const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+      const float lse2 = lsum > 0.f ? st.x * c + __log2f(lsum) : __int_as_float(0xff800000);
+      const int chunk = dd.chunk;
+      const int os = t % kOStages;
       // Stage the bf16 row in the swizzled tile layout (the layout TMA uses),
       // after the stores that last read this staging buffer have drained.
-      const int os = t % kOStages;
       if (warp == kEpiW0 && lane == 0) bulk_wait_read_le1();
       named_bar(1, 128);
       const uint32_t so_addr = smem_u32(so + os * Cfg::kOBytes);
 #pragma unroll
       for (int a = 0; a < D / 64; ++a) {
+        uint32_t ov[64];
+        tmem_ld32(lane_base + Cfg::kColO + sb * D + a * 64, *reinterpret_cast<uint32_t(*)[32]>(&ov[0]));
+        tmem_ld32(lane_base + Cfg::kColO + sb * D + a * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&ov[32]));
+        tmem_ld_wait();
+        if (a == D / 64 - 1) {
+          // The O buffer is free once its values are in registers.
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&o_free[sb]);
+        }
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
-          const float* f = reinterpret_cast<const float*>(&ov[a * 64 + ch * 8]);
+          const float* f = reinterpret_cast<const float*>(&ov[ch * 8]);
           st_shared_v4(so_addr + a * 128 * 128 + row * 128 + ((ch ^ (row & 7)) << 4),
                        pack_bf16x2(f[0] * inv, f[1] * inv), pack_bf16x2(f[2] * inv, f[3] * inv),
                        pack_bf16x2(f[4] * inv, f[5] * inv), pack_bf16x2(f[6] * inv, f[7] * inv));
         }
       }
-      if (e >= 0) args.part_lse[(static_cast<size_t>(slot) * args.n_q + q) * args.h_q + r * G + hh] = lse2;
+      args.part_lse[static_cast<size_t>(chunk) * 128 + row] = e >= 0 ? lse2 : __int_as_float(0xff800000);
       fence_proxy_async_smem();
       named_bar(1, 128);
       // One thread issues, commits and later waits for the chunk's tile
-      // stores (bulk groups are tracked per thread).
+      // stores (bulk groups are tracked per thread): one box per d atom.
       if (warp == kEpiW0 && lane == 0) {
-        for (int qq = 0; qq < n_here; ++qq) {
-          const int eq = dd.entry[qq];
-          for (int a = 0; a < D / 64; ++a)
-            tma_store_3d(&tm_po, so + os * Cfg::kOBytes + a * 128 * 128 + qq * G * 128, a * 64, r * G,
-                         (eq & 31) * args.n_q + (eq >> 5));
-        }
+        for (int a = 0; a < D / 64; ++a)
+          tma_store_2d(&tm_po, so + os * Cfg::kOBytes + a * 128 * 128, a * 64, chunk * 128);
         bulk_commit();
       }
       __syncwarp();
@@ -488,39 +510,47 @@ __global__ void sched_count_kernel(const int32_t* ids, long long total, int h_kv
   atomicAdd(&cnt[(wave * h_kv + r) * nb + b], 1);
 }
 
-// One CTA: exclusive scan of cnt -> offs, and the compacted list of non-empty lists.
-__global__ void __launch_bounds__(1024) sched_scan_kernel(const int* cnt, int n, int* offs, int* lists,
-                                                          int* n_lists) {
-  __shared__ int s_a[1024], s_b[1024];
-  __shared__ int carry_a, carry_b;
+// One CTA: exclusive scans of cnt -> offs and of ceil(cnt / qpc) -> chunk_off,
+// and the compacted list of non-empty lists.
+__global__ void __launch_bounds__(1024) sched_scan_kernel(const int* cnt, int n, int qpc, int* offs, int* chunk_off,
+                                                          int* lists, int* n_lists) {
+  __shared__ int s_a[1024], s_b[1024], s_c[1024];
+  __shared__ int carry_a, carry_b, carry_c;
   if (threadIdx.x == 0) {
     carry_a = 0;
     carry_b = 0;
+    carry_c = 0;
   }
   __syncthreads();
   for (int base = 0; base < n; base += 1024) {
     const int i = base + threadIdx.x;
     const int v = i < n ? cnt[i] : 0;
     const int nz = v > 0 ? 1 : 0;
+    const int nc = (v + qpc - 1) / qpc;
     s_a[threadIdx.x] = v;
     s_b[threadIdx.x] = nz;
+    s_c[threadIdx.x] = nc;
     __syncthreads();
     for (int off = 1; off < 1024; off <<= 1) {
       const int ta = threadIdx.x >= off ? s_a[threadIdx.x - off] : 0;
       const int tb = threadIdx.x >= off ? s_b[threadIdx.x - off] : 0;
+      const int tc = threadIdx.x >= off ? s_c[threadIdx.x - off] : 0;
       __syncthreads();
       s_a[threadIdx.x] += ta;
       s_b[threadIdx.x] += tb;
+      s_c[threadIdx.x] += tc;
       __syncthreads();
     }
     if (i < n) {
       offs[i] = carry_a + s_a[threadIdx.x] - v;
+      chunk_off[i] = carry_c + s_c[threadIdx.x] - nc;
       if (nz) lists[carry_b + s_b[threadIdx.x] - 1] = i;
     }
     __syncthreads();
     if (threadIdx.x == 1023) {
       carry_a += s_a[1023];
       carry_b += s_b[1023];
+      carry_c += s_c[1023];
     }
     __syncthreads();
   }
@@ -530,8 +560,8 @@ __global__ void __launch_bounds__(1024) sched_scan_kernel(const int* cnt, int n,
   }
 }
 
-__global__ void sched_fill_kernel(const int32_t* ids, long long total, int h_kv, int topk, int nb, const int* offs,
-                                  int* fill, int* entries) {
+__global__ void sched_fill_kernel(const int32_t* ids, long long total, int h_kv, int topk, int nb, int G,
+                                  const int* offs, const int* chunk_off, int* fill, int* entries, int* prow_of) {
   const long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (e >= total) return;
   const int b = ids[e];
@@ -540,37 +570,41 @@ __global__ void sched_fill_kernel(const int32_t* ids, long long total, int h_kv,
   const int r = static_cast<int>((e / topk) % h_kv);
   const int q = static_cast<int>(e / (static_cast<long long>(topk) * h_kv));
   const int rb = ((q / kWave) * h_kv + r) * nb + b;
-  const int pos = offs[rb] + atomicAdd(&fill[rb], 1);
-  entries[pos] = (q << 5) | slot;
+  const int k = atomicAdd(&fill[rb], 1);    // position inside the list
+  entries[offs[rb] + k] = (q << 5) | slot;
+  const int qpc = 128 / G;
+  prow_of[e] = (chunk_off[rb] + k / qpc) * 128 + (k % qpc) * G;
 }
 
 // ---------------------------------------------------------------------------
 // merge: O[q, h] = sum over valid slots of 2^(lse2_s - L) o_s
 // ---------------------------------------------------------------------------
 template <int D>
-__global__ void __launch_bounds__(256) merge_partials_kernel(const int32_t* ids, const uint16_t* part_o,
-                                                             const float* part_lse, uint16_t* o, int n_q, int h_q,
-                                                             int h_kv, int topk, int nb) {
+__global__ void __launch_bounds__(256) merge_partials_kernel(const int32_t* ids, const int* prow_of,
+                                                             const uint16_t* part_o, const float* part_lse,
+                                                             uint16_t* o, int h_q, int h_kv, int topk, int nb) {
   // One CTA per (query, group); thread = (head within group, 8-column chunk).
+  // prow_of[(q, r, slot)] is the first partial row (chunk * 128 + query-in-
+  // chunk * G) the block-major kernel wrote for that selection.
   const int qr = blockIdx.x;
   const int q = qr / h_kv, r = qr % h_kv;
   const int G = h_q / h_kv;
   constexpr int kChunks = D / 8;
   const int32_t* my_ids = ids + static_cast<size_t>(qr) * topk;
+  const int* my_rows = prow_of + static_cast<size_t>(qr) * topk;
   for (int w = threadIdx.x; w < G * kChunks; w += blockDim.x) {
     const int hh = w / kChunks, ch = w % kChunks;
-    const int h = r * G + hh;
     float L = __int_as_float(0xff800000);
     for (int s = 0; s < topk; ++s) {
       if (my_ids[s] < 0 || my_ids[s] >= nb) continue;   // the schedule skips these too
-      L = fmaxf(L, part_lse[(static_cast<size_t>(s) * n_q + q) * h_q + h]);
+      L = fmaxf(L, part_lse[static_cast<size_t>(my_rows[s]) + hh]);
     }
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     float den = 0.f;
     if (L != __int_as_float(0xff800000)) {
       for (int s = 0; s < topk; ++s) {
         if (my_ids[s] < 0 || my_ids[s] >= nb) continue;
-        const size_t prow = (static_cast<size_t>(s) * n_q + q) * h_q + h;
+        const size_t prow = static_cast<size_t>(my_rows[s]) + hh;
         const float ls = part_lse[prow];
         if (ls == __int_as_float(0xff800000)) continue;
         const float wgt = ex2_approx(ls - L);
@@ -590,7 +624,7 @@ __global__ void __launch_bounds__(256) merge_partials_kernel(const int32_t* ids,
     out.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
     out.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
     out.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
-    *reinterpret_cast<uint4*>(o + (static_cast<size_t>(q) * h_q + h) * D + ch * 8) = out;
+    *reinterpret_cast<uint4*>(o + (static_cast<size_t>(q) * h_q + r * G + hh) * D + ch * 8) = out;
   }
 }
 
@@ -619,10 +653,10 @@ cudaError_t launch_kvo_g(int G, const CUtensorMap* m, const KvoArgs& a, int grid
 }
 
 struct SparseWs {
-  int *cnt, *fill, *offs, *lists, *n_lists, *work, *entries;
+  int *cnt, *fill, *offs, *chunk_off, *lists, *n_lists, *work, *entries, *prow_of;
   uint16_t* part_o;
   float* part_lse;
-  size_t bytes;
+  size_t max_chunks, bytes;
 };
 
 SparseWs carve(const msa_params& p, int n_q, int n_kv, void* base) {
@@ -630,6 +664,7 @@ SparseWs carve(const msa_params& p, int n_q, int n_kv, void* base) {
   const int n_waves = (n_q + kWave - 1) / kWave;
   const size_t nl = static_cast<size_t>(n_waves) * p.h_kv * nb;
   const size_t nnz = static_cast<size_t>(n_q) * p.h_kv * p.topk;
+  const int qpc = 128 / (p.h_q / p.h_kv);
   uint8_t* w = static_cast<uint8_t*>(base);
   size_t off = 0;
   SparseWs s;
@@ -644,10 +679,14 @@ SparseWs carve(const msa_params& p, int n_q, int n_kv, void* base) {
   s.work = s.cnt ? s.cnt + 2 * nl : nullptr;
   s.n_lists = s.cnt ? s.cnt + 2 * nl + 1 : nullptr;
   s.offs = reinterpret_cast<int*>(take((nl + 1) * 4));
+  s.chunk_off = reinterpret_cast<int*>(take(nl * 4));
   s.lists = reinterpret_cast<int*>(take(nl * 4));
   s.entries = reinterpret_cast<int*>(take(nnz * 4));
-  s.part_lse = reinterpret_cast<float*>(take(static_cast<size_t>(p.topk) * n_q * p.h_q * 4));
-  s.part_o = reinterpret_cast<uint16_t*>(take(static_cast<size_t>(p.topk) * n_q * p.h_q * p.d * 2));
+  s.prow_of = reinterpret_cast<int*>(take(nnz * 4));
+  // Every list rounds up to whole chunks: at most nnz / qpc + nl chunks.
+  s.max_chunks = (nnz + qpc - 1) / qpc + nl;
+  s.part_lse = reinterpret_cast<float*>(take(s.max_chunks * 128 * 4));
+  s.part_o = reinterpret_cast<uint16_t*>(take(s.max_chunks * 128 * static_cast<size_t>(p.d) * 2));
   s.bytes = off;
   return s;
 }
@@ -677,18 +716,18 @@ int run_sparse_attn_kvouter(const msa_params& p, const void* q, const CUtensorMa
   if (cudaMemsetAsync(s.cnt, 0, (2 * static_cast<size_t>(nl) + 2) * 4, stream) != cudaSuccess) return MSA_ERR_CUDA;
   const int gsz = static_cast<int>((total + kSchedThreads - 1) / kSchedThreads);
   sched_count_kernel<<<gsz, kSchedThreads, 0, stream>>>(block_ids, total, p.h_kv, p.topk, nb, s.cnt);
-  sched_scan_kernel<<<1, 1024, 0, stream>>>(s.cnt, nl, s.offs, s.lists, s.n_lists);
-  sched_fill_kernel<<<gsz, kSchedThreads, 0, stream>>>(block_ids, total, p.h_kv, p.topk, nb, s.offs, s.fill,
-                                                       s.entries);
+  sched_scan_kernel<<<1, 1024, 0, stream>>>(s.cnt, nl, 128 / G, s.offs, s.chunk_off, s.lists, s.n_lists);
+  sched_fill_kernel<<<gsz, kSchedThreads, 0, stream>>>(block_ids, total, p.h_kv, p.topk, nb, G, s.offs,
+                                                       s.chunk_off, s.fill, s.entries, s.prow_of);
   if (cudaGetLastError() != cudaSuccess) return MSA_ERR_CUDA;
 
   KvoArgs a;
   a.offs = s.offs;
+  a.chunk_off = s.chunk_off;
   a.entries = s.entries;
   a.lists = s.lists;
   a.n_lists = s.n_lists;
   a.work_counter = s.work;
-  a.part_o = s.part_o;
   a.part_lse = s.part_lse;
   a.status = status;
   a.n_q = n_q;
@@ -706,12 +745,11 @@ int run_sparse_attn_kvouter(const msa_params& p, const void* q, const CUtensorMa
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = sms;
   CUtensorMap maps[4] = {tq, tk, tv, tq};
-  {  // partial outputs [topk * n_q][h_q][d]: one box = the G head rows of one (slot, query)
-    const uint64_t dims[3] = {static_cast<uint64_t>(p.d), static_cast<uint64_t>(p.h_q),
-                              static_cast<uint64_t>(p.topk) * n_q};
-    const uint64_t strides[2] = {static_cast<uint64_t>(p.d) * 2, static_cast<uint64_t>(p.h_q) * p.d * 2};
-    const uint32_t box[3] = {64, static_cast<uint32_t>(G), 1};
-    if (!encode_tma_bf16(&maps[3], 3, s.part_o, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MSA_ERR_CUDA;
+  {  // chunk-major partial rows [max_chunks * 128][d]: one box = 128 rows x 64 columns
+    const uint64_t dims[2] = {static_cast<uint64_t>(p.d), static_cast<uint64_t>(s.max_chunks) * 128};
+    const uint64_t strides[1] = {static_cast<uint64_t>(p.d) * 2};
+    const uint32_t box[2] = {64, 128};
+    if (!encode_tma_bf16(&maps[3], 2, s.part_o, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MSA_ERR_CUDA;
   }
   cudaError_t e;
   if (p.d == 64) {
@@ -724,11 +762,11 @@ int run_sparse_attn_kvouter(const msa_params& p, const void* q, const CUtensorMa
   if (e != cudaSuccess) return MSA_ERR_CUDA;
   const int mgrid = n_q * p.h_kv;
   if (p.d == 64)
-    merge_partials_kernel<64><<<mgrid, 256, 0, stream>>>(block_ids, s.part_o, s.part_lse, static_cast<uint16_t*>(o),
-                                                          n_q, p.h_q, p.h_kv, p.topk, nb);
+    merge_partials_kernel<64><<<mgrid, 256, 0, stream>>>(block_ids, s.prow_of, s.part_o, s.part_lse,
+                                                          static_cast<uint16_t*>(o), p.h_q, p.h_kv, p.topk, nb);
   else
-    merge_partials_kernel<128><<<mgrid, 256, 0, stream>>>(block_ids, s.part_o, s.part_lse,
-                                                           static_cast<uint16_t*>(o), n_q, p.h_q, p.h_kv, p.topk, nb);
+    merge_partials_kernel<128><<<mgrid, 256, 0, stream>>>(block_ids, s.prow_of, s.part_o, s.part_lse,
+                                                           static_cast<uint16_t*>(o), p.h_q, p.h_kv, p.topk, nb);
   return cudaGetLastError() == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
 }
 

@@ -141,6 +141,12 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void*
       "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int c0, int c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(c0), "r"(c1)
+               : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until the shared-memory sources of all committed bulk stores were read.
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
@@ -300,6 +306,24 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float r;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
   return r;
+}
+
+// 2^x on the FMA/ALU pipes (x <= 0 or -inf), to offload the MUFU unit.
+// Cody-Waite style range reduction: n = nearest integer to x via the 1.5*2^23
+// rounding constant, f = x - n in [-1/2, 1/2], 2^f from a degree-3 polynomial,
+// and 2^n added to the exponent field.  The coefficients are a weighted
+// least-squares fit of 2^f on [-1/2, 1/2] minimising relative error (Lawson
+// reweighting on Chebyshev nodes); max relative error 7.5e-5, far below the
+// bf16 rounding of P.  x < -126 returns 0 (masked keys, negligible terms).
+__device__ __forceinline__ float exp2_poly(float x) {
+  const float t = x + 12582912.0f;
+  const float n = t - 12582912.0f;
+  const float f = x - n;
+  float p = fmaf(0.05517148971557617f, f, 0.2426111102104187f);
+  p = fmaf(p, f, 0.6932610273361206f);
+  p = fmaf(p, f, 0.9999280571937561f);
+  const float r = __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+  return x < -126.0f ? 0.0f : r;
 }
 
 // Pack two floats to bf16x2 (round to nearest even): lo -> bits 0-15.
