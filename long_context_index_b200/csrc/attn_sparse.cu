@@ -511,52 +511,90 @@ __global__ void sched_count_kernel(const int32_t* ids, long long total, int h_kv
 }
 
 // One CTA: exclusive scans of cnt -> offs and of ceil(cnt / qpc) -> chunk_off,
-// and the compacted list of non-empty lists.
+// and the compacted list of non-empty lists.  Each thread owns 8 consecutive
+// entries per pass; the per-thread totals are scanned with warp shuffles and
+// one cross-warp step, carrying the running totals between passes.
 __global__ void __launch_bounds__(1024) sched_scan_kernel(const int* cnt, int n, int qpc, int* offs, int* chunk_off,
                                                           int* lists, int* n_lists) {
-  __shared__ int s_a[1024], s_b[1024], s_c[1024];
-  __shared__ int carry_a, carry_b, carry_c;
-  if (threadIdx.x == 0) {
-    carry_a = 0;
-    carry_b = 0;
-    carry_c = 0;
-  }
+  constexpr int kPer = 8;
+  __shared__ int wsum[3][32];
+  __shared__ int carry[3];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x < 3) carry[threadIdx.x] = 0;
   __syncthreads();
-  for (int base = 0; base < n; base += 1024) {
-    const int i = base + threadIdx.x;
-    const int v = i < n ? cnt[i] : 0;
-    const int nz = v > 0 ? 1 : 0;
-    const int nc = (v + qpc - 1) / qpc;
-    s_a[threadIdx.x] = v;
-    s_b[threadIdx.x] = nz;
-    s_c[threadIdx.x] = nc;
-    __syncthreads();
-    for (int off = 1; off < 1024; off <<= 1) {
-      const int ta = threadIdx.x >= off ? s_a[threadIdx.x - off] : 0;
-      const int tb = threadIdx.x >= off ? s_b[threadIdx.x - off] : 0;
-      const int tc = threadIdx.x >= off ? s_c[threadIdx.x - off] : 0;
-      __syncthreads();
-      s_a[threadIdx.x] += ta;
-      s_b[threadIdx.x] += tb;
-      s_c[threadIdx.x] += tc;
-      __syncthreads();
+  for (int base = 0; base < n; base += 1024 * kPer) {
+    const int i0 = base + threadIdx.x * kPer;
+    int v[kPer];
+    int ta = 0, tb = 0, tc = 0;
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      v[k] = i0 + k < n ? cnt[i0 + k] : 0;
+      ta += v[k];
+      tb += v[k] > 0;
+      tc += (v[k] + qpc - 1) / qpc;
     }
-    if (i < n) {
-      offs[i] = carry_a + s_a[threadIdx.x] - v;
-      chunk_off[i] = carry_c + s_c[threadIdx.x] - nc;
-      if (nz) lists[carry_b + s_b[threadIdx.x] - 1] = i;
+    // Inclusive warp scan of the thread totals.
+    int ia = ta, ib = tb, ic = tc;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int xa = __shfl_up_sync(0xffffffffu, ia, off);
+      const int xb = __shfl_up_sync(0xffffffffu, ib, off);
+      const int xc = __shfl_up_sync(0xffffffffu, ic, off);
+      if (lane >= off) {
+        ia += xa;
+        ib += xb;
+        ic += xc;
+      }
+    }
+    if (lane == 31) {
+      wsum[0][warp] = ia;
+      wsum[1][warp] = ib;
+      wsum[2][warp] = ic;
     }
     __syncthreads();
-    if (threadIdx.x == 1023) {
-      carry_a += s_a[1023];
-      carry_b += s_b[1023];
-      carry_c += s_c[1023];
+    if (warp == 0) {
+      int a = wsum[0][lane], b = wsum[1][lane], c = wsum[2][lane];
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int xa = __shfl_up_sync(0xffffffffu, a, off);
+        const int xb = __shfl_up_sync(0xffffffffu, b, off);
+        const int xc = __shfl_up_sync(0xffffffffu, c, off);
+        if (lane >= off) {
+          a += xa;
+          b += xb;
+          c += xc;
+        }
+      }
+      wsum[0][lane] = a;   // inclusive over warps
+      wsum[1][lane] = b;
+      wsum[2][lane] = c;
+    }
+    __syncthreads();
+    int pa = carry[0] + (warp ? wsum[0][warp - 1] : 0) + ia - ta;
+    int pb = carry[1] + (warp ? wsum[1][warp - 1] : 0) + ib - tb;
+    int pc = carry[2] + (warp ? wsum[2][warp - 1] : 0) + ic - tc;
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      const int i = i0 + k;
+      if (i < n) {
+        offs[i] = pa;
+        chunk_off[i] = pc;
+        if (v[k] > 0) lists[pb++] = i;
+      }
+      pa += v[k];
+      pc += (v[k] + qpc - 1) / qpc;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      carry[0] += wsum[0][31];
+      carry[1] += wsum[1][31];
+      carry[2] += wsum[2][31];
     }
     __syncthreads();
   }
   if (threadIdx.x == 0) {
-    offs[n] = carry_a;
-    *n_lists = carry_b;
+    offs[n] = carry[0];
+    *n_lists = carry[1];
   }
 }
 
@@ -585,7 +623,10 @@ __global__ void __launch_bounds__(256) merge_partials_kernel(const int32_t* ids,
                                                              uint16_t* o, int h_q, int h_kv, int topk, int nb) {
   // One CTA per (query, group); thread = (head within group, 8-column chunk).
   // prow_of[(q, r, slot)] is the first partial row (chunk * 128 + query-in-
-  // chunk * G) the block-major kernel wrote for that selection.
+  // chunk * G) the block-major kernel wrote for that selection.  Slots are
+  // read 8 at a time with independent loads and folded in with an online
+  // log-sum-exp, so the loads of a group are all in flight together.
+  constexpr int kGrp = 8;
   const int qr = blockIdx.x;
   const int q = qr / h_kv, r = qr % h_kv;
   const int G = h_q / h_kv;
@@ -594,27 +635,38 @@ __global__ void __launch_bounds__(256) merge_partials_kernel(const int32_t* ids,
   const int* my_rows = prow_of + static_cast<size_t>(qr) * topk;
   for (int w = threadIdx.x; w < G * kChunks; w += blockDim.x) {
     const int hh = w / kChunks, ch = w % kChunks;
-    float L = __int_as_float(0xff800000);
-    for (int s = 0; s < topk; ++s) {
-      if (my_ids[s] < 0 || my_ids[s] >= nb) continue;   // the schedule skips these too
-      L = fmaxf(L, part_lse[static_cast<size_t>(my_rows[s]) + hh]);
-    }
+    float M = __int_as_float(0xff800000), den = 0.f;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    float den = 0.f;
-    if (L != __int_as_float(0xff800000)) {
-      for (int s = 0; s < topk; ++s) {
-        if (my_ids[s] < 0 || my_ids[s] >= nb) continue;
-        const size_t prow = static_cast<size_t>(my_rows[s]) + hh;
-        const float ls = part_lse[prow];
-        if (ls == __int_as_float(0xff800000)) continue;
-        const float wgt = ex2_approx(ls - L);
+    for (int s0 = 0; s0 < topk; s0 += kGrp) {
+      float ls[kGrp];
+      uint4 v[kGrp];
+#pragma unroll
+      for (int j = 0; j < kGrp; ++j) {
+        const int s = s0 + j;
+        const int b = s < topk ? my_ids[s] : -1;
+        const bool ok = b >= 0 && b < nb;   // the schedule skips the others too
+        const size_t prow = ok ? static_cast<size_t>(my_rows[s]) + hh : 0;
+        ls[j] = ok ? part_lse[prow] : __int_as_float(0xff800000);
+        v[j] = ok ? *reinterpret_cast<const uint4*>(part_o + prow * D + ch * 8) : make_uint4(0, 0, 0, 0);
+      }
+      float gm = M;
+#pragma unroll
+      for (int j = 0; j < kGrp; ++j) gm = fmaxf(gm, ls[j]);
+      if (gm == __int_as_float(0xff800000)) continue;
+      const float alpha = ex2_approx(M - gm);   // 0 when M is still -inf
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] *= alpha;
+      den *= alpha;
+      M = gm;
+#pragma unroll
+      for (int j = 0; j < kGrp; ++j) {
+        const float wgt = ex2_approx(ls[j] - gm);   // 0 for empty slots
         den += wgt;
-        const uint4 v = *reinterpret_cast<const uint4*>(part_o + prow * D + ch * 8);
-        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+        const uint32_t u[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          acc[2 * i] += wgt * __uint_as_float(u[i] << 16);
-          acc[2 * i + 1] += wgt * __uint_as_float(u[i] & 0xffff0000u);
+          acc[2 * i] = fmaf(wgt, __uint_as_float(u[i] << 16), acc[2 * i]);
+          acc[2 * i + 1] = fmaf(wgt, __uint_as_float(u[i] & 0xffff0000u), acc[2 * i + 1]);
         }
       }
     }
