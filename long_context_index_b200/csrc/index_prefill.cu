@@ -229,25 +229,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int bb = 0; bb < kBlocksPerTile; ++bb) bmax[bb] = __int_as_float(0xff800000);
       const int j0 = t * kKeys;
       if (g < groups_here) {
+        // The 128-column row in two halves (two TMEM loads in flight per
+        // wait); per block, four independent 3-input max chains.
+        float m4[kBlocksPerTile][4];
 #pragma unroll
-        for (int c = 0; c < kKeys / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(taddr_row + acc * 256 + c * 32, v);
+        for (int bb = 0; bb < kBlocksPerTile; ++bb)
+          m4[bb][0] = m4[bb][1] = m4[bb][2] = m4[bb][3] = __int_as_float(0xff800000);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t v[64];
+          tmem_ld32(taddr_row + acc * 256 + h * 64, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+          tmem_ld32(taddr_row + acc * 256 + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
           tmem_ld_wait();
-          const int jc = j0 + c * 32;
-          float m = __int_as_float(0xff800000);
-          if (jc + 32 <= kv_lim) {
+          const int jh = j0 + h * 64;
+          if (jh + 64 > kv_lim) {   // keys this row must not see
 #pragma unroll
-            for (int e = 0; e < 30; e += 3)
-              m = max3f(m, fmaxf(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), __uint_as_float(v[e + 2]));
-            m = max3f(m, __uint_as_float(v[30]), __uint_as_float(v[31]));
-          } else if (jc < kv_lim) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (jc + e < kv_lim) m = fmaxf(m, __uint_as_float(v[e]));
+            for (int e = 0; e < 64; ++e)
+              if (jh + e >= kv_lim) v[e] = 0xff800000u;   // -inf
           }
-          bmax[(c * 32) / BK] = fmaxf(bmax[(c * 32) / BK], m);
+          constexpr int kBpH = 64 / BK > 0 ? 64 / BK : 1;   // blocks touched per half
+#pragma unroll
+          for (int e = 0; e < 64; e += 8) {
+            const int bb = (h * 64 + e) / BK;
+            const int k = (e / 8) & 3;
+            m4[bb][k] = max3f(m4[bb][k], fmaxf(__uint_as_float(v[e]), __uint_as_float(v[e + 1])),
+                              max3f(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]), __uint_as_float(v[e + 4])));
+            m4[bb][k] =
+                max3f(m4[bb][k], __uint_as_float(v[e + 5]), fmaxf(__uint_as_float(v[e + 6]), __uint_as_float(v[e + 7])));
+          }
+          (void)kBpH;
         }
+#pragma unroll
+        for (int bb = 0; bb < kBlocksPerTile; ++bb)
+          bmax[bb] = fmaxf(fmaxf(m4[bb][0], m4[bb][1]), fmaxf(m4[bb][2], m4[bb][3]));
       }
       // Release the accumulator stage to the MMA warp.
       tc_fence_before();
