@@ -150,6 +150,30 @@ MSA_API int msa_sparse_attn_decode(const msa_params* p, const void* q, const voi
  */
 MSA_API int msa_device_status(const void* ws, void* stream);
 
+/*
+ * Allocation-free variant of msa_sparse_attn_decode, for callers that cannot
+ * allocate device memory (no workspace argument).  The paper has no
+ * counterpart: this is a deployment convenience.  Arguments and results are
+ * exactly those of msa_sparse_attn_decode.
+ *   * Scratch: a file-scope device array of MSA_NOALLOC_SCRATCH_BYTES that
+ *     every GPU which loads the library holds until process exit.  A problem
+ *     whose scratch would not fit (see msa_workspace_size(MSA_OP_DECODE, ...))
+ *     is rejected with MSA_ERR_WORKSPACE before anything is launched.
+ *   * The first call on a device looks up the array's device address (once
+ *     per device, with that device current); make that first call before any
+ *     stream capture.
+ *   * Every call on a device shares the one array: calls that overlap on the
+ *     GPU (different streams, no ordering between them) race and may return
+ *     wrong results.  Serialise them, e.g. on one stream.
+ *   * The array keeps the last call's contents; the call itself clears what
+ *     must start at zero.  msa_device_status() does not apply to it.
+ */
+#define MSA_NOALLOC_SCRATCH_BYTES (16u << 20)
+MSA_API int msa_sparse_attn_decode_noalloc(const msa_params* p, const void* q, const void* q_idx,
+                                           const void* k_cache, const void* v_cache, const void* k_idx_cache,
+                                           const int64_t* cu_kv, int batch, int max_kv, int dense,
+                                           int32_t* block_ids, void* o, void* stream);
+
 /* Human-readable text of a status code (static storage). */
 MSA_API const char* msa_status_string(int status);
 

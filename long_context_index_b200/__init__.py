@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(_HERE, "libmsa.so")
 OP_INDEX_TOPK, OP_PREFILL, OP_DECODE = 0, 1, 2
 
 SYMBOLS = ("msa_workspace_size", "msa_index_topk", "msa_sparse_attn_prefill", "msa_sparse_attn_decode",
-           "msa_device_status", "msa_status_string")
+           "msa_device_status", "msa_status_string", "msa_sparse_attn_decode_noalloc")
 
 
 class MSAError(RuntimeError):
@@ -63,6 +63,8 @@ def lib():
         L.msa_index_topk.argtypes = [P, vp, vp, i32, i32, i32, vp, vp, sz, vp]
         L.msa_sparse_attn_prefill.argtypes = [P, vp, vp, vp, vp, i32, i32, i32, vp, vp, sz, vp]
         L.msa_sparse_attn_decode.argtypes = [P, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, vp, vp, sz, vp]
+        L.msa_sparse_attn_decode_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, vp, vp]
+        L.msa_sparse_attn_decode_noalloc.restype = i32
         L.msa_device_status.argtypes = [vp, vp]
         L.msa_status_string.argtypes = [i32]
         L.msa_status_string.restype = C.c_char_p

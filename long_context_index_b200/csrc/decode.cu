@@ -24,6 +24,7 @@
 // The dense run skips 1-2 and lets step 3 enumerate every causal block.
 #include <cstdint>
 #include <cuda_runtime.h>
+#include <mutex>
 
 #include "msa_internal.h"
 #include "ptx.cuh"
@@ -601,3 +602,54 @@ int run_sparse_attn_decode(const msa_params& p, const void* q, const void* q_idx
 }
 
 }  // namespace msa
+
+// ---------------------------------------------------------------------------
+// Allocation-free decode step.
+//
+// For callers that cannot allocate device memory at all: code running where
+// cudaMalloc is not allowed (for example while a serving runtime owns and
+// pre-partitions every byte of the GPU, or a plugin that is handed only its
+// input and output buffers).  The scratch the decode step needs lives in a
+// fixed file-scope device array of MSA_NOALLOC_SCRATCH_BYTES, which every GPU
+// that loads this library holds until the process exits.
+// ---------------------------------------------------------------------------
+namespace msa {
+namespace {
+
+constexpr int kMaxDevices = 64;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[MSA_NOALLOC_SCRATCH_BYTES];
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of this device's copy of the array.  In host code the
+// array's name is only a host-side stand-in, never a device address, so the
+// address is looked up once per device with that device current.
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MSA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return MSA_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return MSA_OK;
+}
+
+}  // namespace
+}  // namespace msa
+
+extern "C" MSA_API int msa_sparse_attn_decode_noalloc(const msa_params* p, const void* q, const void* q_idx,
+                                                      const void* k_cache, const void* v_cache,
+                                                      const void* k_idx_cache, const int64_t* cu_kv, int batch,
+                                                      int max_kv, int dense, int32_t* block_ids, void* o,
+                                                      void* stream) {
+  void* scratch = nullptr;
+  const int rc = msa::noalloc_scratch(&scratch);
+  if (rc) return rc;
+  // Same validation and kernels as msa_sparse_attn_decode; a problem whose
+  // scratch exceeds the array is rejected there with MSA_ERR_WORKSPACE.
+  return msa_sparse_attn_decode(p, q, q_idx, k_cache, v_cache, k_idx_cache, cu_kv, batch, max_kv, dense, block_ids,
+                                o, scratch, MSA_NOALLOC_SCRATCH_BYTES, stream);
+}

@@ -77,7 +77,7 @@ def test_prefill_and_decode_reject_bad_arguments():
     L = msa.lib()
     p = P()
     assert L.msa_sparse_attn_prefill(C.byref(p), 16, 16, 16, None, 10, 5, 0, 16, 256, 1 << 20, None) == -1
-    assert L.msa_sparse_attn_prefill(C.byref(p), 16, 16, 16, 8, 10, 10, 0, 16, 256, 1 << 20, None) == -3
+    assert L.msa_sparse_attn_prefill(C.byref(p), 16, 16, 16, 8, 10, 10, 0, 16, 256, 1 << 40, None) == -3
     assert L.msa_sparse_attn_decode(C.byref(p), 16, 16, 16, 16, 16, 16, 0, 100, 0, 16, 16, 256, 1 << 30,
                                     None) == -1
     assert L.msa_sparse_attn_decode(C.byref(p), 16, 16, 16, 16, 16, 16, 4, 100, 0, 16, 16, 256, 10, None) == -4
