@@ -50,7 +50,11 @@ L2_BYTES = 126 * 1024 * 1024
 
 # DRAM traffic per launch from the committed ncu captures, keyed by kernel,
 # with the digest of the kernel source it was measured on (stale -> null).
-TRAFFIC = {}
+TRAFFIC = {
+    # schedule + KV-outer + merge (msa_sparse_attn_prefill) at 128K, from
+    # profiles/bench_prefill_128k_decode_b64_launches.md
+    "attn_prefill": (14.087e9 + 35.567e9 + 35.023e9 + 2.142e9 + 0.080e9, "1563746e8dd8", "attn_sparse.cu"),
+}
 
 
 def load_peaks():
