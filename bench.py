@@ -142,17 +142,31 @@ def bf16(torch, t):
     return t.view(torch.bfloat16) if t.dtype == torch.int16 else t
 
 
+def rank_workloads(case: str, rank: int):
+    """The (prefill, decode) problems rank `rank` runs: the same shapes on
+    every rank, each rank its own seed, so N ranks process N independent
+    problems (weak scaling; no data crosses ranks)."""
+    pre, dec = cases(case)
+    off = 1000 * rank
+    return (Workload(**{**pre.__dict__, "seed": pre.seed + off}),
+            Workload(**{**dec.__dict__, "seed": dec.seed + off}))
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    """Max of a per-rank time over all ranks (every rank calls this)."""
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def run_ours(args, rank, world, torch, dist):
     import long_context_index_b200 as msa
     from long_context_index_b200 import flops
 
-    PREFILL, DECODE = cases(args.case)
-
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream()
-    seed_off = 1000 * rank   # each rank its own independent problem
-    wp = Workload(**{**PREFILL.__dict__, "seed": PREFILL.seed + seed_off})
-    wd = Workload(**{**DECODE.__dict__, "seed": DECODE.seed + seed_off})
+    wp, wd = rank_workloads(args.case, rank)
     tp = make_prefill(wp)
     td = make_decode(wd)
     pp = msa.Params.make(wp.h_q, wp.h_kv, wp.d, wp.d_idx, wp.block_k, wp.topk)
@@ -221,9 +235,7 @@ def run_ours(args, rank, world, torch, dist):
         if rc:
             raise RuntimeError("device status %d after the timed steps" % rc)
     if world > 1:
-        tt = torch.tensor([t_total], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_total = float(tt.item())
+        t_total = max_over_ranks(t_total, dist, dev)
     ms_step = t_total / args.steps
     tokens_step = n + B
     value = tokens_step * world / (ms_step / 1e3)
@@ -285,9 +297,7 @@ def run_ours(args, rank, world, torch, dist):
         torch.cuda.synchronize()
         t_e2e = a.elapsed_time(b)
         if world > 1:
-            tt = torch.tensor([t_e2e], dtype=torch.float64, device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            t_e2e = float(tt.item())
+            t_e2e = max_over_ranks(t_e2e, dist, dev)
         e2e_value = tokens_step * world / (t_e2e / args.steps / 1e3)
 
     peaks, peak_src = load_peaks()

@@ -22,7 +22,8 @@ LIB_PATH = os.path.join(_HERE, "libmsa.so")
 OP_INDEX_TOPK, OP_PREFILL, OP_DECODE = 0, 1, 2
 
 SYMBOLS = ("msa_workspace_size", "msa_index_topk", "msa_sparse_attn_prefill", "msa_sparse_attn_decode",
-           "msa_device_status", "msa_status_string", "msa_sparse_attn_decode_noalloc")
+           "msa_device_status", "msa_status_string", "msa_sparse_attn_decode_noalloc",
+           "msa_test_never_ready_wait")
 
 
 class MSAError(RuntimeError):
@@ -65,6 +66,8 @@ def lib():
         L.msa_sparse_attn_decode.argtypes = [P, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, vp, vp, sz, vp]
         L.msa_sparse_attn_decode_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, vp, vp]
         L.msa_sparse_attn_decode_noalloc.restype = i32
+        L.msa_test_never_ready_wait.argtypes = [vp, sz, C.c_longlong, vp]
+        L.msa_test_never_ready_wait.restype = i32
         L.msa_device_status.argtypes = [vp, vp]
         L.msa_status_string.argtypes = [i32]
         L.msa_status_string.restype = C.c_char_p

@@ -79,6 +79,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 struct WaitCtx {
   volatile int* abort_flag;  // shared memory
   int* status;               // global memory, may be null
+  unsigned long long deadline_ns = kWaitNs;
 };
 
 static __device__ __noinline__ void wait_timed_out(const WaitCtx& w) {
@@ -94,7 +95,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*w.abort_flag) return false;
-    if (globaltimer() - t0 > kWaitNs) {
+    if (globaltimer() - t0 > w.deadline_ns) {
       wait_timed_out(w);
       return false;
     }

@@ -13,8 +13,11 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def declared_symbols():
-    src = open(os.path.join(ROOT, "include", "msa.h")).read()
-    return sorted(set(re.findall(r"^MSA_API [^(]*?\b(msa_\w+)\(", src, re.M)))
+    names = set()
+    for h in ("msa.h", "msa_testing.h"):
+        src = open(os.path.join(ROOT, "include", h)).read()
+        names |= set(re.findall(r"^MSA_API [^(]*?\b(msa_\w+)\(", src, re.M))
+    return sorted(names)
 
 
 def test_library_exports_every_declared_symbol():

@@ -69,3 +69,7 @@ def test_decode_b64_64k_128k():
 
 def test_decode_b64_64k_128k_dense_sampled():
     run_case(WORKLOADS["decode_b64_64k_128k"], dense=True, seqs=[0, 17, 63])
+
+
+def test_decode_b8_1m():
+    run_case(WORKLOADS["decode_b8_1m"])

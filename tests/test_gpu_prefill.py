@@ -103,3 +103,10 @@ def test_prefill_32k_sampled_rows():
 def test_prefill_128k_sampled_rows():
     w = WORKLOADS["prefill_128k"]
     run_case(w, rows=sampled(w, 32))
+
+
+def test_chunked_prefill_1m_sampled_rows():
+    w = WORKLOADS["chunked_prefill_1m"]
+    rng = np.random.default_rng(4)
+    rows = list(rng.integers(0, w.n_q, 12)) + [0, w.n_q - 1]
+    run_case(w, rows=rows)
