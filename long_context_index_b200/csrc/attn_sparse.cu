@@ -18,8 +18,10 @@
 //        K_b, V_b once by TMA, then streams chunks of 128/G queries of the
 //        list (each query's G head rows of group r are one 3-D TMA box), and
 //        publishes a descriptor per chunk in a 4-deep ring.
-//      * warp 1 issues S = Q K_b^T into one of two TMEM S buffers and
-//        O = P V_b (P read back from TMEM) into one of two TMEM O buffers.
+//      * warp 1 issues S = Q K_b^T into the TMEM S buffer, and O = P V_b (P
+//        read from one of two TMEM P buffers) into one of two TMEM O buffers.
+//        S is released as soon as the softmax has loaded it, so the next S
+//        MMA queues behind the previous PV and the tensor pipe stays fed.
 //      * warps 2..9 (softmax): two threads per row, each owning 64 of the 128
 //        columns; the exact softmax of the row over the block's visible keys
 //        (causal only in the local block); the two halves exchange only their
@@ -65,8 +67,11 @@ struct KvoCfg {
   static constexpr int kOBytes = 128 * D * 2;          // staged bf16 partial tile
   static constexpr int kSmemData = kQStages * kQBytes + kKVStages * 2 * kKVBytes + kOStages * kOBytes;
   static constexpr int kSmemBytes = kSmemData + 12288 + 1024;
-  static constexpr int kColS = 0;        // S/P buffers: [0, BK), [BK, 2BK)
-  static constexpr int kColO = 2 * BK;   // O buffers: [2BK, 2BK + D), [2BK + D, 2BK + 2D)
+  // TMEM: one S buffer (freed as soon as the softmax has loaded it), two P
+  // buffers (bf16 pairs, BK/2 columns each), two O buffers.
+  static constexpr int kColS = 0;        // S: [0, BK)
+  static constexpr int kColP = BK;       // P: [BK, BK + BK/2), [BK + BK/2, 2BK)
+  static constexpr int kColO = 2 * BK;   // O: [2BK, 2BK + D), [2BK + D, 2BK + 2D)
   static constexpr int kTmemCols = (2 * BK + 2 * D) <= 256 ? 256 : 512;
 };
 
@@ -118,9 +123,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* kv_empty = kv_full + kKVStages;
   uint64_t* d_full = kv_empty + kKVStages;                   // [kDesc]
   uint64_t* d_empty = d_full + kDesc;
-  uint64_t* s_full = d_empty + kDesc;                        // [2]
-  uint64_t* s_free = s_full + 2;
-  uint64_t* p_full = s_free + 2;
+  uint64_t* s_full = d_empty + kDesc;                        // [1] S ready
+  uint64_t* s_free = s_full + 1;                             // [1] S loaded by the softmax
+  uint64_t* p_free = s_free + 1;                             // [2] P consumed by its PV
+  uint64_t* p_full = p_free + 2;
   uint64_t* o_full = p_full + 2;
   uint64_t* o_free = o_full + 2;
   uint64_t* ml_full = o_free + 2;                            // [kDesc]
@@ -143,9 +149,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&d_empty[s], 13);  // MMA thread + 8 softmax warps + 4 epilogue warps
       mbar_init(&ml_full[s], 8);   // 8 softmax warps
     }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 8);          // the 8 softmax warps, once their S loads completed
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&s_full[s], 1);
-      mbar_init(&s_free[s], 1);
+      mbar_init(&p_free[s], 1);
       mbar_init(&p_full[s], 8);
       mbar_init(&o_full[s], 1);
       mbar_init(&o_free[s], 4);
@@ -270,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&o_free[sb], ((j >> 1) & 1) ^ 1, wc)) return false;
         tc_fence_after();
         const uint32_t sv_addr = skv_addr + kvs * 2 * Cfg::kKVBytes + Cfg::kKVBytes;
-        const uint32_t p_tmem = tmem + Cfg::kColS + sb * BK;
+        const uint32_t p_tmem = tmem + Cfg::kColP + sb * (BK / 2);
         const uint32_t o_tmem = tmem + Cfg::kColO + sb * D;
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
@@ -278,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_ts(o_tmem, p_tmem + kk * 8, bdesc, idesc_o, kk > 0 ? 1u : 0u);
         }
         umma_commit(&o_full[sb]);
-        umma_commit(&s_free[sb]);
+        umma_commit(&p_free[sb]);
         if (last) umma_commit(&kv_empty[kvs]);
         return true;
       };
@@ -298,7 +305,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++kvc;
         }
         if (!mbar_wait(&q_full[qs], (t / kQStages) & 1, wc)) { ok = false; break; }
-        if (!mbar_wait(&s_free[sb], ((t >> 1) & 1) ^ 1, wc)) { ok = false; break; }
+        // S(t) reuses the single S buffer once the softmax has loaded S(t-1).
+        if (!mbar_wait(s_free, (t & 1) ^ 1, wc)) { ok = false; break; }
         tc_fence_after();
         const uint32_t sk_addr = skv_addr + kvs * 2 * Cfg::kKVBytes;
 #pragma unroll
@@ -308,10 +316,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t adesc =
               smem_desc(sq_addr + qs * Cfg::kQBytes + atom * 128 * 128 + koff, 16, 1024, kSwizzle128B);
           const uint64_t bdesc = smem_desc(sk_addr + atom * BK * 128 + koff, 16, 1024, kSwizzle128B);
-          umma_ss(tmem + Cfg::kColS + sb * BK, adesc, bdesc, idesc_s, ks > 0 ? 1u : 0u);
+          umma_ss(tmem + Cfg::kColS, adesc, bdesc, idesc_s, ks > 0 ? 1u : 0u);
         }
         umma_commit(&q_empty[qs]);
-        umma_commit(&s_full[sb]);
+        umma_commit(s_full);
         if (pending && !issue_pv(t - 1, prev_kvs, prev_last)) { ok = false; break; }
         if (last) {
           // The last chunk of a list frees the K/V stage the producer waits on
@@ -355,15 +363,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int kv_lim = args.causal ? min(p + 1, args.n_kv) : args.n_kv;
         lim = min(BK, kv_lim - b * BK) - half * HC;
       }
-      const int sb = t & 1;
-      if (!mbar_wait(&s_full[sb], (t >> 1) & 1, wc)) break;
+      const int sb = t & 1;   // P buffer
+      if (!mbar_wait(s_full, t & 1, wc)) break;
       tc_fence_after();
-      const uint32_t s_tmem = lane_base + Cfg::kColS + sb * BK;
+      const uint32_t s_tmem = lane_base + Cfg::kColS;
       uint32_t sv[HC];
 #pragma unroll
       for (int cc = 0; cc < HC / 32; ++cc)
         tmem_ld32(s_tmem + half * HC + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[cc * 32]));
       tmem_ld_wait();
+      // S is in registers: hand the S buffer back so the next S MMA can start.
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free);
       if (lim < HC) {
 #pragma unroll
         for (int i = 0; i < HC; ++i)
@@ -386,8 +398,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       xs[half * 128 + row] = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
       named_bar(2 + quarter, 64);
       const float mx = fmaxf(xs[row], xs[128 + row]);
-      // Both halves' S values are in registers past this barrier, so P may
-      // overwrite any S column.
       const float bias = mx == __int_as_float(0xff800000) ? 0.f : mx * c;
       float ls[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t pk[HC / 2];
@@ -401,10 +411,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         pk[i / 2] = pack_bf16x2(p0, p1);
         pk[i / 2 + 1] = pack_bf16x2(p2, p3);
       }
+      // P(t) goes to P buffer t & 1 once the PV of chunk t - 2 has read it.
+      if (!mbar_wait(&p_free[sb], ((t >> 1) & 1) ^ 1, wc)) break;
+      tc_fence_after();
+      const uint32_t p_tmem = lane_base + Cfg::kColP + sb * (BK / 2);
 #pragma unroll
       for (int cc = 0; cc < HC / 64; ++cc)
-        tmem_st32(s_tmem + half * (HC / 2) + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[cc * 32]));
-      if (HC / 2 == 16) tmem_st16(s_tmem + half * (HC / 2), *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
+        tmem_st32(p_tmem + half * (HC / 2) + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[cc * 32]));
+      if (HC / 2 == 16) tmem_st16(p_tmem + half * (HC / 2), *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
       const float lsum = (ls[0] + ls[1]) + (ls[2] + ls[3]);
       if (half == 0)
         ml[ds * 128 + row] = make_float2(mx, lsum);
