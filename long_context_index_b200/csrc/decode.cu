@@ -12,15 +12,17 @@
 //      to Q_idx and K_idx alike, makes each loaded 16-byte vector a fragment;
 //      the dot product does not depend on the order of d_idx).  Max-pools per
 //      block and keeps the chunk's top (k - 1) non-local blocks per group.
-//   2. decode_topk_merge_kernel  one warp per (sequence, group): top (k - 1)
-//      of the chunk lists (score desc, block asc: exact because every global
-//      winner is a winner of its chunk), plus the local block, ascending.
+//   2. merge (in the index kernel's last CTA of each sequence, found with an
+//      atomic counter): one warp per group takes the top (k - 1) of the chunk
+//      lists (score desc, block asc: exact because every global winner is a
+//      winner of its chunk), plus the local block, ascending.
 //   3. decode_attn_kernel    grid (splits, group x head tile, batch).  Each
 //      CTA stages whole K/V blocks with cp.async (16-byte, coalesced), shares
 //      them among the 16 heads of its head tile, and runs QK^T and PV on
 //      mma.sync with an fp32 online softmax; writes an (m, l, o) partial.
-//   4. decode_combine_kernel  per (sequence, head): LSE-weighted sum of the
-//      partials, rounded to bf16.
+//   4. combine (in the attention kernel's last CTA of each (sequence, group,
+//      head tile)): per head, the LSE-weighted sum of the split partials,
+//      rounded to bf16.
 // The dense run skips 1-2 and lets step 3 enumerate every causal block.
 #include <cstdint>
 #include <cuda_runtime.h>
@@ -35,6 +37,7 @@ namespace {
 constexpr int kIdxThreads = 256;    // 8 warps
 constexpr int kIdxChunkBlocks = 64; // CB: blocks per index CTA
 constexpr int kAttnThreads = 128;   // 4 warps, 32 keys each
+constexpr int kMergeRegCand = 8;    // per-lane register cache of the merge
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kNegInf = -__builtin_huge_valf();
 
@@ -63,8 +66,10 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool v
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
                : "memory");
 }
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 __device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
@@ -91,7 +96,9 @@ struct DecArgs {
   uint16_t* o;              // [B, h_q, d]
   float* cand_s;            // [B, max_chunks, h_kv, kfree]
   int* cand_b;
-  float* part;              // [B, h_q, splits, d + 2]  (o[d], m, l)
+  float* part;              // [B, h_q, splits, d + 4]  (o[d], m, l, 2 pad)
+  int* seq_count;           // [B] index CTAs finished per sequence (zeroed per call)
+  int* grp_count;           // [B, h_kv, head_tiles] attention CTAs finished (zeroed per call)
   int batch, h_q, h_kv, topk, causal, force_local, kfree, max_chunks;
   int splits, slots_per_split, dense, head_tiles;
   float scale_log2;
@@ -100,6 +107,9 @@ struct DecArgs {
 // ---------------------------------------------------------------------------
 // 1. index scan: block max-pool + per-chunk top-(k-1) per group
 // ---------------------------------------------------------------------------
+template <int BK>
+__device__ void merge_topk_warp(const DecArgs& a, int b, int r, int lane, int* chosen);
+
 template <int DIDX, int BK>
 __global__ void __launch_bounds__(kIdxThreads) decode_index_kernel(const DecArgs a) {
   constexpr int kHalves = DIDX / 32;   // 16-byte vectors per token row per thread
@@ -164,6 +174,8 @@ __global__ void __launch_bounds__(kIdxThreads) decode_index_kernel(const DecArgs
   }
   __syncthreads();
 
+  __shared__ int chosen[8][33];
+  __shared__ int s_last;
   // Per group: top-kfree eligible non-local blocks of this chunk.
   const int p = L - 1;
   const int b_loc = p / BK;
@@ -200,16 +212,22 @@ __global__ void __launch_bounds__(kIdxThreads) decode_index_kernel(const DecArgs
       }
     }
   }
+  // The last CTA of this sequence to finish merges the chunk lists.
+  const int nch = min((nb + kIdxChunkBlocks - 1) / kIdxChunkBlocks, a.max_chunks);
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = atomicAdd(&a.seq_count[b], 1) == nch - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  for (int r = warp; r < a.h_kv; r += kIdxThreads / 32) merge_topk_warp<BK>(a, b, r, lane, chosen[warp]);
 }
 
 // ---------------------------------------------------------------------------
 // 2. merge of the chunk lists + local block -> block_ids (ascending, -1 pad)
 // ---------------------------------------------------------------------------
 template <int BK>
-__global__ void __launch_bounds__(32) decode_topk_merge_kernel(const DecArgs a) {
-  const int b = blockIdx.x / a.h_kv;
-  const int r = blockIdx.x % a.h_kv;
-  const int lane = threadIdx.x;
+__device__ void merge_topk_warp(const DecArgs& a, int b, int r, int lane, int* chosen) {
   const int L = static_cast<int>(a.cu_kv[b + 1] - a.cu_kv[b]);
   const int nb = (L + BK - 1) / BK;
   // Clamp to the chunks the workspace holds (a caller that understated max_kv
@@ -217,36 +235,74 @@ __global__ void __launch_bounds__(32) decode_topk_merge_kernel(const DecArgs a) 
   const int nch = min((nb + kIdxChunkBlocks - 1) / kIdxChunkBlocks, a.max_chunks);
   const int ncand = nch * a.kfree;
   const int b_loc = (L - 1) / BK;
-  __shared__ int chosen[33];
   int nsel = 0;
-  // Repeated warp argmax over the candidates with a strictly decreasing bound:
-  // each round picks the best candidate that is worse than the previous pick.
-  float last_s = __builtin_huge_valf();
-  int last_b = -1;
-  for (int k = 0; k < a.kfree; ++k) {
-    float bs = kNegInf;
-    int bi = 0x7fffffff;
-    for (int c = lane; c < ncand; c += 32) {
-      const int ch = c / a.kfree, slot = c % a.kfree;
-      const size_t idx = ((static_cast<size_t>(b) * a.max_chunks + ch) * a.h_kv + r) * a.kfree + slot;
-      const int cb = a.cand_b[idx];
-      if (cb < 0) continue;
-      const float cs = a.cand_s[idx];
-      // Only candidates strictly after the previous pick in (score desc, block asc).
-      if (k > 0 && !better(last_s, last_b, cs, cb)) continue;
-      if (bi == 0x7fffffff || better(cs, cb, bs, bi)) { bs = cs; bi = cb; }
-    }
+  if (ncand <= 32 * kMergeRegCand) {
+    // Small candidate sets (up to 16 chunks of 16) live in registers: one
+    // load per candidate, then repeated warp argmax; the owner lane retires
+    // each pick (block ids are unique across chunks).
+    float cs[kMergeRegCand];
+    int cb[kMergeRegCand];
 #pragma unroll
-    for (int x = 16; x > 0; x >>= 1) {
-      const float os = __shfl_xor_sync(0xffffffffu, bs, x);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, x);
-      if (oi != 0x7fffffff && (bi == 0x7fffffff || better(os, oi, bs, bi))) { bs = os; bi = oi; }
+    for (int i = 0; i < kMergeRegCand; ++i) {
+      const int c = lane + 32 * i;
+      cs[i] = kNegInf;
+      cb[i] = -1;
+      if (c < ncand) {
+        const int ch = c / a.kfree, slot = c % a.kfree;
+        const size_t idx = ((static_cast<size_t>(b) * a.max_chunks + ch) * a.h_kv + r) * a.kfree + slot;
+        cb[i] = __ldcg(a.cand_b + idx);
+        cs[i] = __ldcg(a.cand_s + idx);
+      }
     }
-    if (bi == 0x7fffffff) break;
-    if (lane == 0) chosen[nsel] = bi;
-    ++nsel;
-    last_s = bs;
-    last_b = bi;
+    for (int k = 0; k < a.kfree; ++k) {
+      float bs = kNegInf;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < kMergeRegCand; ++i)
+        if (cb[i] >= 0 && (bi == 0x7fffffff || better(cs[i], cb[i], bs, bi))) { bs = cs[i]; bi = cb[i]; }
+#pragma unroll
+      for (int x = 16; x > 0; x >>= 1) {
+        const float os = __shfl_xor_sync(0xffffffffu, bs, x);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, x);
+        if (oi != 0x7fffffff && (bi == 0x7fffffff || better(os, oi, bs, bi))) { bs = os; bi = oi; }
+      }
+      if (bi == 0x7fffffff) break;
+      if (lane == 0) chosen[nsel] = bi;
+      ++nsel;
+#pragma unroll
+      for (int i = 0; i < kMergeRegCand; ++i)
+        if (cb[i] == bi) cb[i] = -1;
+    }
+  } else {
+    // Repeated warp argmax over the candidates with a strictly decreasing bound:
+    // each round picks the best candidate that is worse than the previous pick.
+    float last_s = __builtin_huge_valf();
+    int last_b = -1;
+    for (int k = 0; k < a.kfree; ++k) {
+      float bs = kNegInf;
+      int bi = 0x7fffffff;
+      for (int c = lane; c < ncand; c += 32) {
+        const int ch = c / a.kfree, slot = c % a.kfree;
+        const size_t idx = ((static_cast<size_t>(b) * a.max_chunks + ch) * a.h_kv + r) * a.kfree + slot;
+        const int cb = __ldcg(a.cand_b + idx);
+        if (cb < 0) continue;
+        const float cs = __ldcg(a.cand_s + idx);
+        // Only candidates strictly after the previous pick in (score desc, block asc).
+        if (k > 0 && !better(last_s, last_b, cs, cb)) continue;
+        if (bi == 0x7fffffff || better(cs, cb, bs, bi)) { bs = cs; bi = cb; }
+      }
+  #pragma unroll
+      for (int x = 16; x > 0; x >>= 1) {
+        const float os = __shfl_xor_sync(0xffffffffu, bs, x);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, x);
+        if (oi != 0x7fffffff && (bi == 0x7fffffff || better(os, oi, bs, bi))) { bs = os; bi = oi; }
+      }
+      if (bi == 0x7fffffff) break;
+      if (lane == 0) chosen[nsel] = bi;
+      ++nsel;
+      last_s = bs;
+      last_b = bi;
+    }
   }
   if (lane == 0) {
     if (a.force_local) chosen[nsel++] = b_loc;
@@ -260,6 +316,15 @@ __global__ void __launch_bounds__(32) decode_topk_merge_kernel(const DecArgs a) 
     int32_t* out = a.block_ids + (static_cast<size_t>(b) * a.h_kv + r) * a.topk;
     for (int i = 0; i < a.topk; ++i) out[i] = i < nsel ? chosen[i] : -1;
   }
+  __syncwarp();
+}
+
+// topk == 1 with the forced local block: no scan, every sequence's ids are
+// its local block.
+template <int BK>
+__global__ void __launch_bounds__(32) decode_local_only_kernel(const DecArgs a) {
+  __shared__ int chosen[33];
+  merge_topk_warp<BK>(a, blockIdx.x / a.h_kv, blockIdx.x % a.h_kv, threadIdx.x, chosen);
 }
 
 // ---------------------------------------------------------------------------
@@ -296,13 +361,52 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const DecArgs
   const int L = static_cast<int>(a.cu_kv[b + 1] - off);
   const int nb = (L + BK - 1) / BK;
 
-  // Q rows of this head tile (zero rows beyond the group).
-  for (int c = tid; c < 16 * kChunks; c += kAttnThreads) {
-    const int row = c / kChunks, ch = c % kChunks;
-    cp_async16(swz<D>(smem_u32(sQ), row, ch), a.q + (static_cast<size_t>(b) * a.h_q + h0 + min(row, rows - 1)) * D + ch * 8,
-               row < rows);
-  }
-  cp_async_wait_all();
+  const int s_begin = split * a.slots_per_split;
+  const int n_slots = a.dense ? nb : a.topk;
+  const int s_end = min(n_slots, s_begin + a.slots_per_split);
+  const int32_t* ids = a.block_ids + (static_cast<size_t>(b) * a.h_kv + r) * a.topk;
+  // Next slot at or after s holding a block of this sequence (padding is -1).
+  auto next_valid = [&](int s) {
+    for (; s < s_end; ++s) {
+      const int blk = a.dense ? s : ids[s];
+      if (blk >= 0 && blk < nb) break;
+    }
+    return s;
+  };
+  // Two cp.async groups per block: K (with Q on the first block), then V, so
+  // that Q K^T and the softmax run while V is still arriving.
+  auto load_kv = [&](int blk, bool with_q) {
+    const int j0 = blk * BK;
+    if (with_q) {
+      for (int c = tid; c < 16 * kChunks; c += kAttnThreads) {
+        const int row = c / kChunks, ch = c % kChunks;
+        cp_async16(swz<D>(smem_u32(sQ), row, ch),
+                   a.q + (static_cast<size_t>(b) * a.h_q + h0 + min(row, rows - 1)) * D + ch * 8, row < rows);
+      }
+    }
+    if (blk >= 0) {
+      for (int c = tid; c < BK * kChunks; c += kAttnThreads) {
+        const int row = c / kChunks, ch = c % kChunks;
+        const bool ok = j0 + row < L;
+        const size_t src = ((static_cast<size_t>(off) + (ok ? j0 + row : 0)) * a.h_kv + r) * D + ch * 8;
+        cp_async16(swz<D>(smem_u32(sK), row, ch), a.k_cache + src, ok);
+      }
+    }
+    cp_async_commit();
+    if (blk >= 0) {
+      for (int c = tid; c < BK * kChunks; c += kAttnThreads) {
+        const int row = c / kChunks, ch = c % kChunks;
+        const bool ok = j0 + row < L;
+        const size_t src = ((static_cast<size_t>(off) + (ok ? j0 + row : 0)) * a.h_kv + r) * D + ch * 8;
+        cp_async16(swz<D>(smem_u32(sV), row, ch), a.v_cache + src, ok);
+      }
+    }
+    cp_async_commit();
+  };
+
+  int s = next_valid(s_begin);
+  load_kv(s < s_end ? (a.dense ? s : ids[s]) : -1, true);
+  cp_async_wait<1>();
   __syncthreads();
   uint32_t qf[D / 16][4];
 #pragma unroll
@@ -317,23 +421,9 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const DecArgs
   for (int i = 0; i < D / 8; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
   float m_lo = kNegInf, m_hi = kNegInf, l_lo = 0.f, l_hi = 0.f;   // rows g, g+8
 
-  const int s_begin = split * a.slots_per_split;
-  const int n_slots = a.dense ? nb : a.topk;
-  const int s_end = min(n_slots, s_begin + a.slots_per_split);
-  for (int s = s_begin; s < s_end; ++s) {
-    const int blk = a.dense ? s : a.block_ids[(static_cast<size_t>(b) * a.h_kv + r) * a.topk + s];
-    if (blk < 0 || blk >= nb) continue;    // padding
+  while (s < s_end) {
+    const int blk = a.dense ? s : ids[s];
     const int j0 = blk * BK;
-    __syncthreads();   // previous block fully consumed
-    for (int c = tid; c < BK * kChunks; c += kAttnThreads) {
-      const int row = c / kChunks, ch = c % kChunks;
-      const bool ok = j0 + row < L;
-      const size_t src = ((static_cast<size_t>(off) + (ok ? j0 + row : 0)) * a.h_kv + r) * D + ch * 8;
-      cp_async16(swz<D>(smem_u32(sK), row, ch), a.k_cache + src, ok);
-      cp_async16(swz<D>(smem_u32(sV), row, ch), a.v_cache + src, ok);
-    }
-    cp_async_wait_all();
-    __syncthreads();
 
     // S = Q K^T for this warp's KPW keys (NT n-tiles of 8).
     float sacc[NT][4];
@@ -394,6 +484,8 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const DecArgs
       oacc[i][2] *= al_hi;
       oacc[i][3] *= al_hi;
     }
+    cp_async_wait<0>();
+    __syncthreads();   // V landed for every warp
     // O += P V (KS steps of 16 keys).
 #pragma unroll
     for (int kk = 0; kk < KS; ++kk) {
@@ -407,7 +499,15 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const DecArgs
         mma_bf16_16816(oacc[dt + 1], a0, a1, a2, a3, b2, b3);
       }
     }
+    s = next_valid(s + 1);
+    if (s < s_end) {
+      __syncthreads();   // this block's K and V fully consumed
+      load_kv(a.dense ? s : ids[s], false);
+      cp_async_wait<1>();
+      __syncthreads();
+    }
   }
+  cp_async_wait<0>();
 
   // Row sums over the 4 threads of a row.
 #pragma unroll
@@ -442,7 +542,7 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const DecArgs
     sO[(warp * 16 + g + 8) * D + col + 1] = oacc[dt][3] * sc_hi;
   }
   __syncthreads();
-  const size_t stride = D + 2;
+  const size_t stride = D + 4;   // 16-byte rows for the float4 combine
   for (int e = tid; e < 16 * D; e += kAttnThreads) {
     const int row = e / D, col = e % D;
     if (row >= rows) continue;
@@ -462,32 +562,441 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const DecArgs
     pp[D] = M;
     pp[D + 1] = Lsum;
   }
+  // The last split CTA of this (sequence, group, head tile) combines: per
+  // row, weights w_s = exp2(m_s - M) / sum_s w_s l_s, then O = sum_s w_s o_s.
+  __shared__ int s_last;
+  __shared__ float s_w[16][32];
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = atomicAdd(&a.grp_count[blockIdx.z * gridDim.y + blockIdx.y], 1) == a.splits - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const float* pbase = a.part + (static_cast<size_t>(b) * a.h_q + h0) * a.splits * stride;
+  for (int row = warp; row < rows; row += kAttnThreads / 32) {
+    const float* pr = pbase + static_cast<size_t>(row) * a.splits * stride;
+    const float m = lane < a.splits ? __ldcg(pr + lane * stride + D) : kNegInf;
+    const float l = lane < a.splits ? __ldcg(pr + lane * stride + D + 1) : 0.f;
+    float M = m;
+#pragma unroll
+    for (int x = 16; x > 0; x >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, x));
+    const float w = (m == kNegInf) ? 0.f : ex2_approx(m - M);
+    float den = w * l;
+#pragma unroll
+    for (int x = 16; x > 0; x >>= 1) den += __shfl_xor_sync(0xffffffffu, den, x);
+    s_w[row][lane] = den > 0.f ? w / den : 0.f;
+  }
+  __syncthreads();
+  for (int e = tid; e < rows * (D / 4); e += kAttnThreads) {
+    const int row = e / (D / 4), c4 = e % (D / 4);
+    const float* pr = pbase + static_cast<size_t>(row) * a.splits * stride + c4 * 4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+    for (int sp = 0; sp < a.splits; ++sp) {
+      const float ws = s_w[row][sp];
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(pr + sp * stride));
+      acc.x += ws * v.x;
+      acc.y += ws * v.y;
+      acc.z += ws * v.z;
+      acc.w += ws * v.w;
+    }
+    uint2 out;
+    out.x = pack_bf16x2(acc.x, acc.y);
+    out.y = pack_bf16x2(acc.z, acc.w);
+    *reinterpret_cast<uint2*>(a.o + (static_cast<size_t>(b) * a.h_q + h0 + row) * D + c4 * 4) = out;
+  }
 }
 
 // ---------------------------------------------------------------------------
-// 4. combine the split partials of each (sequence, head)
+// 3s. sparse decode attention, persistent and TMA-fed
 // ---------------------------------------------------------------------------
-template <int D>
-__global__ void __launch_bounds__(D) decode_combine_kernel(const DecArgs a) {
-  const int bh = blockIdx.x;   // b * h_q + h
-  const int col = threadIdx.x;
-  const size_t stride = D + 2;
-  const float* pp = a.part + static_cast<size_t>(bh) * a.splits * stride;
-  float M = kNegInf;
-  for (int s = 0; s < a.splits; ++s) M = fmaxf(M, pp[s * stride + D]);
-  float num = 0.f, den = 0.f;
-  if (M != kNegInf) {
-    for (int s = 0; s < a.splits; ++s) {
-      const float m = pp[s * stride + D];
-      if (m == kNegInf) continue;
-      const float w = ex2_approx(m - M);
-      num += w * pp[s * stride + col];
-      den += w * pp[s * stride + D + 1];
-    }
+// Work is a flat list of items g = u * topk + slot over units
+// u = (b, r, head tile); a grid of kStreamCtas CTAs gives CTA c the contiguous
+// range [c T / n, (c + 1) T / n), so every SM streams the same number of K/V
+// blocks whatever the batch and selection look like.  Per CTA: one producer
+// warp issues TMA loads (Q tile, K block, V block) into a ring of stages;
+// four consumer warps run the online softmax on mma.sync.  Warp w computes
+// S for keys [w BK/4, (w+1) BK/4) of the block, the four warps agree on the
+// row maxima through shared memory, write P (bf16) to shared memory, and warp
+// w then accumulates O for output columns [w D/4, (w+1) D/4) over the whole
+// block, so no cross-warp reduction of O is ever needed.  A unit that lies in
+// one CTA is normalised and written directly; a unit split between CTAs
+// leaves an (o, m, l) partial per CTA and the last of them to finish merges.
+constexpr int kStreamConsumers = 4;
+constexpr int kStreamThreads = 32 * (kStreamConsumers + 1);
+constexpr int kStreamCtas = 148;       // persistent grid: one CTA per SM
+constexpr int kStreamIdsCap = 1024;    // items per CTA held in shared memory
+
+template <int D, int BK>
+struct StreamCfg {
+  static constexpr int kHalves = D / 64;                  // 128-byte column halves
+  static constexpr int kQBytes = 16 * 128 * kHalves;      // 16 head rows x D
+  static constexpr int kKBytes = BK * 128 * kHalves;      // BK keys x D
+  static constexpr int kStageBytes = kQBytes + 2 * kKBytes;
+  static constexpr int kFit = (212 * 1024) / kStageBytes;
+  static constexpr int kStages = kFit > 8 ? 8 : kFit;
+  static constexpr int kPBytes = 16 * BK * 2;
+  static constexpr int kOffP = kStages * kStageBytes;
+  static constexpr int kOffRed = kOffP + kPBytes;                       // red_m[4][16], red_l[4][16]
+  static constexpr int kOffIds = kOffRed + 2 * kStreamConsumers * 16 * 4;
+  static constexpr int kOffMeta = kOffIds + kStreamIdsCap * 4;          // int4 per stage
+  static constexpr int kOffBar = kOffMeta + kStages * 16;               // full[], empty[]
+  static constexpr int kOffFlags = kOffBar + 2 * kStages * 8;
+  static constexpr int kSmemBytes = kOffFlags + 16;
+  static_assert(kStages >= 2, "stage ring");
+  static_assert(kSmemBytes + 1024 <= 227 * 1024, "shared memory");
+};
+
+struct StreamArgs {
+  const int32_t* block_ids;   // [B, h_kv, topk]
+  const int64_t* cu_kv;       // [B + 1]
+  uint16_t* o;                // [B, h_q, d]
+  float* part;                // [n_cta + U][16][d + 4]
+  int* unit_count;            // [U] CTAs finished per unit (zeroed per call)
+  int* status;
+  long long total_items;      // T = U * topk
+  int n_cta, h_q, h_kv, topk, head_tiles, group;
+  float scale_log2;
+};
+
+// Byte offset of 16-byte chunk ch of row x in a TMA 128B-swizzled tile of
+// `rows` rows stored as D/64 column halves of rows x 128 bytes.
+__device__ __forceinline__ uint32_t sw128(uint32_t base, int rows, int x, int ch) {
+  return base + (ch >> 3) * rows * 128 + x * 128 + (((ch & 7) ^ (x & 7)) << 4);
+}
+
+__device__ __forceinline__ int cta_of_item(long long g, long long T, int n) {
+  return static_cast<int>(((g + 1) * n - 1) / T);
+}
+
+template <int D, int BK>
+__global__ void __launch_bounds__(kStreamThreads, 1)
+    decode_attn_stream_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                              const __grid_constant__ CUtensorMap tm_v, const StreamArgs a) {
+  using C = StreamCfg<D, BK>;
+  constexpr int KPW = BK / kStreamConsumers;   // S keys per warp
+  constexpr int NT = KPW / 8;
+  constexpr int NCOL = D / kStreamConsumers;   // O columns per warp
+  constexpr int NTO = NCOL / 8;
+  constexpr int PST = D + 4;                   // partial row stride (floats)
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float* red_m = reinterpret_cast<float*>(smem + C::kOffRed);
+  float* red_l = red_m + kStreamConsumers * 16;
+  int* s_ids = reinterpret_cast<int*>(smem + C::kOffIds);
+  int4* meta = reinterpret_cast<int4*>(smem + C::kOffMeta);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* empty = full + C::kStages;
+  int* flags = reinterpret_cast<int*>(smem + C::kOffFlags);   // [0] abort, [1] last
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sP = sbase + C::kOffP;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const long long T = a.total_items;
+  const int cta = blockIdx.x;
+  const long long g0 = cta * T / a.n_cta, g1 = (cta + 1) * T / a.n_cta;
+  const int n_items = static_cast<int>(g1 - g0);
+  const int upb = a.h_kv * a.head_tiles;   // units per sequence
+
+  // Block ids of this CTA's items, -1 where the slot is padding or out of range.
+  for (int i = tid; i < n_items; i += kStreamThreads) {
+    const long long g = g0 + i;
+    const long long u = g / a.topk;
+    const int slot = static_cast<int>(g - u * a.topk);
+    const int b = static_cast<int>(u / upb), r = static_cast<int>(u % upb) / a.head_tiles;
+    const int L = static_cast<int>(a.cu_kv[b + 1] - a.cu_kv[b]);
+    const int nb = (L + BK - 1) / BK;
+    const int blk = a.block_ids[(static_cast<size_t>(b) * a.h_kv + r) * a.topk + slot];
+    s_ids[i] = (blk >= 0 && blk < nb) ? blk : -1;
   }
-  const float v = den > 0.f ? num / den : 0.f;
-  const uint32_t pk = pack_bf16x2(v, 0.f);
-  a.o[static_cast<size_t>(bh) * D + col] = static_cast<uint16_t>(pk & 0xffffu);
+  if (tid == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kStreamConsumers);
+    }
+    flags[0] = 0;
+    flags[1] = 0;
+    flags[2] = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  WaitCtx wc{reinterpret_cast<volatile int*>(&flags[0]), a.status};
+
+  if (warp == kStreamConsumers) {
+    // ---------------- producer ----------------
+    if (lane != 0) return;
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    long long cur_u = -1;
+    long long off = 0;
+    int L = 0, qrow = 0, r = 0;
+    int issued = 0;
+    for (int i = 0; i < n_items; ++i) {
+      const int blk = s_ids[i];
+      if (blk < 0) continue;
+      const long long u = (g0 + i) / a.topk;
+      if (u != cur_u) {
+        const int b = static_cast<int>(u / upb), rt = static_cast<int>(u % upb);
+        r = rt / a.head_tiles;
+        qrow = b * a.h_q + r * a.group + (rt % a.head_tiles) * 16;
+        off = a.cu_kv[b];
+        L = static_cast<int>(a.cu_kv[b + 1] - off);
+        cur_u = u;
+      }
+      const int stage = issued % C::kStages;
+      const uint32_t ph = (issued / C::kStages) & 1;
+      if (!mbar_wait(&empty[stage], ph ^ 1, wc)) break;
+      const int j0 = blk * BK;
+      // The last (partial) block is fetched as the BK keys ending at L, so no
+      // box reaches past this sequence; rows before j0 are masked.
+      const int kbase = j0 + BK <= L ? j0 : L - BK;
+      meta[stage] = make_int4(j0, kbase, min(j0 + BK, L), 0);
+      mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+      uint8_t* st = smem + stage * C::kStageBytes;
+      const int krow = static_cast<int>(off + kbase);
+#pragma unroll
+      for (int h = 0; h < C::kHalves; ++h) {
+        tma_load_2d(st + h * 16 * 128, &tm_q, &full[stage], h * 64, qrow);
+        tma_load_3d(st + C::kQBytes + h * BK * 128, &tm_k, &full[stage], h * 64, r, krow);
+        tma_load_3d(st + C::kQBytes + C::kKBytes + h * BK * 128, &tm_v, &full[stage], h * 64, r, krow);
+      }
+      ++issued;
+    }
+    // Loads still in flight (only possible after an abort) land before exit.
+    WaitCtx drain{reinterpret_cast<volatile int*>(&flags[2]), a.status};
+    for (int k = issued > C::kStages ? issued - C::kStages : 0; k < issued; ++k)
+      mbar_wait(&full[k % C::kStages], (k / C::kStages) & 1, drain);
+    return;
+  }
+
+  // ---------------- consumers (warps 0..3) ----------------
+  const int g = lane >> 2, t = lane & 3;
+  const int mi = lane >> 3, rr = lane & 7;
+  float oacc[NTO][4];
+  float m_lo = kNegInf, m_hi = kNegInf, l_lo = 0.f, l_hi = 0.f;
+#pragma unroll
+  for (int i = 0; i < NTO; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
+  int consumed = 0;
+
+  for (int i = 0; i < n_items; ++i) {
+    const long long gi = g0 + i;
+    const long long u = gi / a.topk;
+    if (s_ids[i] >= 0) {
+      const int stage = consumed % C::kStages;
+      const uint32_t ph = (consumed / C::kStages) & 1;
+      ++consumed;
+      mbar_wait(&full[stage], ph, wc);   // on timeout the flag is set and the data is ignored
+      const int4 md = meta[stage];
+      const int j0 = md.x, kbase = md.y, jend = md.z;
+      const uint32_t sQ = sbase + stage * C::kStageBytes;
+      const uint32_t sK = sQ + C::kQBytes;
+      const uint32_t sV = sK + C::kKBytes;
+
+      uint32_t qf[D / 16][4];
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks)
+        ldsm_x4(sw128(sQ, 16, (mi & 1) * 8 + rr, 2 * ks + (mi >> 1)), qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3]);
+      float sacc[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ks += 2) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(sw128(sK, BK, warp * KPW + nt * 8 + rr, 2 * ks + mi), b0, b1, b2, b3);
+          mma_bf16_16816(sacc[nt], qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], b0, b1);
+          mma_bf16_16816(sacc[nt], qf[ks + 1][0], qf[ks + 1][1], qf[ks + 1][2], qf[ks + 1][3], b2, b3);
+        }
+      }
+      float mx_lo = kNegInf, mx_hi = kNegInf;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int key = kbase + warp * KPW + nt * 8 + 2 * t + e;
+          const bool ok = key >= j0 && key < jend;
+          sacc[nt][e] = ok ? sacc[nt][e] * a.scale_log2 : kNegInf;
+          sacc[nt][2 + e] = ok ? sacc[nt][2 + e] * a.scale_log2 : kNegInf;
+          mx_lo = fmaxf(mx_lo, sacc[nt][e]);
+          mx_hi = fmaxf(mx_hi, sacc[nt][2 + e]);
+        }
+      }
+#pragma unroll
+      for (int x = 1; x < 4; x <<= 1) {
+        mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, x));
+        mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, x));
+      }
+      if (t == 0) {
+        red_m[warp * 16 + g] = mx_lo;
+        red_m[warp * 16 + g + 8] = mx_hi;
+      }
+      named_bar(1, 32 * kStreamConsumers);
+#pragma unroll
+      for (int w = 0; w < kStreamConsumers; ++w) {
+        mx_lo = fmaxf(mx_lo, red_m[w * 16 + g]);
+        mx_hi = fmaxf(mx_hi, red_m[w * 16 + g + 8]);
+      }
+      const float mn_lo = fmaxf(m_lo, mx_lo), mn_hi = fmaxf(m_hi, mx_hi);
+      const float al_lo = mn_lo == kNegInf ? 1.f : ex2_approx(m_lo - mn_lo);
+      const float al_hi = mn_hi == kNegInf ? 1.f : ex2_approx(m_hi - mn_hi);
+      const float bi_lo = mn_lo == kNegInf ? 0.f : mn_lo, bi_hi = mn_hi == kNegInf ? 0.f : mn_hi;
+      m_lo = mn_lo;
+      m_hi = mn_hi;
+      float ps_lo = 0.f, ps_hi = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const float p0 = ex2_approx(sacc[nt][0] - bi_lo), p1 = ex2_approx(sacc[nt][1] - bi_lo);
+        const float p2 = ex2_approx(sacc[nt][2] - bi_hi), p3 = ex2_approx(sacc[nt][3] - bi_hi);
+        ps_lo += p0 + p1;
+        ps_hi += p2 + p3;
+        const int ch = warp * NT + nt;
+        asm volatile("st.shared.b32 [%0], %1;" ::"r"(sP + g * (BK * 2) + ((ch ^ (g & 7)) << 4) + 4 * t),
+                     "r"(pack_bf16x2(p0, p1)));
+        asm volatile("st.shared.b32 [%0], %1;" ::"r"(sP + (g + 8) * (BK * 2) + ((ch ^ (g & 7)) << 4) + 4 * t),
+                     "r"(pack_bf16x2(p2, p3)));
+      }
+#pragma unroll
+      for (int x = 1; x < 4; x <<= 1) {
+        ps_lo += __shfl_xor_sync(0xffffffffu, ps_lo, x);
+        ps_hi += __shfl_xor_sync(0xffffffffu, ps_hi, x);
+      }
+      if (t == 0) {
+        red_l[warp * 16 + g] = ps_lo;
+        red_l[warp * 16 + g + 8] = ps_hi;
+      }
+      // Rows of a partial block before j0 hold other keys: zero this warp's
+      // V columns there so that 0 * V stays 0 whatever those rows contain.
+      const bool zap = kbase < j0;
+      if (zap) {
+        const int nz = j0 - kbase;
+        for (int e = lane; e < nz * NTO; e += 32) {
+          const int x = e / NTO, ch = warp * NTO + e % NTO;
+          asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(sw128(sV, BK, x, ch)), "r"(0u)
+                       : "memory");
+        }
+      }
+      named_bar(1, 32 * kStreamConsumers);
+      float ls_lo = 0.f, ls_hi = 0.f;
+#pragma unroll
+      for (int w = 0; w < kStreamConsumers; ++w) {
+        ls_lo += red_l[w * 16 + g];
+        ls_hi += red_l[w * 16 + g + 8];
+      }
+      l_lo = l_lo * al_lo + ls_lo;
+      l_hi = l_hi * al_hi + ls_hi;
+#pragma unroll
+      for (int i2 = 0; i2 < NTO; ++i2) {
+        oacc[i2][0] *= al_lo;
+        oacc[i2][1] *= al_lo;
+        oacc[i2][2] *= al_hi;
+        oacc[i2][3] *= al_hi;
+      }
+#pragma unroll
+      for (int kk = 0; kk < BK / 16; ++kk) {
+        uint32_t a0, a1, a2, a3;
+        const int prow = (mi & 1) * 8 + rr, pch = 2 * kk + (mi >> 1);
+        ldsm_x4(sP + prow * (BK * 2) + ((pch ^ (prow & 7)) << 4), a0, a1, a2, a3);
+#pragma unroll
+        for (int dt = 0; dt < NTO; dt += 2) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(sw128(sV, BK, kk * 16 + (mi & 1) * 8 + rr, warp * NTO + dt + (mi >> 1)), b0, b1, b2, b3);
+          mma_bf16_16816(oacc[dt], a0, a1, a2, a3, b0, b1);
+          mma_bf16_16816(oacc[dt + 1], a0, a1, a2, a3, b2, b3);
+        }
+      }
+      if (zap) fence_proxy_async_smem();   // generic writes before the stage's next TMA fill
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[stage]);
+    }
+
+    // End of this CTA's share of unit u: write it out.
+    if ((gi + 1) % a.topk != 0 && i + 1 != n_items) continue;
+    const int b = static_cast<int>(u / upb), rt = static_cast<int>(u % upb);
+    const int r = rt / a.head_tiles, ht = rt % a.head_tiles;
+    const int rows = min(16, a.group - ht * 16);
+    const int h0 = r * a.group + ht * 16;
+    const int c_lo = cta_of_item(u * a.topk, T, a.n_cta);
+    const int c_hi = cta_of_item(u * a.topk + a.topk - 1, T, a.n_cta);
+    uint16_t* orow = a.o + (static_cast<size_t>(b) * a.h_q + h0) * D;
+    if (c_lo == c_hi) {
+      const float in_lo = l_lo > 0.f ? 1.f / l_lo : 0.f, in_hi = l_hi > 0.f ? 1.f / l_hi : 0.f;
+#pragma unroll
+      for (int dt = 0; dt < NTO; ++dt) {
+        const int col = warp * NCOL + dt * 8 + 2 * t;
+        if (g < rows)
+          *reinterpret_cast<uint32_t*>(orow + g * D + col) = pack_bf16x2(oacc[dt][0] * in_lo, oacc[dt][1] * in_lo);
+        if (g + 8 < rows)
+          *reinterpret_cast<uint32_t*>(orow + (g + 8) * D + col) =
+              pack_bf16x2(oacc[dt][2] * in_hi, oacc[dt][3] * in_hi);
+      }
+    } else {
+      float* pp = a.part + (static_cast<size_t>(cta) + u) * 16 * PST;
+#pragma unroll
+      for (int dt = 0; dt < NTO; ++dt) {
+        const int col = warp * NCOL + dt * 8 + 2 * t;
+        *reinterpret_cast<float2*>(pp + g * PST + col) = make_float2(oacc[dt][0], oacc[dt][1]);
+        *reinterpret_cast<float2*>(pp + (g + 8) * PST + col) = make_float2(oacc[dt][2], oacc[dt][3]);
+      }
+      if (warp == 0 && t == 0) {
+        *reinterpret_cast<float2*>(pp + g * PST + D) = make_float2(m_lo, l_lo);
+        *reinterpret_cast<float2*>(pp + (g + 8) * PST + D) = make_float2(m_hi, l_hi);
+      }
+      __threadfence();
+      named_bar(1, 32 * kStreamConsumers);
+      if (tid == 0) {
+        flags[1] = atomicAdd(&a.unit_count[u], 1) == c_hi - c_lo;
+        __threadfence();
+      }
+      named_bar(1, 32 * kStreamConsumers);
+      if (flags[1]) {
+        // Last CTA of the unit: LSE-weighted merge of the c_hi - c_lo + 1 partials.
+        float M_lo = kNegInf, M_hi = kNegInf;
+        for (int c = c_lo; c <= c_hi; ++c) {
+          const float* q = a.part + (static_cast<size_t>(c) + u) * 16 * PST;
+          M_lo = fmaxf(M_lo, __ldcg(q + g * PST + D));
+          M_hi = fmaxf(M_hi, __ldcg(q + (g + 8) * PST + D));
+        }
+        float acc[NTO][4];
+#pragma unroll
+        for (int dt = 0; dt < NTO; ++dt) acc[dt][0] = acc[dt][1] = acc[dt][2] = acc[dt][3] = 0.f;
+        float den_lo = 0.f, den_hi = 0.f;
+        for (int c = c_lo; c <= c_hi; ++c) {
+          const float* q = a.part + (static_cast<size_t>(c) + u) * 16 * PST;
+          const float2 ml_lo = __ldcg(reinterpret_cast<const float2*>(q + g * PST + D));
+          const float2 ml_hi = __ldcg(reinterpret_cast<const float2*>(q + (g + 8) * PST + D));
+          const float w_lo = ml_lo.x == kNegInf ? 0.f : ex2_approx(ml_lo.x - M_lo);
+          const float w_hi = ml_hi.x == kNegInf ? 0.f : ex2_approx(ml_hi.x - M_hi);
+          den_lo += w_lo * ml_lo.y;
+          den_hi += w_hi * ml_hi.y;
+#pragma unroll
+          for (int dt = 0; dt < NTO; ++dt) {
+            const int col = warp * NCOL + dt * 8 + 2 * t;
+            const float2 v0 = __ldcg(reinterpret_cast<const float2*>(q + g * PST + col));
+            const float2 v1 = __ldcg(reinterpret_cast<const float2*>(q + (g + 8) * PST + col));
+            acc[dt][0] += w_lo * v0.x;
+            acc[dt][1] += w_lo * v0.y;
+            acc[dt][2] += w_hi * v1.x;
+            acc[dt][3] += w_hi * v1.y;
+          }
+        }
+        const float in_lo = den_lo > 0.f ? 1.f / den_lo : 0.f, in_hi = den_hi > 0.f ? 1.f / den_hi : 0.f;
+#pragma unroll
+        for (int dt = 0; dt < NTO; ++dt) {
+          const int col = warp * NCOL + dt * 8 + 2 * t;
+          if (g < rows)
+            *reinterpret_cast<uint32_t*>(orow + g * D + col) = pack_bf16x2(acc[dt][0] * in_lo, acc[dt][1] * in_lo);
+          if (g + 8 < rows)
+            *reinterpret_cast<uint32_t*>(orow + (g + 8) * D + col) =
+                pack_bf16x2(acc[dt][2] * in_hi, acc[dt][3] * in_hi);
+        }
+      }
+    }
+    m_lo = m_hi = kNegInf;
+    l_lo = l_hi = 0.f;
+#pragma unroll
+    for (int i2 = 0; i2 < NTO; ++i2) oacc[i2][0] = oacc[i2][1] = oacc[i2][2] = oacc[i2][3] = 0.f;
+  }
 }
 
 // Split plan shared by the workspace query and the launch.
@@ -521,38 +1030,102 @@ int launch_attn_combine(const DecArgs& a, cudaStream_t st) {
     return MSA_ERR_CUDA;
   dim3 grid(a.splits, a.h_kv * a.head_tiles, a.batch);
   kern<<<grid, kAttnThreads, smem, st>>>(a);
-  if (cudaGetLastError() != cudaSuccess) return MSA_ERR_CUDA;
-  decode_combine_kernel<D><<<a.batch * a.h_q, D, 0, st>>>(a);
+  return cudaGetLastError() == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
+}
+
+long long stream_items(const msa_params& p, int batch) {
+  return static_cast<long long>(batch) * p.h_kv * ((p.h_q / p.h_kv + 15) / 16) * p.topk;
+}
+
+int stream_ctas(long long T) {
+  long long n = (T + kStreamIdsCap - 1) / kStreamIdsCap;
+  if (n < kStreamCtas) n = kStreamCtas;
+  return static_cast<int>(n < T ? n : T);
+}
+
+template <int D, int BK>
+int launch_attn_stream(const DecArgs& a, int max_kv, int* status, cudaStream_t st) {
+  using C = StreamCfg<D, BK>;
+  CUtensorMap tq, tk, tv;
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(D), static_cast<uint64_t>(a.batch) * a.h_q};
+    const uint64_t strides[1] = {static_cast<uint64_t>(D) * 2};
+    const uint32_t box[2] = {64, 16};
+    if (!encode_tma_bf16(&tq, 2, a.q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MSA_ERR_CUDA;
+  }
+  {
+    // Rows of the packed caches: the sum of L_b is at most batch * max_kv.
+    const uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(a.h_kv),
+                              static_cast<uint64_t>(a.batch) * max_kv};
+    const uint64_t strides[2] = {static_cast<uint64_t>(D) * 2, static_cast<uint64_t>(a.h_kv) * D * 2};
+    const uint32_t box[3] = {64, 1, BK};
+    if (!encode_tma_bf16(&tk, 3, a.k_cache, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MSA_ERR_CUDA;
+    if (!encode_tma_bf16(&tv, 3, a.v_cache, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MSA_ERR_CUDA;
+  }
+  StreamArgs s;
+  s.block_ids = a.block_ids;
+  s.cu_kv = a.cu_kv;
+  s.o = a.o;
+  s.part = a.part;
+  s.unit_count = a.grp_count;
+  s.status = status;
+  s.total_items = static_cast<long long>(a.batch) * a.h_kv * a.head_tiles * a.topk;
+  s.n_cta = stream_ctas(s.total_items);
+  s.h_q = a.h_q;
+  s.h_kv = a.h_kv;
+  s.topk = a.topk;
+  s.head_tiles = a.head_tiles;
+  s.group = a.h_q / a.h_kv;
+  s.scale_log2 = a.scale_log2;
+  const int smem = C::kSmemBytes + 1024;
+  auto kern = decode_attn_stream_kernel<D, BK>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return MSA_ERR_CUDA;
+  kern<<<s.n_cta, kStreamThreads, smem, st>>>(tq, tk, tv, s);
   return cudaGetLastError() == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
 }
 
 template <int DIDX, int BK>
 int launch_index(const DecArgs& a, cudaStream_t st) {
-  if (a.kfree > 0) {   // topk == 1 with the forced local block needs no scan
+  if (a.kfree > 0) {
     dim3 grid(a.max_chunks, a.batch);
     decode_index_kernel<DIDX, BK><<<grid, kIdxThreads, 0, st>>>(a);
-    if (cudaGetLastError() != cudaSuccess) return MSA_ERR_CUDA;
+  } else {   // topk == 1 with the forced local block needs no scan
+    decode_local_only_kernel<BK><<<a.batch * a.h_kv, 32, 0, st>>>(a);
   }
-  decode_topk_merge_kernel<BK><<<a.batch * a.h_kv, 32, 0, st>>>(a);
   return cudaGetLastError() == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
 }
 
 }  // namespace
+
+// Completion counters at the front of the decode workspace: [B] index CTAs
+// per sequence, then [B, h_kv, head_tiles] attention CTAs.  The caller zeroes
+// them (with the status word) before every call.
+size_t decode_counter_bytes(const msa_params& p, int batch) {
+  const size_t n = static_cast<size_t>(batch) * (1 + p.h_kv * ((p.h_q / p.h_kv + 15) / 16));
+  return align_up(n * 4, 256);
+}
 
 size_t decode_workspace_bytes(const msa_params& p, int batch, int max_kv) {
   const int kfree = p.topk;   // upper bound on topk - force_local
   const size_t cand = static_cast<size_t>(batch) * max_chunks_for(p, max_kv) * p.h_kv * kfree;
   const SplitPlan sd = plan_splits(p, max_kv, 1), ss = plan_splits(p, max_kv, 0);
   const int splits = sd.splits > ss.splits ? sd.splits : ss.splits;
-  const size_t part = static_cast<size_t>(batch) * p.h_q * splits * (p.d + 2);
-  return align_up(cand * 4, 256) * 2 + align_up(part * 4, 256);
+  const size_t part_dense = static_cast<size_t>(batch) * p.h_q * splits * (p.d + 4);
+  const long long T = stream_items(p, batch);
+  const long long units = T / p.topk;
+  const size_t part_stream = static_cast<size_t>(stream_ctas(T) + units) * 16 * (p.d + 4);
+  const size_t part = part_dense > part_stream ? part_dense : part_stream;
+  return decode_counter_bytes(p, batch) + align_up(cand * 4, 256) * 2 + align_up(part * 4, 256);
 }
 
 int run_sparse_attn_decode(const msa_params& p, const void* q, const void* q_idx, const void* k_cache,
                            const void* v_cache, const void* k_idx_cache, const int64_t* cu_kv, int batch,
                            int max_kv, int dense, int32_t* block_ids, void* o, void* ws, size_t /*ws_bytes*/,
-                           int* /*status*/, cudaStream_t stream) {
+                           int* status, cudaStream_t stream) {
   if (p.h_kv > 8) return MSA_ERR_UNSUPPORTED;
+  // TMA row coordinates of the caches are 32-bit.
+  if (!dense && static_cast<long long>(batch) * max_kv > 0x7fffffffLL) return MSA_ERR_UNSUPPORTED;
   DecArgs a;
   a.q = static_cast<const uint16_t*>(q);
   a.q_idx = static_cast<const uint16_t*>(q_idx);
@@ -580,6 +1153,9 @@ int run_sparse_attn_decode(const msa_params& p, const void* q, const void* q_idx
   a.scale_log2 = scale * kLog2e;
   const size_t cand = static_cast<size_t>(batch) * a.max_chunks * p.h_kv * p.topk;
   uint8_t* w = static_cast<uint8_t*>(ws);
+  a.seq_count = reinterpret_cast<int*>(w);
+  a.grp_count = a.seq_count + batch;
+  w += decode_counter_bytes(p, batch);
   a.cand_s = reinterpret_cast<float*>(w);
   a.cand_b = reinterpret_cast<int*>(w + align_up(cand * 4, 256));
   a.part = reinterpret_cast<float*>(w + 2 * align_up(cand * 4, 256));
@@ -595,6 +1171,13 @@ int run_sparse_attn_decode(const msa_params& p, const void* q, const void* q_idx
     }
   }
   if (rc) return rc;
+  if (!dense) {
+    if (p.d == 64)
+      return p.block_k == 64 ? launch_attn_stream<64, 64>(a, max_kv, status, stream)
+                             : launch_attn_stream<64, 128>(a, max_kv, status, stream);
+    return p.block_k == 64 ? launch_attn_stream<128, 64>(a, max_kv, status, stream)
+                           : launch_attn_stream<128, 128>(a, max_kv, status, stream);
+  }
   if (p.d == 64) {
     return p.block_k == 64 ? launch_attn_combine<64, 64>(a, stream) : launch_attn_combine<64, 128>(a, stream);
   }

@@ -156,7 +156,8 @@ int msa_sparse_attn_decode(const msa_params* p, const void* q, const void* q_idx
   if ((reinterpret_cast<uintptr_t>(cu_kv) & 7u) != 0) return MSA_ERR_MISALIGNED;
   if (!dense && (!aligned16(q_idx) || !aligned16(k_idx_cache) || !aligned16(block_ids))) return MSA_ERR_MISALIGNED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if ((rc = clear_status(ws, st))) return rc;
+  // One memset clears the status word and the decode completion counters.
+  if (cudaMemsetAsync(ws, 0, kWsHeader + decode_counter_bytes(*p, batch), st) != cudaSuccess) return MSA_ERR_CUDA;
   return run_sparse_attn_decode(*p, q, q_idx, k_cache, v_cache, k_idx_cache, cu_kv, batch, max_kv, dense,
                                 block_ids, o, static_cast<uint8_t*>(ws) + kWsHeader, ws_bytes - kWsHeader,
                                 static_cast<int*>(ws), st);

@@ -38,6 +38,7 @@ int run_sparse_attn_kvouter(const msa_params& p, const void* q, const CUtensorMa
                             size_t ws_bytes, int* status, cudaStream_t stream);
 
 // Decode step.
+size_t decode_counter_bytes(const msa_params& p, int batch);
 size_t decode_workspace_bytes(const msa_params& p, int batch, int max_kv);
 int run_sparse_attn_decode(const msa_params& p, const void* q, const void* q_idx, const void* k_cache,
                            const void* v_cache, const void* k_idx_cache, const int64_t* cu_kv, int batch,

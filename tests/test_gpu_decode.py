@@ -54,6 +54,8 @@ def test_small_decode_dense():
     dict(batch=7, kv_min=64, kv_max=64),           # one full block per sequence
     dict(batch=3, kv_min=1, kv_max=3),             # tiny caches
     dict(topk=1, batch=3),                         # the local block alone
+    dict(h_q=4, h_kv=4, d=128, d_idx=32, block_k=128, topk=3, batch=9, kv_min=100, kv_max=3000),  # group of 1
+    dict(h_q=128, h_kv=1, d=128, d_idx=64, block_k=64, topk=8, batch=2, kv_min=2000, kv_max=4000),  # 8 head tiles
 ])
 def test_shapes(kw):
     run_case(small(seed=kw.get("batch", 1) * 31 + kw.get("kv_max", 0), **kw))
@@ -73,3 +75,10 @@ def test_decode_b64_64k_128k_dense_sampled():
 
 def test_decode_b8_1m():
     run_case(WORKLOADS["decode_b8_1m"])
+
+
+def test_many_items_per_cta():
+    # 2048 x 8 x 16 = 262144 (sequence, group, slot) items: more than 1024 per
+    # CTA at 148 CTAs, so the persistent attention grid grows; sampled rows.
+    w = small(h_q=32, h_kv=8, d=64, d_idx=32, block_k=64, topk=16, batch=2048, kv_min=100, kv_max=1500, seed=77)
+    run_case(w, seqs=[0, 1, 777, 2047])
