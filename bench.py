@@ -349,7 +349,11 @@ def run_ours(args, rank, world, torch, dist):
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "note": "prefill inputs and outputs cross PCIe every step; decode KV caches stay resident"},
         # ours per step: index 1; sparse prefill 5 (count, scan, fill, KV-outer, merge); decode 4
-        "gpu_launches": 10 * args.steps,
+        # Per step: index top-k (1); sparse prefill: schedule count, scan and
+        # fill (3), block-major attention (1), partial merge (1); decode:
+        # persistent index scan with the merge folded in (1), persistent
+        # attention with the combine folded in (1).
+        "gpu_launches": 8 * args.steps,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.case == "full":

@@ -122,7 +122,11 @@ MSA_API int msa_sparse_attn_prefill(const msa_params* p, const void* q, const vo
 /*
  * One batched decode step: for every sequence b the query at position
  * L_b - 1 runs the index branch over its whole index-key cache, then the main
- * branch over the selected blocks (split over KV blocks, then combined).
+ * branch over the selected blocks.  Both sparse kernels are persistent: the
+ * index scan splits the blocks of all sequences into equal ranges per CTA,
+ * the attention splits the (sequence, group, slot) list the same way, and
+ * partial results of a sequence or group split between CTAs are merged by the
+ * last CTA to finish it.
  *   q            bf16 [batch, h_q, d]
  *   q_idx        bf16 [batch, h_kv, d_idx]
  *   k_cache,
@@ -134,7 +138,8 @@ MSA_API int msa_sparse_attn_prefill(const msa_params* p, const void* q, const vo
  *                and block_ids is not written)
  *   block_ids    int32 [batch, h_kv, topk] output (may be NULL when dense)
  *   o            bf16 [batch, h_q, d] output
- * Every L_b must be in [1, max_kv].
+ * Every L_b must be in [1, max_kv].  With dense = 0, batch <= 4096 and
+ * batch * max_kv < 2^31 (MSA_ERR_UNSUPPORTED otherwise).
  */
 MSA_API int msa_sparse_attn_decode(const msa_params* p, const void* q, const void* q_idx, const void* k_cache,
                            const void* v_cache, const void* k_idx_cache, const int64_t* cu_kv, int batch,

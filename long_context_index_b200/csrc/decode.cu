@@ -35,7 +35,10 @@ namespace msa {
 namespace {
 
 constexpr int kIdxThreads = 256;    // 8 warps
-constexpr int kIdxChunkBlocks = 64; // CB: blocks per index CTA
+constexpr int kIdxCtasPerSm = 3;
+constexpr int kIdxCtas = 148 * kIdxCtasPerSm;   // persistent index grid
+constexpr int kIdxWCap = 1024;      // blocks per index CTA held in shared memory
+constexpr int kIdxMaxBatch = 4096;  // sequences whose block prefix fits shared memory
 constexpr int kAttnThreads = 128;   // 4 warps, 32 keys each
 constexpr int kMergeRegCand = 8;    // per-lane register cache of the merge
 constexpr float kLog2e = 1.4426950408889634f;
@@ -94,49 +97,116 @@ struct DecArgs {
   const int64_t* cu_kv;     // [B + 1]
   int32_t* block_ids;       // [B, h_kv, topk]
   uint16_t* o;              // [B, h_q, d]
-  float* cand_s;            // [B, max_chunks, h_kv, kfree]
+  float* cand_s;            // [idx_ctas + B, h_kv, kfree]
   int* cand_b;
   float* part;              // [B, h_q, splits, d + 4]  (o[d], m, l, 2 pad)
   int* seq_count;           // [B] index CTAs finished per sequence (zeroed per call)
   int* grp_count;           // [B, h_kv, head_tiles] attention CTAs finished (zeroed per call)
-  int batch, h_q, h_kv, topk, causal, force_local, kfree, max_chunks;
+  int batch, h_q, h_kv, topk, causal, force_local, kfree, idx_ctas, idx_wmax;
   int splits, slots_per_split, dense, head_tiles;
   float scale_log2;
 };
 
 // ---------------------------------------------------------------------------
-// 1. index scan: block max-pool + per-chunk top-(k-1) per group
+// 1. index scan, persistent.  The blocks of all sequences, laid end to end
+//    (sequence b owns global blocks [P_b, P_b+1) with P the prefix of
+//    ceil(L_b / BK)), are split into idx_ctas equal contiguous ranges, one per
+//    CTA, so every CTA streams the same number of index-key bytes whatever the
+//    length mix.  A CTA scores its blocks (max-pool per block and group), then
+//    keeps, per (sequence, group) it touched, the top (k - 1) non-local blocks
+//    of its share as candidates in slot (CTA + sequence), a slot no other
+//    (CTA, sequence) pair can take because both orders agree.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ int idx_cta_of(long long gblk, long long T, int n) {
+  return static_cast<int>(((gblk + 1) * n - 1) / T);
+}
+
 template <int BK>
-__device__ void merge_topk_warp(const DecArgs& a, int b, int r, int lane, int* chosen);
+__device__ void merge_topk_warp(const DecArgs& a, int b, int r, int lane, int* chosen, int c_lo, int nseg,
+                                long long T, int n);
 
 template <int DIDX, int BK>
-__global__ void __launch_bounds__(kIdxThreads) decode_index_kernel(const DecArgs a) {
+__global__ void __launch_bounds__(kIdxThreads, kIdxCtasPerSm) decode_index_kernel(const DecArgs a) {
   constexpr int kHalves = DIDX / 32;   // 16-byte vectors per token row per thread
-  __shared__ float smax[8][kIdxChunkBlocks];
-  const int b = blockIdx.y;
-  const int chunk = blockIdx.x;
-  const int64_t off = a.cu_kv[b];
-  const int L = static_cast<int>(a.cu_kv[b + 1] - off);
-  const int nb = (L + BK - 1) / BK;
-  const int blk0 = chunk * kIdxChunkBlocks;
-  if (blk0 >= nb) return;
-  const int nblk = min(kIdxChunkBlocks, nb - blk0);
+  constexpr int kWarps = kIdxThreads / 32;
+  extern __shared__ __align__(16) uint8_t ismem[];
+  const int B = a.batch;
+  const int wmax = a.idx_wmax;
+  int* pfx = reinterpret_cast<int*>(ismem);                                       // [B + 1]
+  float* smax = reinterpret_cast<float*>(ismem + ((B + 1) * 4 + 15) / 16 * 16);   // [h_kv][wmax]
+  int* lastq = reinterpret_cast<int*>(smax + a.h_kv * wmax);                      // [wmax + 1]
+  __shared__ int warp_tot[kWarps];
+  __shared__ int chosen[kWarps][33];
+  __shared__ int n_last;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
+  const int n = a.idx_ctas, cta = blockIdx.x;
 
-  // Q_idx fragment (B operand): column n = group g, permuted d_idx order.
-  uint4 qv[kHalves];
+  // Block prefix over the sequences (each CTA builds its own copy).
+  int running = 0;
+  for (int base = 0; base < B; base += kIdxThreads) {
+    const int bb = base + threadIdx.x;
+    const int nb = bb < B ? static_cast<int>((a.cu_kv[bb + 1] - a.cu_kv[bb] + BK - 1) / BK) : 0;
+    int v = nb;
 #pragma unroll
-  for (int h = 0; h < kHalves; ++h) {
-    qv[h] = make_uint4(0, 0, 0, 0);
-    if (g < a.h_kv)
-      qv[h] = *reinterpret_cast<const uint4*>(a.q_idx + (static_cast<size_t>(b) * a.h_kv + g) * DIDX + 8 * t + 32 * h);
+    for (int x = 1; x < 32; x <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, v, x);
+      if (lane >= x) v += y;
+    }
+    if (lane == 31) warp_tot[warp] = v;
+    __syncthreads();
+    int before = 0, tot = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      before += w < warp ? warp_tot[w] : 0;
+      tot += warp_tot[w];
+    }
+    if (bb < B) pfx[bb] = running + before + v - nb;
+    running += tot;
+    __syncthreads();
   }
-  const uint16_t* kbase = a.k_idx + static_cast<size_t>(off) * DIDX;
+  if (threadIdx.x == 0) {
+    pfx[B] = running;
+    n_last = 0;
+  }
+  __syncthreads();
+  const long long T = pfx[B];
+  const int G0 = static_cast<int>(cta * T / n);
+  const int W = min(static_cast<int>((cta + 1) * T / n) - G0, wmax);   // clamp: only a understated max_kv exceeds it
+  if (W <= 0) return;
+  const int G1 = G0 + W;
+  auto seq_of = [&](int gb) {   // largest b with pfx[b] <= gb
+    int lo = 0, hi = B - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (pfx[mid] <= gb) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+  };
 
-  for (int lb = warp; lb < nblk; lb += kIdxThreads / 32) {
-    const int j0 = (blk0 + lb) * BK;
+  // Score: warp w takes blocks w, w + 8, ... of the range.
+  int cur = -1, cur_end = 0, cur_p = 0, L = 0;
+  const uint16_t* kbase = a.k_idx;
+  uint4 qv[kHalves];
+  for (int i = warp; i < W; i += kWarps) {
+    const int gb = G0 + i;
+    if (cur < 0 || gb >= cur_end) {
+      cur = seq_of(gb);
+      cur_p = pfx[cur];
+      cur_end = pfx[cur + 1];
+      const int64_t off = a.cu_kv[cur];
+      L = static_cast<int>(a.cu_kv[cur + 1] - off);
+      kbase = a.k_idx + static_cast<size_t>(off) * DIDX;
+      // Q_idx fragment (B operand): column n = group g, permuted d_idx order.
+#pragma unroll
+      for (int h = 0; h < kHalves; ++h) {
+        qv[h] = make_uint4(0, 0, 0, 0);
+        if (g < a.h_kv)
+          qv[h] = *reinterpret_cast<const uint4*>(a.q_idx + (static_cast<size_t>(cur) * a.h_kv + g) * DIDX + 8 * t +
+                                                   32 * h);
+      }
+    }
+    const int j0 = (gb - cur_p) * BK;
     float m0 = kNegInf, m1 = kNegInf;   // groups 2t, 2t+1
 #pragma unroll 2
     for (int mt = 0; mt < BK / 16; ++mt) {
@@ -168,78 +238,102 @@ __global__ void __launch_bounds__(kIdxThreads) decode_index_kernel(const DecArgs
       m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, x));
     }
     if (g == 0) {
-      smax[2 * t][lb] = m0;
-      smax[2 * t + 1][lb] = m1;
+      if (2 * t < a.h_kv) smax[(2 * t) * wmax + i] = m0;
+      if (2 * t + 1 < a.h_kv) smax[(2 * t + 1) * wmax + i] = m1;
     }
   }
   __syncthreads();
 
-  __shared__ int chosen[8][33];
-  __shared__ int s_last;
-  // Per group: top-kfree eligible non-local blocks of this chunk.
-  const int p = L - 1;
-  const int b_loc = p / BK;
-  for (int r = warp; r < a.h_kv; r += kIdxThreads / 32) {
-    float s0 = kNegInf, s1 = kNegInf;
-    int i0 = -1, i1 = -1;
-    {
-      const int lb0 = lane, lb1 = lane + 32;
-      // Decode: every cached key is visible (j <= p), so every block is eligible.
-      if (lb0 < nblk && !(a.force_local && blk0 + lb0 == b_loc)) { s0 = smax[r][lb0]; i0 = blk0 + lb0; }
-      if (lb1 < nblk && !(a.force_local && blk0 + lb1 == b_loc)) { s1 = smax[r][lb1]; i1 = blk0 + lb1; }
-      if (i1 >= 0 && (i0 < 0 || better(s1, i1, s0, i0))) {
-        float ts = s0; s0 = s1; s1 = ts;
-        int ti = i0; i0 = i1; i1 = ti;
+  // Per (sequence, group) share: top-kfree non-local blocks by repeated warp
+  // argmax with a strictly decreasing (score desc, block asc) bound.  Decode
+  // sees every cached key (j <= p), so every block is eligible.
+  const int b_first = seq_of(G0), b_last = seq_of(G1 - 1);
+  const int nsegs = b_last - b_first + 1;
+  for (int pi = warp; pi < nsegs * a.h_kv; pi += kWarps) {
+    const int sb = b_first + pi / a.h_kv, r = pi % a.h_kv;
+    const int p0 = pfx[sb];
+    const int i_lo = max(p0, G0) - G0, i_hi = min(pfx[sb + 1], G1) - G0;
+    const int i_loc = a.force_local ? pfx[sb + 1] - 1 - G0 : -1;   // the local block is the last one
+    const size_t base = ((static_cast<size_t>(cta) + sb) * a.h_kv + r) * a.kfree;
+    float last_s = __builtin_huge_valf();
+    int last_b = -1;
+    int k = 0;
+    for (; k < a.kfree; ++k) {
+      float bs = kNegInf;
+      int bi = 0x7fffffff;
+      for (int i = i_lo + lane; i < i_hi; i += 32) {
+        if (i == i_loc) continue;
+        const float sc = smax[r * wmax + i];
+        const int blk = G0 + i - p0;
+        if (k > 0 && !better(last_s, last_b, sc, blk)) continue;
+        if (bi == 0x7fffffff || better(sc, blk, bs, bi)) { bs = sc; bi = blk; }
       }
-    }
-    const size_t base = ((static_cast<size_t>(b) * a.max_chunks + chunk) * a.h_kv + r) * a.kfree;
-    for (int k = 0; k < a.kfree; ++k) {
-      float bs = i0 >= 0 ? s0 : kNegInf;
-      int bi = i0 >= 0 ? i0 : 0x7fffffff;
 #pragma unroll
       for (int x = 16; x > 0; x >>= 1) {
         const float os = __shfl_xor_sync(0xffffffffu, bs, x);
         const int oi = __shfl_xor_sync(0xffffffffu, bi, x);
         if (oi != 0x7fffffff && (bi == 0x7fffffff || better(os, oi, bs, bi))) { bs = os; bi = oi; }
       }
+      if (bi == 0x7fffffff) break;
       if (lane == 0) {
-        a.cand_s[base + k] = bi == 0x7fffffff ? kNegInf : bs;
-        a.cand_b[base + k] = bi == 0x7fffffff ? -1 : bi;
+        a.cand_s[base + k] = bs;
+        a.cand_b[base + k] = bi;
       }
-      if (i0 >= 0 && i0 == bi) {   // the owner pops its head
-        s0 = s1; i0 = i1;
-        s1 = kNegInf; i1 = -1;
-      }
+      last_s = bs;
+      last_b = bi;
     }
+    if (lane == 0)
+      for (; k < a.kfree; ++k) {
+        a.cand_s[base + k] = kNegInf;
+        a.cand_b[base + k] = -1;
+      }
   }
-  // The last CTA of this sequence to finish merges the chunk lists.
-  const int nch = min((nb + kIdxChunkBlocks - 1) / kIdxChunkBlocks, a.max_chunks);
+
+  // Arrive once per sequence touched, adding the blocks scored here; the CTA
+  // that completes a sequence's block count merges it.  (Counting blocks,
+  // not CTAs, keeps this right when the grid has more CTAs than blocks and
+  // some ranges are empty.)
   __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) s_last = atomicAdd(&a.seq_count[b], 1) == nch - 1;
+  for (int sidx = threadIdx.x; sidx < nsegs; sidx += kIdxThreads) {
+    const int sb = b_first + sidx;
+    const int lo = max(pfx[sb], G0), hi = min(pfx[sb + 1], G1);
+    if (atomicAdd(&a.seq_count[sb], hi - lo) + (hi - lo) == pfx[sb + 1] - pfx[sb]) lastq[atomicAdd(&n_last, 1)] = sb;
+  }
   __syncthreads();
-  if (!s_last) return;
+  if (n_last == 0) return;
   __threadfence();
-  for (int r = warp; r < a.h_kv; r += kIdxThreads / 32) merge_topk_warp<BK>(a, b, r, lane, chosen[warp]);
+  for (int pi = warp; pi < n_last * a.h_kv; pi += kWarps) {
+    const int sb = lastq[pi / a.h_kv], r = pi % a.h_kv;
+    const int c_lo = idx_cta_of(pfx[sb], T, n), c_hi = idx_cta_of(pfx[sb + 1] - 1, T, n);
+    merge_topk_warp<BK>(a, sb, r, lane, chosen[warp], c_lo, c_hi - c_lo + 1, T, n);
+  }
 }
 
 // ---------------------------------------------------------------------------
-// 2. merge of the chunk lists + local block -> block_ids (ascending, -1 pad)
+// 2. merge of the per-CTA candidate lists + local block -> block_ids
+//    (ascending, -1 pad).  Exact: every global winner is a winner of the
+//    share that holds it.
 // ---------------------------------------------------------------------------
+// Shares come from CTAs c_lo .. c_lo + nseg - 1 of an n-CTA grid over T
+// blocks; a CTA whose range is empty wrote nothing and is skipped.
 template <int BK>
-__device__ void merge_topk_warp(const DecArgs& a, int b, int r, int lane, int* chosen) {
+__device__ void merge_topk_warp(const DecArgs& a, int b, int r, int lane, int* chosen, int c_lo, int nseg,
+                                long long T, int n) {
   const int L = static_cast<int>(a.cu_kv[b + 1] - a.cu_kv[b]);
-  const int nb = (L + BK - 1) / BK;
-  // Clamp to the chunks the workspace holds (a caller that understated max_kv
-  // gets a wrong answer, never an out-of-bounds read).
-  const int nch = min((nb + kIdxChunkBlocks - 1) / kIdxChunkBlocks, a.max_chunks);
-  const int ncand = nch * a.kfree;
   const int b_loc = (L - 1) / BK;
+  const int ncand = nseg * a.kfree;
+  auto cand_index = [&](int c) -> long long {   // -1: share of an empty range
+    const int sg = c / a.kfree, slot = c - sg * a.kfree;
+    const long long cc = c_lo + sg;
+    if ((cc + 1) * T / n == cc * T / n) return -1;
+    return ((cc + b) * a.h_kv + r) * a.kfree + slot;
+  };
   int nsel = 0;
   if (ncand <= 32 * kMergeRegCand) {
-    // Small candidate sets (up to 16 chunks of 16) live in registers: one
-    // load per candidate, then repeated warp argmax; the owner lane retires
-    // each pick (block ids are unique across chunks).
+    // Small candidate sets live in registers: one load per candidate, then
+    // repeated warp argmax; the owner lane retires each pick (block ids are
+    // unique across shares).
     float cs[kMergeRegCand];
     int cb[kMergeRegCand];
 #pragma unroll
@@ -247,9 +341,8 @@ __device__ void merge_topk_warp(const DecArgs& a, int b, int r, int lane, int* c
       const int c = lane + 32 * i;
       cs[i] = kNegInf;
       cb[i] = -1;
-      if (c < ncand) {
-        const int ch = c / a.kfree, slot = c % a.kfree;
-        const size_t idx = ((static_cast<size_t>(b) * a.max_chunks + ch) * a.h_kv + r) * a.kfree + slot;
+      const long long idx = c < ncand ? cand_index(c) : -1;
+      if (idx >= 0) {
         cb[i] = __ldcg(a.cand_b + idx);
         cs[i] = __ldcg(a.cand_s + idx);
       }
@@ -274,24 +367,23 @@ __device__ void merge_topk_warp(const DecArgs& a, int b, int r, int lane, int* c
         if (cb[i] == bi) cb[i] = -1;
     }
   } else {
-    // Repeated warp argmax over the candidates with a strictly decreasing bound:
-    // each round picks the best candidate that is worse than the previous pick.
+    // Repeated warp argmax with a strictly decreasing bound: each round picks
+    // the best candidate that is worse than the previous pick.
     float last_s = __builtin_huge_valf();
     int last_b = -1;
     for (int k = 0; k < a.kfree; ++k) {
       float bs = kNegInf;
       int bi = 0x7fffffff;
       for (int c = lane; c < ncand; c += 32) {
-        const int ch = c / a.kfree, slot = c % a.kfree;
-        const size_t idx = ((static_cast<size_t>(b) * a.max_chunks + ch) * a.h_kv + r) * a.kfree + slot;
+        const long long idx = cand_index(c);
+        if (idx < 0) continue;
         const int cb = __ldcg(a.cand_b + idx);
         if (cb < 0) continue;
         const float cs = __ldcg(a.cand_s + idx);
-        // Only candidates strictly after the previous pick in (score desc, block asc).
         if (k > 0 && !better(last_s, last_b, cs, cb)) continue;
         if (bi == 0x7fffffff || better(cs, cb, bs, bi)) { bs = cs; bi = cb; }
       }
-  #pragma unroll
+#pragma unroll
       for (int x = 16; x > 0; x >>= 1) {
         const float os = __shfl_xor_sync(0xffffffffu, bs, x);
         const int oi = __shfl_xor_sync(0xffffffffu, bi, x);
@@ -324,7 +416,7 @@ __device__ void merge_topk_warp(const DecArgs& a, int b, int r, int lane, int* c
 template <int BK>
 __global__ void __launch_bounds__(32) decode_local_only_kernel(const DecArgs a) {
   __shared__ int chosen[33];
-  merge_topk_warp<BK>(a, blockIdx.x / a.h_kv, blockIdx.x % a.h_kv, threadIdx.x, chosen);
+  merge_topk_warp<BK>(a, blockIdx.x / a.h_kv, blockIdx.x % a.h_kv, threadIdx.x, chosen, 0, 0, 1, 1);
 }
 
 // ---------------------------------------------------------------------------
@@ -1017,9 +1109,24 @@ SplitPlan plan_splits(const msa_params& p, int max_kv, int dense) {
   return s;
 }
 
-int max_chunks_for(const msa_params& p, int max_kv) {
-  const int nb = (max_kv + p.block_k - 1) / p.block_k;
-  return (nb + kIdxChunkBlocks - 1) / kIdxChunkBlocks;
+// Index grid: at least kIdxCtas CTAs, and enough that no CTA holds more than
+// kIdxWCap blocks when every sequence is max_kv long.
+struct IdxPlan {
+  int ctas, wmax;
+  size_t smem;
+};
+
+IdxPlan plan_index(const msa_params& p, int batch, int max_kv) {
+  IdxPlan ip;
+  const long long tmax = static_cast<long long>(batch) * ((max_kv + p.block_k - 1) / p.block_k);
+  long long n = (tmax + kIdxWCap - 1) / kIdxWCap;
+  if (n < kIdxCtas) n = kIdxCtas;
+  ip.ctas = static_cast<int>(n);
+  ip.wmax = static_cast<int>((tmax + n - 1) / n);
+  if (ip.wmax < 1) ip.wmax = 1;
+  ip.smem = align_up(static_cast<size_t>(batch + 1) * 4, 16) + static_cast<size_t>(p.h_kv) * ip.wmax * 4 +
+            static_cast<size_t>(ip.wmax + 1) * 4;
+  return ip;
 }
 
 template <int D, int BK>
@@ -1086,10 +1193,13 @@ int launch_attn_stream(const DecArgs& a, int max_kv, int* status, cudaStream_t s
 }
 
 template <int DIDX, int BK>
-int launch_index(const DecArgs& a, cudaStream_t st) {
+int launch_index(const DecArgs& a, size_t smem, cudaStream_t st) {
   if (a.kfree > 0) {
-    dim3 grid(a.max_chunks, a.batch);
-    decode_index_kernel<DIDX, BK><<<grid, kIdxThreads, 0, st>>>(a);
+    auto kern = decode_index_kernel<DIDX, BK>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+        cudaSuccess)
+      return MSA_ERR_CUDA;
+    kern<<<a.idx_ctas, kIdxThreads, smem, st>>>(a);
   } else {   // topk == 1 with the forced local block needs no scan
     decode_local_only_kernel<BK><<<a.batch * a.h_kv, 32, 0, st>>>(a);
   }
@@ -1108,7 +1218,7 @@ size_t decode_counter_bytes(const msa_params& p, int batch) {
 
 size_t decode_workspace_bytes(const msa_params& p, int batch, int max_kv) {
   const int kfree = p.topk;   // upper bound on topk - force_local
-  const size_t cand = static_cast<size_t>(batch) * max_chunks_for(p, max_kv) * p.h_kv * kfree;
+  const size_t cand = static_cast<size_t>(plan_index(p, batch, max_kv).ctas + batch) * p.h_kv * kfree;
   const SplitPlan sd = plan_splits(p, max_kv, 1), ss = plan_splits(p, max_kv, 0);
   const int splits = sd.splits > ss.splits ? sd.splits : ss.splits;
   const size_t part_dense = static_cast<size_t>(batch) * p.h_q * splits * (p.d + 4);
@@ -1126,6 +1236,8 @@ int run_sparse_attn_decode(const msa_params& p, const void* q, const void* q_idx
   if (p.h_kv > 8) return MSA_ERR_UNSUPPORTED;
   // TMA row coordinates of the caches are 32-bit.
   if (!dense && static_cast<long long>(batch) * max_kv > 0x7fffffffLL) return MSA_ERR_UNSUPPORTED;
+  // The index scan keeps the block prefix of all sequences in shared memory.
+  if (!dense && batch > kIdxMaxBatch) return MSA_ERR_UNSUPPORTED;
   DecArgs a;
   a.q = static_cast<const uint16_t*>(q);
   a.q_idx = static_cast<const uint16_t*>(q_idx);
@@ -1142,7 +1254,9 @@ int run_sparse_attn_decode(const msa_params& p, const void* q, const void* q_idx
   a.causal = p.causal;
   a.force_local = p.force_local;
   a.kfree = p.topk - (p.force_local ? 1 : 0);
-  a.max_chunks = max_chunks_for(p, max_kv);
+  const IdxPlan ip = plan_index(p, batch, max_kv);
+  a.idx_ctas = ip.ctas;
+  a.idx_wmax = ip.wmax;
   const SplitPlan sp = plan_splits(p, max_kv, dense);
   a.splits = sp.splits;
   a.slots_per_split = sp.slots_per_split;
@@ -1151,7 +1265,7 @@ int run_sparse_attn_decode(const msa_params& p, const void* q, const void* q_idx
   a.head_tiles = (G + 15) / 16;
   const float scale = p.scale > 0.f ? p.scale : 1.0f / sqrtf(static_cast<float>(p.d));
   a.scale_log2 = scale * kLog2e;
-  const size_t cand = static_cast<size_t>(batch) * a.max_chunks * p.h_kv * p.topk;
+  const size_t cand = static_cast<size_t>(ip.ctas + batch) * p.h_kv * p.topk;
   uint8_t* w = static_cast<uint8_t*>(ws);
   a.seq_count = reinterpret_cast<int*>(w);
   a.grp_count = a.seq_count + batch;
@@ -1163,11 +1277,11 @@ int run_sparse_attn_decode(const msa_params& p, const void* q, const void* q_idx
   int rc = MSA_OK;
   if (!dense) {
     if (p.block_k == 64) {
-      rc = p.d_idx == 32 ? launch_index<32, 64>(a, stream)
-                         : (p.d_idx == 64 ? launch_index<64, 64>(a, stream) : launch_index<128, 64>(a, stream));
+      rc = p.d_idx == 32 ? launch_index<32, 64>(a, ip.smem, stream)
+                         : (p.d_idx == 64 ? launch_index<64, 64>(a, ip.smem, stream) : launch_index<128, 64>(a, ip.smem, stream));
     } else {
-      rc = p.d_idx == 32 ? launch_index<32, 128>(a, stream)
-                         : (p.d_idx == 64 ? launch_index<64, 128>(a, stream) : launch_index<128, 128>(a, stream));
+      rc = p.d_idx == 32 ? launch_index<32, 128>(a, ip.smem, stream)
+                         : (p.d_idx == 64 ? launch_index<64, 128>(a, ip.smem, stream) : launch_index<128, 128>(a, ip.smem, stream));
     }
   }
   if (rc) return rc;
