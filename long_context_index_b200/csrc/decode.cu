@@ -329,16 +329,19 @@ __device__ void merge_topk_warp(const DecArgs& a, int b, int r, int lane, int* c
     if ((cc + 1) * T / n == cc * T / n) return -1;
     return ((cc + b) * a.h_kv + r) * a.kfree + slot;
   };
-  int nsel = 0;
-  if (ncand <= 32 * kMergeRegCand) {
-    // Small candidate sets live in registers: one load per candidate, then
-    // repeated warp argmax; the owner lane retires each pick (block ids are
-    // unique across shares).
+  // Streaming merge: candidates arrive in chunks of 32 * kMergeRegCand (one
+  // coalesced load per lane and slot); each chunk is merged with the running
+  // top-kfree list, lane k holding its k-th entry, by kfree rounds of warp
+  // argmax whose winner is retired by its owner (block ids are unique across
+  // shares).
+  float run_s = kNegInf;
+  int run_b = -1;
+  for (int c0 = 0; c0 < ncand; c0 += 32 * kMergeRegCand) {
     float cs[kMergeRegCand];
     int cb[kMergeRegCand];
 #pragma unroll
     for (int i = 0; i < kMergeRegCand; ++i) {
-      const int c = lane + 32 * i;
+      const int c = c0 + lane + 32 * i;
       cs[i] = kNegInf;
       cb[i] = -1;
       const long long idx = c < ncand ? cand_index(c) : -1;
@@ -347,9 +350,11 @@ __device__ void merge_topk_warp(const DecArgs& a, int b, int r, int lane, int* c
         cs[i] = __ldcg(a.cand_s + idx);
       }
     }
+    float new_s = kNegInf;
+    int new_b = -1;
     for (int k = 0; k < a.kfree; ++k) {
-      float bs = kNegInf;
-      int bi = 0x7fffffff;
+      float bs = run_s;
+      int bi = run_b >= 0 ? run_b : 0x7fffffff;
 #pragma unroll
       for (int i = 0; i < kMergeRegCand; ++i)
         if (cb[i] >= 0 && (bi == 0x7fffffff || better(cs[i], cb[i], bs, bi))) { bs = cs[i]; bi = cb[i]; }
@@ -360,42 +365,22 @@ __device__ void merge_topk_warp(const DecArgs& a, int b, int r, int lane, int* c
         if (oi != 0x7fffffff && (bi == 0x7fffffff || better(os, oi, bs, bi))) { bs = os; bi = oi; }
       }
       if (bi == 0x7fffffff) break;
-      if (lane == 0) chosen[nsel] = bi;
-      ++nsel;
+      if (lane == k) {
+        new_s = bs;
+        new_b = bi;
+      }
+      if (run_b == bi) run_b = -1;
 #pragma unroll
       for (int i = 0; i < kMergeRegCand; ++i)
         if (cb[i] == bi) cb[i] = -1;
     }
-  } else {
-    // Repeated warp argmax with a strictly decreasing bound: each round picks
-    // the best candidate that is worse than the previous pick.
-    float last_s = __builtin_huge_valf();
-    int last_b = -1;
-    for (int k = 0; k < a.kfree; ++k) {
-      float bs = kNegInf;
-      int bi = 0x7fffffff;
-      for (int c = lane; c < ncand; c += 32) {
-        const long long idx = cand_index(c);
-        if (idx < 0) continue;
-        const int cb = __ldcg(a.cand_b + idx);
-        if (cb < 0) continue;
-        const float cs = __ldcg(a.cand_s + idx);
-        if (k > 0 && !better(last_s, last_b, cs, cb)) continue;
-        if (bi == 0x7fffffff || better(cs, cb, bs, bi)) { bs = cs; bi = cb; }
-      }
-#pragma unroll
-      for (int x = 16; x > 0; x >>= 1) {
-        const float os = __shfl_xor_sync(0xffffffffu, bs, x);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, x);
-        if (oi != 0x7fffffff && (bi == 0x7fffffff || better(os, oi, bs, bi))) { bs = os; bi = oi; }
-      }
-      if (bi == 0x7fffffff) break;
-      if (lane == 0) chosen[nsel] = bi;
-      ++nsel;
-      last_s = bs;
-      last_b = bi;
-    }
+    run_s = new_s;
+    run_b = new_b;
   }
+  const int nsel0 = __popc(__ballot_sync(0xffffffffu, run_b >= 0));   // lanes 0 .. nsel0 - 1
+  if (run_b >= 0) chosen[lane] = run_b;
+  __syncwarp();
+  int nsel = nsel0;
   if (lane == 0) {
     if (a.force_local) chosen[nsel++] = b_loc;
     // insertion sort (<= 32 entries)
