@@ -45,16 +45,19 @@
 namespace msa {
 namespace {
 
-constexpr int kThreads = 448;   // 14 warps
+constexpr int kThreads = 480;   // 15 warps
 constexpr int kSoftW0 = 2;      // softmax warps 2..9: two per TMEM lane quarter, 64 columns each
 constexpr int kEpiW0 = 10;      // epilogue warps 10..13
+constexpr int kPvW = 14;        // PV issuer (S is issued by warp 1): each SMSP's issue port is shared
+                                // with two softmax warps, so one thread issuing both would cap the rate
 // One K/V stage suffices because a CTA switches blocks only once per
 // (group, block) list (hundreds of chunks); the partial tile is staged in
 // two shared-memory buffers for the TMA stores.
-constexpr int kQStages = 2;
+constexpr int kQStages = 3;
 constexpr int kKVStages = 1;
-constexpr int kOStages = 2;
-constexpr int kDesc = 4;        // descriptor ring depth
+constexpr int kOStages = 1;
+constexpr int kDesc = 8;        // descriptor ring depth (a slot is held until the epilogue is done)
+constexpr int kCtrlBytes = 20480;   // descriptors, softmax stats, staged entries, barriers
 constexpr int kSchedThreads = 256;
 constexpr int kStageEntries = 256;   // list entries staged in shared memory at a time
 constexpr int kWave = 4096;          // query rows per wave (L2-resident Q working set)
@@ -66,7 +69,7 @@ struct KvoCfg {
   static constexpr int kKVBytes = BK * D * 2;          // one of K or V
   static constexpr int kOBytes = 128 * D * 2;          // staged bf16 partial tile
   static constexpr int kSmemData = kQStages * kQBytes + kKVStages * 2 * kKVBytes + kOStages * kOBytes;
-  static constexpr int kSmemBytes = kSmemData + 12288 + 1024;
+  static constexpr int kSmemBytes = kSmemData + kCtrlBytes + 1024;
   // TMEM: one S buffer (freed as soon as the softmax has loaded it), two P
   // buffers (bf16 pairs, BK/2 columns each), two O buffers.
   static constexpr int kColS = 0;        // S: [0, BK)
@@ -83,7 +86,7 @@ struct Desc {
   int first_of_kv, last_of_kv, end, chunk;   // chunk: global chunk id (partial tile index)
 };
 
-static_assert(kDesc * (sizeof(Desc) + 128 * 12) + 4 * 128 * 4 + kStageEntries * 4 + 32 * 8 + 16 <= 12288,
+static_assert(kDesc * (sizeof(Desc) + 128 * 12) + 4 * 128 * 4 + kStageEntries * 4 + 64 * 8 + 16 <= kCtrlBytes,
               "control block of attn_kvouter_kernel exceeds its shared-memory reservation");
 
 struct KvoArgs {
@@ -119,9 +122,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(stage + kStageEntries);
   uint64_t* q_full = bars;                                   // [kQStages]
   uint64_t* q_empty = q_full + kQStages;
-  uint64_t* kv_full = q_empty + kQStages;                    // [kKVStages]
-  uint64_t* kv_empty = kv_full + kKVStages;
-  uint64_t* d_full = kv_empty + kKVStages;                   // [kDesc]
+  // K and V of a stage have their own barriers: the next list's K can land
+  // once the current list's last S has read K, while its last PV still
+  // reads V.
+  uint64_t* k_full = q_empty + kQStages;                     // [kKVStages]
+  uint64_t* k_empty = k_full + kKVStages;
+  uint64_t* v_full = k_empty + kKVStages;
+  uint64_t* v_empty = v_full + kKVStages;
+  uint64_t* d_full = v_empty + kKVStages;                    // [kDesc]
   uint64_t* d_empty = d_full + kDesc;
   uint64_t* s_full = d_empty + kDesc;                        // [1] S ready
   uint64_t* s_free = s_full + 1;                             // [1] S loaded by the softmax
@@ -141,12 +149,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&q_empty[s], 1);
     }
     for (int s = 0; s < kKVStages; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     for (int s = 0; s < kDesc; ++s) {
       mbar_init(&d_full[s], 1);
-      mbar_init(&d_empty[s], 13);  // MMA thread + 8 softmax warps + 4 epilogue warps
+      mbar_init(&d_empty[s], 14);  // S and PV issuers + 8 softmax warps + 4 epilogue warps
       mbar_init(&ml_full[s], 8);   // 8 softmax warps
     }
     mbar_init(s_full, 1);
@@ -170,6 +180,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const WaitCtx wc{abort_flag, args.status};
   const int n_lists = *args.n_lists;
+  // Gathered Q rows are re-read by up to k lists of their wave: keep them in
+  // L2; partial tiles are read once, much later: let them leave first.
+  const uint64_t q_policy = l2_evict_last();
+  const uint64_t part_policy = l2_evict_first();
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer (whole warp)
@@ -194,15 +208,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int start = args.offs[rb], cnt = args.offs[rb + 1] - start;
       const int chunk0 = args.chunk_off[rb];
       const int kvs = kvc % kKVStages;
+      const uint32_t kv_ph = ((kvc / kKVStages) & 1) ^ 1;
+      uint8_t* sk = skv + kvs * 2 * Cfg::kKVBytes;
       if (lane == 0) {
-        ok = mbar_wait(&kv_empty[kvs], ((kvc / kKVStages) & 1) ^ 1, wc);
+        ok = mbar_wait(&k_empty[kvs], kv_ph, wc);
         if (ok) {
-          mbar_arrive_expect_tx(&kv_full[kvs], 2 * Cfg::kKVBytes);
-          uint8_t* sk = skv + kvs * 2 * Cfg::kKVBytes;
-          for (int a = 0; a < Cfg::kAtoms; ++a) {
-            tma_load_3d(sk + a * BK * 128, &tm_k, &kv_full[kvs], a * 64, r, b * BK);
-            tma_load_3d(sk + Cfg::kKVBytes + a * BK * 128, &tm_v, &kv_full[kvs], a * 64, r, b * BK);
-          }
+          mbar_arrive_expect_tx(&k_full[kvs], Cfg::kKVBytes);
+          for (int a = 0; a < Cfg::kAtoms; ++a)
+            tma_load_3d(sk + a * BK * 128, &tm_k, &k_full[kvs], a * 64, r, b * BK);
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -246,12 +259,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           dd.entry[qi] = e;
           const int q = e >= 0 ? (e >> 5) : args.n_q;   // past the end: TMA fills zeros
           for (int a = 0; a < Cfg::kAtoms; ++a)
-            tma_load_3d(sq + qs * Cfg::kQBytes + a * 128 * 128 + qi * G * 128, &tm_q, &q_full[qs], a * 64,
-                        r * G, q);
+            tma_load_3d_hint(sq + qs * Cfg::kQBytes + a * 128 * 128 + qi * G * 128, &tm_q, &q_full[qs], a * 64,
+                             r * G, q, q_policy);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&d_full[ds]);
         ++t;
+        if (c0 == 0) {
+          // V after the first chunk is out: S and the softmax of that chunk
+          // run while the previous list's last PV releases the V buffer.
+          if (lane == 0) {
+            ok = mbar_wait(&v_empty[kvs], kv_ph, wc);
+            if (ok) {
+              mbar_arrive_expect_tx(&v_full[kvs], Cfg::kKVBytes);
+              for (int a = 0; a < Cfg::kAtoms; ++a)
+                tma_load_3d(sk + Cfg::kKVBytes + a * BK * 128, &tm_v, &v_full[kvs], a * 64, r, b * BK);
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) break;
+        }
       }
     }
     // End marker for the consumers.
@@ -263,77 +290,75 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    // ---------------------------------------------------------------- UMMA
+    // ---------------------------------------------------------------- UMMA: S = Q K^T
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, BK, false, false);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
-      const uint32_t sq_addr = smem_u32(sq);
-      const uint32_t skv_addr = smem_u32(skv);
-      int kvc = 0;
-      int prev_kvs = 0, prev_last = 0;
-      auto issue_pv = [&](int j, int kvs, int last) -> bool {
-        const int sb = j & 1;
-        if (!mbar_wait(&p_full[sb], (j >> 1) & 1, wc)) return false;
-        if (!mbar_wait(&o_free[sb], ((j >> 1) & 1) ^ 1, wc)) return false;
-        tc_fence_after();
-        const uint32_t sv_addr = skv_addr + kvs * 2 * Cfg::kKVBytes + Cfg::kKVBytes;
-        const uint32_t p_tmem = tmem + Cfg::kColP + sb * (BK / 2);
-        const uint32_t o_tmem = tmem + Cfg::kColO + sb * D;
-#pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk) {
-          const uint64_t bdesc = smem_desc(sv_addr + kk * 2048, BK * 128, 1024, kSwizzle128B);
-          umma_ts(o_tmem, p_tmem + kk * 8, bdesc, idesc_o, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(&o_full[sb]);
-        umma_commit(&p_free[sb]);
-        if (last) umma_commit(&kv_empty[kvs]);
-        return true;
-      };
-      int t = 0;
-      bool ok = true;
-      bool pending = false;   // PV of chunk t-1 not yet issued
-      while (ok) {
+      // Descriptors differ only in their start-address field (address >> 4,
+      // bits 0-13, never carrying out for shared-memory addresses), so they
+      // are a base plus an offset.
+      const uint64_t q_desc0 = smem_desc(smem_u32(sq), 16, 1024, kSwizzle128B);
+      const uint64_t k_desc0 = smem_desc(smem_u32(skv), 16, 1024, kSwizzle128B);
+      int kvc = 0;   // lists whose K was awaited
+      for (int t = 0;; ++t) {
         const int ds = t % kDesc;
-        if (!mbar_wait(&d_full[ds], (t / kDesc) & 1, wc)) { ok = false; break; }
+        if (!mbar_wait(&d_full[ds], (t / kDesc) & 1, wc)) break;
         const Desc& dd = desc[ds];
         const int end = dd.end, kvs = dd.kvs, first = dd.first_of_kv, last = dd.last_of_kv;
         mbar_arrive(&d_empty[ds]);
         if (end) break;
-        const int qs = t % kQStages, sb = t & 1;
+        const int qs = t % kQStages;
         if (first) {
-          if (!mbar_wait(&kv_full[kvs], (kvc / kKVStages) & 1, wc)) { ok = false; break; }
+          if (!mbar_wait(&k_full[kvs], (kvc / kKVStages) & 1, wc)) break;
           ++kvc;
         }
-        if (!mbar_wait(&q_full[qs], (t / kQStages) & 1, wc)) { ok = false; break; }
+        if (!mbar_wait(&q_full[qs], (t / kQStages) & 1, wc)) break;
         // S(t) reuses the single S buffer once the softmax has loaded S(t-1).
-        if (!mbar_wait(s_free, (t & 1) ^ 1, wc)) { ok = false; break; }
+        if (!mbar_wait(s_free, (t & 1) ^ 1, wc)) break;
         tc_fence_after();
-        const uint32_t sk_addr = skv_addr + kvs * 2 * Cfg::kKVBytes;
+        const uint64_t qd = q_desc0 + ((qs * Cfg::kQBytes) >> 4);
+        const uint64_t kd = k_desc0 + ((kvs * 2 * Cfg::kKVBytes) >> 4);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-          const int atom = ks / 4;
-          const uint32_t koff = (ks % 4) * 32;
-          const uint64_t adesc =
-              smem_desc(sq_addr + qs * Cfg::kQBytes + atom * 128 * 128 + koff, 16, 1024, kSwizzle128B);
-          const uint64_t bdesc = smem_desc(sk_addr + atom * BK * 128 + koff, 16, 1024, kSwizzle128B);
-          umma_ss(tmem + Cfg::kColS, adesc, bdesc, idesc_s, ks > 0 ? 1u : 0u);
+          const uint32_t off = (ks / 4) * (128 * 128) + (ks % 4) * 32;
+          const uint32_t koff = (ks / 4) * (BK * 128) + (ks % 4) * 32;
+          umma_ss(tmem + Cfg::kColS, qd + (off >> 4), kd + (koff >> 4), idesc_s, ks > 0 ? 1u : 0u);
         }
         umma_commit(&q_empty[qs]);
         umma_commit(s_full);
-        if (pending && !issue_pv(t - 1, prev_kvs, prev_last)) { ok = false; break; }
-        if (last) {
-          // The last chunk of a list frees the K/V stage the producer waits on
-          // before it publishes the next list, so its PV cannot be deferred.
-          if (!issue_pv(t, kvs, last)) { ok = false; break; }
-          pending = false;
-        } else {
-          pending = true;
-          prev_kvs = kvs;
-          prev_last = last;
-        }
-        ++t;
+        if (last) umma_commit(&k_empty[kvs]);   // this list's last read of K
       }
-      if (ok && pending) issue_pv(t - 1, prev_kvs, prev_last);
+    }
+  } else if (warp == kPvW) {
+    // ---------------------------------------------------------------- UMMA: O = P V
+    if (lane == 0) {
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
+      const uint64_t v_desc0 = smem_desc(smem_u32(skv) + Cfg::kKVBytes, BK * 128, 1024, kSwizzle128B);
+      int vc = 0;   // lists whose V was awaited
+      for (int t = 0;; ++t) {
+        const int ds = t % kDesc;
+        if (!mbar_wait(&d_full[ds], (t / kDesc) & 1, wc)) break;
+        const Desc& dd = desc[ds];
+        const int end = dd.end, kvs = dd.kvs, first = dd.first_of_kv, last = dd.last_of_kv;
+        mbar_arrive(&d_empty[ds]);
+        if (end) break;
+        const int sb = t & 1;
+        if (first) {
+          if (!mbar_wait(&v_full[kvs], (vc / kKVStages) & 1, wc)) break;
+          ++vc;
+        }
+        if (!mbar_wait(&p_full[sb], (t >> 1) & 1, wc)) break;
+        if (!mbar_wait(&o_free[sb], ((t >> 1) & 1) ^ 1, wc)) break;
+        tc_fence_after();
+        const uint64_t vd = v_desc0 + ((kvs * 2 * Cfg::kKVBytes) >> 4);
+        const uint32_t p_tmem = tmem + Cfg::kColP + sb * (BK / 2);
+        const uint32_t o_tmem = tmem + Cfg::kColO + sb * D;
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk)
+          umma_ts(o_tmem, p_tmem + kk * 8, vd + ((kk * 2048) >> 4), idesc_o, kk > 0 ? 1u : 0u);
+        umma_commit(&o_full[sb]);
+        umma_commit(&p_free[sb]);
+        if (last) umma_commit(&v_empty[kvs]);   // this list's last read of V
+      }
     }
   } else if (warp >= kSoftW0 && warp < kEpiW0) {
     // ---------------------------------------------------------------- softmax
@@ -432,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&ml_full[ds]);
       }
     }
-  } else if (warp >= kEpiW0) {
+  } else if (warp >= kEpiW0 && warp < kEpiW0 + 4) {
     // ---------------------------------------------------------------- epilogue
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
@@ -463,7 +488,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int os = t % kOStages;
       // Stage the bf16 row in the swizzled tile layout (the layout TMA uses),
       // after the stores that last read this staging buffer have drained.
-      if (warp == kEpiW0 && lane == 0) bulk_wait_read_le1();
+      if (warp == kEpiW0 && lane == 0) {
+        if (kOStages == 1)
+          bulk_wait_read0();
+        else
+          bulk_wait_read_le1();
+      }
       named_bar(1, 128);
       const uint32_t so_addr = smem_u32(so + os * Cfg::kOBytes);
 #pragma unroll
@@ -493,7 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // stores (bulk groups are tracked per thread): one box per d atom.
       if (warp == kEpiW0 && lane == 0) {
         for (int a = 0; a < D / 64; ++a)
-          tma_store_2d(&tm_po, so + os * Cfg::kOBytes + a * 128 * 128, a * 64, chunk * 128);
+          tma_store_2d_hint(&tm_po, so + os * Cfg::kOBytes + a * 128 * 128, a * 64, chunk * 128, part_policy);
         bulk_commit();
       }
       __syncwarp();
