@@ -179,8 +179,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && n_ktiles > 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(kRows, kKeys, false, false);
       constexpr uint32_t sbo = 8 * Cfg::kSwB;   // 8-row core-matrix group stride
-      const uint32_t sq_addr = smem_u32(sq);
-      const uint32_t sk_addr = smem_u32(sk);
+      // Descriptors differ only in the start-address field (address >> 4 in
+      // bits 0-13, no carry for shared-memory addresses): base + offset, so
+      // the issuing thread spends few instructions per MMA (it shares its
+      // SMSP's issue port with two epilogue warps).
+      const uint64_t q_desc0 = smem_desc(smem_u32(sq), 16, sbo, Cfg::kSwz);
+      const uint64_t k_desc0 = smem_desc(smem_u32(sk), 16, sbo, Cfg::kSwz);
       bool ok = mbar_wait(q_full, 0, wc);
       for (int t = 0; ok && t < n_ktiles; ++t) {
         const int s = t % Cfg::kStages;
@@ -188,17 +192,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&acc_empty[acc], ((t >> 1) & 1) ^ 1, wc)) break;
         if (!mbar_wait(&full[s], (t / Cfg::kStages) & 1, wc)) break;
         tc_fence_after();
-        for (int g = 0; g < groups_here; ++g) {
+        const uint64_t kd = k_desc0 + ((s * Cfg::kAtoms * kKeys * Cfg::kSwB) >> 4);
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          if (g >= groups_here) break;
           const uint32_t d_tmem = tmem + acc * 256 + g * 128;
 #pragma unroll
           for (int ks = 0; ks < DIDX / 16; ++ks) {
-            const int atom = ks / (Cfg::kSwB / 32);
-            const uint32_t koff = (ks % (Cfg::kSwB / 32)) * 32;
-            const uint64_t adesc =
-                smem_desc(sq_addr + (g * Cfg::kAtoms + atom) * kRows * Cfg::kSwB + koff, 16, sbo, Cfg::kSwz);
-            const uint64_t bdesc =
-                smem_desc(sk_addr + (s * Cfg::kAtoms + atom) * kKeys * Cfg::kSwB + koff, 16, sbo, Cfg::kSwz);
-            umma_ss(d_tmem, adesc, bdesc, idesc, ks > 0 ? 1u : 0u);
+            constexpr int kPerAtom = Cfg::kSwB / 32;
+            const uint32_t aoff = ((g * Cfg::kAtoms + ks / kPerAtom) * kRows * Cfg::kSwB + (ks % kPerAtom) * 32) >> 4;
+            const uint32_t boff = ((ks / kPerAtom) * kKeys * Cfg::kSwB + (ks % kPerAtom) * 32) >> 4;
+            umma_ss(d_tmem, q_desc0 + aoff, kd + boff, idesc, ks > 0 ? 1u : 0u);
           }
         }
         umma_commit(&empty[s]);       // smem stage free once these MMAs finish
