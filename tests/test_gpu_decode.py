@@ -82,3 +82,40 @@ def test_many_items_per_cta():
     # CTA at 148 CTAs, so the persistent attention grid grows; sampled rows.
     w = small(h_q=32, h_kv=8, d=64, d_idx=32, block_k=64, topk=16, batch=2048, kv_min=100, kv_max=1500, seed=77)
     run_case(w, seqs=[0, 1, 777, 2047])
+
+
+def test_decode_equals_prefill_row_at_last_position():
+    # Entry-point consistency: a decode step and a one-row chunked prefill at
+    # q_pos0 = L_b - 1 over the same caches run different kernels but must
+    # select the same blocks (bit for bit) and agree on O within tolerance.
+    w = small(h_q=64, h_kv=4, d=128, d_idx=64, block_k=128, topk=16, batch=4, kv_min=3000, kv_max=9000, seed=91)
+    t = make_decode(w)
+    p = msa.Params.make(w.h_q, w.h_kv, w.d, w.d_idx, w.block_k, w.topk)
+    ids, o = msa.sparse_attn_decode(p, dev(t["q"]), dev(t["q_idx"]), dev(t["k_cache"]), dev(t["v_cache"]),
+                                    dev(t["k_idx_cache"]), dev(t["cu_kv"]), int(t["lens"].max()))
+    torch.cuda.synchronize()
+    cu = t["cu_kv"]
+    for b in range(w.batch):
+        lo, hi = int(cu[b]), int(cu[b + 1])
+        L = hi - lo
+        pid = msa.index_topk(p, dev(t["q_idx"][b:b + 1]), dev(t["k_idx_cache"][lo:hi]), L - 1)
+        po = msa.sparse_attn_prefill(p, dev(t["q"][b:b + 1]), dev(t["k_cache"][lo:hi]), dev(t["v_cache"][lo:hi]),
+                                     pid, L - 1)
+        torch.cuda.synchronize()
+        assert torch.equal(pid[0].cpu(), ids[b].cpu()), b
+        assert_close(host_f64(o[b]), host_f64(po[0]), what="decode vs prefill row, sequence %d" % b)
+
+
+def test_sparse_decode_rejects_batches_beyond_the_index_prefix():
+    # The sparse index scan keeps the block prefix of every sequence in shared
+    # memory: batches above 4096 are refused before any launch.
+    B = 4097
+    p = msa.Params.make(8, 2, 64, 32, 64, 4)
+    q = torch.zeros((B, 8, 64), dtype=torch.bfloat16, device="cuda")
+    qi = torch.zeros((B, 2, 32), dtype=torch.bfloat16, device="cuda")
+    kc = torch.zeros((B, 2, 64), dtype=torch.bfloat16, device="cuda")
+    ki = torch.zeros((B, 1, 32), dtype=torch.bfloat16, device="cuda")
+    cu = torch.arange(B + 1, dtype=torch.int64, device="cuda")
+    with pytest.raises(msa.MSAError) as err:
+        msa.sparse_attn_decode(p, q, qi, kc, kc, ki, cu, 1)
+    assert err.value.code == -2
