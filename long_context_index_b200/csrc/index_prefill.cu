@@ -9,19 +9,23 @@
 //             ties to the lower block index, emitted ascending, -1 padded.
 // Selection compares raw scores and never exponentiates (section 4.4.1).
 //
-// Design (one CTA = 128 query rows x 2 groups):
-//   * warp 0, one lane: TMA producer.  Loads the two Q_idx tiles (A operands,
-//     resident for the CTA) and streams 128-key K_idx tiles (B operand, shared
-//     by both groups) through an NST-deep shared-memory ring.
-//   * warp 1, one lane: UMMA issuer.  Per key tile, two 128x128xd_idx
-//     tcgen05.mma (one per group) into one of two TMEM accumulator stages
-//     (2 stages x 2 groups x 128 fp32 columns = all 512 columns), so the MMA
-//     of tile t+1 overlaps the epilogue of tile t.
-//   * warps 4..11: epilogue.  Thread = (TMEM lane = query row, group).  Reads
-//     its row of S from TMEM, masks invisible keys, max-pools per block with
-//     3-input max, and keeps a register top-k list (insertion only when the
-//     candidate beats the current k-th score, so ties keep the earlier, lower
-//     block).  M is never written to memory.
+// Design (one CTA = 128 query rows x one group):
+//   * warp 0, one lane: TMA producer.  Loads the Q_idx tile (A operand,
+//     resident for the CTA) and streams 256-key K_idx tiles (B operand)
+//     through an NST-deep shared-memory ring.
+//   * warp 1, one lane: UMMA issuer.  Per key tile, one 128x256xd_idx
+//     tcgen05.mma chain into one of two TMEM accumulator stages (2 x 256 fp32
+//     columns = all 512 columns), so the MMA of tile t+1 overlaps the
+//     epilogue of tile t.  N = 256 halves the MMA instructions per flop: the
+//     issuing thread shares its SMSP's issue port with two epilogue warps,
+//     and a contended issue slot costs more than the MMA itself.
+//   * warps 4..11: epilogue.  Thread = (TMEM lane = query row, half of the
+//     tile's 256 columns).  Reads its 128 columns of S from TMEM, masks
+//     invisible keys, max-pools per block with 3-input max, and keeps a
+//     register top-k list of the blocks in its halves (insertion only when
+//     the candidate beats the current k-th score, so ties keep the earlier,
+//     lower block).  At the end the two half-lists of a row are merged by
+//     (score desc, block asc).  M is never written to memory.
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -33,7 +37,7 @@ namespace msa {
 namespace {
 
 constexpr int kRows = 128;      // query rows per CTA (UMMA M)
-constexpr int kKeys = 128;      // keys per tile (UMMA N)
+constexpr int kKeys = 256;      // keys per tile (UMMA N)
 constexpr int kThreads = 384;   // 12 warps
 constexpr int kEpiWarp0 = 4;    // first epilogue warp
 
@@ -42,9 +46,10 @@ struct IdxCfg {
   static constexpr int kSwB = DIDX * 2 >= 128 ? 128 : DIDX * 2;   // swizzle span (bytes)
   static constexpr int kAtoms = DIDX * 2 / kSwB;                  // swizzle atoms along K
   static constexpr uint32_t kSwz = kSwB == 128 ? kSwizzle128B : kSwizzle64B;
-  static constexpr int kTileBytes = kRows * DIDX * 2;             // one 128 x DIDX bf16 tile
-  static constexpr int kStages = DIDX == 128 ? 4 : (DIDX == 64 ? 6 : 8);
-  static constexpr int kSmemQ = 2 * kTileBytes;
+  static constexpr int kQBytes = kRows * DIDX * 2;                // the 128 x DIDX Q_idx tile
+  static constexpr int kTileBytes = kKeys * DIDX * 2;             // one 256 x DIDX K_idx tile
+  static constexpr int kStages = DIDX == 128 ? 2 : (DIDX == 64 ? 5 : 8);
+  static constexpr int kSmemQ = kQBytes;
   static constexpr int kSmemK = kStages * kTileBytes;
   static constexpr int kSmemBytes = kSmemQ + kSmemK + 1024 /*barriers etc.*/ + 1024 /*align*/;
 };
@@ -53,7 +58,7 @@ struct IdxArgs {
   int32_t* block_ids;
   int* status;
   int n_q, n_kv, q_pos0, h_kv, topk, causal, force_local;
-  int n_tiles, n_pairs;
+  int n_tiles;
 };
 
 // Sorted-descending register list of KMAX (score, block) pairs.  Slots
@@ -98,7 +103,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   using Cfg = IdxCfg<DIDX>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sq = smem;                       // [2 groups][atoms][128 rows][kSwB]
+  uint8_t* sq = smem;                       // [atoms][128 rows][kSwB]
   uint8_t* sk = smem + Cfg::kSmemQ;         // [stages][atoms][128 keys][kSwB]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sk + Cfg::kSmemK);
   uint64_t* full = bars;                    // [kStages]
@@ -111,11 +116,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = warp_id();
   const int lane = lane_id();
-  const int tile = args.n_tiles - 1 - static_cast<int>(blockIdx.x) / args.n_pairs;  // heavy tiles first
-  const int pair = static_cast<int>(blockIdx.x) % args.n_pairs;
+  const int tile = args.n_tiles - 1 - static_cast<int>(blockIdx.x) / args.h_kv;  // heavy tiles first
+  const int grp = static_cast<int>(blockIdx.x) % args.h_kv;
   const int i0 = tile * kRows;
   const int rows_here = min(kRows, args.n_q - i0);
-  const int groups_here = min(2, args.h_kv - 2 * pair);
 
   // Key range this CTA must score.  A row at position p needs keys < kv_lim(p)
   // where kv_lim = p + 1 (causal) or n_kv; with force_local its own block is
@@ -159,11 +163,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && n_ktiles > 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
-      mbar_arrive_expect_tx(q_full, groups_here * Cfg::kTileBytes);
-      for (int g = 0; g < groups_here; ++g)
-        for (int a = 0; a < Cfg::kAtoms; ++a)
-          tma_load_3d(sq + (g * Cfg::kAtoms + a) * kRows * Cfg::kSwB, &tm_q, q_full, a * (Cfg::kSwB / 2),
-                      2 * pair + g, i0);
+      mbar_arrive_expect_tx(q_full, Cfg::kQBytes);
+      for (int a = 0; a < Cfg::kAtoms; ++a)
+        tma_load_3d(sq + a * kRows * Cfg::kSwB, &tm_q, q_full, a * (Cfg::kSwB / 2), grp, i0);
       for (int t = 0; t < n_ktiles; ++t) {
         const int s = t % Cfg::kStages;
         const uint32_t ph = (t / Cfg::kStages) & 1;
@@ -193,17 +195,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&full[s], (t / Cfg::kStages) & 1, wc)) break;
         tc_fence_after();
         const uint64_t kd = k_desc0 + ((s * Cfg::kAtoms * kKeys * Cfg::kSwB) >> 4);
+        const uint32_t d_tmem = tmem + acc * kKeys;
 #pragma unroll
-        for (int g = 0; g < 2; ++g) {
-          if (g >= groups_here) break;
-          const uint32_t d_tmem = tmem + acc * 256 + g * 128;
-#pragma unroll
-          for (int ks = 0; ks < DIDX / 16; ++ks) {
-            constexpr int kPerAtom = Cfg::kSwB / 32;
-            const uint32_t aoff = ((g * Cfg::kAtoms + ks / kPerAtom) * kRows * Cfg::kSwB + (ks % kPerAtom) * 32) >> 4;
-            const uint32_t boff = ((ks / kPerAtom) * kKeys * Cfg::kSwB + (ks % kPerAtom) * 32) >> 4;
-            umma_ss(d_tmem, q_desc0 + aoff, kd + boff, idesc, ks > 0 ? 1u : 0u);
-          }
+        for (int ks = 0; ks < DIDX / 16; ++ks) {
+          constexpr int kPerAtom = Cfg::kSwB / 32;
+          const uint32_t aoff = ((ks / kPerAtom) * kRows * Cfg::kSwB + (ks % kPerAtom) * 32) >> 4;
+          const uint32_t boff = ((ks / kPerAtom) * kKeys * Cfg::kSwB + (ks % kPerAtom) * 32) >> 4;
+          umma_ss(d_tmem, q_desc0 + aoff, kd + boff, idesc, ks > 0 ? 1u : 0u);
         }
         umma_commit(&empty[s]);       // smem stage free once these MMAs finish
         umma_commit(&acc_full[acc]);  // accumulator ready for the epilogue
@@ -212,38 +210,38 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp >= kEpiWarp0) {
     // ---------------------------------------------------------------- epilogue
     const int quarter = warp & 3;
-    const int g = (warp - kEpiWarp0) >> 2;   // group within the pair
+    const int half = (warp - kEpiWarp0) >> 2;   // columns [128 half, 128 half + 128) of each tile
     const int row = quarter * 32 + lane;
-    const bool row_ok = row < rows_here && g < groups_here;
+    const bool row_ok = row < rows_here;
     const int p = args.q_pos0 + i0 + row;
     const int kv_lim = args.causal ? min(p + 1, args.n_kv) : args.n_kv;
     const int b_loc = p / BK;
     const int k_free = args.topk - (args.force_local ? 1 : 0);
     TopK<KMAX> tk;
     tk.init(k_free);
-    const uint32_t taddr_row = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + g * 128;
+    const uint32_t taddr_row = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + half * 128;
 
     for (int t = 0; t < n_ktiles; ++t) {
       const int acc = t & 1;
       if (!mbar_wait(&acc_full[acc], (t >> 1) & 1, wc)) break;
       tc_fence_after();
-      constexpr int kBlocksPerTile = kKeys / BK;
-      float bmax[kBlocksPerTile];
+      constexpr int kBlocksPerHalf = 128 / BK;
+      float bmax[kBlocksPerHalf];
 #pragma unroll
-      for (int bb = 0; bb < kBlocksPerTile; ++bb) bmax[bb] = __int_as_float(0xff800000);
-      const int j0 = t * kKeys;
-      if (g < groups_here) {
-        // The 128-column row in two halves (two TMEM loads in flight per
+      for (int bb = 0; bb < kBlocksPerHalf; ++bb) bmax[bb] = __int_as_float(0xff800000);
+      const int j0 = t * kKeys + half * 128;
+      if (j0 < kv_end) {
+        // 128 columns in two 64-column pieces (two TMEM loads in flight per
         // wait); per block, four independent 3-input max chains.
-        float m4[kBlocksPerTile][4];
+        float m4[kBlocksPerHalf][4];
 #pragma unroll
-        for (int bb = 0; bb < kBlocksPerTile; ++bb)
+        for (int bb = 0; bb < kBlocksPerHalf; ++bb)
           m4[bb][0] = m4[bb][1] = m4[bb][2] = m4[bb][3] = __int_as_float(0xff800000);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           uint32_t v[64];
-          tmem_ld32(taddr_row + acc * 256 + h * 64, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-          tmem_ld32(taddr_row + acc * 256 + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+          tmem_ld32(taddr_row + acc * kKeys + h * 64, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+          tmem_ld32(taddr_row + acc * kKeys + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
           tmem_ld_wait();
           const int jh = j0 + h * 64;
           if (jh + 64 > kv_lim) {   // keys this row must not see
@@ -251,7 +249,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int e = 0; e < 64; ++e)
               if (jh + e >= kv_lim) v[e] = 0xff800000u;   // -inf
           }
-          constexpr int kBpH = 64 / BK > 0 ? 64 / BK : 1;   // blocks touched per half
 #pragma unroll
           for (int e = 0; e < 64; e += 8) {
             const int bb = (h * 64 + e) / BK;
@@ -261,19 +258,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             m4[bb][k] =
                 max3f(m4[bb][k], __uint_as_float(v[e + 5]), fmaxf(__uint_as_float(v[e + 6]), __uint_as_float(v[e + 7])));
           }
-          (void)kBpH;
         }
 #pragma unroll
-        for (int bb = 0; bb < kBlocksPerTile; ++bb)
+        for (int bb = 0; bb < kBlocksPerHalf; ++bb)
           bmax[bb] = fmaxf(fmaxf(m4[bb][0], m4[bb][1]), fmaxf(m4[bb][2], m4[bb][3]));
       }
       // Release the accumulator stage to the MMA warp.
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[acc]);
-      if (row_ok) {
+      if (row_ok && j0 < kv_end) {
 #pragma unroll
-        for (int bb = 0; bb < kBlocksPerTile; ++bb) {
+        for (int bb = 0; bb < kBlocksPerHalf; ++bb) {
           const int b = (j0 / BK) + bb;
           const bool eligible = static_cast<long long>(b) * BK < kv_lim && !(args.force_local && b == b_loc);
           const float x = bmax[bb];
@@ -282,11 +278,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
 
-    if (row_ok) {
-      // Final set: live list entries plus the local block, ascending, -1 padded.
+    // Merge the two half-lists of each row: both go to shared memory (the K
+    // ring is idle once every tile has been consumed), then the half-0 thread
+    // takes the top k_free by (score desc, block asc), adds the local block
+    // and writes the ids ascending, -1 padded.
+    named_bar(1, 256);   // every epilogue thread is past its last accumulator read
+    float* msc = reinterpret_cast<float*>(sk) + (half * kRows + row) * KMAX;
+    int* mid = reinterpret_cast<int*>(sk + 2 * kRows * KMAX * 4) + (half * kRows + row) * KMAX;
+#pragma unroll
+    for (int i = 0; i < KMAX; ++i) {
+      msc[i] = tk.sc[i];
+      mid[i] = tk.id[i];
+    }
+    named_bar(1, 256);
+    if (half == 0 && row_ok) {
+      const float* asc = msc;
+      const int* aid = mid;
+      const float* bsc = msc + kRows * KMAX;
+      const int* bid = mid + kRows * KMAX;
+      int ia = KMAX - k_free, ib = KMAX - k_free;   // live parts, each sorted (score desc, block asc)
       int ids[KMAX + 1];
 #pragma unroll
-      for (int i = 0; i < KMAX; ++i) ids[i] = tk.id[i] < 0 ? 0x7fffffff : tk.id[i];
+      for (int i = 0; i < KMAX + 1; ++i) ids[i] = 0x7fffffff;
+#pragma unroll
+      for (int k = 0; k < KMAX; ++k) {
+        if (k < k_free) {
+          const bool a_ok = ia < KMAX && aid[ia] >= 0;
+          const bool b_ok = ib < KMAX && bid[ib] >= 0;
+          if (a_ok || b_ok) {
+            const bool take_a =
+                a_ok && (!b_ok || asc[ia] > bsc[ib] || (asc[ia] == bsc[ib] && aid[ia] < bid[ib]));
+            ids[k] = take_a ? aid[ia] : bid[ib];
+            ia += take_a ? 1 : 0;
+            ib += take_a ? 0 : 1;
+          }
+        }
+      }
       ids[KMAX] = args.force_local ? b_loc : 0x7fffffff;
       // Odd-even transposition sort on static indices (stays in registers).
 #pragma unroll
@@ -299,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ids[i + 1] = hi;
         }
       }
-      int32_t* out = args.block_ids + (static_cast<size_t>(i0 + row) * args.h_kv + 2 * pair + g) * args.topk;
+      int32_t* out = args.block_ids + (static_cast<size_t>(i0 + row) * args.h_kv + grp) * args.topk;
 #pragma unroll
       for (int i = 0; i < KMAX + 1; ++i)
         if (i < args.topk) out[i] = ids[i] == 0x7fffffff ? -1 : ids[i];
@@ -321,7 +348,7 @@ cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const IdxArgs
   const int smem = IdxCfg<DIDX>::kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(a.n_tiles * a.n_pairs);
+  dim3 grid(a.n_tiles * a.h_kv);
   kern<<<grid, kThreads, smem, st>>>(tq, tk, a);
   return cudaGetLastError();
 }
@@ -356,7 +383,7 @@ int run_index_topk_prefill(const msa_params& p, const void* q_idx, const void* k
   {
     const uint64_t dims[2] = {static_cast<uint64_t>(p.d_idx), static_cast<uint64_t>(n_kv)};
     const uint64_t strides[1] = {static_cast<uint64_t>(p.d_idx) * 2};
-    const uint32_t box[2] = {static_cast<uint32_t>(sw_elems), 128};
+    const uint32_t box[2] = {static_cast<uint32_t>(sw_elems), static_cast<uint32_t>(kKeys)};
     if (!encode_tma_bf16(&tk, 2, k_idx, dims, strides, box, swz)) return MSA_ERR_CUDA;
   }
   IdxArgs a;
@@ -370,7 +397,6 @@ int run_index_topk_prefill(const msa_params& p, const void* q_idx, const void* k
   a.causal = p.causal;
   a.force_local = p.force_local;
   a.n_tiles = (n_q + kRows - 1) / kRows;
-  a.n_pairs = (p.h_kv + 1) / 2;
   cudaError_t e;
   switch (p.d_idx) {
     case 32: e = launch_b<32>(p.block_k, tq, tk, a, stream); break;
