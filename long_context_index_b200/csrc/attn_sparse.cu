@@ -462,7 +462,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const int qi = row / G;
-    const int hh = row % G;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const float c = args.scale_log2;
     for (int t = 0;; ++t) {
@@ -475,7 +474,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       const int e = qi < dd.count ? dd.entry[qi] : -1;
-      const int r = dd.r;
       const int sb = t & 1;
       if (!mbar_wait(&o_full[sb], (t >> 1) & 1, wc)) break;
       if (!mbar_wait(&ml_full[ds], (t / kDesc) & 1, wc)) break;
