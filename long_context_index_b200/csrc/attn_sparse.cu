@@ -424,15 +424,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       named_bar(2 + quarter, 64);
       const float mx = fmaxf(xs[row], xs[128 + row]);
       const float bias = mx == __int_as_float(0xff800000) ? 0.f : mx * c;
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};   // two pairs of partial sums
       uint32_t pk[HC / 2];
 #pragma unroll
       for (int i = 0; i < HC; i += 4) {
-        const float p0 = ex2_approx(fmaf(__uint_as_float(sv[i]), c, -bias));
-        const float p1 = ex2_approx(fmaf(__uint_as_float(sv[i + 1]), c, -bias));
-        const float p2 = ex2_approx(fmaf(__uint_as_float(sv[i + 2]), c, -bias));
-        const float p3 = ex2_approx(fmaf(__uint_as_float(sv[i + 3]), c, -bias));
-        ls[(i / 4) & 3] += (p0 + p1) + (p2 + p3);
+        float x0, x1, x2, x3;
+        ffma2(x0, x1, __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]), c, c, -bias, -bias);
+        ffma2(x2, x3, __uint_as_float(sv[i + 2]), __uint_as_float(sv[i + 3]), c, c, -bias, -bias);
+        const float p0 = ex2_approx(x0), p1 = ex2_approx(x1), p2 = ex2_approx(x2), p3 = ex2_approx(x3);
+        float s0, s1;
+        fadd2(s0, s1, p0, p1, p2, p3);
+        const int k = ((i / 4) & 1) * 2;
+        fadd2(ls[k], ls[k + 1], ls[k], ls[k + 1], s0, s1);
         pk[i / 2] = pack_bf16x2(p0, p1);
         pk[i / 2 + 1] = pack_bf16x2(p2, p3);
       }
@@ -509,9 +512,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
           const float* f = reinterpret_cast<const float*>(&ov[ch * 8]);
-          st_shared_v4(so_addr + a * 128 * 128 + row * 128 + ((ch ^ (row & 7)) << 4),
-                       pack_bf16x2(f[0] * inv, f[1] * inv), pack_bf16x2(f[2] * inv, f[3] * inv),
-                       pack_bf16x2(f[4] * inv, f[5] * inv), pack_bf16x2(f[6] * inv, f[7] * inv));
+          float g[8];
+#pragma unroll
+          for (int j = 0; j < 8; j += 2) fmul2(g[j], g[j + 1], f[j], f[j + 1], inv, inv);
+          st_shared_v4(so_addr + a * 128 * 128 + row * 128 + ((ch ^ (row & 7)) << 4), pack_bf16x2(g[0], g[1]),
+                       pack_bf16x2(g[2], g[3]), pack_bf16x2(g[4], g[5]), pack_bf16x2(g[6], g[7]));
         }
       }
       args.part_lse[static_cast<size_t>(chunk) * 128 + row] = e >= 0 ? lse2 : __int_as_float(0xff800000);
