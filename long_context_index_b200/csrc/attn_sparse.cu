@@ -291,74 +291,85 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- UMMA: S = Q K^T
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, BK, false, false);
-      // Descriptors differ only in their start-address field (address >> 4,
-      // bits 0-13, never carrying out for shared-memory addresses), so they
-      // are a base plus an offset.
-      const uint64_t q_desc0 = smem_desc(smem_u32(sq), 16, 1024, kSwizzle128B);
-      const uint64_t k_desc0 = smem_desc(smem_u32(skv), 16, 1024, kSwizzle128B);
-      int kvc = 0;   // lists whose K was awaited
-      for (int t = 0;; ++t) {
-        const int ds = t % kDesc;
-        if (!mbar_wait(&d_full[ds], (t / kDesc) & 1, wc)) break;
-        const Desc& dd = desc[ds];
-        const int end = dd.end, kvs = dd.kvs, first = dd.first_of_kv, last = dd.last_of_kv;
-        mbar_arrive(&d_empty[ds]);
-        if (end) break;
-        const int qs = t % kQStages;
-        if (first) {
-          if (!mbar_wait(&k_full[kvs], (kvc / kKVStages) & 1, wc)) break;
-          ++kvc;
-        }
-        if (!mbar_wait(&q_full[qs], (t / kQStages) & 1, wc)) break;
-        // S(t) reuses the single S buffer once the softmax has loaded S(t-1).
-        if (!mbar_wait(s_free, (t & 1) ^ 1, wc)) break;
-        tc_fence_after();
-        const uint64_t qd = q_desc0 + ((qs * Cfg::kQBytes) >> 4);
-        const uint64_t kd = k_desc0 + ((kvs * 2 * Cfg::kKVBytes) >> 4);
+    // Both issuers run their loops with the whole warp (warp-uniform waits
+    // and descriptor math) and issue from one elected lane: a divergent
+    // single-lane loop loses most issue slots to the softmax and epilogue
+    // warps sharing its SMSP (measured: 108 against 272 cycles per MMA with
+    // three busy warps).
+    constexpr uint32_t idesc_s = idesc_bf16_f32(128, BK, false, false);
+    // Descriptors differ only in their start-address field (address >> 4,
+    // bits 0-13, never carrying out for shared-memory addresses), so they
+    // are a base plus an offset.
+    const uint64_t q_desc0 = smem_desc(smem_u32(sq), 16, 1024, kSwizzle128B);
+    const uint64_t k_desc0 = smem_desc(smem_u32(skv), 16, 1024, kSwizzle128B);
+    int kvc = 0;   // lists whose K was awaited
+    for (int t = 0;; ++t) {
+      const int ds = t % kDesc;
+      if (!__all_sync(0xffffffffu, mbar_wait(&d_full[ds], (t / kDesc) & 1, wc))) break;
+      const Desc& dd = desc[ds];
+      const int end = dd.end, kvs = dd.kvs, first = dd.first_of_kv, last = dd.last_of_kv;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&d_empty[ds]);
+      if (end) break;
+      const int qs = t % kQStages;
+      if (first) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&k_full[kvs], (kvc / kKVStages) & 1, wc))) break;
+        ++kvc;
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait(&q_full[qs], (t / kQStages) & 1, wc))) break;
+      // S(t) reuses the single S buffer once the softmax has loaded S(t-1).
+      if (!__all_sync(0xffffffffu, mbar_wait(s_free, (t & 1) ^ 1, wc))) break;
+      tc_fence_after();
+      const uint64_t qd = q_desc0 + ((qs * Cfg::kQBytes) >> 4);
+      const uint64_t kd = k_desc0 + ((kvs * 2 * Cfg::kKVBytes) >> 4);
+      const bool leader = elect_one();
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t off = (ks / 4) * (128 * 128) + (ks % 4) * 32;
-          const uint32_t koff = (ks / 4) * (BK * 128) + (ks % 4) * 32;
-          umma_ss(tmem + Cfg::kColS, qd + (off >> 4), kd + (koff >> 4), idesc_s, ks > 0 ? 1u : 0u);
-        }
+      for (int ks = 0; ks < D / 16; ++ks) {
+        const uint32_t off = (ks / 4) * (128 * 128) + (ks % 4) * 32;
+        const uint32_t koff = (ks / 4) * (BK * 128) + (ks % 4) * 32;
+        if (leader) umma_ss(tmem + Cfg::kColS, qd + (off >> 4), kd + (koff >> 4), idesc_s, ks > 0 ? 1u : 0u);
+      }
+      if (leader) {
         umma_commit(&q_empty[qs]);
         umma_commit(s_full);
         if (last) umma_commit(&k_empty[kvs]);   // this list's last read of K
       }
+      __syncwarp();
     }
   } else if (warp == kPvW) {
     // ---------------------------------------------------------------- UMMA: O = P V
-    if (lane == 0) {
-      constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
-      const uint64_t v_desc0 = smem_desc(smem_u32(skv) + Cfg::kKVBytes, BK * 128, 1024, kSwizzle128B);
-      int vc = 0;   // lists whose V was awaited
-      for (int t = 0;; ++t) {
-        const int ds = t % kDesc;
-        if (!mbar_wait(&d_full[ds], (t / kDesc) & 1, wc)) break;
-        const Desc& dd = desc[ds];
-        const int end = dd.end, kvs = dd.kvs, first = dd.first_of_kv, last = dd.last_of_kv;
-        mbar_arrive(&d_empty[ds]);
-        if (end) break;
-        const int sb = t & 1;
-        if (first) {
-          if (!mbar_wait(&v_full[kvs], (vc / kKVStages) & 1, wc)) break;
-          ++vc;
-        }
-        if (!mbar_wait(&p_full[sb], (t >> 1) & 1, wc)) break;
-        if (!mbar_wait(&o_free[sb], ((t >> 1) & 1) ^ 1, wc)) break;
-        tc_fence_after();
-        const uint64_t vd = v_desc0 + ((kvs * 2 * Cfg::kKVBytes) >> 4);
-        const uint32_t p_tmem = tmem + Cfg::kColP + sb * (BK / 2);
-        const uint32_t o_tmem = tmem + Cfg::kColO + sb * D;
+    constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
+    const uint64_t v_desc0 = smem_desc(smem_u32(skv) + Cfg::kKVBytes, BK * 128, 1024, kSwizzle128B);
+    int vc = 0;   // lists whose V was awaited
+    for (int t = 0;; ++t) {
+      const int ds = t % kDesc;
+      if (!__all_sync(0xffffffffu, mbar_wait(&d_full[ds], (t / kDesc) & 1, wc))) break;
+      const Desc& dd = desc[ds];
+      const int end = dd.end, kvs = dd.kvs, first = dd.first_of_kv, last = dd.last_of_kv;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&d_empty[ds]);
+      if (end) break;
+      const int sb = t & 1;
+      if (first) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&v_full[kvs], (vc / kKVStages) & 1, wc))) break;
+        ++vc;
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait(&p_full[sb], (t >> 1) & 1, wc))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&o_free[sb], ((t >> 1) & 1) ^ 1, wc))) break;
+      tc_fence_after();
+      const uint64_t vd = v_desc0 + ((kvs * 2 * Cfg::kKVBytes) >> 4);
+      const uint32_t p_tmem = tmem + Cfg::kColP + sb * (BK / 2);
+      const uint32_t o_tmem = tmem + Cfg::kColO + sb * D;
+      const bool leader = elect_one();
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk)
-          umma_ts(o_tmem, p_tmem + kk * 8, vd + ((kk * 2048) >> 4), idesc_o, kk > 0 ? 1u : 0u);
+      for (int kk = 0; kk < BK / 16; ++kk)
+        if (leader) umma_ts(o_tmem, p_tmem + kk * 8, vd + ((kk * 2048) >> 4), idesc_o, kk > 0 ? 1u : 0u);
+      if (leader) {
         umma_commit(&o_full[sb]);
         umma_commit(&p_free[sb]);
         if (last) umma_commit(&v_empty[kvs]);   // this list's last read of V
       }
+      __syncwarp();
     }
   } else if (warp >= kSoftW0 && warp < kEpiW0) {
     // ---------------------------------------------------------------- softmax

@@ -178,33 +178,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- UMMA
-    if (lane == 0 && n_ktiles > 0) {
+    // The whole warp runs the loop (warp-uniform waits and descriptor math)
+    // and one elected lane issues: a single-lane divergent issue loop loses
+    // most of its issue slots to the two epilogue warps on this SMSP
+    // (measured: 108 against 272 cycles per MMA with three busy warps).
+    if (n_ktiles > 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(kRows, kKeys, false, false);
       constexpr uint32_t sbo = 8 * Cfg::kSwB;   // 8-row core-matrix group stride
       // Descriptors differ only in the start-address field (address >> 4 in
-      // bits 0-13, no carry for shared-memory addresses): base + offset, so
-      // the issuing thread spends few instructions per MMA (it shares its
-      // SMSP's issue port with two epilogue warps).
+      // bits 0-13, no carry for shared-memory addresses): base + offset.
       const uint64_t q_desc0 = smem_desc(smem_u32(sq), 16, sbo, Cfg::kSwz);
       const uint64_t k_desc0 = smem_desc(smem_u32(sk), 16, sbo, Cfg::kSwz);
-      bool ok = mbar_wait(q_full, 0, wc);
+      bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, wc));
       for (int t = 0; ok && t < n_ktiles; ++t) {
         const int s = t % Cfg::kStages;
         const int acc = t & 1;
-        if (!mbar_wait(&acc_empty[acc], ((t >> 1) & 1) ^ 1, wc)) break;
-        if (!mbar_wait(&full[s], (t / Cfg::kStages) & 1, wc)) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(&acc_empty[acc], ((t >> 1) & 1) ^ 1, wc))) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (t / Cfg::kStages) & 1, wc))) break;
         tc_fence_after();
         const uint64_t kd = k_desc0 + ((s * Cfg::kAtoms * kKeys * Cfg::kSwB) >> 4);
         const uint32_t d_tmem = tmem + acc * kKeys;
+        const bool leader = elect_one();
 #pragma unroll
         for (int ks = 0; ks < DIDX / 16; ++ks) {
           constexpr int kPerAtom = Cfg::kSwB / 32;
           const uint32_t aoff = ((ks / kPerAtom) * kRows * Cfg::kSwB + (ks % kPerAtom) * 32) >> 4;
           const uint32_t boff = ((ks / kPerAtom) * kKeys * Cfg::kSwB + (ks % kPerAtom) * 32) >> 4;
-          umma_ss(d_tmem, q_desc0 + aoff, kd + boff, idesc, ks > 0 ? 1u : 0u);
+          if (leader) umma_ss(d_tmem, q_desc0 + aoff, kd + boff, idesc, ks > 0 ? 1u : 0u);
         }
-        umma_commit(&empty[s]);       // smem stage free once these MMAs finish
-        umma_commit(&acc_full[acc]);  // accumulator ready for the epilogue
+        if (leader) {
+          umma_commit(&empty[s]);       // smem stage free once these MMAs finish
+          umma_commit(&acc_full[acc]);  // accumulator ready for the epilogue
+        }
+        __syncwarp();
       }
     }
   } else if (warp >= kEpiWarp0) {
