@@ -3,27 +3,27 @@
 // For every sequence b the query sits at position p = L_b - 1 of its own
 // contiguous caches.  The step is the prefill math of one row
 // (titansim.online summary of "MiniMax Sparse Attention": eq. (6) and the
-// local-block rule in section 4.2, eq. (8) in section 4.3), split so that the
-// HBM-bound scans use the whole GPU:
+// local-block rule in section 4.2, eq. (8) in section 4.3), as two persistent
+// HBM-streaming launches:
 //
-//   1. decode_index_kernel   grid (chunks of CB blocks, batch).  Streams the
-//      index-key cache once for all groups with 16-byte coalesced loads that
-//      feed mma.sync directly (a fixed permutation of the d_idx axis, applied
-//      to Q_idx and K_idx alike, makes each loaded 16-byte vector a fragment;
-//      the dot product does not depend on the order of d_idx).  Max-pools per
-//      block and keeps the chunk's top (k - 1) non-local blocks per group.
-//   2. merge (in the index kernel's last CTA of each sequence, found with an
-//      atomic counter): one warp per group takes the top (k - 1) of the chunk
-//      lists (score desc, block asc: exact because every global winner is a
-//      winner of its chunk), plus the local block, ascending.
-//   3. decode_attn_kernel    grid (splits, group x head tile, batch).  Each
-//      CTA stages whole K/V blocks with cp.async (16-byte, coalesced), shares
-//      them among the 16 heads of its head tile, and runs QK^T and PV on
-//      mma.sync with an fp32 online softmax; writes an (m, l, o) partial.
-//   4. combine (in the attention kernel's last CTA of each (sequence, group,
-//      head tile)): per head, the LSE-weighted sum of the split partials,
-//      rounded to bf16.
-// The dense run skips 1-2 and lets step 3 enumerate every causal block.
+//   1. decode_index_kernel   The blocks of all sequences, end to end, are cut
+//      into equal ranges, one per CTA.  Streams the index-key cache once for
+//      all groups with 16-byte coalesced loads that feed mma.sync directly (a
+//      fixed permutation of the d_idx axis, applied to Q_idx and K_idx alike,
+//      makes each loaded 16-byte vector a fragment; the dot product does not
+//      depend on the order of d_idx).  Max-pools per block and keeps, per
+//      (sequence, group) share, the top (k - 1) non-local blocks.  The CTA
+//      that completes a sequence's block count merges its shares (score desc,
+//      block asc: exact because every global winner wins within its share),
+//      adds the local block and writes the ids ascending.
+//   2. decode_attn_stream_kernel  The (sequence, group, head tile, slot)
+//      items are cut into equal ranges, one per CTA.  A producer warp
+//      TMA-loads the Q tile and the selected K/V block per item; four consumer
+//      warps run QK^T and PV on mma.sync with an fp32 online softmax.  A unit
+//      split between CTAs is merged by the last of them (LSE weights).
+// The dense run (every causal block) skips the index scan and uses
+// decode_attn_kernel: split-KV CTAs staging K/V with cp.async, combined by
+// the last split of each (sequence, group, head tile).
 #include <cstdint>
 #include <cuda_runtime.h>
 #include <mutex>
@@ -97,9 +97,9 @@ struct DecArgs {
   const int64_t* cu_kv;     // [B + 1]
   int32_t* block_ids;       // [B, h_kv, topk]
   uint16_t* o;              // [B, h_q, d]
-  float* cand_s;            // [idx_ctas + B, h_kv, kfree]
+  float* cand_s;            // [idx_ctas + B, h_kv, kfree] top-k candidates per (CTA, sequence) share
   int* cand_b;
-  float* part;              // [B, h_q, splits, d + 4]  (o[d], m, l, 2 pad)
+  float* part;              // dense: [B, h_q, splits, d + 4] (o[d], m, l, 2 pad); sparse: per-share rows
   int* seq_count;           // [B] index CTAs finished per sequence (zeroed per call)
   int* grp_count;           // [B, h_kv, head_tiles] attention CTAs finished (zeroed per call)
   int batch, h_q, h_kv, topk, causal, force_local, kfree, idx_ctas, idx_wmax;
@@ -1076,21 +1076,16 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
   }
 }
 
-// Split plan shared by the workspace query and the launch.
+// Split plan of the dense run, shared by the workspace query and the launch.
 struct SplitPlan {
   int splits, slots_per_split;
 };
 
-SplitPlan plan_splits(const msa_params& p, int max_kv, int dense) {
+SplitPlan plan_dense_splits(const msa_params& p, int max_kv) {
   SplitPlan s;
-  if (dense) {
-    const int nb = (max_kv + p.block_k - 1) / p.block_k;
-    s.splits = nb < 32 ? nb : 32;
-    s.slots_per_split = (nb + s.splits - 1) / s.splits;
-  } else {
-    s.splits = p.topk;
-    s.slots_per_split = 1;
-  }
+  const int nb = (max_kv + p.block_k - 1) / p.block_k;
+  s.splits = nb < 32 ? nb : 32;
+  s.slots_per_split = (nb + s.splits - 1) / s.splits;
   return s;
 }
 
@@ -1204,9 +1199,7 @@ size_t decode_counter_bytes(const msa_params& p, int batch) {
 size_t decode_workspace_bytes(const msa_params& p, int batch, int max_kv) {
   const int kfree = p.topk;   // upper bound on topk - force_local
   const size_t cand = static_cast<size_t>(plan_index(p, batch, max_kv).ctas + batch) * p.h_kv * kfree;
-  const SplitPlan sd = plan_splits(p, max_kv, 1), ss = plan_splits(p, max_kv, 0);
-  const int splits = sd.splits > ss.splits ? sd.splits : ss.splits;
-  const size_t part_dense = static_cast<size_t>(batch) * p.h_q * splits * (p.d + 4);
+  const size_t part_dense = static_cast<size_t>(batch) * p.h_q * plan_dense_splits(p, max_kv).splits * (p.d + 4);
   const long long T = stream_items(p, batch);
   const long long units = T / p.topk;
   const size_t part_stream = static_cast<size_t>(stream_ctas(T) + units) * 16 * (p.d + 4);
@@ -1242,7 +1235,7 @@ int run_sparse_attn_decode(const msa_params& p, const void* q, const void* q_idx
   const IdxPlan ip = plan_index(p, batch, max_kv);
   a.idx_ctas = ip.ctas;
   a.idx_wmax = ip.wmax;
-  const SplitPlan sp = plan_splits(p, max_kv, dense);
+  const SplitPlan sp = plan_dense_splits(p, max_kv);   // read by the dense run only
   a.splits = sp.splits;
   a.slots_per_split = sp.slots_per_split;
   a.dense = dense;
