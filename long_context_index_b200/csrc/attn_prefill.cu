@@ -194,52 +194,68 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- UMMA
-    if (lane == 0 && nblk > 0) {
+    // The whole warp runs the loop (warp-uniform waits and descriptor math)
+    // and one elected lane issues: a divergent single-lane issue loop loses
+    // most of its issue slots to the softmax warps sharing this SMSP.
+    if (nblk > 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, BK, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
-      const uint32_t sq_addr = smem_u32(sq);
-      const uint32_t skv_addr = smem_u32(skv);
-      bool ok = mbar_wait(q_full, 0, wc);
+      // Descriptors differ only in their start-address field (address >> 4,
+      // bits 0-13): a base plus an offset.
+      const uint64_t q_desc0 = smem_desc(smem_u32(sq), 16, 1024, kSwizzle128B);
+      const uint64_t k_desc0 = smem_desc(smem_u32(skv), 16, 1024, kSwizzle128B);
+      const uint64_t v_desc0 = smem_desc(smem_u32(skv) + Cfg::kKVBytes, BK * 128, 1024, kSwizzle128B);
+      bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, wc));
       auto issue_pv = [&](int j) -> bool {
         const int s = j % kStages;
         const int sb = j & 1;
-        if (!mbar_wait(&p_full[sb], (j >> 1) & 1, wc)) return false;
+        if (!__all_sync(0xffffffffu, mbar_wait(&p_full[sb], (j >> 1) & 1, wc))) return false;
         tc_fence_after();
-        const uint32_t sv_addr = skv_addr + s * 2 * Cfg::kKVBytes + Cfg::kKVBytes;
+        const uint64_t vd = v_desc0 + ((s * 2 * Cfg::kKVBytes) >> 4);
         const uint32_t p_tmem = tmem + (sb ? Cfg::kColS1 : Cfg::kColS0);
+        const bool leader = elect_one();
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
           // B = V block, MN-major: 16 keys per step = 2048 bytes; d atoms are BK*128 bytes apart.
-          const uint64_t bdesc = smem_desc(sv_addr + kk * 2048, BK * 128, 1024, kSwizzle128B);
-          umma_ts(tmem + Cfg::kColO, p_tmem + kk * 8, bdesc, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+          if (leader)
+            umma_ts(tmem + Cfg::kColO, p_tmem + kk * 8, vd + ((kk * 2048) >> 4), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&kv_empty[s]);
-        umma_commit(&s_free[sb]);
-        umma_commit(o_done);
+        if (leader) {
+          umma_commit(&kv_empty[s]);
+          umma_commit(&s_free[sb]);
+          umma_commit(o_done);
+        }
+        __syncwarp();
         return true;
       };
       for (int j = 0; ok && j < nblk; ++j) {
         const int s = j % kStages;
         const int sb = j & 1;
-        if (!mbar_wait(&kv_full[s], (j / kStages) & 1, wc)) break;
-        if (!mbar_wait(&s_free[sb], ((j >> 1) & 1) ^ 1, wc)) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(&kv_full[s], (j / kStages) & 1, wc))) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(&s_free[sb], ((j >> 1) & 1) ^ 1, wc))) break;
         tc_fence_after();
-        const uint32_t sk_addr = skv_addr + s * 2 * Cfg::kKVBytes;
+        const uint64_t kd = k_desc0 + ((s * 2 * Cfg::kKVBytes) >> 4);
+        const bool leader = elect_one();
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-          const int atom = ks / 4;
-          const uint32_t koff = (ks % 4) * 32;
-          const uint64_t adesc = smem_desc(sq_addr + atom * 128 * 128 + koff, 16, 1024, kSwizzle128B);
-          const uint64_t bdesc = smem_desc(sk_addr + atom * BK * 128 + koff, 16, 1024, kSwizzle128B);
-          umma_ss(tmem + (sb ? Cfg::kColS1 : Cfg::kColS0), adesc, bdesc, idesc_s, ks > 0 ? 1u : 0u);
+          const uint32_t aoff = ((ks / 4) * 128 * 128 + (ks % 4) * 32) >> 4;
+          const uint32_t boff = ((ks / 4) * BK * 128 + (ks % 4) * 32) >> 4;
+          if (leader)
+            umma_ss(tmem + (sb ? Cfg::kColS1 : Cfg::kColS0), q_desc0 + aoff, kd + boff, idesc_s, ks > 0 ? 1u : 0u);
         }
-        umma_commit(&s_full[sb]);
+        if (leader) umma_commit(&s_full[sb]);
+        __syncwarp();
         if (j > 0 && !issue_pv(j - 1)) {
           ok = false;
           break;
         }
       }
-      if (ok && issue_pv(nblk - 1)) umma_commit(o_final);
+      if (ok) {
+        const bool done = issue_pv(nblk - 1);
+        const bool leader = elect_one();   // the same lane that issued the MMAs
+        if (done && leader) umma_commit(o_final);
+        __syncwarp();
+      }
     }
   } else if (warp >= kSoftWarp0) {
     // ---------------------------------------------------------------- softmax + epilogue
