@@ -38,10 +38,14 @@ DECODE = WORKLOADS["decode_b64_64k_128k"]
 
 
 def cases(name):
-    """The bench workload, or a smaller instance of the same kernels for ncu
-    captures ("small": 32K prefill and 8 decode sequences)."""
+    """The bench workload, a smaller instance of the same kernels for ncu
+    captures ("small": 32K prefill and 8 decode sequences), or the long-context
+    pair ("long": the last 8192 queries of a 2^20-token chunked prefill and a
+    batch of 8 sequences decoding at 2^20)."""
     if name == "small":
-        return WORKLOADS["prefill_32k"], Workload(**{**DECODE.__dict__, "batch": 8})
+        return WORKLOADS["prefill_32k"], Workload(**{**DECODE.__dict__, "batch": 8, "name": "decode_b8"})
+    if name == "long":
+        return WORKLOADS["chunked_prefill_1m"], WORKLOADS["decode_b8_1m"]
     return PREFILL, DECODE
 
 
@@ -171,7 +175,9 @@ def run_ours(args, rank, world, torch, dist):
     td = make_decode(wd)
     pp = msa.Params.make(wp.h_q, wp.h_kv, wp.d, wp.d_idx, wp.block_k, wp.topk)
     pd = msa.Params.make(wd.h_q, wd.h_kv, wd.d, wd.d_idx, wd.block_k, wd.topk)
-    n = wp.n_q
+    n = wp.n_q                 # prefill query rows
+    n_kv = tp["k"].shape[0]    # prefill keys (n_kv > n: a chunk at the end of a longer context)
+    q_pos0 = int(tp["q_pos0"])
     B = wd.batch
     max_kv = int(td["lens"].max())
 
@@ -185,15 +191,15 @@ def run_ours(args, rank, world, torch, dist):
     o = torch.empty((n, wp.h_q, wp.d), dtype=torch.bfloat16, device=dev)
     dids = torch.empty((B, wd.h_kv, wd.topk), dtype=torch.int32, device=dev)
     do = torch.empty((B, wd.h_q, wd.d), dtype=torch.bfloat16, device=dev)
-    ws_i = torch.empty(msa.workspace_size(msa.OP_INDEX_TOPK, pp, n, n), dtype=torch.uint8, device=dev)
-    ws_p = torch.empty(max(256, msa.workspace_size(msa.OP_PREFILL, pp, n, n)), dtype=torch.uint8, device=dev)
+    ws_i = torch.empty(msa.workspace_size(msa.OP_INDEX_TOPK, pp, n, n_kv), dtype=torch.uint8, device=dev)
+    ws_p = torch.empty(max(256, msa.workspace_size(msa.OP_PREFILL, pp, n, n_kv)), dtype=torch.uint8, device=dev)
     ws_d = torch.empty(msa.workspace_size(msa.OP_DECODE, pd, batch=B, max_kv=max_kv), dtype=torch.uint8,
                        device=dev)
 
     def step():
-        msa.index_topk(pp, d_in["q_idx"], d_in["k_idx"], 0, block_ids=ids, ws=ws_i)
+        msa.index_topk(pp, d_in["q_idx"], d_in["k_idx"], q_pos0, block_ids=ids, ws=ws_i)
         ev[1].record(stream)
-        msa.sparse_attn_prefill(pp, d_in["q"], d_in["k"], d_in["v"], ids, 0, out=o, ws=ws_p)
+        msa.sparse_attn_prefill(pp, d_in["q"], d_in["k"], d_in["v"], ids, q_pos0, out=o, ws=ws_p)
         ev[2].record(stream)
         msa.sparse_attn_decode(pd, dd["q"], dd["q_idx"], dd["k_cache"], dd["v_cache"], dd["k_idx_cache"],
                                dd["cu_kv"], max_kv, block_ids=dids, out=do, ws=ws_d)
@@ -243,8 +249,8 @@ def run_ours(args, rank, world, torch, dist):
     # ---- useful work of this step (from the ids of the last step)
     ids_h = ids.cpu().numpy()
     dids_h = dids.cpu().numpy()
-    f_idx = flops.index_flops(n, n, 0, wp.h_kv, wp.d_idx)
-    sel = flops.selected_keys(ids_h, wp.block_k, n, 0)
+    f_idx = flops.index_flops(n, n_kv, q_pos0, wp.h_kv, wp.d_idx)
+    sel = flops.selected_keys(ids_h, wp.block_k, n_kv, q_pos0)
     f_main = flops.main_flops(sel, wp.h_q, wp.h_kv, wp.d)
     b_dec = flops.decode_bytes(td["lens"], dids_h, wd.h_q, wd.h_kv, wd.d, wd.d_idx, wd.block_k)
 
@@ -253,7 +259,7 @@ def run_ours(args, rank, world, torch, dist):
     if not args.no_dense:
         e0, e1, e2 = E(enable_timing=True), E(enable_timing=True), E(enable_timing=True)
         e0.record(stream)
-        msa.sparse_attn_prefill(pp, d_in["q"], d_in["k"], d_in["v"], None, 0, out=o, ws=ws_p)
+        msa.sparse_attn_prefill(pp, d_in["q"], d_in["k"], d_in["v"], None, q_pos0, out=o, ws=ws_p)
         e1.record(stream)
         msa.sparse_attn_decode(pd, dd["q"], None, dd["k_cache"], dd["v_cache"], None, dd["cu_kv"], max_kv,
                                dense=True, out=do, ws=ws_d)
@@ -274,8 +280,8 @@ def run_ours(args, rank, world, torch, dist):
             d_in[k_].view(torch.int16).copy_(t_, non_blocking=True)
         for k_, t_ in hostd.items():
             dd[k_].view(t_.dtype).copy_(t_, non_blocking=True)
-        msa.index_topk(pp, d_in["q_idx"], d_in["k_idx"], 0, block_ids=ids, ws=ws_i)
-        msa.sparse_attn_prefill(pp, d_in["q"], d_in["k"], d_in["v"], ids, 0, out=o, ws=ws_p)
+        msa.index_topk(pp, d_in["q_idx"], d_in["k_idx"], q_pos0, block_ids=ids, ws=ws_i)
+        msa.sparse_attn_prefill(pp, d_in["q"], d_in["k"], d_in["v"], ids, q_pos0, out=o, ws=ws_p)
         msa.sparse_attn_decode(pd, dd["q"], dd["q_idx"], dd["k_cache"], dd["v_cache"], dd["k_idx_cache"],
                                dd["cu_kv"], max_kv, block_ids=dids, out=do, ws=ws_d)
         out_h.copy_(o.view(torch.int16), non_blocking=True)
@@ -314,7 +320,7 @@ def run_ours(args, rank, world, torch, dist):
     dom = max(kern, key=lambda k_: kern[k_]["ms"])
     dk = kern[dom]
     traffic = None
-    if dom in TRAFFIC and TRAFFIC[dom][1] == src_digest(TRAFFIC[dom][2]):
+    if args.case == "full" and dom in TRAFFIC and TRAFFIC[dom][1] == src_digest(TRAFFIC[dom][2]):
         traffic = TRAFFIC[dom][0]
     line = {
         "metric": METRIC,
@@ -329,11 +335,13 @@ def run_ours(args, rank, world, torch, dist):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded; integer index inputs with planted needles)",
-        "config": {"workload": "%s + %s" % (wp.name, wd.name if wd.batch == 64 else "decode_b%d" % wd.batch),
-                   "seq_len": n, "decode_batch": B,
+        "config": {"workload": "%s + %s" % (wp.name, wd.name),
+                   "seq_len": n_kv, "prefill_rows": n, "decode_batch": B,
                    "h_q": wp.h_q, "h_kv": wp.h_kv, "d": wp.d, "d_idx": wp.d_idx, "block_k": wp.block_k,
                    "topk": wp.topk, "tokens_per_step": tokens_step,
-                   "l2": "inputs larger than L2 (Q alone 2 GiB; decode caches 13 GB), no flush"},
+                   "l2": "inputs larger than L2 (%.1f GB prefill inputs; %.1f GB decode caches), no flush"
+                         % (sum(t_.numel() * t_.element_size() for t_ in host.values()) / 1e9,
+                            sum(dd[k_].numel() * dd[k_].element_size() for k_ in ("k_cache", "v_cache", "k_idx_cache")) / 1e9)},
         "prefill": {"ms": t_idx + t_attn, "tokens_per_s": n * world / ((t_idx + t_attn) / 1e3),
                     "index_ms": t_idx, "attn_ms": t_attn, "useful_tflop": (f_idx + f_main) / 1e12,
                     "tensor_frac": (f_idx + f_main) / ((t_idx + t_attn) / 1e3) / 1e12 / peaks["bf16_tflops"]},
@@ -348,7 +356,6 @@ def run_ours(args, rank, world, torch, dist):
         "kernels": {k_: {kk: vv for kk, vv in v_.items() if kk != "work"} for k_, v_ in kern.items()},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "note": "prefill inputs and outputs cross PCIe every step; decode KV caches stay resident"},
-        # ours per step: index 1; sparse prefill 5 (count, scan, fill, KV-outer, merge); decode 4
         # Per step: index top-k (1); sparse prefill: schedule count, scan and
         # fill (3), block-major attention (1), partial merge (1); decode:
         # persistent index scan with the merge folded in (1), persistent
@@ -423,7 +430,7 @@ def main():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--case", choices=["full", "small"], default="full")
+    ap.add_argument("--case", choices=["full", "small", "long"], default="full")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
