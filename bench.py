@@ -57,7 +57,7 @@ L2_BYTES = 126 * 1024 * 1024
 TRAFFIC = {
     # schedule + KV-outer + merge (msa_sparse_attn_prefill) at 128K, from
     # profiles/bench_prefill_128k_decode_b64_launches.md
-    "attn_prefill": (10.672e9 + 35.566e9 + 35.022e9 + 2.142e9 + 0.080e9, "6d4766b068df", "attn_sparse.cu"),
+    "attn_prefill": (10.672e9 + 35.566e9 + 35.022e9 + 2.142e9 + 0.080e9, "a45989db703f", "attn_sparse.cu"),
 }
 
 

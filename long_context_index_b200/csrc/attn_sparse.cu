@@ -14,24 +14,29 @@
 //      at any moment the CTAs gather the queries of one wave of kWave rows,
 //      whose Q rows (kWave x h_q x d x 2 bytes) stay resident in L2.
 //   2. attn_kvouter_kernel (persistent, warp-specialised, tcgen05):
-//      * warp 0 grabs the next (r, b) list with an atomic counter, loads
-//        K_b, V_b once by TMA, then streams chunks of 128/G queries of the
-//        list (each query's G head rows of group r are one 3-D TMA box), and
-//        publishes a descriptor per chunk in a 4-deep ring.
-//      * warp 1 issues S = Q K_b^T into the TMEM S buffer, and O = P V_b (P
-//        read from one of two TMEM P buffers) into one of two TMEM O buffers.
-//        S is released as soon as the softmax has loaded it, so the next S
-//        MMA queues behind the previous PV and the tensor pipe stays fed.
+//      * warp 0 grabs the next (r, b) list with an atomic counter, loads K_b
+//        by TMA, then streams chunks of 128/G queries of the list (each
+//        query's G head rows of group r are one 3-D TMA box, gathered with an
+//        L2 evict-last policy into a 3-stage ring) and publishes a descriptor
+//        per chunk in an 8-deep ring; V_b follows the list's first chunk.  K
+//        and V have their own barriers, so the next list's K lands once the
+//        last S has read K while the last PV still reads V.
+//      * warp 1 issues S = Q K_b^T into the TMEM S buffer; warp 14 issues
+//        O = P V_b (P read from one of two TMEM P buffers) into one of two
+//        TMEM O buffers.  Both run their loops with the whole warp and issue
+//        from one elected lane with precomputed descriptors: a tcgen05.mma
+//        issuing thread slows with every busy warp on its SMSP.  S is
+//        released as soon as the softmax has loaded it.
 //      * warps 2..9 (softmax): two threads per row, each owning 64 of the 128
 //        columns; the exact softmax of the row over the block's visible keys
 //        (causal only in the local block); the two halves exchange only their
-//        max through shared memory; P is written over S; (m, l_lo, l_hi) go
-//        to the epilogue.  (The exponentials are MUFU-bound: 16 per clock per
-//        SM, so one 128x128 tile costs as many cycles as its two MMAs; two
-//        warps per SM sub-partition keep the MUFU pipe fed.)
+//        max through shared memory; P (bf16) goes to a P buffer; (m, l_lo,
+//        l_hi) go to the epilogue.  (The exponentials are MUFU-bound: 16 per
+//        clock per SM, so one 128x128 tile costs as many cycles as its two
+//        MMAs; two warps per SM sub-partition keep the MUFU pipe fed.)
 //      * warps 10..13 (epilogue): o = O / l in bf16 staged in shared memory and
-//        written by TMA as one contiguous 128-row tile per chunk
-//        (chunk-major partials), lse2 = m c + log2 l beside it.
+//        written by TMA (L2 evict-first) as one contiguous 128-row tile per
+//        chunk (chunk-major partials), lse2 = m c + log2 l beside it.
 //   3. merge_partials_kernel: per (query, group), O = sum_s 2^(lse2_s - L) o_s
 //      over the valid slots, L = log2 sum 2^lse2_s; rounded to bf16.  The
 //      schedule records, per (query, group, slot), the partial row it wrote.
