@@ -138,8 +138,8 @@ MSA_API int msa_sparse_attn_prefill(const msa_params* p, const void* q, const vo
  *                and block_ids is not written)
  *   block_ids    int32 [batch, h_kv, topk] output (may be NULL when dense)
  *   o            bf16 [batch, h_q, d] output
- * Every L_b must be in [1, max_kv].  With dense = 0, batch <= 4096 and
- * batch * max_kv < 2^31 (MSA_ERR_UNSUPPORTED otherwise).
+ * Every L_b must be in [1, max_kv].  h_kv <= 8; with dense = 0 also
+ * batch <= 4096 and batch * max_kv < 2^31 (MSA_ERR_UNSUPPORTED otherwise).
  */
 MSA_API int msa_sparse_attn_decode(const msa_params* p, const void* q, const void* q_idx, const void* k_cache,
                            const void* v_cache, const void* k_idx_cache, const int64_t* cu_kv, int batch,
