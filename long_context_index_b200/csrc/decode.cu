@@ -38,7 +38,7 @@ constexpr int kIdxThreads = 256;    // 8 warps
 constexpr int kIdxCtasPerSm = 3;
 constexpr int kIdxCtas = 148 * kIdxCtasPerSm;   // persistent index grid
 constexpr int kIdxWCap = 1024;      // blocks per index CTA held in shared memory
-constexpr int kIdxMaxBatch = 4096;  // sequences whose block prefix fits shared memory
+constexpr int kIdxMaxBatch = kDecodeMaxBatch;   // sequences whose block prefix fits shared memory
 constexpr int kAttnThreads = 128;   // 4 warps, 32 keys each
 constexpr int kMergeRegCand = 8;    // per-lane register cache of the merge
 constexpr float kLog2e = 1.4426950408889634f;
@@ -1211,7 +1211,7 @@ int run_sparse_attn_decode(const msa_params& p, const void* q, const void* q_idx
                            const void* v_cache, const void* k_idx_cache, const int64_t* cu_kv, int batch,
                            int max_kv, int dense, int32_t* block_ids, void* o, void* ws, size_t /*ws_bytes*/,
                            int* status, cudaStream_t stream) {
-  if (p.h_kv > 8) return MSA_ERR_UNSUPPORTED;
+  if (p.h_kv > kDecodeMaxGroups) return MSA_ERR_UNSUPPORTED;
   // TMA row coordinates of the caches are 32-bit.
   if (!dense && static_cast<long long>(batch) * max_kv > 0x7fffffffLL) return MSA_ERR_UNSUPPORTED;
   // The index scan keeps the block prefix of all sequences in shared memory.

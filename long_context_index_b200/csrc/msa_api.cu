@@ -148,6 +148,11 @@ int msa_sparse_attn_decode(const msa_params* p, const void* q, const void* q_idx
   if (rc) return rc;
   if (batch <= 0 || max_kv <= 0 || (dense != 0 && dense != 1)) return MSA_ERR_INVALID;
   if (max_kv > kMaxRows) return MSA_ERR_UNSUPPORTED;
+  if (p->h_kv > kDecodeMaxGroups) return MSA_ERR_UNSUPPORTED;
+  // Sparse: the block prefix of every sequence sits in shared memory, and TMA
+  // row coordinates of the caches are 32-bit.
+  if (!dense && (batch > kDecodeMaxBatch || static_cast<long long>(batch) * max_kv > 0x7fffffffLL))
+    return MSA_ERR_UNSUPPORTED;
   const size_t need = kWsHeader + align_up(decode_workspace_bytes(*p, batch, max_kv), 256);
   if ((rc = check_ws(ws, ws_bytes, need))) return rc;
   if (!q || !k_cache || !v_cache || !cu_kv || !o) return MSA_ERR_INVALID;

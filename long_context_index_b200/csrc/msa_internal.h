@@ -38,6 +38,9 @@ int run_sparse_attn_kvouter(const msa_params& p, const void* q, const CUtensorMa
                             size_t ws_bytes, int* status, cudaStream_t stream);
 
 // Decode step.
+// Limits of the decode kernels (checked on the host before any launch).
+constexpr int kDecodeMaxGroups = 8;     // h_kv: one index-scan warp per group
+constexpr int kDecodeMaxBatch = 4096;   // sparse: the block prefix of every sequence in shared memory
 size_t decode_counter_bytes(const msa_params& p, int batch);
 size_t decode_workspace_bytes(const msa_params& p, int batch, int max_kv);
 int run_sparse_attn_decode(const msa_params& p, const void* q, const void* q_idx, const void* k_cache,

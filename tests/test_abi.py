@@ -86,3 +86,12 @@ def test_prefill_and_decode_reject_bad_arguments():
     assert L.msa_sparse_attn_decode(C.byref(p), 16, 16, 16, 16, 16, 16, 4, 100, 0, 16, 16, 256, 10, None) == -4
     assert L.msa_sparse_attn_decode(C.byref(p), 16, None, 16, 16, None, 16, 4, 100, 0, None, 16, 256,
                                     1 << 30, None) == -1
+    # Decode limits, refused on the host before any launch: more than 8 groups;
+    # a sparse batch above 4096 or with batch * max_kv >= 2^31 (dense is fine).
+    wide = P(h_q=32, h_kv=16)
+    assert L.msa_sparse_attn_decode(C.byref(wide), 16, 16, 16, 16, 16, 16, 4, 100, 0, 16, 16, 256, 1 << 40,
+                                    None) == -2
+    assert L.msa_sparse_attn_decode(C.byref(p), 16, 16, 16, 16, 16, 16, 4097, 100, 0, 16, 16, 256, 1 << 40,
+                                    None) == -2
+    assert L.msa_sparse_attn_decode(C.byref(p), 16, 16, 16, 16, 16, 16, 4096, 1 << 20, 0, 16, 16, 256,
+                                    1 << 40, None) == -2
