@@ -8,10 +8,13 @@ HBM: the index branch and the main branch of a 128K-token causal prefill
 decode step of 64 sequences with KV lengths in [64K, 128K] (the same model
 shape).  Tokens per step = 131072 prefill + 64 decode tokens.
 
-Prints one JSON line (rank 0).  Under torchrun each rank runs its own
-independent problem (weak scaling, no data-path collective); the time is the
-max over ranks.  ``--impl reference`` times the fp64 CPU oracle on bounded
-samples of the same workload on the host cores instead.
+Prints one JSON line (rank 0).  ``--gpus N`` runs N ranks, one per GPU: under
+torchrun (WORLD_SIZE set) it must equal the world size; run directly with
+N > 1 it relaunches itself under torchrun with N processes.  Each rank runs
+its own independent problem of the same shape (weak scaling, no data-path
+collective); the time is the max over ranks.  ``--impl reference`` times the
+fp64 CPU oracle on bounded samples of the same workload on the host cores
+instead (rank 0 only).
 """
 from __future__ import annotations
 
@@ -39,9 +42,13 @@ DECODE = WORKLOADS["decode_b64_64k_128k"]
 
 def cases(name):
     """The bench workload, a smaller instance of the same kernels for ncu
-    captures ("small": 32K prefill and 8 decode sequences), or the long-context
+    captures ("small": 32K prefill and 8 decode sequences), the long-context
     pair ("long": the last 8192 queries of a 2^20-token chunked prefill and a
-    batch of 8 sequences decoding at 2^20)."""
+    batch of 8 sequences decoding at 2^20), or a tiny pair that runs in
+    seconds ("tiny": the 1K prefill and 4 short decode sequences)."""
+    if name == "tiny":
+        return WORKLOADS["tiny_prefill_1k"], Workload(**{**DECODE.__dict__, "batch": 4, "kv_min": 3000,
+                                                           "kv_max": 9000, "name": "decode_b4_short"})
     if name == "small":
         return WORKLOADS["prefill_32k"], Workload(**{**DECODE.__dict__, "batch": 8, "name": "decode_b8"})
     if name == "long":
@@ -52,13 +59,9 @@ def cases(name):
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_BYTES = 126 * 1024 * 1024
 
-# DRAM traffic per launch from the committed ncu captures, keyed by kernel,
-# with the digest of the kernel source it was measured on (stale -> null).
-TRAFFIC = {
-    # schedule + KV-outer + merge (msa_sparse_attn_prefill) at 128K, from
-    # profiles/bench_prefill_128k_decode_b64_launches.md
-    "attn_prefill": (10.672e9 + 35.566e9 + 35.022e9 + 2.142e9 + 0.080e9, "a45989db703f", "attn_sparse.cu"),
-}
+# DRAM bytes per call of the dominant unit, measured by ncu on the kernel
+# source with the given digest (a stale digest reports null).
+TRAFFIC = {}
 
 
 def load_peaks():
@@ -254,18 +257,33 @@ def run_ours(args, rank, world, torch, dist):
     f_main = flops.main_flops(sel, wp.h_q, wp.h_kv, wp.d)
     b_dec = flops.decode_bytes(td["lens"], dids_h, wd.h_q, wd.h_kv, wd.d, wd.d_idx, wd.block_k)
 
-    # ---- dense run of the same kernels (every causal block), once, untimed above
+    # ---- dense run (every causal block): the same call with no block ids
+    # (prefill) / dense = 1 (decode), warmed up and timed over as many steps
+    # as the sparse run, outside the sparse timed region
     t_dense_p = t_dense_d = None
     if not args.no_dense:
-        e0, e1, e2 = E(enable_timing=True), E(enable_timing=True), E(enable_timing=True)
-        e0.record(stream)
-        msa.sparse_attn_prefill(pp, d_in["q"], d_in["k"], d_in["v"], None, q_pos0, out=o, ws=ws_p)
-        e1.record(stream)
-        msa.sparse_attn_decode(pd, dd["q"], None, dd["k_cache"], dd["v_cache"], None, dd["cu_kv"], max_kv,
-                               dense=True, out=do, ws=ws_d)
-        e2.record(stream)
+        def dense_step(ev_):
+            ev_[0].record(stream)
+            msa.sparse_attn_prefill(pp, d_in["q"], d_in["k"], d_in["v"], None, q_pos0, out=o, ws=ws_p)
+            ev_[1].record(stream)
+            msa.sparse_attn_decode(pd, dd["q"], None, dd["k_cache"], dd["v_cache"], None, dd["cu_kv"], max_kv,
+                                   dense=True, out=do, ws=ws_d)
+            ev_[2].record(stream)
+
+        for _ in range(args.warmup):
+            dense_step([E(enable_timing=True) for _ in range(3)])
+        dev_ = [[E(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+        for s_ in range(args.steps):
+            dense_step(dev_[s_])
         torch.cuda.synchronize()
-        t_dense_p, t_dense_d = e0.elapsed_time(e1), e1.elapsed_time(e2)
+        t_dense_p = statistics.median(e[0].elapsed_time(e[1]) for e in dev_)
+        t_dense_d = statistics.median(e[1].elapsed_time(e[2]) for e in dev_)
+        for wsx in (ws_p, ws_d):
+            rc = msa.device_status(wsx)
+            if rc:
+                raise RuntimeError("device status %d after the dense runs" % rc)
+    med_pre = statistics.median(e[0].elapsed_time(e[2]) for e in evs)
+    med_dec = statistics.median(e[2].elapsed_time(e[3]) for e in evs)
 
     # ---- end to end through the public API with host buffers
     out_h = torch.empty((n, wp.h_q, wp.d), dtype=torch.int16).pin_memory()
@@ -348,8 +366,11 @@ def run_ours(args, rank, world, torch, dist):
         "decode": {"ms": t_dec, "tokens_per_s": B * world / (t_dec / 1e3), "bytes": b_dec,
                    "hbm_frac": b_dec / (t_dec / 1e3) / 1e9 / peaks["hbm_gbs"]},
         "dense": None if t_dense_p is None else {
-            "prefill_ms": t_dense_p, "decode_ms": t_dense_d,
-            "prefill_sparse_speedup": t_dense_p / (t_idx + t_attn), "decode_sparse_speedup": t_dense_d / t_dec},
+            "prefill_ms": t_dense_p, "decode_ms": t_dense_d, "steps": args.steps, "warmup": args.warmup,
+            "stat": "median per step; sparse medians %.3f ms prefill, %.4f ms decode" % (med_pre, med_dec),
+            "kernels": "prefill: query-outer tcgen05 flash kernel over every causal block (a block-major pass "
+                       "would write one partial per (query, block)); decode: split-KV kernel over every block",
+            "prefill_sparse_speedup": t_dense_p / med_pre, "decode_sparse_speedup": t_dense_d / med_dec},
         "roofline": {"kernel": dom, "bound": dk["bound"], "achieved": dk["achieved"], "peak": dk["peak"],
                      "unit": dk["unit"], "frac": dk["frac"], "traffic": traffic,
                      "peak_source": peak_src + (" burst" if dk["bound"] == "tensor" else "")},
@@ -395,6 +416,8 @@ def cpu_baseline(tp, td, wp, wd, rows_n=2048, seqs_n=32):
 def run_reference(args, rank, world):
     if rank != 0:
         return None
+    case = getattr(args, "case", "full") if args is not None else "full"
+    PREFILL, DECODE = cases(case)
     tp = make_prefill(PREFILL)
     td = make_decode(DECODE)
     threads = os.cpu_count() or 1
@@ -415,34 +438,56 @@ def run_reference(args, rank, world):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "prefill_128k + decode_b64_64k_128k", "seq_len": PREFILL.n_q,
+        "config": {"workload": "%s + %s" % (PREFILL.name, DECODE.name), "seq_len": PREFILL.n_kv,
                    "decode_batch": DECODE.batch},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                         "sample": "per step %d random rows of the 128K prefill (index + main branch) and %d "
-                                   "decode sequences" % (rows_n, seqs_n)},
+                         "sample": "per step %d random rows of the %s prefill (index + main branch) and %d "
+                                   "decode sequences" % (rows_n, PREFILL.name, seqs_n)},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
 
-def main():
+def relaunch_command(argv, n_gpus: int, port: int):
+    """The torchrun command that runs this bench with one process per GPU."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", str(n_gpus),
+            "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__)] + list(argv)
+
+
+def free_port() -> int:
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def main(argv=None):
+    argv = sys.argv[1:] if argv is None else argv
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--case", choices=["full", "small", "long"], default="full")
+    ap.add_argument("--case", choices=["full", "small", "long", "tiny"], default="full")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    args = ap.parse_args()
+    args = ap.parse_args(argv)
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        # Run directly with N > 1: one process per GPU under torchrun.
+        return subprocess.call(relaunch_command(argv, args.gpus, free_port()))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        sys.stderr.write("bench.py: --gpus %d but WORLD_SIZE=%d\n" % (args.gpus, world))
+        return 2
     if args.impl == "reference":
         line = run_reference(args, rank, world)
         if line is not None:
             print(json.dumps(line), flush=True)
-        return
+        return 0
     import torch
     import torch.distributed as dist
     from datetime import timedelta
@@ -456,7 +501,8 @@ def main():
     finally:
         if world > 1:
             dist.destroy_process_group()
+    return 0
 
 
 if __name__ == "__main__":
-    main()
+    sys.exit(main())

@@ -113,7 +113,9 @@ MSA_API int msa_index_topk(const msa_params* p, const void* q_idx, const void* k
  *             dense run (every causal block: eq. (1))
  *   o         bf16 [n_q, h_q, d] output (fp32 accumulation, rounded to
  *             nearest even)
- * Ids must be valid (each -1 or a block holding a visible key of the row).
+ * Ids must be valid: each -1 or a block holding a visible key of the row,
+ * and the non-negative ids of a (row, group) pairwise distinct (a repeated id
+ * would be attended twice; msa_index_topk never emits one).
  */
 MSA_API int msa_sparse_attn_prefill(const msa_params* p, const void* q, const void* k, const void* v,
                             const int32_t* block_ids, int n_q, int n_kv, int q_pos0, void* o, void* ws,
@@ -162,8 +164,13 @@ MSA_API int msa_device_status(const void* ws, void* stream);
  * exactly those of msa_sparse_attn_decode.
  *   * Scratch: a file-scope device array of MSA_NOALLOC_SCRATCH_BYTES that
  *     every GPU which loads the library holds until process exit.  A problem
- *     whose scratch would not fit (see msa_workspace_size(MSA_OP_DECODE, ...))
- *     is rejected with MSA_ERR_WORKSPACE before anything is launched.
+ *     whose scratch would not fit is rejected with MSA_ERR_WORKSPACE before
+ *     anything is launched.  The scratch is that of the run requested: the
+ *     sparse run needs completion counters, top-k candidates and one partial
+ *     per (attention CTA, group) share (64 q heads, 4 KV heads, d = 128,
+ *     k = 16: about 10 MB at 64 sequences); the dense run needs 32 split
+ *     partials per head.  msa_workspace_size(MSA_OP_DECODE, ...) reports the
+ *     larger of the two, an upper bound.
  *   * The first call on a device looks up the array's device address (once
  *     per device, with that device current); make that first call before any
  *     stream capture.

@@ -1,10 +1,15 @@
-// attn_prefill.cu -- main branch of a (chunked) prefill on sm_100a.
+// attn_prefill.cu -- main branch of a (chunked) prefill on sm_100a: the
+// dispatch between the sparse (block-major, attn_sparse.cu) and the dense
+// path, and the dense kernel itself.
 //
-// Computes, for every query row i and head h of group r = h / G (titansim.online
-// summary of "MiniMax Sparse Attention", eq. (8), section 4.3):
-//   O_i^(h) = softmax( Q_i^(h) K^(r)[I]^T / sqrt(d) ) V^(r)[I],
-// where I is the set of causally visible keys of the blocks selected for
-// (i, r) -- or of every causal block for the dense run (eq. (1)).
+// The dense run computes eq. (1) of the titansim.online summary of "MiniMax
+// Sparse Attention" (section 2.2) for GQA: for every query row i and head h of
+// group r = h / G,
+//   O_i^(h) = softmax( Q_i^(h) K^(r)[0..p_i]^T / sqrt(d) ) V^(r)[0..p_i],
+// i.e. eq. (8) with every causal block selected.  It is the baseline the
+// sparse path is measured against.  A block-major (KV-outer) pass over every
+// block would write one partial per (query, block) -- at 128K that is 2 TB --
+// so the dense run keeps the query as the outer loop.
 //
 // Kernel design (query-outer, GQA-packed):
 //   * One CTA owns a 128-row tile = QT = 128/G consecutive queries x the G
@@ -21,9 +26,8 @@
 //     the running max grows by more than 2^8 (otherwise P may exceed 1 by at
 //     most 256, which fp32 accumulation absorbs).  P is written back to TMEM as
 //     bf16 over the S buffer it came from.
-//   * The block list of a tile is either every causal block (dense) or the
-//     sorted union of the blocks its QT queries selected; a row masks every
-//     block its own query did not select, and keys after its position.
+//   * A tile walks every block up to its last query's position; a row masks
+//     the keys after its own position.
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -38,7 +42,6 @@ constexpr int kThreads = 256;   // 8 warps
 constexpr int kSoftWarp0 = 4;   // softmax warps 4..7
 constexpr int kStages = 2;      // K/V ring depth
 constexpr float kRescaleLog2 = 8.0f;
-constexpr int kMaxList = 1024;  // max union size (QT * topk <= 1024)
 
 template <int D, int BK>
 struct AttnCfg {
@@ -46,7 +49,7 @@ struct AttnCfg {
   static constexpr int kQBytes = 128 * D * 2;
   static constexpr int kKVBytes = BK * D * 2;
   static constexpr int kSmemData = kQBytes + kStages * 2 * kKVBytes;
-  static constexpr int kSmemBytes = kSmemData + 2 * kMaxList * 4 + 4096 + 1024;
+  static constexpr int kSmemBytes = kSmemData + 4096 + 1024;
   static constexpr int kTmemCols = (2 * BK + D) <= 256 ? 256 : 512;
   static constexpr int kColS0 = 0;
   static constexpr int kColS1 = BK;
@@ -54,10 +57,9 @@ struct AttnCfg {
 };
 
 struct AttnArgs {
-  const int32_t* block_ids;  // [n_q, h_kv, topk] or null (dense)
   uint16_t* o;               // [n_q, h_q, d]
   int* status;
-  int n_q, n_kv, q_pos0, h_q, h_kv, topk, causal;
+  int n_q, n_kv, q_pos0, h_q, h_kv, causal;
   int n_qtiles;
   float scale_log2;          // softmax scale * log2(e)
 };
@@ -72,9 +74,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sq = smem;                                   // [atoms][128 rows][128 B]
   uint8_t* skv = smem + Cfg::kQBytes;                   // [stage][K|V][atoms][BK rows][128 B]
-  int* s_list = reinterpret_cast<int*>(smem + Cfg::kSmemData);   // block list (sorted)
-  int* s_sel = s_list + kMaxList;                       // [QT][topk] selected ids of the tile's queries
-  uint64_t* bars = reinterpret_cast<uint64_t*>(s_sel + kMaxList);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kSmemData);
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;                         // [kStages]
   uint64_t* kv_empty = kv_full + kStages;               // [kStages]
@@ -85,7 +85,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* o_final = o_done + 1;                       // the last PV only
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_final + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
-  int* s_nblk = abort_flag + 1;
 
   const int warp = warp_id();
   const int lane = lane_id();
@@ -93,7 +92,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int r = static_cast<int>(blockIdx.x) % args.h_kv;
   const int i0 = qtile * QT;
   const int q_here = min(QT, args.n_q - i0);
-  const bool dense = args.block_ids == nullptr;
 
   // ---------------------------------------------------------------- setup
   if (threadIdx.x == 0) {
@@ -116,59 +114,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(tmem_slot, Cfg::kTmemCols);
     tmem_relinquish();
   }
-  // Block list of the tile.
-  const int p_first = args.q_pos0 + i0;
-  const int p_last = p_first + q_here - 1;
+  // Blocks of the tile: every block up to its last query's position.
+  const int p_last = args.q_pos0 + i0 + q_here - 1;
   const int nb_total = (args.n_kv + BK - 1) / BK;
-  if (dense) {
-    if (threadIdx.x == 0) *s_nblk = args.causal ? (p_last / BK + 1) : nb_total;
-  } else {
-    const int nsel = q_here * args.topk;
-    for (int t = threadIdx.x; t < QT * args.topk; t += kThreads) {
-      const int qi = t / args.topk;
-      const int v = t < nsel ? args.block_ids[(static_cast<size_t>(i0 + qi) * args.h_kv + r) * args.topk +
-                                              (t % args.topk)]
-                             : -1;
-      s_sel[t] = v;
-      s_list[t] = v < 0 ? 0x7fffffff : v;
-    }
-    __syncthreads();
-    // Bitonic sort of the (power-of-two padded) id list.
-    int n2 = 1;
-    while (n2 < QT * args.topk) n2 <<= 1;
-    for (int t = QT * args.topk + threadIdx.x; t < n2; t += kThreads) s_list[t] = 0x7fffffff;
-    __syncthreads();
-    for (int k = 2; k <= n2; k <<= 1) {
-      for (int j = k >> 1; j > 0; j >>= 1) {
-        for (int t = threadIdx.x; t < n2; t += kThreads) {
-          const int u = t ^ j;
-          if (u > t) {
-            const int a = s_list[t], b = s_list[u];
-            const bool up = (t & k) == 0;
-            if ((a > b) == up) {
-              s_list[t] = b;
-              s_list[u] = a;
-            }
-          }
-        }
-        __syncthreads();
-      }
-    }
-    if (threadIdx.x == 0) {
-      int n = 0;
-      for (int t = 0; t < n2; ++t) {
-        const int v = s_list[t];
-        if (v == 0x7fffffff) break;
-        if (n == 0 || s_list[n - 1] != v) s_list[n++] = v;
-      }
-      *s_nblk = n;
-    }
-  }
+  const int nblk = args.causal ? min(p_last / BK + 1, nb_total) : nb_total;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int nblk = *s_nblk;
   const WaitCtx wc{abort_flag, args.status};
 
   if (warp == 0) {
@@ -181,7 +134,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int a = 0; a < Cfg::kAtoms; ++a) tma_load_3d(sq + a * 128 * 128, &tm_q, q_full, a * 64, r * G, i0);
       for (int j = 0; j < nblk; ++j) {
         const int s = j % kStages;
-        const int b = dense ? j : s_list[j];
+        const int b = j;
         if (!mbar_wait(&kv_empty[s], ((j / kStages) & 1) ^ 1, wc)) break;
         mbar_arrive_expect_tx(&kv_full[s], 2 * Cfg::kKVBytes);
         uint8_t* sk = skv + s * 2 * Cfg::kKVBytes;
@@ -270,19 +223,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float c = args.scale_log2;
     float m_run = __int_as_float(0xff800000);  // running max of raw scores (-inf)
     float l_run = 0.f;
-    const int* my_sel = s_sel + qi * args.topk;
 
     for (int j = 0; j < nblk; ++j) {
       const int sb = j & 1;
-      const int b = dense ? j : s_list[j];
-      // Is block b selected for this row's query?
-      bool row_sel = row_ok;
-      if (!dense && row_ok) {
-        row_sel = false;
-        for (int t = 0; t < args.topk; ++t) row_sel |= my_sel[t] == b;
-      }
-      const int kb0 = b * BK;
-      const int lim = row_sel ? min(BK, kv_lim - kb0) : 0;   // valid keys of this block for the row
+      const int kb0 = j * BK;
+      const int lim = row_ok ? min(BK, kv_lim - kb0) : 0;   // valid keys of this block for the row
       if (!mbar_wait(&s_full[sb], (j >> 1) & 1, wc)) break;
       tc_fence_after();
       uint32_t sv[BK];
@@ -450,7 +395,6 @@ int run_sparse_attn_prefill(const msa_params& p, const void* q, const void* k, c
   if (block_ids)   // sparse: block-major schedule (attn_sparse.cu)
     return run_sparse_attn_kvouter(p, q, tk, tv, block_ids, n_q, n_kv, q_pos0, o, ws, ws_bytes, status, stream);
   AttnArgs a;
-  a.block_ids = block_ids;
   a.o = static_cast<uint16_t*>(o);
   a.status = status;
   a.n_q = n_q;
@@ -458,7 +402,6 @@ int run_sparse_attn_prefill(const msa_params& p, const void* q, const void* k, c
   a.q_pos0 = q_pos0;
   a.h_q = p.h_q;
   a.h_kv = p.h_kv;
-  a.topk = p.topk;
   a.causal = p.causal;
   a.n_qtiles = (n_q + QT - 1) / QT;
   const float scale = p.scale > 0.f ? p.scale : 1.0f / sqrtf(static_cast<float>(p.d));

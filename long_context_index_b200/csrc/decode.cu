@@ -1196,15 +1196,21 @@ size_t decode_counter_bytes(const msa_params& p, int batch) {
   return align_up(n * 4, 256);
 }
 
-size_t decode_workspace_bytes(const msa_params& p, int batch, int max_kv) {
+// Workspace of one call: the counters, then the sparse run's top-k candidates
+// and per-share partials, or the dense run's split partials.  dense < 0 gives
+// the larger of the two (what msa_workspace_size reports, since it does not
+// know which run the caller will make).
+size_t decode_workspace_bytes(const msa_params& p, int batch, int max_kv, int dense) {
   const int kfree = p.topk;   // upper bound on topk - force_local
   const size_t cand = static_cast<size_t>(plan_index(p, batch, max_kv).ctas + batch) * p.h_kv * kfree;
   const size_t part_dense = static_cast<size_t>(batch) * p.h_q * plan_dense_splits(p, max_kv).splits * (p.d + 4);
   const long long T = stream_items(p, batch);
   const long long units = T / p.topk;
   const size_t part_stream = static_cast<size_t>(stream_ctas(T) + units) * 16 * (p.d + 4);
-  const size_t part = part_dense > part_stream ? part_dense : part_stream;
-  return decode_counter_bytes(p, batch) + align_up(cand * 4, 256) * 2 + align_up(part * 4, 256);
+  const size_t sparse = align_up(cand * 4, 256) * 2 + align_up(part_stream * 4, 256);
+  const size_t dense_b = align_up(cand * 4, 256) * 2 + align_up(part_dense * 4, 256);
+  const size_t body = dense > 0 ? dense_b : (dense == 0 ? sparse : (sparse > dense_b ? sparse : dense_b));
+  return decode_counter_bytes(p, batch) + body;
 }
 
 int run_sparse_attn_decode(const msa_params& p, const void* q, const void* q_idx, const void* k_cache,

@@ -103,7 +103,7 @@ size_t msa_workspace_size(int op, const msa_params* p, int n_q, int n_kv, int ba
       return kWsHeader + align_up(prefill_workspace_bytes(*p, n_q, n_kv), 256);
     case MSA_OP_DECODE:
       if (batch <= 0 || max_kv <= 0 || max_kv > kMaxRows) return 0;
-      return kWsHeader + align_up(decode_workspace_bytes(*p, batch, max_kv), 256);
+      return kWsHeader + align_up(decode_workspace_bytes(*p, batch, max_kv, -1), 256);
     default:
       return 0;
   }
@@ -153,7 +153,8 @@ int msa_sparse_attn_decode(const msa_params* p, const void* q, const void* q_idx
   // row coordinates of the caches are 32-bit.
   if (!dense && (batch > kDecodeMaxBatch || static_cast<long long>(batch) * max_kv > 0x7fffffffLL))
     return MSA_ERR_UNSUPPORTED;
-  const size_t need = kWsHeader + align_up(decode_workspace_bytes(*p, batch, max_kv), 256);
+  // The call needs only the scratch of the run it makes (sparse or dense).
+  const size_t need = kWsHeader + align_up(decode_workspace_bytes(*p, batch, max_kv, dense), 256);
   if ((rc = check_ws(ws, ws_bytes, need))) return rc;
   if (!q || !k_cache || !v_cache || !cu_kv || !o) return MSA_ERR_INVALID;
   if (!dense && (!q_idx || !k_idx_cache || !block_ids)) return MSA_ERR_INVALID;

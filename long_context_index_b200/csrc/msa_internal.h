@@ -42,7 +42,8 @@ int run_sparse_attn_kvouter(const msa_params& p, const void* q, const CUtensorMa
 constexpr int kDecodeMaxGroups = 8;     // h_kv: one index-scan warp per group
 constexpr int kDecodeMaxBatch = 4096;   // sparse: the block prefix of every sequence in shared memory
 size_t decode_counter_bytes(const msa_params& p, int batch);
-size_t decode_workspace_bytes(const msa_params& p, int batch, int max_kv);
+// dense: 1 = the dense run, 0 = the sparse run, -1 = the larger of the two.
+size_t decode_workspace_bytes(const msa_params& p, int batch, int max_kv, int dense);
 int run_sparse_attn_decode(const msa_params& p, const void* q, const void* q_idx, const void* k_cache,
                            const void* v_cache, const void* k_idx_cache, const int64_t* cu_kv, int batch,
                            int max_kv, int dense, int32_t* block_ids, void* o, void* ws, size_t ws_bytes,

@@ -338,25 +338,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return r;
 }
 
-// 2^x on the FMA/ALU pipes (x <= 0 or -inf), to offload the MUFU unit.
-// Cody-Waite style range reduction: n = nearest integer to x via the 1.5*2^23
-// rounding constant, f = x - n in [-1/2, 1/2], 2^f from a degree-3 polynomial,
-// and 2^n added to the exponent field.  The coefficients are a weighted
-// least-squares fit of 2^f on [-1/2, 1/2] minimising relative error (Lawson
-// reweighting on Chebyshev nodes); max relative error 7.5e-5, far below the
-// bf16 rounding of P.  x < -126 returns 0 (masked keys, negligible terms).
-__device__ __forceinline__ float exp2_poly(float x) {
-  const float t = x + 12582912.0f;
-  const float n = t - 12582912.0f;
-  const float f = x - n;
-  float p = fmaf(0.05517148971557617f, f, 0.2426111102104187f);
-  p = fmaf(p, f, 0.6932610273361206f);
-  p = fmaf(p, f, 0.9999280571937561f);
-  const float r = __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-  return x < -126.0f ? 0.0f : r;
-}
-
-// Pack two floats to bf16x2 (round to nearest even): lo -> bits 0-15.
 // Paired fp32 arithmetic (one instruction for two lanes of work, sm_100+):
 // halves the issue slots of elementwise softmax and epilogue math.
 __device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
@@ -382,6 +363,7 @@ __device__ __forceinline__ void fmul2(float& d0, float& d1, float a0, float a1, 
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
+// Pack two floats to bf16x2 (round to nearest even): lo -> bits 0-15.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

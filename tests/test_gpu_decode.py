@@ -77,6 +77,11 @@ def test_decode_b8_1m():
     run_case(WORKLOADS["decode_b8_1m"])
 
 
+def test_decode_b8_1m_dense():
+    # The dense decode run at 2^20 that the decode sparse/dense ratio divides by.
+    run_case(WORKLOADS["decode_b8_1m"], dense=True)
+
+
 def test_many_items_per_cta():
     # 2048 x 8 x 16 = 262144 (sequence, group, slot) items: more than 1024 per
     # CTA at 148 CTAs, so the persistent attention grid grows; sampled rows.

@@ -100,9 +100,27 @@ def test_prefill_32k_sampled_rows():
     run_case(w, rows=sampled(w, 64))
 
 
+# Rows on both sides of the block-major schedule's query-wave boundaries
+# (waves of 4096 rows), where a list of one wave ends and the next begins.
+WAVE_EDGES = [4095, 4096, 8191, 8192, 65535, 65536]
+
+
 def test_prefill_128k_sampled_rows():
     w = WORKLOADS["prefill_128k"]
-    run_case(w, rows=sampled(w, 32))
+    run_case(w, rows=sampled(w, 32) + WAVE_EDGES)
+
+
+def test_prefill_128k_dense_sampled_rows():
+    # The dense run (every causal block, eq. (1)) that the sparse/dense ratio
+    # of the benchmark divides by, on 64 sampled rows of the 128K prefill.
+    w = WORKLOADS["prefill_128k"]
+    run_case(w, rows=sampled(w, 59, seed=5), dense=True)
+
+
+def test_chunked_prefill_1m_dense_sampled_rows():
+    w = WORKLOADS["chunked_prefill_1m"]
+    rng = np.random.default_rng(6)
+    run_case(w, rows=list(rng.integers(0, w.n_q, 62)) + [0, w.n_q - 1], dense=True)
 
 
 def test_chunked_prefill_1m_sampled_rows():

@@ -46,3 +46,41 @@ def test_two_gloo_ranks():
     assert sp0 != sp1 and sd0 != sd1                  # independent problems
     assert t0 == t1 == 15.0                           # max over ranks on every rank
     assert ref1 is None                               # the reference arm is rank 0's alone
+
+
+def _bench_env():
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    env["PYTHONPATH"] = bench.ROOT
+    return env
+
+
+def test_bench_gpus_flag_launches_that_many_ranks():
+    # `bench.py --gpus 2` run directly relaunches itself under torchrun with
+    # two processes; the reference arm (CPU only) prints from rank 0 and
+    # reports the world size it ran with.
+    import json
+    import subprocess
+    import sys
+    cmd = [sys.executable, os.path.join(bench.ROOT, "bench.py"), "--gpus", "2", "--impl", "reference",
+           "--case", "tiny", "--steps", "1", "--warmup", "0"]
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=600, env=_bench_env())
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1          # rank 0 alone prints
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2
+
+
+def test_bench_gpus_flag_must_match_world_size():
+    import subprocess
+    import sys
+    env = _bench_env()
+    env.update(WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    cmd = [sys.executable, os.path.join(bench.ROOT, "bench.py"), "--gpus", "2", "--impl", "reference",
+           "--case", "tiny", "--steps", "1", "--warmup", "0"]
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=120, env=env)
+    assert r.returncode != 0 and "WORLD_SIZE" in r.stderr
+    c = bench.relaunch_command(["--gpus", "4"], 4, 29500)
+    assert c[1:4] == ["-m", "torch.distributed.run", "--nnodes=1"] and "--nproc-per-node" in c
+    assert c[c.index("--nproc-per-node") + 1] == "4" and c[c.index("--master-addr") + 1] == "127.0.0.1"
