@@ -44,8 +44,15 @@ def cases(name):
     """The bench workload, a smaller instance of the same kernels for ncu
     captures ("small": 32K prefill and 8 decode sequences), the long-context
     pair ("long": the last 8192 queries of a 2^20-token chunked prefill and a
-    batch of 8 sequences decoding at 2^20), or a tiny pair that runs in
-    seconds ("tiny": the 1K prefill and 4 short decode sequences)."""
+    batch of 8 sequences decoding at 2^20), a profiling pair small enough for
+    multi-pass ncu captures ("prof": the last 4096 queries of a 65536-token
+    context, about 1 GB of partials, and 8 sequences of 16K-32K tokens), or a
+    tiny pair that runs in seconds ("tiny": the 1K prefill and 4 short decode
+    sequences)."""
+    if name == "prof":
+        return (Workload(**{**WORKLOADS["prefill_32k"].__dict__, "n_q": 4096, "n_kv": 65536,
+                            "name": "chunked_prefill_64k_4k"}),
+                Workload(**{**DECODE.__dict__, "batch": 8, "kv_min": 16384, "kv_max": 32768, "name": "decode_b8_32k"}))
     if name == "tiny":
         return WORKLOADS["tiny_prefill_1k"], Workload(**{**DECODE.__dict__, "batch": 4, "kv_min": 3000,
                                                            "kv_max": 9000, "name": "decode_b4_short"})
@@ -467,7 +474,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--case", choices=["full", "small", "long", "tiny"], default="full")
+    ap.add_argument("--case", choices=["full", "small", "long", "prof", "tiny"], default="full")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")

@@ -179,9 +179,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------------- UMMA
     // The whole warp runs the loop (warp-uniform waits and descriptor math)
-    // and one elected lane issues: a single-lane divergent issue loop loses
-    // most of its issue slots to the two epilogue warps on this SMSP
-    // (measured: 108 against 272 cycles per MMA with three busy warps).
+    // and each MMA is predicated on an elected lane: a single-lane divergent
+    // issue loop loses most of its issue slots to the two epilogue warps on
+    // this SMSP (measured: 108 against 272 cycles per MMA with three busy
+    // warps).
     if (n_ktiles > 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(kRows, kKeys, false, false);
       constexpr uint32_t sbo = 8 * Cfg::kSwB;   // 8-row core-matrix group stride
@@ -198,18 +199,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint64_t kd = k_desc0 + ((s * Cfg::kAtoms * kKeys * Cfg::kSwB) >> 4);
         const uint32_t d_tmem = tmem + acc * kKeys;
-        const bool leader = elect_one();
 #pragma unroll
         for (int ks = 0; ks < DIDX / 16; ++ks) {
           constexpr int kPerAtom = Cfg::kSwB / 32;
           const uint32_t aoff = ((ks / kPerAtom) * kRows * Cfg::kSwB + (ks % kPerAtom) * 32) >> 4;
           const uint32_t boff = ((ks / kPerAtom) * kKeys * Cfg::kSwB + (ks % kPerAtom) * 32) >> 4;
-          if (leader) umma_ss(d_tmem, q_desc0 + aoff, kd + boff, idesc, ks > 0 ? 1u : 0u);
+          umma_ss_elect(d_tmem, q_desc0 + aoff, kd + boff, idesc, ks > 0 ? 1u : 0u);
         }
-        if (leader) {
-          umma_commit(&empty[s]);       // smem stage free once these MMAs finish
-          umma_commit(&acc_full[acc]);  // accumulator ready for the epilogue
-        }
+        umma_commit_elect(&empty[s]);       // smem stage free once these MMAs finish
+        umma_commit_elect(&acc_full[acc]);  // accumulator ready for the epilogue
         __syncwarp();
       }
     }

@@ -22,7 +22,7 @@ _LIB = os.path.join(_HERE, "libmsa_oracle.so")
 class Params(C.Structure):
     _fields_ = [("h_q", C.c_int), ("h_kv", C.c_int), ("d", C.c_int), ("d_idx", C.c_int),
                 ("block_k", C.c_int), ("topk", C.c_int), ("causal", C.c_int),
-                ("force_local", C.c_int), ("scale", C.c_double), ("threads", C.c_int)]
+                ("force_local", C.c_int), ("scale", C.c_double), ("threads", C.c_int), ("pool", C.c_int)]
 
 
 def build(force: bool = False) -> str:
@@ -57,9 +57,13 @@ def lib():
     return _lib
 
 
-def params(h_q, h_kv, d, d_idx, block_k, topk, causal=1, force_local=1, scale=0.0, threads=0) -> Params:
+POOL_MAX, POOL_MEAN = 0, 1
+
+
+def params(h_q, h_kv, d, d_idx, block_k, topk, causal=1, force_local=1, scale=0.0, threads=0,
+           pool=POOL_MAX) -> Params:
     return Params(h_q, h_kv, d, d_idx, block_k, topk, int(causal), int(force_local), float(scale),
-                  int(threads))
+                  int(threads), int(pool))
 
 
 def _u16(a) -> np.ndarray:

@@ -13,7 +13,8 @@
 //        eq. (8)  main-branch softmax attention over the gathered blocks (4.3);
 //        section 4.4.1: softmax is monotone, so selection ranks raw scores.
 //   [M]  m.163.com post, "Step 1 Index Attention": Q_idx in R^{n x h x d},
-//        K_idx in R^{n x 1 x d}: one index query per GQA group, one shared key.
+//        K_idx in R^{n x 1 x d}: one index query per GQA group, one shared key;
+//        and its comparison of the block max-pool with MoBA's mean pooling.
 //
 // Every input is a bf16 bit pattern widened exactly to double; all arithmetic
 // is double.  Rows are independent, so the OpenMP split over (row, group)
@@ -48,6 +49,7 @@ typedef struct {
   int h_q, h_kv, d, d_idx, block_k, topk, causal, force_local;
   double scale;   // main-branch softmax scale; <= 0 means 1/sqrt(d)
   int threads;    // OpenMP threads; <= 0 means the runtime default
+  int pool;       // block pooling of the token scores: 0 = max (eq. 6), 1 = mean (MoBA-style ablation)
 } msa_oracle_params;
 
 }  // extern "C"
@@ -89,6 +91,13 @@ int check(const msa_oracle_params* P, int n_q, int n_kv, long long q_pos0) {
 // Eq. (6), [T] section 4.2: block scores of one (query row, group).
 //   S_j = <Q_idx_i^(r), K_idx_j> / sqrt(d_idx)        (token score)
 //   M_b = max over j in B_b with j visible of S_j     (causal block max-pool)
+// With P.pool = 1, M_b is instead the mean of S_j over the visible keys of
+// the block: the mean pooling of MoBA that [M] compares the max-pool with
+// (the mean of <q, k_j> is <q, mean of k_j>, MoBA's block score).  A mean
+// over a partial block is a ratio that the kernel ranks in fp32, so the
+// ranking key here is the same fp32 rounding of (sum of raw dot products) /
+// (visible keys), times 1/sqrt(d_idx); with integer-valued index inputs the
+// sum is exact and the key is exactly the kernel's.
 // Blocks with no visible key get -inf (they are not eligible).
 void block_scores_row(const msa_oracle_params& P, const uint16_t* q_idx, const uint16_t* k_idx,
                       int n_kv, int i, long long p, int r, double* M) {
@@ -97,16 +106,24 @@ void block_scores_row(const msa_oracle_params& P, const uint16_t* q_idx, const u
   const uint16_t* qv = q_idx + (static_cast<size_t>(i) * P.h_kv + r) * P.d_idx;
   for (int b = 0; b < nb; ++b) {
     double best = kNegInf;
+    double raw_sum = 0.0;
+    long long count = 0;
     for (long long j = static_cast<long long>(b) * P.block_k;
          j < std::min<long long>(static_cast<long long>(b + 1) * P.block_k, n_kv); ++j) {
       if (!visible(P, p, j, n_kv)) continue;
       const uint16_t* kv = k_idx + static_cast<size_t>(j) * P.d_idx;  // K_idx[j, 0, :]
       double s = 0.0;
       for (int t = 0; t < P.d_idx; ++t) s += bf16(qv[t]) * bf16(kv[t]);
+      raw_sum += s;
+      ++count;
       s *= inv;
       if (s > best) best = s;
     }
-    M[b] = best;
+    if (P.pool == 1)
+      M[b] = count == 0 ? kNegInf
+                        : static_cast<double>(static_cast<float>(raw_sum / static_cast<double>(count))) * inv;
+    else
+      M[b] = best;
   }
 }
 
