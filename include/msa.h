@@ -82,6 +82,9 @@ typedef struct {
   int causal;      /* 1: key j visible from position p iff j <= p; 0: all keys */
   int force_local; /* 1: the block holding the query position is always selected */
   float scale;     /* main-branch softmax scale; <= 0 means 1/sqrt(d) */
+  int pool;        /* block pooling of the index scores: 0 = max (eq. (6)); 1 = mean over the block's visible
+                      keys (the MoBA-style mean pooling the m.163.com post compares max-pooling with), ranked
+                      by the fp32 quotient of the exact score sum and the key count */
 } msa_params;
 
 /*

@@ -20,6 +20,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmsa.so")
 
 OP_INDEX_TOPK, OP_PREFILL, OP_DECODE = 0, 1, 2
+POOL_MAX, POOL_MEAN = 0, 1   # msa_params.pool
 
 SYMBOLS = ("msa_workspace_size", "msa_index_topk", "msa_sparse_attn_prefill", "msa_sparse_attn_decode",
            "msa_device_status", "msa_status_string", "msa_sparse_attn_decode_noalloc",
@@ -36,11 +37,11 @@ class Params(C.Structure):
     """Mirror of ``msa_params`` (include/msa.h)."""
     _fields_ = [("h_q", C.c_int), ("h_kv", C.c_int), ("d", C.c_int), ("d_idx", C.c_int),
                 ("block_k", C.c_int), ("topk", C.c_int), ("causal", C.c_int), ("force_local", C.c_int),
-                ("scale", C.c_float)]
+                ("scale", C.c_float), ("pool", C.c_int)]
 
     @classmethod
-    def make(cls, h_q, h_kv, d, d_idx, block_k, topk, causal=True, force_local=True, scale=0.0):
-        return cls(h_q, h_kv, d, d_idx, block_k, topk, int(causal), int(force_local), float(scale))
+    def make(cls, h_q, h_kv, d, d_idx, block_k, topk, causal=True, force_local=True, scale=0.0, pool=0):
+        return cls(h_q, h_kv, d, d_idx, block_k, topk, int(causal), int(force_local), float(scale), int(pool))
 
 
 _lib = None

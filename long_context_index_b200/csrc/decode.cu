@@ -103,7 +103,7 @@ struct DecArgs {
   int* seq_count;           // [B] index CTAs finished per sequence (zeroed per call)
   int* grp_count;           // [B, h_kv, head_tiles] attention CTAs finished (zeroed per call)
   int batch, h_q, h_kv, topk, causal, force_local, kfree, idx_ctas, idx_wmax;
-  int splits, slots_per_split, dense, head_tiles;
+  int splits, slots_per_split, dense, head_tiles, pool;
   float scale_log2;
 };
 
@@ -125,7 +125,7 @@ template <int BK>
 __device__ void merge_topk_warp(const DecArgs& a, int b, int r, int lane, int* chosen, int c_lo, int nseg,
                                 long long T, int n);
 
-template <int DIDX, int BK>
+template <int DIDX, int BK, int POOL>
 __global__ void __launch_bounds__(kIdxThreads, kIdxCtasPerSm) decode_index_kernel(const DecArgs a) {
   constexpr int kHalves = DIDX / 32;   // 16-byte vectors per token row per thread
   constexpr int kWarps = kIdxThreads / 32;
@@ -207,7 +207,9 @@ __global__ void __launch_bounds__(kIdxThreads, kIdxCtasPerSm) decode_index_kerne
       }
     }
     const int j0 = (gb - cur_p) * BK;
-    float m0 = kNegInf, m1 = kNegInf;   // groups 2t, 2t+1
+    // Groups 2t, 2t+1: running max (max-pool) or sum (mean-pool; the sum of
+    // integer-valued scores is exact in fp32, in any order, below 2^24).
+    float m0 = POOL ? 0.f : kNegInf, m1 = POOL ? 0.f : kNegInf;
 #pragma unroll 2
     for (int mt = 0; mt < BK / 16; ++mt) {
       const int ja = j0 + mt * 16 + g, jb = ja + 8;
@@ -223,19 +225,32 @@ __global__ void __launch_bounds__(kIdxThreads, kIdxCtasPerSm) decode_index_kerne
         mma_bf16_16816(c, ra[h].x, rb[h].x, ra[h].y, rb[h].y, qv[h].x, qv[h].y);
         mma_bf16_16816(c, ra[h].z, rb[h].z, ra[h].w, rb[h].w, qv[h].z, qv[h].w);
       }
-      if (ja < L) {
-        m0 = fmaxf(m0, c[0]);
-        m1 = fmaxf(m1, c[1]);
-      }
-      if (jb < L) {
-        m0 = fmaxf(m0, c[2]);
-        m1 = fmaxf(m1, c[3]);
+      if (POOL) {   // keys past L loaded zeros, so their scores add 0
+        m0 += c[0] + c[2];
+        m1 += c[1] + c[3];
+      } else {
+        if (ja < L) {
+          m0 = fmaxf(m0, c[0]);
+          m1 = fmaxf(m1, c[1]);
+        }
+        if (jb < L) {
+          m0 = fmaxf(m0, c[2]);
+          m1 = fmaxf(m1, c[3]);
+        }
       }
     }
 #pragma unroll
     for (int x = 4; x < 32; x <<= 1) {
-      m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, x));
-      m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, x));
+      const float o0 = __shfl_xor_sync(0xffffffffu, m0, x), o1 = __shfl_xor_sync(0xffffffffu, m1, x);
+      m0 = POOL ? m0 + o0 : fmaxf(m0, o0);
+      m1 = POOL ? m1 + o1 : fmaxf(m1, o1);
+    }
+    if (POOL) {
+      // Mean over the block's keys, ranked in fp32: a full block divides by
+      // B_k exactly, the partial last block rounds the quotient.
+      const int cnt = min(BK, L - j0);
+      m0 = cnt >= BK ? m0 * (1.0f / BK) : __fdiv_rn(m0, static_cast<float>(cnt));
+      m1 = cnt >= BK ? m1 * (1.0f / BK) : __fdiv_rn(m1, static_cast<float>(cnt));
     }
     if (g == 0) {
       if (2 * t < a.h_kv) smax[(2 * t) * wmax + i] = m0;
@@ -1175,7 +1190,7 @@ int launch_attn_stream(const DecArgs& a, int max_kv, int* status, cudaStream_t s
 template <int DIDX, int BK>
 int launch_index(const DecArgs& a, size_t smem, cudaStream_t st) {
   if (a.kfree > 0) {
-    auto kern = decode_index_kernel<DIDX, BK>;
+    auto kern = a.pool ? decode_index_kernel<DIDX, BK, 1> : decode_index_kernel<DIDX, BK, 0>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
         cudaSuccess)
       return MSA_ERR_CUDA;
@@ -1238,6 +1253,7 @@ int run_sparse_attn_decode(const msa_params& p, const void* q, const void* q_idx
   a.causal = p.causal;
   a.force_local = p.force_local;
   a.kfree = p.topk - (p.force_local ? 1 : 0);
+  a.pool = p.pool;
   const IdxPlan ip = plan_index(p, batch, max_kv);
   a.idx_ctas = ip.ctas;
   a.idx_wmax = ip.wmax;

@@ -4,7 +4,9 @@
 // "MiniMax Sparse Attention", eq. (6), section 4.2):
 //   S_ij = <Q_idx_i^(r), K_idx_j>                  (the 1/sqrt(d_idx) factor is
 //                                                   positive: order-preserving)
-//   M_ib = max over visible j in block b of S_ij   (causal block max-pool)
+//   M_ib = max over visible j in block b of S_ij   (causal block max-pool;
+//          with pool = mean, the mean over the visible keys of the block,
+//          the MoBA-style pooling the m.163.com post compares it with)
 //   I_i^(r) = local block + the best (topk - 1) other eligible blocks by M,
 //             ties to the lower block index, emitted ascending, -1 padded.
 // Selection compares raw scores and never exponentiates (section 4.4.1).
@@ -40,6 +42,8 @@ constexpr int kRows = 128;      // query rows per CTA (UMMA M)
 constexpr int kKeys = 256;      // keys per tile (UMMA N)
 constexpr int kThreads = 384;   // 12 warps
 constexpr int kEpiWarp0 = 4;    // first epilogue warp
+constexpr int kPoolMax = 0;     // msa_params.pool: block max-pool (eq. (6))
+constexpr int kPoolMean = 1;    //                  block mean-pool (MoBA-style ablation)
 
 template <int DIDX>
 struct IdxCfg {
@@ -57,7 +61,7 @@ struct IdxCfg {
 struct IdxArgs {
   int32_t* block_ids;
   int* status;
-  int n_q, n_kv, q_pos0, h_kv, topk, causal, force_local;
+  int n_q, n_kv, q_pos0, h_kv, topk, causal, force_local, pool;
   int n_tiles;
 };
 
@@ -96,7 +100,7 @@ struct TopK {
   }
 };
 
-template <int DIDX, int BK, int KMAX>
+template <int DIDX, int BK, int KMAX, int POOL>
 __global__ void __launch_bounds__(kThreads, 1)
     index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                               const IdxArgs args) {
@@ -236,11 +240,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int j0 = t * kKeys + half * 128;
       if (j0 < kv_end) {
         // 128 columns in two 64-column pieces (two TMEM loads in flight per
-        // wait); per block, four independent 3-input max chains.
+        // wait); per block, four independent 3-input max chains (max-pool)
+        // or add chains (mean-pool: masked keys add 0, and the sum of
+        // integer-valued scores is exact in fp32 below 2^24).
+        constexpr uint32_t kMasked = POOL == kPoolMax ? 0xff800000u : 0u;   // -inf / 0
         float m4[kBlocksPerHalf][4];
 #pragma unroll
         for (int bb = 0; bb < kBlocksPerHalf; ++bb)
-          m4[bb][0] = m4[bb][1] = m4[bb][2] = m4[bb][3] = __int_as_float(0xff800000);
+          m4[bb][0] = m4[bb][1] = m4[bb][2] = m4[bb][3] = __uint_as_float(kMasked);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           uint32_t v[64];
@@ -251,21 +258,41 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (jh + 64 > kv_lim) {   // keys this row must not see
 #pragma unroll
             for (int e = 0; e < 64; ++e)
-              if (jh + e >= kv_lim) v[e] = 0xff800000u;   // -inf
+              if (jh + e >= kv_lim) v[e] = kMasked;
           }
 #pragma unroll
           for (int e = 0; e < 64; e += 8) {
             const int bb = (h * 64 + e) / BK;
             const int k = (e / 8) & 3;
-            m4[bb][k] = max3f(m4[bb][k], fmaxf(__uint_as_float(v[e]), __uint_as_float(v[e + 1])),
-                              max3f(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]), __uint_as_float(v[e + 4])));
-            m4[bb][k] =
-                max3f(m4[bb][k], __uint_as_float(v[e + 5]), fmaxf(__uint_as_float(v[e + 6]), __uint_as_float(v[e + 7])));
+            if (POOL == kPoolMax) {
+              m4[bb][k] = max3f(m4[bb][k], fmaxf(__uint_as_float(v[e]), __uint_as_float(v[e + 1])),
+                                max3f(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]), __uint_as_float(v[e + 4])));
+              m4[bb][k] = max3f(m4[bb][k], __uint_as_float(v[e + 5]),
+                                fmaxf(__uint_as_float(v[e + 6]), __uint_as_float(v[e + 7])));
+            } else {
+              float a0, a1, b0, b1;
+              fadd2(a0, a1, __uint_as_float(v[e]), __uint_as_float(v[e + 1]), __uint_as_float(v[e + 2]),
+                    __uint_as_float(v[e + 3]));
+              fadd2(b0, b1, __uint_as_float(v[e + 4]), __uint_as_float(v[e + 5]), __uint_as_float(v[e + 6]),
+                    __uint_as_float(v[e + 7]));
+              fadd2(a0, a1, a0, a1, b0, b1);
+              m4[bb][k] += a0 + a1;
+            }
           }
         }
 #pragma unroll
-        for (int bb = 0; bb < kBlocksPerHalf; ++bb)
-          bmax[bb] = fmaxf(fmaxf(m4[bb][0], m4[bb][1]), fmaxf(m4[bb][2], m4[bb][3]));
+        for (int bb = 0; bb < kBlocksPerHalf; ++bb) {
+          if (POOL == kPoolMax) {
+            bmax[bb] = fmaxf(fmaxf(m4[bb][0], m4[bb][1]), fmaxf(m4[bb][2], m4[bb][3]));
+          } else {
+            // Mean over the visible keys of the block, ranked in fp32: a full
+            // block divides by B_k exactly, a partial one rounds the quotient.
+            const float sum = (m4[bb][0] + m4[bb][1]) + (m4[bb][2] + m4[bb][3]);
+            const int cnt = min(BK, kv_lim - (j0 + bb * BK));
+            bmax[bb] = cnt >= BK ? sum * (1.0f / BK)
+                                 : (cnt > 0 ? __fdiv_rn(sum, static_cast<float>(cnt)) : __int_as_float(0xff800000));
+          }
+        }
       }
       // Release the accumulator stage to the MMA warp.
       tc_fence_before();
@@ -346,9 +373,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int DIDX, int BK, int KMAX>
+template <int DIDX, int BK, int KMAX, int POOL>
 cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const IdxArgs& a, cudaStream_t st) {
-  auto kern = index_topk_prefill_kernel<DIDX, BK, KMAX>;
+  auto kern = index_topk_prefill_kernel<DIDX, BK, KMAX, POOL>;
   const int smem = IdxCfg<DIDX>::kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -359,8 +386,9 @@ cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const IdxArgs
 
 template <int DIDX, int BK>
 cudaError_t launch_k(const CUtensorMap& tq, const CUtensorMap& tk, const IdxArgs& a, cudaStream_t st) {
-  if (a.topk <= 16) return launch_t<DIDX, BK, 16>(tq, tk, a, st);
-  return launch_t<DIDX, BK, 32>(tq, tk, a, st);
+  if (a.pool == kPoolMean)
+    return a.topk <= 16 ? launch_t<DIDX, BK, 16, kPoolMean>(tq, tk, a, st) : launch_t<DIDX, BK, 32, kPoolMean>(tq, tk, a, st);
+  return a.topk <= 16 ? launch_t<DIDX, BK, 16, kPoolMax>(tq, tk, a, st) : launch_t<DIDX, BK, 32, kPoolMax>(tq, tk, a, st);
 }
 
 template <int DIDX>
@@ -400,6 +428,7 @@ int run_index_topk_prefill(const msa_params& p, const void* q_idx, const void* k
   a.topk = p.topk;
   a.causal = p.causal;
   a.force_local = p.force_local;
+  a.pool = p.pool;
   a.n_tiles = (n_q + kRows - 1) / kRows;
   cudaError_t e;
   switch (p.d_idx) {

@@ -21,6 +21,7 @@ int check_params(const msa_params* p) {
   if (p->h_q <= 0 || p->h_kv <= 0 || p->d <= 0 || p->d_idx <= 0 || p->block_k <= 0 || p->topk <= 0)
     return MSA_ERR_INVALID;
   if ((p->causal != 0 && p->causal != 1) || (p->force_local != 0 && p->force_local != 1)) return MSA_ERR_INVALID;
+  if (p->pool != 0 && p->pool != 1) return MSA_ERR_INVALID;
   if (p->h_q % p->h_kv != 0) return MSA_ERR_UNSUPPORTED;
   const int g = p->h_q / p->h_kv;
   if (g > 128 || 128 % g != 0) return MSA_ERR_UNSUPPORTED;

@@ -18,10 +18,10 @@ def host_f64(t: torch.Tensor) -> np.ndarray:
     return t.float().cpu().numpy().astype(np.float64)
 
 
-def params_pair(h_q, h_kv, d, d_idx, block_k, topk, causal=1, force_local=1, scale=0.0):
+def params_pair(h_q, h_kv, d, d_idx, block_k, topk, causal=1, force_local=1, scale=0.0, pool=0):
     """The same problem as library parameters and as oracle parameters."""
-    return (msa.Params.make(h_q, h_kv, d, d_idx, block_k, topk, causal, force_local, scale),
-            oracle.params(h_q, h_kv, d, d_idx, block_k, topk, causal, force_local, scale))
+    return (msa.Params.make(h_q, h_kv, d, d_idx, block_k, topk, causal, force_local, scale, pool),
+            oracle.params(h_q, h_kv, d, d_idx, block_k, topk, causal, force_local, scale, pool=pool))
 
 
 def assert_close(got: np.ndarray, ref: np.ndarray, atol=1e-2, rtol=1e-2, what=""):

@@ -49,6 +49,8 @@ def test_workspace_size_is_host_only_and_validates():
     assert msa.workspace_size(msa.OP_INDEX_TOPK, P(h_q=6, h_kv=4), 10, 10) == 0
     assert msa.workspace_size(msa.OP_DECODE, P(), batch=0, max_kv=10) == 0
     assert msa.workspace_size(7, P(), 10, 10) == 0
+    assert msa.workspace_size(msa.OP_INDEX_TOPK, P(pool=msa.POOL_MEAN), 10, 10) >= 256
+    assert msa.workspace_size(msa.OP_INDEX_TOPK, P(pool=-1), 10, 10) == 0
 
 
 def call_index(p, n_q=128, n_kv=128, q_pos0=0, qi=16, ki=16, ids=16, ws=256, ws_bytes=1 << 20):
@@ -58,6 +60,7 @@ def call_index(p, n_q=128, n_kv=128, q_pos0=0, qi=16, ki=16, ids=16, ws=256, ws_
 @pytest.mark.parametrize("kw,code", [
     (dict(d=96), -2), (dict(d_idx=48), -2), (dict(block_k=32), -2), (dict(topk=33), -2),
     (dict(h_q=48, h_kv=32), -2), (dict(h_q=6, h_kv=4), -2), (dict(topk=0), -1), (dict(causal=2), -1),
+    (dict(pool=2), -1),
 ])
 def test_index_rejects_bad_params(kw, code):
     assert call_index(P(**kw)) == code

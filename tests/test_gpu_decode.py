@@ -19,9 +19,9 @@ def small(**kw):
     return Workload(**base)
 
 
-def run_case(w, seqs=None, dense=False, force_local=1):
+def run_case(w, seqs=None, dense=False, force_local=1, pool=0):
     t = make_decode(w)
-    p, po = params_pair(w.h_q, w.h_kv, w.d, w.d_idx, w.block_k, w.topk, 1, force_local)
+    p, po = params_pair(w.h_q, w.h_kv, w.d, w.d_idx, w.block_k, w.topk, 1, force_local, pool=pool)
     ids, o = msa.sparse_attn_decode(p, dev(t["q"]), dev(t["q_idx"]), dev(t["k_cache"]), dev(t["v_cache"]),
                                     dev(t["k_idx_cache"]), dev(t["cu_kv"]), int(t["lens"].max()), dense=dense)
     torch.cuda.synchronize()
@@ -63,6 +63,15 @@ def test_shapes(kw):
 
 def test_force_local_off():
     run_case(small(seed=41), force_local=0)
+
+
+@pytest.mark.parametrize("force_local", [1, 0])
+def test_mean_pool_decode(force_local):
+    # Mean-pool ablation: ids bit for bit, including the partial last block
+    # (ranked when force_local = 0).
+    run_case(small(seed=43, batch=6, kv_min=100, kv_max=3000), force_local=force_local, pool=msa.POOL_MEAN)
+    run_case(small(h_q=64, h_kv=4, d=128, d_idx=64, block_k=128, topk=16, batch=3, kv_min=5000, kv_max=20000,
+                   seed=44), force_local=force_local, pool=msa.POOL_MEAN)
 
 
 def test_decode_b64_64k_128k():

@@ -15,10 +15,10 @@ from tests.gpu_util import dev, params_pair
 pytestmark = pytest.mark.gpu
 
 
-def run_case(w: Workload, n_q=None, n_kv=None, rows=None, causal=1, force_local=1, topk=None):
+def run_case(w: Workload, n_q=None, n_kv=None, rows=None, causal=1, force_local=1, topk=None, pool=0):
     t = make_prefill(w, n_q=n_q, n_kv=n_kv)
     k = w.topk if topk is None else topk
-    p, po = params_pair(w.h_q, w.h_kv, w.d, w.d_idx, w.block_k, k, causal, force_local)
+    p, po = params_pair(w.h_q, w.h_kv, w.d, w.d_idx, w.block_k, k, causal, force_local, pool=pool)
     ids = msa.index_topk(p, dev(t["q_idx"]), dev(t["k_idx"]), q_pos0=t["q_pos0"])
     torch.cuda.synchronize()
     got = ids.cpu().numpy()
@@ -131,3 +131,32 @@ def test_chunked_prefill_1m_sampled_rows():
     ref = oracle.index_topk(po, t["q_idx"], t["k_idx"], q_pos0=t["q_pos0"], rows=rows)
     assert np.array_equal(got[rows], ref)
     check_needles(t, got, w)
+
+
+# Mean-pool ablation (the MoBA-style pooling the m.163.com post compares the
+# max-pool with): ids must still match the oracle bit for bit, partial
+# (ragged or causal) blocks included.
+@pytest.mark.parametrize("kw", [
+    dict(n_q=1000, n_kv=1000),
+    dict(n_q=77, n_kv=1000),
+    dict(n_q=700, n_kv=900, d_idx=128, block_k=128, topk=5),
+    dict(n_q=600, n_kv=600, topk=32, block_k=64),
+])
+@pytest.mark.parametrize("force_local", [1, 0])
+def test_mean_pool_shapes(kw, force_local):
+    run_case(small(seed=kw.get("n_q", 1) + 17, **kw), force_local=force_local, pool=msa.POOL_MEAN)
+
+
+def test_mean_pool_prefill_32k_sampled_rows():
+    w = WORKLOADS["prefill_32k"]
+    rng = np.random.default_rng(11)
+    run_case(w, rows=list(rng.integers(0, w.n_q, 48)) + [0, 127, 128, w.n_q - 1], pool=msa.POOL_MEAN)
+
+
+def test_mean_and_max_pool_select_differently():
+    # On the 32K workload the two poolings must disagree somewhere (the
+    # ablation is not a no-op), while each matches its oracle above.
+    w = WORKLOADS["prefill_32k"]
+    _, a = run_case(w, rows=[w.n_q - 1], pool=msa.POOL_MAX)
+    _, b = run_case(w, rows=[w.n_q - 1], pool=msa.POOL_MEAN)
+    assert not np.array_equal(a, b)
