@@ -70,6 +70,8 @@ extern "C" {
 #define MSA_OP_INDEX_TOPK 0
 #define MSA_OP_PREFILL 1
 #define MSA_OP_DECODE 2
+#define MSA_OP_INDEX_TOPK_VARLEN 3 /* n_q = total rows, batch = sequences */
+#define MSA_OP_PREFILL_VARLEN 4    /* n_q = total rows, batch = sequences */
 
 /* Problem parameters (the pages' notation: H_q, H_kv, d_h, d_idx, B_k, k). */
 typedef struct {
@@ -152,8 +154,41 @@ MSA_API int msa_sparse_attn_decode(const msa_params* p, const void* q, const voi
                            void* stream);
 
 /*
+ * Packed batches of independent prefills (the serving form: many sequences
+ * of different lengths in one call).  Sequence s owns rows
+ * [cu_seqlens[s], cu_seqlens[s + 1]) of every tensor below; its query i sits
+ * at position i of the sequence (a full causal prefill of each sequence), it
+ * sees only its own keys, and its block ids are local to it.  Per sequence
+ * the result is exactly that of msa_index_topk / msa_sparse_attn_prefill on
+ * its rows (titansim.online section 4.2 and eq. (8), section 4.3).
+ *   cu_seqlens    int32 [batch + 1] DEVICE prefix of the sequence lengths:
+ *                 cu_seqlens[0] = 0, non-decreasing, cu_seqlens[batch] = total.
+ *                 A violation is found on the device: nothing is computed and
+ *                 msa_device_status() reports MSA_ERR_INVALID.
+ *   topk_per_seq  int32 [batch] DEVICE, or NULL: the number of blocks kept
+ *                 for each sequence (adaptive k; the future-work direction of
+ *                 titansim.online section 5.3), clamped to [1, p->topk]; the
+ *                 ids beyond it are -1.  NULL keeps p->topk for every sequence.
+ *   q_idx [total, h_kv, d_idx], k_idx [total, 1, d_idx], block_ids
+ *   [total, h_kv, topk], q [total, h_q, d], k, v [total, h_kv, d],
+ *   o [total, h_q, d]; layouts and types as for the single-sequence calls.
+ * The prefill runs the sparse (block-major) path only: block_ids must not be
+ * NULL.  batch >= 1; total <= 2^24.  Workspace: msa_workspace_size with
+ * MSA_OP_INDEX_TOPK_VARLEN / MSA_OP_PREFILL_VARLEN, n_q = total and
+ * batch = the number of sequences.
+ */
+MSA_API int msa_index_topk_varlen(const msa_params* p, const void* q_idx, const void* k_idx,
+                                  const int32_t* cu_seqlens, int batch, int total, const int32_t* topk_per_seq,
+                                  int32_t* block_ids, void* ws, size_t ws_bytes, void* stream);
+MSA_API int msa_sparse_attn_prefill_varlen(const msa_params* p, const void* q, const void* k, const void* v,
+                                           const int32_t* cu_seqlens, int batch, int total,
+                                           const int32_t* block_ids, void* o, void* ws, size_t ws_bytes,
+                                           void* stream);
+
+/*
  * Device status recorded by the last call that used workspace `ws`: MSA_OK,
- * or MSA_ERR_TIMEOUT when one of its kernels gave up a bounded wait.  Every
+ * MSA_ERR_TIMEOUT when one of its kernels gave up a bounded wait, or
+ * MSA_ERR_INVALID when a varlen call found cu_seqlens invalid.  Every
  * call clears the status word (the first 4 bytes of its workspace) before
  * launching.  Synchronises `stream` first; returns MSA_ERR_CUDA if that or the
  * 4-byte read fails.

@@ -13,18 +13,19 @@ import os
 from typing import Optional
 
 __all__ = ["MSAError", "Params", "lib", "workspace_size", "index_topk", "sparse_attn_prefill",
-           "sparse_attn_decode", "device_status", "status_string", "OP_INDEX_TOPK", "OP_PREFILL",
-           "OP_DECODE"]
+           "sparse_attn_decode", "index_topk_varlen", "sparse_attn_prefill_varlen", "device_status",
+           "status_string", "OP_INDEX_TOPK", "OP_PREFILL", "OP_DECODE", "OP_INDEX_TOPK_VARLEN",
+           "OP_PREFILL_VARLEN", "POOL_MAX", "POOL_MEAN"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmsa.so")
 
-OP_INDEX_TOPK, OP_PREFILL, OP_DECODE = 0, 1, 2
+OP_INDEX_TOPK, OP_PREFILL, OP_DECODE, OP_INDEX_TOPK_VARLEN, OP_PREFILL_VARLEN = 0, 1, 2, 3, 4
 POOL_MAX, POOL_MEAN = 0, 1   # msa_params.pool
 
 SYMBOLS = ("msa_workspace_size", "msa_index_topk", "msa_sparse_attn_prefill", "msa_sparse_attn_decode",
-           "msa_device_status", "msa_status_string", "msa_sparse_attn_decode_noalloc",
-           "msa_test_never_ready_wait")
+           "msa_index_topk_varlen", "msa_sparse_attn_prefill_varlen", "msa_device_status", "msa_status_string",
+           "msa_sparse_attn_decode_noalloc", "msa_test_never_ready_wait")
 
 
 class MSAError(RuntimeError):
@@ -65,6 +66,8 @@ def lib():
         L.msa_index_topk.argtypes = [P, vp, vp, i32, i32, i32, vp, vp, sz, vp]
         L.msa_sparse_attn_prefill.argtypes = [P, vp, vp, vp, vp, i32, i32, i32, vp, vp, sz, vp]
         L.msa_sparse_attn_decode.argtypes = [P, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, vp, vp, sz, vp]
+        L.msa_index_topk_varlen.argtypes = [P, vp, vp, vp, i32, i32, vp, vp, vp, sz, vp]
+        L.msa_sparse_attn_prefill_varlen.argtypes = [P, vp, vp, vp, vp, i32, i32, vp, vp, vp, sz, vp]
         L.msa_sparse_attn_decode_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, vp, vp]
         L.msa_sparse_attn_decode_noalloc.restype = i32
         L.msa_test_never_ready_wait.argtypes = [vp, sz, C.c_longlong, vp]
@@ -72,7 +75,8 @@ def lib():
         L.msa_device_status.argtypes = [vp, vp]
         L.msa_status_string.argtypes = [i32]
         L.msa_status_string.restype = C.c_char_p
-        for f in ("msa_index_topk", "msa_sparse_attn_prefill", "msa_sparse_attn_decode", "msa_device_status"):
+        for f in ("msa_index_topk", "msa_sparse_attn_prefill", "msa_sparse_attn_decode", "msa_device_status",
+                  "msa_index_topk_varlen", "msa_sparse_attn_prefill_varlen"):
             getattr(L, f).restype = i32
         _lib = L
     return _lib
@@ -201,6 +205,54 @@ def sparse_attn_decode(p: Params, q, q_idx, k_cache, v_cache, k_idx_cache, cu_kv
         raise MSAError(rc, "msa_sparse_attn_decode")
     _after(ws, stream, "msa_sparse_attn_decode")
     return block_ids, out
+
+
+def index_topk_varlen(p: Params, q_idx, k_idx, cu_seqlens, topk_per_seq=None, block_ids=None, ws=None,
+                      stream=None):
+    """Index branch of a packed batch of sequences (rows [cu[s], cu[s+1]) each):
+    block ids [total, h_kv, topk], local to each sequence, -1 padded.
+    ``topk_per_seq`` (int32 [batch], optional): blocks kept per sequence."""
+    torch = _torch()
+    total = q_idx.shape[0]
+    batch = cu_seqlens.shape[0] - 1
+    _check(q_idx, "q_idx", _bf16(), (total, p.h_kv, p.d_idx))
+    _check(k_idx, "k_idx", _bf16(), (total, 1, p.d_idx))
+    _check(cu_seqlens, "cu_seqlens", (torch.int32,), (batch + 1,))
+    if topk_per_seq is not None:
+        _check(topk_per_seq, "topk_per_seq", (torch.int32,), (batch,))
+    if block_ids is None:
+        block_ids = torch.empty((total, p.h_kv, p.topk), dtype=torch.int32, device=q_idx.device)
+    _check(block_ids, "block_ids", (torch.int32,), (total, p.h_kv, p.topk))
+    ws = _workspace(OP_INDEX_TOPK_VARLEN, p, total, total, batch=batch, ws=ws, device=q_idx.device)
+    rc = lib().msa_index_topk_varlen(C.byref(p), _ptr(q_idx), _ptr(k_idx), _ptr(cu_seqlens), batch, total,
+                                     _ptr(topk_per_seq), _ptr(block_ids), _ptr(ws), ws.numel(), _stream(stream))
+    if rc:
+        raise MSAError(rc, "msa_index_topk_varlen")
+    _after(ws, stream, "msa_index_topk_varlen")
+    return block_ids
+
+
+def sparse_attn_prefill_varlen(p: Params, q, k, v, cu_seqlens, block_ids, out=None, ws=None, stream=None):
+    """Main branch of a packed batch of sequences: O [total, h_q, d] bf16."""
+    torch = _torch()
+    total = q.shape[0]
+    batch = cu_seqlens.shape[0] - 1
+    _check(q, "q", _bf16(), (total, p.h_q, p.d))
+    _check(k, "k", _bf16(), (total, p.h_kv, p.d))
+    _check(v, "v", _bf16(), (total, p.h_kv, p.d))
+    _check(cu_seqlens, "cu_seqlens", (torch.int32,), (batch + 1,))
+    _check(block_ids, "block_ids", (torch.int32,), (total, p.h_kv, p.topk))
+    if out is None:
+        out = torch.empty((total, p.h_q, p.d), dtype=torch.bfloat16, device=q.device)
+    _check(out, "out", _bf16(), (total, p.h_q, p.d))
+    ws = _workspace(OP_PREFILL_VARLEN, p, total, total, batch=batch, ws=ws, device=q.device)
+    rc = lib().msa_sparse_attn_prefill_varlen(C.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), batch,
+                                              total, _ptr(block_ids), _ptr(out), _ptr(ws), ws.numel(),
+                                              _stream(stream))
+    if rc:
+        raise MSAError(rc, "msa_sparse_attn_prefill_varlen")
+    _after(ws, stream, "msa_sparse_attn_prefill_varlen")
+    return out
 
 
 def _after(ws, stream, what):

@@ -367,13 +367,13 @@ cudaError_t launch_g(int G, const CUtensorMap& tq, const CUtensorMap& tk, const 
 
 }  // namespace
 
-size_t prefill_workspace_bytes(const msa_params& p, int n_q, int n_kv) {
-  return sparse_prefill_workspace_bytes(p, n_q, n_kv);
+size_t prefill_workspace_bytes(const msa_params& p, int n_q, int n_kv, int batch) {
+  return sparse_prefill_workspace_bytes(p, n_q, n_kv, batch);
 }
 
 int run_sparse_attn_prefill(const msa_params& p, const void* q, const void* k, const void* v,
                             const int32_t* block_ids, int n_q, int n_kv, int q_pos0, void* o, void* ws,
-                            size_t ws_bytes, int* status, cudaStream_t stream) {
+                            size_t ws_bytes, int* status, cudaStream_t stream, const Varlen* vl) {
   if (n_q == 0) return MSA_OK;
   const int G = p.h_q / p.h_kv;
   const int QT = 128 / G;
@@ -393,7 +393,8 @@ int run_sparse_attn_prefill(const msa_params& p, const void* q, const void* k, c
     if (!encode_tma_bf16(&tv, 3, v, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MSA_ERR_CUDA;
   }
   if (block_ids)   // sparse: block-major schedule (attn_sparse.cu)
-    return run_sparse_attn_kvouter(p, q, tk, tv, block_ids, n_q, n_kv, q_pos0, o, ws, ws_bytes, status, stream);
+    return run_sparse_attn_kvouter(p, q, tk, tv, block_ids, n_q, n_kv, q_pos0, o, ws, ws_bytes, status, stream, vl);
+  if (vl) return MSA_ERR_INVALID;   // packed batches run sparse only
   AttnArgs a;
   a.o = static_cast<uint16_t*>(o);
   a.status = status;

@@ -72,8 +72,9 @@ struct KvoCfg {
 // One chunk of gathered queries of a (group, block) list.
 struct Desc {
   int entry[128];   // (query << 5) | slot, for the first `count` rows' queries
-  int r, b, count, kvs;
+  int r, b, count, kvs;                      // b: block index within its sequence
   int first_of_kv, last_of_kv, end, chunk;   // chunk: global chunk id (partial tile index)
+  int seq_row0, seq_len;                     // the block's sequence: first row, length
 };
 
 static_assert(kDesc * sizeof(Desc) + kStageEntries * 4 + 64 * 8 + 16 <= kCtrlBytes,
@@ -91,7 +92,21 @@ struct KvoArgs {
   int* status;
   int n_q, n_kv, q_pos0, h_q, h_kv, topk, causal, nb;
   float scale_log2;
+  const int* cu_seqlens;   // packed batch of sequences (varlen), or null: one (chunked) prefill
+  const int* blk_pfx;      // [batch + 1] prefix of ceil(L_s / B_k): global block = blk_pfx[s] + local block
+  int batch;
 };
+
+// Sequence of a query row / of a global block in a packed batch: the largest
+// s with pfx[s] <= x, for a non-decreasing pfx[0..batch].
+__device__ __forceinline__ int seq_search(const int* pfx, int batch, int x) {
+  int lo = 0, hi = batch - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (pfx[mid] <= x) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
 
 template <int D, int BK, int G>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -181,7 +196,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       li = __shfl_sync(0xffffffffu, li, 0);
       if (li >= n_lists) break;
       const int rb = args.lists[li];
-      const int r = (rb / args.nb) % args.h_kv, b = rb % args.nb;
+      const int r = (rb / args.nb) % args.h_kv, gb = rb % args.nb;
+      // The block's sequence: its key rows start at seq_row0 + b * BK.
+      int b = gb, seq_row0 = 0, seq_len = args.n_kv;
+      if (args.cu_seqlens) {
+        const int sq_ = seq_search(args.blk_pfx, args.batch, gb);
+        b = gb - args.blk_pfx[sq_];
+        seq_row0 = args.cu_seqlens[sq_];
+        seq_len = args.cu_seqlens[sq_ + 1] - seq_row0;
+      }
+      const int kv_row = seq_row0 + b * BK;
       const int start = args.offs[rb], cnt = args.offs[rb + 1] - start;
       const int chunk0 = args.chunk_off[rb];
       const int kvs = kvc % kKVStages;
@@ -192,7 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) {
           mbar_arrive_expect_tx(&k_full[kvs], Cfg::kKVBytes);
           for (int a = 0; a < Cfg::kAtoms; ++a)
-            tma_load_3d(sk + a * BK * 128, &tm_k, &k_full[kvs], a * 64, r, b * BK);
+            tma_load_3d(sk + a * BK * 128, &tm_k, &k_full[kvs], a * 64, r, kv_row);
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -228,6 +252,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           dd.last_of_kv = c0 + QPC >= cnt;
           dd.end = 0;
           dd.chunk = chunk0 + c0 / QPC;
+          dd.seq_row0 = seq_row0;
+          dd.seq_len = seq_len;
           mbar_arrive_expect_tx(&q_full[qs], Cfg::kQBytes);
         }
         __syncwarp();
@@ -250,7 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (ok) {
               mbar_arrive_expect_tx(&v_full[kvs], Cfg::kKVBytes);
               for (int a = 0; a < Cfg::kAtoms; ++a)
-                tma_load_3d(sk + Cfg::kKVBytes + a * BK * 128, &tm_v, &v_full[kvs], a * 64, r, b * BK);
+                tma_load_3d(sk + Cfg::kKVBytes + a * BK * 128, &tm_v, &v_full[kvs], a * 64, r, kv_row);
             }
           }
           ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -403,16 +429,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Desc& dd = desc[ds];
       const int end = dd.end;
       const int e = (!end && qi < dd.count) ? dd.entry[qi] : -1;
-      const int b = dd.b, chunk = dd.chunk;
+      const int b = dd.b, chunk = dd.chunk, seq_row0 = dd.seq_row0, seq_len = dd.seq_len;
       __syncwarp();
       if (lane == 0) mbar_arrive(&d_empty[ds]);
       // The previous chunk's epilogue runs while the tensor core computes S(t).
       if (j > 0 && !epilogue(j - 1)) break;
       if (end) break;
-      int lim = 0;   // visible keys of this block for the row
+      int lim = 0;   // visible keys of this block for the row (positions local to its sequence)
       if (e >= 0) {
-        const int p = args.q_pos0 + (e >> 5);
-        const int kv_lim = args.causal ? min(p + 1, args.n_kv) : args.n_kv;
+        const int p = (args.cu_seqlens ? 0 : args.q_pos0) + (e >> 5) - seq_row0;
+        const int kv_lim = args.causal ? min(p + 1, seq_len) : seq_len;
         lim = min(BK, kv_lim - b * BK);
       }
       if (!mbar_wait(&s_full[g], j & 1, wc)) break;
@@ -479,14 +505,34 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------
 // schedule: block_ids -> per-(group, block) lists of (query, slot)
 // ---------------------------------------------------------------------------
-__global__ void sched_count_kernel(const int32_t* ids, long long total, int h_kv, int topk, int nb, int* cnt) {
+// Schedule geometry shared by the three kernels: a selection (query q, block
+// b local to q's sequence) maps to global block blk_pfx[s] + b of the packed
+// batch (one sequence: the block itself); -1 when b is no block of q's
+// sequence.
+struct SchedGeom {
+  const int* cu_seqlens;   // or null: one sequence of n_kv keys
+  const int* blk_pfx;
+  int batch, nb_one, bk;   // nb_one: blocks of the single sequence
+  int nb;                  // blocks of the schedule (bound of every global block)
+  __device__ __forceinline__ int global_block(int q, int b) const {
+    if (b < 0) return -1;
+    if (!cu_seqlens) return b < nb_one ? b : -1;
+    const int s = seq_search(cu_seqlens, batch, q);
+    const int L = cu_seqlens[s + 1] - cu_seqlens[s];
+    const int gb = blk_pfx[s] + b;
+    return (b < (L + bk - 1) / bk && gb < nb) ? gb : -1;
+  }
+};
+
+__global__ void sched_count_kernel(const int32_t* ids, long long total, int h_kv, int topk, int nb, SchedGeom geo,
+                                   int* cnt) {
   const long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (e >= total) return;
-  const int b = ids[e];
-  if (b < 0 || b >= nb) return;
+  const int q = static_cast<int>(e / (static_cast<long long>(topk) * h_kv));
+  const int gb = geo.global_block(q, ids[e]);
+  if (gb < 0) return;
   const int r = static_cast<int>((e / topk) % h_kv);
-  const int wave = static_cast<int>(e / (static_cast<long long>(topk) * h_kv)) / kWave;
-  atomicAdd(&cnt[(wave * h_kv + r) * nb + b], 1);
+  atomicAdd(&cnt[((q / kWave) * h_kv + r) * nb + gb], 1);
 }
 
 // One CTA: exclusive scans of cnt -> offs and of ceil(cnt / qpc) -> chunk_off,
@@ -578,15 +624,19 @@ __global__ void __launch_bounds__(1024) sched_scan_kernel(const int* cnt, int n,
 }
 
 __global__ void sched_fill_kernel(const int32_t* ids, long long total, int h_kv, int topk, int nb, int G,
-                                  const int* offs, const int* chunk_off, int* fill, int* entries, int* prow_of) {
+                                  SchedGeom geo, const int* offs, const int* chunk_off, int* fill, int* entries,
+                                  int* prow_of) {
   const long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (e >= total) return;
-  const int b = ids[e];
-  if (b < 0 || b >= nb) return;
+  const int q = static_cast<int>(e / (static_cast<long long>(topk) * h_kv));
+  const int gb = geo.global_block(q, ids[e]);
+  if (gb < 0) {
+    prow_of[e] = -1;   // padding: the merge skips it
+    return;
+  }
   const int slot = static_cast<int>(e % topk);
   const int r = static_cast<int>((e / topk) % h_kv);
-  const int q = static_cast<int>(e / (static_cast<long long>(topk) * h_kv));
-  const int rb = ((q / kWave) * h_kv + r) * nb + b;
+  const int rb = ((q / kWave) * h_kv + r) * nb + gb;
   const int k = atomicAdd(&fill[rb], 1);    // position inside the list
   entries[offs[rb] + k] = (q << 5) | slot;
   const int qpc = 128 / G;
@@ -597,9 +647,9 @@ __global__ void sched_fill_kernel(const int32_t* ids, long long total, int h_kv,
 // merge: O[q, h] = sum over valid slots of 2^(lse2_s - L) o_s
 // ---------------------------------------------------------------------------
 template <int D>
-__global__ void __launch_bounds__(256) merge_partials_kernel(const int32_t* ids, const int* prow_of,
-                                                             const uint16_t* part_o, const float* part_lse,
-                                                             uint16_t* o, int h_q, int h_kv, int topk, int nb) {
+__global__ void __launch_bounds__(256) merge_partials_kernel(const int* prow_of, const uint16_t* part_o,
+                                                             const float* part_lse, uint16_t* o, int h_q, int h_kv,
+                                                             int topk) {
   // One CTA per (query, group); thread = (8-column slice, head within the
   // group), heads fastest, so a warp reads whole 16 * G-byte runs of the
   // column-slice layout.  prow_of[(q, r, slot)] is the first partial row
@@ -612,7 +662,6 @@ __global__ void __launch_bounds__(256) merge_partials_kernel(const int32_t* ids,
   const int q = qr / h_kv, r = qr % h_kv;
   const int G = h_q / h_kv;
   constexpr int kChunks = D / 8;
-  const int32_t* my_ids = ids + static_cast<size_t>(qr) * topk;
   const int* my_rows = prow_of + static_cast<size_t>(qr) * topk;
   for (int w = threadIdx.x; w < G * kChunks; w += blockDim.x) {
     const int hh = w % G, ch = w / G;
@@ -624,9 +673,9 @@ __global__ void __launch_bounds__(256) merge_partials_kernel(const int32_t* ids,
 #pragma unroll
       for (int j = 0; j < kGrp; ++j) {
         const int s = s0 + j;
-        const int b = s < topk ? my_ids[s] : -1;
-        const bool ok = b >= 0 && b < nb;   // the schedule skips the others too
-        const size_t prow = ok ? static_cast<size_t>(my_rows[s]) + hh : 0;
+        const int pr = s < topk ? my_rows[s] : -1;   // -1: padding or no block of this sequence
+        const bool ok = pr >= 0;
+        const size_t prow = ok ? static_cast<size_t>(pr) + hh : 0;
         const size_t at = (((prow >> 7) * kChunks + ch) * 128 + (prow & 127)) * 8;
         ls[j] = ok ? part_lse[prow] : __int_as_float(0xff800000);
         v[j] = ok ? *reinterpret_cast<const uint4*>(part_o + at) : make_uint4(0, 0, 0, 0);
@@ -693,8 +742,15 @@ struct SparseWs {
   size_t max_chunks, bytes;
 };
 
-SparseWs carve(const msa_params& p, int n_q, int n_kv, void* base) {
-  const int nb = (n_kv + p.block_k - 1) / p.block_k;
+// Blocks of the schedule: those of the one sequence, or, for a packed batch
+// of `batch` sequences with n_kv rows in all, at most ceil(n_kv / B_k) +
+// batch (each sequence adds at most one partial block).
+int sched_blocks(const msa_params& p, int n_kv, int batch) {
+  return (n_kv + p.block_k - 1) / p.block_k + (batch > 0 ? batch : 0);
+}
+
+SparseWs carve(const msa_params& p, int n_q, int n_kv, int batch, void* base) {
+  const int nb = sched_blocks(p, n_kv, batch);
   const int n_waves = (n_q + kWave - 1) / kWave;
   const size_t nl = static_cast<size_t>(n_waves) * p.h_kv * nb;
   const size_t nnz = static_cast<size_t>(n_q) * p.h_kv * p.topk;
@@ -727,14 +783,15 @@ SparseWs carve(const msa_params& p, int n_q, int n_kv, void* base) {
 
 }  // namespace
 
-size_t sparse_prefill_workspace_bytes(const msa_params& p, int n_q, int n_kv) {
-  return carve(p, n_q, n_kv, nullptr).bytes;
+size_t sparse_prefill_workspace_bytes(const msa_params& p, int n_q, int n_kv, int batch) {
+  return carve(p, n_q, n_kv, batch, nullptr).bytes;
 }
 
 int run_sparse_attn_kvouter(const msa_params& p, const void* q, const CUtensorMap& tk, const CUtensorMap& tv,
                             const int32_t* block_ids, int n_q, int n_kv, int q_pos0, void* o, void* ws,
-                            size_t ws_bytes, int* status, cudaStream_t stream) {
-  SparseWs s = carve(p, n_q, n_kv, ws);
+                            size_t ws_bytes, int* status, cudaStream_t stream, const Varlen* vl) {
+  const int batch = vl ? vl->batch : 0;
+  SparseWs s = carve(p, n_q, n_kv, batch, ws);
   if (ws_bytes < s.bytes) return MSA_ERR_WORKSPACE;
   const int G = p.h_q / p.h_kv;
   CUtensorMap tq;   // one box = the G head rows of one query of one group
@@ -744,14 +801,21 @@ int run_sparse_attn_kvouter(const msa_params& p, const void* q, const CUtensorMa
     const uint32_t box[3] = {64, static_cast<uint32_t>(G), 1};
     if (!encode_tma_bf16(&tq, 3, q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MSA_ERR_CUDA;
   }
-  const int nb = (n_kv + p.block_k - 1) / p.block_k;
+  const int nb = sched_blocks(p, n_kv, batch);
   const int nl = ((n_q + kWave - 1) / kWave) * p.h_kv * nb;
   const long long total = static_cast<long long>(n_q) * p.h_kv * p.topk;
+  SchedGeom geo;
+  geo.cu_seqlens = vl ? vl->cu_seqlens : nullptr;
+  geo.blk_pfx = vl ? vl->blk_pfx : nullptr;
+  geo.batch = batch;
+  geo.nb_one = (n_kv + p.block_k - 1) / p.block_k;
+  geo.bk = p.block_k;
+  geo.nb = nb;
   if (cudaMemsetAsync(s.cnt, 0, (2 * static_cast<size_t>(nl) + 2) * 4, stream) != cudaSuccess) return MSA_ERR_CUDA;
   const int gsz = static_cast<int>((total + kSchedThreads - 1) / kSchedThreads);
-  sched_count_kernel<<<gsz, kSchedThreads, 0, stream>>>(block_ids, total, p.h_kv, p.topk, nb, s.cnt);
+  sched_count_kernel<<<gsz, kSchedThreads, 0, stream>>>(block_ids, total, p.h_kv, p.topk, nb, geo, s.cnt);
   sched_scan_kernel<<<1, 1024, 0, stream>>>(s.cnt, nl, 128 / G, s.offs, s.chunk_off, s.lists, s.n_lists);
-  sched_fill_kernel<<<gsz, kSchedThreads, 0, stream>>>(block_ids, total, p.h_kv, p.topk, nb, G, s.offs,
+  sched_fill_kernel<<<gsz, kSchedThreads, 0, stream>>>(block_ids, total, p.h_kv, p.topk, nb, G, geo, s.offs,
                                                        s.chunk_off, s.fill, s.entries, s.prow_of);
   if (cudaGetLastError() != cudaSuccess) return MSA_ERR_CUDA;
 
@@ -773,6 +837,9 @@ int run_sparse_attn_kvouter(const msa_params& p, const void* q, const CUtensorMa
   a.topk = p.topk;
   a.causal = p.causal;
   a.nb = nb;
+  a.cu_seqlens = geo.cu_seqlens;
+  a.blk_pfx = geo.blk_pfx;
+  a.batch = batch;
   const float scale = p.scale > 0.f ? p.scale : 1.0f / sqrtf(static_cast<float>(p.d));
   a.scale_log2 = scale * 1.4426950408889634f;
   int dev = 0, sms = 148;
@@ -791,11 +858,11 @@ int run_sparse_attn_kvouter(const msa_params& p, const void* q, const CUtensorMa
   if (e != cudaSuccess) return MSA_ERR_CUDA;
   const int mgrid = n_q * p.h_kv;
   if (p.d == 64)
-    merge_partials_kernel<64><<<mgrid, 256, 0, stream>>>(block_ids, s.prow_of, s.part_o, s.part_lse,
-                                                          static_cast<uint16_t*>(o), p.h_q, p.h_kv, p.topk, nb);
+    merge_partials_kernel<64><<<mgrid, 256, 0, stream>>>(s.prow_of, s.part_o, s.part_lse, static_cast<uint16_t*>(o),
+                                                          p.h_q, p.h_kv, p.topk);
   else
-    merge_partials_kernel<128><<<mgrid, 256, 0, stream>>>(block_ids, s.prow_of, s.part_o, s.part_lse,
-                                                           static_cast<uint16_t*>(o), p.h_q, p.h_kv, p.topk, nb);
+    merge_partials_kernel<128><<<mgrid, 256, 0, stream>>>(s.prow_of, s.part_o, s.part_lse, static_cast<uint16_t*>(o),
+                                                           p.h_q, p.h_kv, p.topk);
   return cudaGetLastError() == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
 }
 

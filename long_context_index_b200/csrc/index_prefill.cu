@@ -63,6 +63,13 @@ struct IdxArgs {
   int* status;
   int n_q, n_kv, q_pos0, h_kv, topk, causal, force_local, pool;
   int n_tiles;
+  // Packed batch of independent causal prefills (varlen), or null: sequence
+  // s owns rows [cu_seqlens[s], cu_seqlens[s + 1]) of Q_idx, K_idx and the
+  // ids, positions restart at 0, and block ids are local to the sequence.
+  const int* cu_seqlens;   // [batch + 1]
+  const int* tile_pfx;     // [batch + 1] prefix of ceil(L_s / 128) (query tiles per sequence)
+  const int* topk_seq;     // [batch] selected blocks of each sequence (adaptive k), or null: topk
+  int batch;
 };
 
 // Sorted-descending register list of KMAX (score, block) pairs.  Slots
@@ -120,18 +127,36 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = warp_id();
   const int lane = lane_id();
-  const int tile = args.n_tiles - 1 - static_cast<int>(blockIdx.x) / args.h_kv;  // heavy tiles first
   const int grp = static_cast<int>(blockIdx.x) % args.h_kv;
+  // The problem this CTA belongs to: the whole call, or one sequence of a
+  // packed batch (row_base = its first row; local positions from 0).
+  int tile, n_q = args.n_q, n_kv = args.n_kv, q_pos0 = args.q_pos0, row_base = 0, k_sel = args.topk;
+  if (args.cu_seqlens) {
+    const int tl = static_cast<int>(blockIdx.x) / args.h_kv;
+    if (tl >= args.tile_pfx[args.batch]) return;   // CTA-uniform, before any barrier or TMEM use
+    int lo = 0, hi = args.batch - 1;               // sequence: largest s with tile_pfx[s] <= tl
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (args.tile_pfx[mid] <= tl) lo = mid; else hi = mid - 1;
+    }
+    row_base = args.cu_seqlens[lo];
+    n_q = n_kv = args.cu_seqlens[lo + 1] - row_base;
+    q_pos0 = 0;
+    tile = args.tile_pfx[lo + 1] - 1 - tl;         // a sequence's heavy (late) tiles first
+    if (args.topk_seq) k_sel = min(max(args.topk_seq[lo], 1), args.topk);
+  } else {
+    tile = args.n_tiles - 1 - static_cast<int>(blockIdx.x) / args.h_kv;  // heavy tiles first
+  }
   const int i0 = tile * kRows;
-  const int rows_here = min(kRows, args.n_q - i0);
+  const int rows_here = min(kRows, n_q - i0);
 
   // Key range this CTA must score.  A row at position p needs keys < kv_lim(p)
   // where kv_lim = p + 1 (causal) or n_kv; with force_local its own block is
   // not scored, so it needs only keys below the start of that block.
-  const int p_last = args.q_pos0 + i0 + rows_here - 1;
+  const int p_last = q_pos0 + i0 + rows_here - 1;
   int kv_end;
   if (!args.causal) {
-    kv_end = args.n_kv;
+    kv_end = n_kv;
   } else if (args.force_local) {
     kv_end = (p_last / BK) * BK;
   } else {
@@ -169,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_k);
       mbar_arrive_expect_tx(q_full, Cfg::kQBytes);
       for (int a = 0; a < Cfg::kAtoms; ++a)
-        tma_load_3d(sq + a * kRows * Cfg::kSwB, &tm_q, q_full, a * (Cfg::kSwB / 2), grp, i0);
+        tma_load_3d(sq + a * kRows * Cfg::kSwB, &tm_q, q_full, a * (Cfg::kSwB / 2), grp, row_base + i0);
       for (int t = 0; t < n_ktiles; ++t) {
         const int s = t % Cfg::kStages;
         const uint32_t ph = (t / Cfg::kStages) & 1;
@@ -177,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&full[s], Cfg::kTileBytes);
         for (int a = 0; a < Cfg::kAtoms; ++a)
           tma_load_2d(sk + (s * Cfg::kAtoms + a) * kKeys * Cfg::kSwB, &tm_k, &full[s], a * (Cfg::kSwB / 2),
-                      t * kKeys);
+                      row_base + t * kKeys);
       }
     }
   } else if (warp == 1) {
@@ -221,10 +246,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int half = (warp - kEpiWarp0) >> 2;   // columns [128 half, 128 half + 128) of each tile
     const int row = quarter * 32 + lane;
     const bool row_ok = row < rows_here;
-    const int p = args.q_pos0 + i0 + row;
-    const int kv_lim = args.causal ? min(p + 1, args.n_kv) : args.n_kv;
+    const int p = q_pos0 + i0 + row;
+    const int kv_lim = args.causal ? min(p + 1, n_kv) : n_kv;
     const int b_loc = p / BK;
-    const int k_free = args.topk - (args.force_local ? 1 : 0);
+    const int k_free = k_sel - (args.force_local ? 1 : 0);
     TopK<KMAX> tk;
     tk.init(k_free);
     const uint32_t taddr_row = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + half * 128;
@@ -357,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ids[i + 1] = hi;
         }
       }
-      int32_t* out = args.block_ids + (static_cast<size_t>(i0 + row) * args.h_kv + grp) * args.topk;
+      int32_t* out = args.block_ids + (static_cast<size_t>(row_base + i0 + row) * args.h_kv + grp) * args.topk;
 #pragma unroll
       for (int i = 0; i < KMAX + 1; ++i)
         if (i < args.topk) out[i] = ids[i] == 0x7fffffff ? -1 : ids[i];
@@ -400,7 +425,7 @@ cudaError_t launch_b(int bk, const CUtensorMap& tq, const CUtensorMap& tk, const
 }  // namespace
 
 int run_index_topk_prefill(const msa_params& p, const void* q_idx, const void* k_idx, int n_q, int n_kv,
-                           int q_pos0, int32_t* block_ids, int* status, cudaStream_t stream) {
+                           int q_pos0, int32_t* block_ids, int* status, cudaStream_t stream, const Varlen* vl) {
   if (n_q == 0) return MSA_OK;
   const int sw_elems = p.d_idx >= 64 ? 64 : p.d_idx;    // TMA box inner extent (elements)
   const CUtensorMapSwizzle swz = p.d_idx >= 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
@@ -430,6 +455,13 @@ int run_index_topk_prefill(const msa_params& p, const void* q_idx, const void* k
   a.force_local = p.force_local;
   a.pool = p.pool;
   a.n_tiles = (n_q + kRows - 1) / kRows;
+  a.cu_seqlens = vl ? vl->cu_seqlens : nullptr;
+  a.tile_pfx = vl ? vl->tile_pfx : nullptr;
+  a.topk_seq = vl ? vl->topk_seq : nullptr;
+  a.batch = vl ? vl->batch : 0;
+  // A packed batch has at most n_tiles + batch query tiles (each sequence adds
+  // at most one partial tile); CTAs past the last tile exit at once.
+  if (vl) a.n_tiles += vl->batch;
   cudaError_t e;
   switch (p.d_idx) {
     case 32: e = launch_b<32>(p.block_k, tq, tk, a, stream); break;

@@ -105,6 +105,10 @@ size_t msa_workspace_size(int op, const msa_params* p, int n_q, int n_kv, int ba
     case MSA_OP_DECODE:
       if (batch <= 0 || max_kv <= 0 || max_kv > kMaxRows) return 0;
       return kWsHeader + align_up(decode_workspace_bytes(*p, batch, max_kv, -1), 256);
+    case MSA_OP_INDEX_TOPK_VARLEN:
+    case MSA_OP_PREFILL_VARLEN:
+      if (batch <= 0 || check_rows(n_q, n_q > 0 ? n_q : 1, 0) != MSA_OK) return 0;
+      return varlen_workspace_bytes(op, *p, batch, n_q);
     default:
       return 0;
   }
@@ -170,13 +174,52 @@ int msa_sparse_attn_decode(const msa_params* p, const void* q, const void* q_idx
                                 static_cast<int*>(ws), st);
 }
 
+namespace {
+int varlen_call(int op, const msa_params* p, const void* a0, const void* a1, const void* a2, const int32_t* cu,
+                int batch, int total, const int32_t* topk_seq, const int32_t* ids_in, int32_t* ids_out, void* o,
+                void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_params(p);
+  if (rc) return rc;
+  if (batch <= 0 || total < 0 || !cu) return MSA_ERR_INVALID;
+  if (total > kMaxRows || batch > kMaxRows) return MSA_ERR_UNSUPPORTED;
+  if ((rc = check_ws(ws, ws_bytes, varlen_workspace_bytes(op, *p, batch, total)))) return rc;
+  if ((reinterpret_cast<uintptr_t>(cu) & 3u) != 0) return MSA_ERR_MISALIGNED;
+  if (topk_seq && (reinterpret_cast<uintptr_t>(topk_seq) & 3u) != 0) return MSA_ERR_MISALIGNED;
+  if (total > 0) {
+    if (!a0 || !a1 || (op == MSA_OP_PREFILL_VARLEN && (!a2 || !ids_in || !o)) ||
+        (op == MSA_OP_INDEX_TOPK_VARLEN && !ids_out))
+      return MSA_ERR_INVALID;
+    if (!aligned16(a0) || !aligned16(a1) || (a2 && !aligned16(a2)) || (o && !aligned16(o)) ||
+        (ids_in && !aligned16(ids_in)) || (ids_out && !aligned16(ids_out)))
+      return MSA_ERR_MISALIGNED;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((rc = clear_status(ws, st))) return rc;
+  return run_varlen(op, *p, a0, a1, a2, cu, batch, total, topk_seq, ids_in, ids_out, o, ws, ws_bytes, st);
+}
+}  // namespace
+
+int msa_index_topk_varlen(const msa_params* p, const void* q_idx, const void* k_idx, const int32_t* cu_seqlens,
+                          int batch, int total, const int32_t* topk_per_seq, int32_t* block_ids, void* ws,
+                          size_t ws_bytes, void* stream) {
+  return varlen_call(MSA_OP_INDEX_TOPK_VARLEN, p, q_idx, k_idx, nullptr, cu_seqlens, batch, total, topk_per_seq,
+                     nullptr, block_ids, nullptr, ws, ws_bytes, stream);
+}
+
+int msa_sparse_attn_prefill_varlen(const msa_params* p, const void* q, const void* k, const void* v,
+                                   const int32_t* cu_seqlens, int batch, int total, const int32_t* block_ids,
+                                   void* o, void* ws, size_t ws_bytes, void* stream) {
+  return varlen_call(MSA_OP_PREFILL_VARLEN, p, q, k, v, cu_seqlens, batch, total, nullptr, block_ids, nullptr, o, ws,
+                     ws_bytes, stream);
+}
+
 int msa_device_status(const void* ws, void* stream) {
   if (!ws) return MSA_ERR_INVALID;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(st) != cudaSuccess) return MSA_ERR_CUDA;
   int s = 0;
   if (cudaMemcpy(&s, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MSA_ERR_CUDA;
-  return s == kDevOk ? MSA_OK : MSA_ERR_TIMEOUT;
+  return s == kDevOk ? MSA_OK : (s == kDevBadInput ? MSA_ERR_INVALID : MSA_ERR_TIMEOUT);
 }
 
 const char* msa_status_string(int status) {

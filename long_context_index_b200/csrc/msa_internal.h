@@ -22,20 +22,50 @@ constexpr size_t kWsHeader = 256;
 bool encode_tma_bf16(CUtensorMap* map, int rank, const void* base, const uint64_t* dims,
                      const uint64_t* strides, const uint32_t* box, CUtensorMapSwizzle swizzle);
 
+// A packed batch of independent causal prefills (the varlen entry points):
+// sequence s owns rows [cu_seqlens[s], cu_seqlens[s + 1]) of every tensor.
+// The prefixes are built on the device by run_varlen_prep.
+struct Varlen {
+  const int* cu_seqlens;   // device [batch + 1]
+  const int* tile_pfx;     // device [batch + 1]: prefix of ceil(L_s / 128) (index query tiles)
+  const int* blk_pfx;      // device [batch + 1]: prefix of ceil(L_s / B_k) (KV blocks)
+  const int* topk_seq;     // device [batch] per-sequence k (index branch only), or null
+  int batch;
+};
+
+// Device status word value for a packed batch whose cu_seqlens is not a
+// valid prefix (cu[0] = 0, non-decreasing, cu[batch] = total rows).
+constexpr int kDevBadInput = 2;
+
+// Builds tile_pfx and blk_pfx from cu_seqlens (one CTA); an invalid
+// cu_seqlens sets the status word and zero prefixes, so no sequence has work.
+int run_varlen_prep(const int* cu_seqlens, int batch, int total, int block_k, int* tile_pfx, int* blk_pfx,
+                    int* status, cudaStream_t stream);
+
 int run_index_topk_prefill(const msa_params& p, const void* q_idx, const void* k_idx, int n_q, int n_kv,
-                           int q_pos0, int32_t* block_ids, int* status, cudaStream_t stream);
+                           int q_pos0, int32_t* block_ids, int* status, cudaStream_t stream,
+                           const Varlen* vl = nullptr);
+
+// The varlen entry points (varlen.cu): workspace bytes (header included) and
+// the run of MSA_OP_INDEX_TOPK_VARLEN (a0, a1 = q_idx, k_idx; ids_out) or
+// MSA_OP_PREFILL_VARLEN (a0, a1, a2 = q, k, v; ids_in; o).
+size_t varlen_workspace_bytes(int op, const msa_params& p, int batch, int total);
+int run_varlen(int op, const msa_params& p, const void* a0, const void* a1, const void* a2, const int32_t* cu,
+               int batch, int total, const int32_t* topk_seq, const int32_t* ids_in, int32_t* ids_out, void* o,
+               void* ws, size_t ws_bytes, cudaStream_t stream);
 
 // Prefill main branch.  ws/ws_bytes: the op's workspace after the header.
-size_t prefill_workspace_bytes(const msa_params& p, int n_q, int n_kv);
+// batch > 0: a packed batch of that many sequences (n_q = n_kv = total rows).
+size_t prefill_workspace_bytes(const msa_params& p, int n_q, int n_kv, int batch = 0);
 int run_sparse_attn_prefill(const msa_params& p, const void* q, const void* k, const void* v,
                             const int32_t* block_ids, int n_q, int n_kv, int q_pos0, void* o, void* ws,
-                            size_t ws_bytes, int* status, cudaStream_t stream);
+                            size_t ws_bytes, int* status, cudaStream_t stream, const Varlen* vl = nullptr);
 
 // Block-major sparse prefill (attn_sparse.cu).
-size_t sparse_prefill_workspace_bytes(const msa_params& p, int n_q, int n_kv);
+size_t sparse_prefill_workspace_bytes(const msa_params& p, int n_q, int n_kv, int batch);
 int run_sparse_attn_kvouter(const msa_params& p, const void* q, const CUtensorMap& tk, const CUtensorMap& tv,
                             const int32_t* block_ids, int n_q, int n_kv, int q_pos0, void* o, void* ws,
-                            size_t ws_bytes, int* status, cudaStream_t stream);
+                            size_t ws_bytes, int* status, cudaStream_t stream, const Varlen* vl);
 
 // Decode step.
 // Limits of the decode kernels (checked on the host before any launch).

@@ -155,3 +155,57 @@ def decode(P: Params, q, q_idx, k_cache, v_cache, k_idx_cache, cu_kv, seqs=None,
     if rc:
         raise ValueError("oracle decode: bad arguments (%d)" % rc)
     return ids, o
+
+
+# ---------------------------------------------------------------------------
+# Packed batches (cu_seqlens): each sequence is an independent problem, so the
+# oracle of the batch is the single-sequence oracle on each sequence's rows.
+# ---------------------------------------------------------------------------
+def _seq_rows(cu, rows):
+    """Per sequence: (s, lo, hi, local row indices or None for all rows, positions in `rows`)."""
+    cu = np.asarray(cu, dtype=np.int64)
+    out = []
+    if rows is None:
+        for s in range(len(cu) - 1):
+            out.append((s, int(cu[s]), int(cu[s + 1]), None, None))
+        return out
+    rows = np.asarray(rows, dtype=np.int64)
+    seq = np.searchsorted(cu, rows, side="right") - 1
+    for s in np.unique(seq):
+        sel = np.nonzero(seq == s)[0]
+        out.append((int(s), int(cu[s]), int(cu[s + 1]), rows[sel] - cu[s], sel))
+    return out
+
+
+def index_topk_varlen(P: Params, q_idx, k_idx, cu_seqlens, topk_per_seq=None, rows=None) -> np.ndarray:
+    """Block ids of a packed batch [rows or total, h_kv, topk]: each sequence
+    selects with its own k (topk_per_seq, clamped to [1, topk]) and pads to
+    topk with -1; ids are local to the sequence."""
+    n = q_idx.shape[0] if rows is None else len(rows)
+    out = np.full((n, P.h_kv, P.topk), -1, dtype=np.int32)
+    for s, lo, hi, loc, pos in _seq_rows(cu_seqlens, rows):
+        if hi <= lo:
+            continue
+        k = P.topk if topk_per_seq is None else int(min(max(int(topk_per_seq[s]), 1), P.topk))
+        Ps = Params(*[getattr(P, f[0]) for f in P._fields_])
+        Ps.topk = k
+        ids = index_topk(Ps, q_idx[lo:hi], k_idx[lo:hi], 0, rows=loc)
+        if pos is None:
+            out[lo:hi, :, :k] = ids
+        else:
+            out[pos, :, :k] = ids
+    return out
+
+
+def sparse_attn_varlen(P: Params, q, k, v, ids, cu_seqlens, rows=None) -> np.ndarray:
+    """Main branch of a packed batch over the given ids (one list per listed row)."""
+    n = q.shape[0] if rows is None else len(rows)
+    out = np.zeros((n, P.h_q, P.d), dtype=np.float64)
+    for s, lo, hi, loc, pos in _seq_rows(cu_seqlens, rows):
+        if hi <= lo:
+            continue
+        if pos is None:
+            out[lo:hi] = sparse_attn(P, q[lo:hi], k[lo:hi], v[lo:hi], ids[lo:hi], 0)
+        else:
+            out[pos] = sparse_attn(P, q[lo:hi], k[lo:hi], v[lo:hi], ids[pos], 0, rows=loc)
+    return out

@@ -230,3 +230,40 @@ def make_decode(w: Workload, batch: Optional[int] = None, kv_min: Optional[int] 
                     needles.append((b, r, pk))
     out["needles"] = needles
     return out
+
+
+def make_varlen_prefill(w: Workload, lens: Optional[List[int]] = None) -> dict:
+    """A packed batch of independent causal prefills (cu_seqlens layout).
+
+    ``w.batch`` sequences with lengths drawn uniformly from
+    [w.kv_min, w.kv_max] (or the given ``lens``); sequence s is drawn like a
+    full prefill of its own length with seed (w.seed, s) -- values, index
+    integers and needles -- and the sequences are stored back to back.
+    Returns q, k, v, q_idx, k_idx (packed, uint16 bf16 bits), lens,
+    cu_seqlens (int32 [batch + 1]) and needles as (sequence, group,
+    query_row, key_position) in sequence-local coordinates.
+    """
+    if lens is None:
+        g = _rng(w.seed, _T_LENS, 0)
+        lens = g.integers(w.kv_min, w.kv_max + 1, size=w.batch).tolist()
+    parts = []
+    needles = []
+    for s, L in enumerate(lens):
+        ws = Workload(**{**w.__dict__, "kind": "prefill", "seed": w.seed * 1000003 + s, "n_q": int(L),
+                         "n_kv": int(L)})
+        t = make_prefill(ws) if L > 0 else None
+        if t is not None:
+            needles += [(s, r, i, pk) for (r, i, pk) in t["needles"]]
+        parts.append(t)
+    cu = np.zeros(len(lens) + 1, dtype=np.int32)
+    cu[1:] = np.cumsum(lens)
+    shapes = {"q": (w.h_q, w.d), "k": (w.h_kv, w.d), "v": (w.h_kv, w.d), "q_idx": (w.h_kv, w.d_idx),
+              "k_idx": (1, w.d_idx)}
+    out = {}
+    for name, sh in shapes.items():
+        chunks = [t[name] for t in parts if t is not None]
+        out[name] = (np.concatenate(chunks, axis=0) if chunks else np.zeros((0,) + sh, dtype=np.uint16))
+    out["lens"] = np.asarray(lens, dtype=np.int64)
+    out["cu_seqlens"] = cu
+    out["needles"] = needles
+    return out

@@ -110,3 +110,37 @@ def test_mean_topk_matches_numpy_means_and_exhaustive_search(k, force_local):
             want = brute_force_select(row, i // B, k, force_local)
             got = [x for x in ids[i, r] if x >= 0]
             assert got == want, (i, r, got, want)
+
+
+# ----------------------------------------------------------------------------
+# Packed batches and adaptive k (oracle helpers built on the pinned functions)
+# ----------------------------------------------------------------------------
+def test_varlen_batch_of_one_is_the_single_sequence_oracle():
+    from synth import Workload, make_varlen_prefill
+    w = Workload("v", "varlen", h_q=4, h_kv=2, d=8, d_idx=4, block_k=8, topk=3, seed=9, batch=1, needles=0)
+    t = make_varlen_prefill(w, lens=[70])
+    prm = P(h_q=4, h_kv=2, d=8, d_idx=4, block_k=8, topk=3, pool=oracle.POOL_MAX)
+    a = oracle.index_topk_varlen(prm, t["q_idx"], t["k_idx"], t["cu_seqlens"])
+    assert np.array_equal(a, oracle.index_topk(prm, t["q_idx"], t["k_idx"]))
+
+
+def test_adaptive_k_keeps_a_prefix_of_the_ranking():
+    # Selecting k_s blocks keeps exactly the k_s best of the ranking that a
+    # larger k uses: every id kept at k_s is kept at topk, and the count is
+    # min(k_s, eligible blocks).
+    from synth import Workload, make_varlen_prefill
+    w = Workload("v", "varlen", h_q=4, h_kv=2, d=8, d_idx=4, block_k=8, topk=6, seed=10, batch=3, needles=0)
+    t = make_varlen_prefill(w, lens=[90, 33, 120])
+    prm = P(h_q=4, h_kv=2, d=8, d_idx=4, block_k=8, topk=6, pool=oracle.POOL_MAX)
+    full = oracle.index_topk_varlen(prm, t["q_idx"], t["k_idx"], t["cu_seqlens"])
+    ks = [2, 6, 1]
+    part = oracle.index_topk_varlen(prm, t["q_idx"], t["k_idx"], t["cu_seqlens"], topk_per_seq=ks)
+    cu = t["cu_seqlens"]
+    for s in range(3):
+        for i in range(cu[s], cu[s + 1]):
+            for r in range(2):
+                a = set(part[i, r][part[i, r] >= 0].tolist())
+                b = set(full[i, r][full[i, r] >= 0].tolist())
+                assert a <= b and len(a) == min(ks[s], len(b))
+                local = (i - cu[s]) // 8
+                assert local in a            # the local block is always kept
