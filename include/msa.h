@@ -186,6 +186,21 @@ MSA_API int msa_sparse_attn_prefill_varlen(const msa_params* p, const void* q, c
                                            void* stream);
 
 /*
+ * msa_sparse_attn_decode with adaptive k: sequence b keeps
+ * min(max(topk_per_seq[b], 1), p->topk) blocks (its local block included when
+ * force_local), its remaining ids being -1 -- the per-sequence choice of k
+ * that titansim.online section 5.3 names as future work.  topk_per_seq is
+ * int32 [batch] DEVICE memory, or NULL (every sequence keeps p->topk: exactly
+ * msa_sparse_attn_decode).  Ignored when dense.  Everything else as for
+ * msa_sparse_attn_decode; the workspace is the same.
+ */
+MSA_API int msa_sparse_attn_decode_adaptive_k(const msa_params* p, const void* q, const void* q_idx,
+                                              const void* k_cache, const void* v_cache, const void* k_idx_cache,
+                                              const int64_t* cu_kv, const int32_t* topk_per_seq, int batch,
+                                              int max_kv, int dense, int32_t* block_ids, void* o, void* ws,
+                                              size_t ws_bytes, void* stream);
+
+/*
  * Device status recorded by the last call that used workspace `ws`: MSA_OK,
  * MSA_ERR_TIMEOUT when one of its kernels gave up a bounded wait, or
  * MSA_ERR_INVALID when a varlen call found cu_seqlens invalid.  Every

@@ -24,7 +24,8 @@ OP_INDEX_TOPK, OP_PREFILL, OP_DECODE, OP_INDEX_TOPK_VARLEN, OP_PREFILL_VARLEN = 
 POOL_MAX, POOL_MEAN = 0, 1   # msa_params.pool
 
 SYMBOLS = ("msa_workspace_size", "msa_index_topk", "msa_sparse_attn_prefill", "msa_sparse_attn_decode",
-           "msa_index_topk_varlen", "msa_sparse_attn_prefill_varlen", "msa_device_status", "msa_status_string",
+           "msa_index_topk_varlen", "msa_sparse_attn_prefill_varlen", "msa_sparse_attn_decode_adaptive_k",
+           "msa_device_status", "msa_status_string",
            "msa_sparse_attn_decode_noalloc", "msa_test_never_ready_wait")
 
 
@@ -66,6 +67,8 @@ def lib():
         L.msa_index_topk.argtypes = [P, vp, vp, i32, i32, i32, vp, vp, sz, vp]
         L.msa_sparse_attn_prefill.argtypes = [P, vp, vp, vp, vp, i32, i32, i32, vp, vp, sz, vp]
         L.msa_sparse_attn_decode.argtypes = [P, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, vp, vp, sz, vp]
+        L.msa_sparse_attn_decode_adaptive_k.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, vp,
+                                                        vp, sz, vp]
         L.msa_index_topk_varlen.argtypes = [P, vp, vp, vp, i32, i32, vp, vp, vp, sz, vp]
         L.msa_sparse_attn_prefill_varlen.argtypes = [P, vp, vp, vp, vp, i32, i32, vp, vp, vp, sz, vp]
         L.msa_sparse_attn_decode_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, vp, vp]
@@ -76,7 +79,7 @@ def lib():
         L.msa_status_string.argtypes = [i32]
         L.msa_status_string.restype = C.c_char_p
         for f in ("msa_index_topk", "msa_sparse_attn_prefill", "msa_sparse_attn_decode", "msa_device_status",
-                  "msa_index_topk_varlen", "msa_sparse_attn_prefill_varlen"):
+                  "msa_index_topk_varlen", "msa_sparse_attn_prefill_varlen", "msa_sparse_attn_decode_adaptive_k"):
             getattr(L, f).restype = i32
         _lib = L
     return _lib
@@ -177,8 +180,9 @@ def sparse_attn_prefill(p: Params, q, k, v, block_ids=None, q_pos0: int = 0, out
 
 
 def sparse_attn_decode(p: Params, q, q_idx, k_cache, v_cache, k_idx_cache, cu_kv, max_kv: int, dense=False,
-                       block_ids=None, out=None, ws=None, stream=None):
-    """One decode step: (block_ids [B, h_kv, topk] or None when dense, O [B, h_q, d])."""
+                       block_ids=None, out=None, ws=None, stream=None, topk_per_seq=None):
+    """One decode step: (block_ids [B, h_kv, topk] or None when dense, O [B, h_q, d]).
+    ``topk_per_seq`` (int32 [B], optional): blocks kept per sequence (adaptive k)."""
     torch = _torch()
     B = q.shape[0]
     tot = k_cache.shape[0]
@@ -196,11 +200,19 @@ def sparse_attn_decode(p: Params, q, q_idx, k_cache, v_cache, k_idx_cache, cu_kv
         out = torch.empty((B, p.h_q, p.d), dtype=torch.bfloat16, device=q.device)
     _check(out, "out", _bf16(), (B, p.h_q, p.d))
     ws = _workspace(OP_DECODE, p, batch=B, max_kv=max_kv, ws=ws, device=q.device)
-    rc = lib().msa_sparse_attn_decode(C.byref(p), _ptr(q), _ptr(q_idx) if not dense else None,
-                                      _ptr(k_cache), _ptr(v_cache), _ptr(k_idx_cache) if not dense else None,
-                                      _ptr(cu_kv), B, int(max_kv), int(bool(dense)),
-                                      _ptr(block_ids) if not dense else None, _ptr(out), _ptr(ws), ws.numel(),
-                                      _stream(stream))
+    if topk_per_seq is not None:
+        _check(topk_per_seq, "topk_per_seq", (torch.int32,), (B,))
+        rc = lib().msa_sparse_attn_decode_adaptive_k(
+            C.byref(p), _ptr(q), _ptr(q_idx) if not dense else None, _ptr(k_cache), _ptr(v_cache),
+            _ptr(k_idx_cache) if not dense else None, _ptr(cu_kv), _ptr(topk_per_seq), B, int(max_kv),
+            int(bool(dense)), _ptr(block_ids) if not dense else None, _ptr(out), _ptr(ws), ws.numel(),
+            _stream(stream))
+    else:
+        rc = lib().msa_sparse_attn_decode(C.byref(p), _ptr(q), _ptr(q_idx) if not dense else None,
+                                          _ptr(k_cache), _ptr(v_cache), _ptr(k_idx_cache) if not dense else None,
+                                          _ptr(cu_kv), B, int(max_kv), int(bool(dense)),
+                                          _ptr(block_ids) if not dense else None, _ptr(out), _ptr(ws), ws.numel(),
+                                          _stream(stream))
     if rc:
         raise MSAError(rc, "msa_sparse_attn_decode")
     _after(ws, stream, "msa_sparse_attn_decode")

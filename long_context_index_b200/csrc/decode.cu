@@ -105,6 +105,7 @@ struct DecArgs {
   int batch, h_q, h_kv, topk, causal, force_local, kfree, idx_ctas, idx_wmax;
   int splits, slots_per_split, dense, head_tiles, pool;
   float scale_log2;
+  const int32_t* topk_seq;  // [B] blocks kept per sequence (adaptive k), or null: topk
 };
 
 // ---------------------------------------------------------------------------
@@ -338,6 +339,10 @@ __device__ void merge_topk_warp(const DecArgs& a, int b, int r, int lane, int* c
   const int L = static_cast<int>(a.cu_kv[b + 1] - a.cu_kv[b]);
   const int b_loc = (L - 1) / BK;
   const int ncand = nseg * a.kfree;
+  // Adaptive k: this sequence keeps its own number of blocks.  Every share
+  // kept its top kfree >= kfree_b, so the global top kfree_b is among them.
+  const int kb = a.topk_seq ? min(max(static_cast<int>(a.topk_seq[b]), 1), a.topk) : a.topk;
+  const int kfree_b = min(a.kfree, kb - (a.force_local ? 1 : 0));
   auto cand_index = [&](int c) -> long long {   // -1: share of an empty range
     const int sg = c / a.kfree, slot = c - sg * a.kfree;
     const long long cc = c_lo + sg;
@@ -367,7 +372,7 @@ __device__ void merge_topk_warp(const DecArgs& a, int b, int r, int lane, int* c
     }
     float new_s = kNegInf;
     int new_b = -1;
-    for (int k = 0; k < a.kfree; ++k) {
+    for (int k = 0; k < kfree_b; ++k) {
       float bs = run_s;
       int bi = run_b >= 0 ? run_b : 0x7fffffff;
 #pragma unroll
@@ -1231,7 +1236,7 @@ size_t decode_workspace_bytes(const msa_params& p, int batch, int max_kv, int de
 int run_sparse_attn_decode(const msa_params& p, const void* q, const void* q_idx, const void* k_cache,
                            const void* v_cache, const void* k_idx_cache, const int64_t* cu_kv, int batch,
                            int max_kv, int dense, int32_t* block_ids, void* o, void* ws, size_t /*ws_bytes*/,
-                           int* status, cudaStream_t stream) {
+                           int* status, cudaStream_t stream, const int32_t* topk_seq) {
   if (p.h_kv > kDecodeMaxGroups) return MSA_ERR_UNSUPPORTED;
   // TMA row coordinates of the caches are 32-bit.
   if (!dense && static_cast<long long>(batch) * max_kv > 0x7fffffffLL) return MSA_ERR_UNSUPPORTED;
@@ -1254,6 +1259,7 @@ int run_sparse_attn_decode(const msa_params& p, const void* q, const void* q_idx
   a.force_local = p.force_local;
   a.kfree = p.topk - (p.force_local ? 1 : 0);
   a.pool = p.pool;
+  a.topk_seq = topk_seq;
   const IdxPlan ip = plan_index(p, batch, max_kv);
   a.idx_ctas = ip.ctas;
   a.idx_wmax = ip.wmax;

@@ -145,10 +145,10 @@ int msa_sparse_attn_prefill(const msa_params* p, const void* q, const void* k, c
                                  static_cast<int*>(ws), st);
 }
 
-int msa_sparse_attn_decode(const msa_params* p, const void* q, const void* q_idx, const void* k_cache,
-                           const void* v_cache, const void* k_idx_cache, const int64_t* cu_kv, int batch,
-                           int max_kv, int dense, int32_t* block_ids, void* o, void* ws, size_t ws_bytes,
-                           void* stream) {
+int msa_sparse_attn_decode_adaptive_k(const msa_params* p, const void* q, const void* q_idx, const void* k_cache,
+                                      const void* v_cache, const void* k_idx_cache, const int64_t* cu_kv,
+                                      const int32_t* topk_per_seq, int batch, int max_kv, int dense,
+                                      int32_t* block_ids, void* o, void* ws, size_t ws_bytes, void* stream) {
   int rc = check_params(p);
   if (rc) return rc;
   if (batch <= 0 || max_kv <= 0 || (dense != 0 && dense != 1)) return MSA_ERR_INVALID;
@@ -165,13 +165,22 @@ int msa_sparse_attn_decode(const msa_params* p, const void* q, const void* q_idx
   if (!dense && (!q_idx || !k_idx_cache || !block_ids)) return MSA_ERR_INVALID;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o)) return MSA_ERR_MISALIGNED;
   if ((reinterpret_cast<uintptr_t>(cu_kv) & 7u) != 0) return MSA_ERR_MISALIGNED;
+  if (topk_per_seq && (reinterpret_cast<uintptr_t>(topk_per_seq) & 3u) != 0) return MSA_ERR_MISALIGNED;
   if (!dense && (!aligned16(q_idx) || !aligned16(k_idx_cache) || !aligned16(block_ids))) return MSA_ERR_MISALIGNED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // One memset clears the status word and the decode completion counters.
   if (cudaMemsetAsync(ws, 0, kWsHeader + decode_counter_bytes(*p, batch), st) != cudaSuccess) return MSA_ERR_CUDA;
   return run_sparse_attn_decode(*p, q, q_idx, k_cache, v_cache, k_idx_cache, cu_kv, batch, max_kv, dense,
                                 block_ids, o, static_cast<uint8_t*>(ws) + kWsHeader, ws_bytes - kWsHeader,
-                                static_cast<int*>(ws), st);
+                                static_cast<int*>(ws), st, dense ? nullptr : topk_per_seq);
+}
+
+int msa_sparse_attn_decode(const msa_params* p, const void* q, const void* q_idx, const void* k_cache,
+                           const void* v_cache, const void* k_idx_cache, const int64_t* cu_kv, int batch,
+                           int max_kv, int dense, int32_t* block_ids, void* o, void* ws, size_t ws_bytes,
+                           void* stream) {
+  return msa_sparse_attn_decode_adaptive_k(p, q, q_idx, k_cache, v_cache, k_idx_cache, cu_kv, nullptr, batch, max_kv,
+                                           dense, block_ids, o, ws, ws_bytes, stream);
 }
 
 namespace {

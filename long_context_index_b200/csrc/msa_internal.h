@@ -77,7 +77,7 @@ size_t decode_workspace_bytes(const msa_params& p, int batch, int max_kv, int de
 int run_sparse_attn_decode(const msa_params& p, const void* q, const void* q_idx, const void* k_cache,
                            const void* v_cache, const void* k_idx_cache, const int64_t* cu_kv, int batch,
                            int max_kv, int dense, int32_t* block_ids, void* o, void* ws, size_t ws_bytes,
-                           int* status, cudaStream_t stream);
+                           int* status, cudaStream_t stream, const int32_t* topk_seq = nullptr);
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 

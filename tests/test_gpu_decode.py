@@ -98,6 +98,28 @@ def test_many_items_per_cta():
     run_case(w, seqs=[0, 1, 777, 2047])
 
 
+@pytest.mark.parametrize("pool", [0, 1])
+def test_adaptive_k_per_sequence(pool):
+    # Each sequence keeps its own number of blocks: ids equal the oracle's
+    # selection with that k (local block included), padded with -1.
+    w = small(h_q=64, h_kv=4, d=128, d_idx=64, block_k=128, topk=16, batch=7, kv_min=3000, kv_max=30000, seed=45)
+    t = make_decode(w)
+    ks = np.array([16, 1, 5, 2, 40, 9, 16], dtype=np.int32)
+    p, _ = params_pair(w.h_q, w.h_kv, w.d, w.d_idx, w.block_k, w.topk, pool=pool)
+    ids, o = msa.sparse_attn_decode(p, dev(t["q"]), dev(t["q_idx"]), dev(t["k_cache"]), dev(t["v_cache"]),
+                                    dev(t["k_idx_cache"]), dev(t["cu_kv"]), int(t["lens"].max()),
+                                    topk_per_seq=torch.from_numpy(ks).cuda())
+    torch.cuda.synchronize()
+    got_ids, got_o = ids.cpu().numpy(), host_f64(o)
+    for b in range(w.batch):
+        kb = int(min(max(ks[b], 1), w.topk))
+        _, po = params_pair(w.h_q, w.h_kv, w.d, w.d_idx, w.block_k, kb, pool=pool)
+        ids_ref, o_ref = oracle.decode(po, t["q"], t["q_idx"], t["k_cache"], t["v_cache"], t["k_idx_cache"],
+                                       t["cu_kv"], seqs=[b])
+        assert np.array_equal(got_ids[b, :, :kb], ids_ref[0]) and np.all(got_ids[b, :, kb:] == -1), b
+        assert_close(got_o[b], o_ref[0], what="adaptive-k decode O, sequence %d" % b)
+
+
 def test_decode_equals_prefill_row_at_last_position():
     # Entry-point consistency: a decode step and a one-row chunked prefill at
     # q_pos0 = L_b - 1 over the same caches run different kernels but must
