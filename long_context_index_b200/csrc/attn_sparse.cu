@@ -13,27 +13,38 @@
 //      query's ids).  Lists are handed out in (wave, group, block) order, so
 //      at any moment the CTAs gather the queries of one wave of kWave rows,
 //      whose Q rows (kWave x h_q x d x 2 bytes) stay resident in L2.
-//   2. attn_kvouter_kernel (persistent, warp-specialised, tcgen05; 12 warps):
+//   2. attn_kvouter_kernel (persistent, warp-specialised, tcgen05):
 //      * warp 0 grabs the next (r, b) list with an atomic counter, loads K_b
 //        by TMA, then streams chunks of 128/G queries of the list (each
 //        query's G head rows of group r are one 3-D TMA box, gathered with an
-//        L2 evict-last policy into a 4-stage ring) and publishes a descriptor
+//        L2 evict-last policy into a 3-stage ring) and publishes a descriptor
 //        per chunk in an 8-deep ring; V_b follows the list's first chunk.  K
 //        and V have their own barriers, so the next list's K lands once the
 //        last S has read K while the last PV still reads V.
-//      * warp 1 issues S = Q K_b^T into TMEM S buffer (chunk & 1); warp 2
-//        issues O = P V_b (P read from that S buffer, where the softmax wrote
-//        it over S) into TMEM O buffer (chunk & 1).  Both run their loops
-//        with the whole warp and issue from one elected lane with
-//        precomputed descriptors.
-//      * warps 4..7 and 8..11 are two softmax groups that take even and odd
-//        chunks: one thread owns a whole 128-column row (the row max needs no
-//        exchange), so while one group exponentiates (MUFU-bound: 16 per
-//        clock per SM, as many cycles per tile as its two MMAs) the other
-//        loads S, writes P or runs its epilogue.  Each group also writes its
-//        own previous chunk's partial (o = O / l in bf16, coalesced 16-byte
-//        stores in a column-slice layout, L2 evict-first) and lse2 = m c +
-//        log2 l, while the tensor core runs the next S into its buffer.
+//      * warp 1 issues S = Q K_b^T into the TMEM S buffer; warp 14 issues
+//        O = P V_b (P read from one of two TMEM P buffers) into one of two
+//        TMEM O buffers.  Both run their loops with the whole warp and issue
+//        from one elected lane with precomputed descriptors: a tcgen05.mma
+//        issuing thread slows with every busy warp on its SMSP.  S is
+//        released as soon as the softmax has loaded it.
+//      * warps 2..9 (softmax): two threads per row, each owning 64 of the 128
+//        columns; the exact softmax of the row over the block's visible keys
+//        (causal only in the local block); the two halves exchange only their
+//        max through shared memory; P (bf16) goes to a P buffer; (m, l_lo,
+//        l_hi) go to the epilogue.  (The exponentials are MUFU-bound: 16 per
+//        clock per SM, so one 128x128 tile costs as many cycles as its two
+//        MMAs; two warps per SM sub-partition keep the MUFU pipe fed.)
+//      * warps 10..13 (epilogue): o = O / l in bf16 staged in shared memory and
+//        written by TMA (L2 evict-first) as one contiguous 128-row tile per
+//        chunk (chunk-major partials), lse2 = m c + log2 l beside it.
+//   3. merge_partials_kernel: per (query, group), O = sum_s 2^(lse2_s - L) o_s
+//      over the valid slots, L = log2 sum 2^lse2_s; rounded to bf16.  The
+//      schedule records, per (query, group, slot), the partial row it wrote.
+//
+// A packed batch of sequences (varlen) runs the same kernels: a selection
+// (query q, block b of q's sequence) goes to global block blk_pfx[s] + b, so
+// lists never mix sequences, and the softmax masks with positions local to
+// the sequence.
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -44,12 +55,19 @@
 namespace msa {
 namespace {
 
-constexpr int kThreads = 384;   // 12 warps
-constexpr int kSoftW0 = 4;      // softmax groups: warps 4..7 (even chunks), 8..11 (odd chunks)
-constexpr int kQStages = 4;
-constexpr int kKVStages = 1;    // a CTA switches blocks once per (group, block) list (hundreds of chunks)
-constexpr int kDesc = 8;        // descriptor ring depth
-constexpr int kCtrlBytes = 8192;    // descriptors, staged entries, barriers
+constexpr int kThreads = 480;   // 15 warps
+constexpr int kSoftW0 = 2;      // softmax warps 2..9: two per TMEM lane quarter, 64 columns each
+constexpr int kEpiW0 = 10;      // epilogue warps 10..13
+constexpr int kPvW = 14;        // PV issuer (S is issued by warp 1): each SMSP's issue port is shared
+                                // with two softmax warps, so one thread issuing both would cap the rate
+// One K/V stage suffices because a CTA switches blocks only once per
+// (group, block) list (hundreds of chunks); the partial tile is staged in
+// two shared-memory buffers for the TMA stores.
+constexpr int kQStages = 3;
+constexpr int kKVStages = 1;
+constexpr int kOStages = 1;
+constexpr int kDesc = 8;        // descriptor ring depth (a slot is held until the epilogue is done)
+constexpr int kCtrlBytes = 20480;   // descriptors, softmax stats, staged entries, barriers
 constexpr int kSchedThreads = 256;
 constexpr int kStageEntries = 256;   // list entries staged in shared memory at a time
 constexpr int kWave = 4096;          // query rows per wave (L2-resident Q working set)
@@ -59,17 +77,19 @@ struct KvoCfg {
   static constexpr int kAtoms = D / 64;
   static constexpr int kQBytes = 128 * D * 2;
   static constexpr int kKVBytes = BK * D * 2;          // one of K or V
-  static constexpr int kSmemData = kQStages * kQBytes + kKVStages * 2 * kKVBytes;
+  static constexpr int kOBytes = 128 * D * 2;          // staged bf16 partial tile
+  static constexpr int kSmemData = kQStages * kQBytes + kKVStages * 2 * kKVBytes + kOStages * kOBytes;
   static constexpr int kSmemBytes = kSmemData + kCtrlBytes + 1024;
-  // TMEM: two S buffers (P is written over S, bf16 pairs in the first BK/2
-  // columns), two O buffers; buffer (chunk & 1).
-  static constexpr int kColS = 0;        // S/P: [g BK, g BK + BK)
-  static constexpr int kColO = 2 * BK;   // O: [2BK + g D, 2BK + g D + D)
+  // TMEM: one S buffer (freed as soon as the softmax has loaded it), two P
+  // buffers (bf16 pairs, BK/2 columns each), two O buffers.
+  static constexpr int kColS = 0;        // S: [0, BK)
+  static constexpr int kColP = BK;       // P: [BK, BK + BK/2), [BK + BK/2, 2BK)
+  static constexpr int kColO = 2 * BK;   // O: [2BK, 2BK + D), [2BK + D, 2BK + 2D)
   static constexpr int kTmemCols = (2 * BK + 2 * D) <= 256 ? 256 : 512;
-  static_assert(kSmemBytes <= 227 * 1024, "shared memory of attn_kvouter_kernel");
 };
 
-// One chunk of gathered queries of a (group, block) list.
+// One chunk of gathered queries of a (group, block) list.  (Declared before
+// KvoCfg's users; the shared-memory budget check follows it.)
 struct Desc {
   int entry[128];   // (query << 5) | slot, for the first `count` rows' queries
   int r, b, count, kvs;                      // b: block index within its sequence
@@ -77,7 +97,7 @@ struct Desc {
   int seq_row0, seq_len;                     // the block's sequence: first row, length
 };
 
-static_assert(kDesc * sizeof(Desc) + kStageEntries * 4 + 64 * 8 + 16 <= kCtrlBytes,
+static_assert(kDesc * (sizeof(Desc) + 128 * 12) + 4 * 128 * 4 + kStageEntries * 4 + 64 * 8 + 16 <= kCtrlBytes,
               "control block of attn_kvouter_kernel exceeds its shared-memory reservation");
 
 struct KvoArgs {
@@ -87,7 +107,6 @@ struct KvoArgs {
   const int* lists;      // non-empty list ids ((wave * h_kv + r) * nb + b)
   const int* n_lists;
   int* work_counter;
-  uint16_t* part_o;      // [chunks][D/8][128][8] bf16 partial rows (column slices)
   float* part_lse;       // [chunks * 128] lse2 of each partial row
   int* status;
   int n_q, n_kv, q_pos0, h_q, h_kv, topk, causal, nb;
@@ -111,30 +130,40 @@ __device__ __forceinline__ int seq_search(const int* pfx, int batch, int x) {
 template <int D, int BK, int G>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                        const __grid_constant__ CUtensorMap tm_v, const KvoArgs args) {
+                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_po,
+                        const KvoArgs args) {
   using Cfg = KvoCfg<D, BK>;
   constexpr int QPC = 128 / G;   // queries per chunk
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sq = smem;                                        // [stage][atoms][128][128 B]
   uint8_t* skv = smem + kQStages * Cfg::kQBytes;             // [stage][K|V][atoms][BK][128 B]
+  uint8_t* so = skv + kKVStages * 2 * Cfg::kKVBytes;         // [stage][atoms][128][128 B] partial tile
   Desc* desc = reinterpret_cast<Desc*>(smem + Cfg::kSmemData);
-  int* stage = reinterpret_cast<int*>(desc + kDesc);         // [kStageEntries] staged list entries
+  float2* ml = reinterpret_cast<float2*>(desc + kDesc);      // [kDesc][128] (m, l of columns 0..63)
+  float* lhi = reinterpret_cast<float*>(ml + kDesc * 128);   // [kDesc][128] l of columns 64..127
+  float* smx = lhi + kDesc * 128;                            // [2 parity][2 halves][128] row-max exchange
+  int* stage = reinterpret_cast<int*>(smx + 4 * 128);        // [kStageEntries] staged list entries
   uint64_t* bars = reinterpret_cast<uint64_t*>(stage + kStageEntries);
   uint64_t* q_full = bars;                                   // [kQStages]
   uint64_t* q_empty = q_full + kQStages;
+  // K and V of a stage have their own barriers: the next list's K can land
+  // once the current list's last S has read K, while its last PV still
+  // reads V.
   uint64_t* k_full = q_empty + kQStages;                     // [kKVStages]
   uint64_t* k_empty = k_full + kKVStages;
   uint64_t* v_full = k_empty + kKVStages;
   uint64_t* v_empty = v_full + kKVStages;
   uint64_t* d_full = v_empty + kKVStages;                    // [kDesc]
   uint64_t* d_empty = d_full + kDesc;
-  uint64_t* s_full = d_empty + kDesc;                        // [2] S(t) in S buffer t & 1
-  uint64_t* s_free = s_full + 2;                             // [2] P(t) read by its PV
-  uint64_t* p_full = s_free + 2;                             // [2] P(t) written
-  uint64_t* o_full = p_full + 2;                             // [2] O(t) complete
-  uint64_t* o_free = o_full + 2;                             // [2] O(t) loaded by the epilogue
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_free + 2);
+  uint64_t* s_full = d_empty + kDesc;                        // [1] S ready
+  uint64_t* s_free = s_full + 1;                             // [1] S loaded by the softmax
+  uint64_t* p_free = s_free + 1;                             // [2] P consumed by its PV
+  uint64_t* p_full = p_free + 2;
+  uint64_t* o_full = p_full + 2;
+  uint64_t* o_free = o_full + 2;
+  uint64_t* ml_full = o_free + 2;                            // [kDesc]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ml_full + kDesc);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = warp_id();
@@ -152,14 +181,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < kDesc; ++s) {
       mbar_init(&d_full[s], 1);
-      mbar_init(&d_empty[s], 6);   // S and PV issuers + the 4 warps of the chunk's softmax group
+      mbar_init(&d_empty[s], 14);  // S and PV issuers + 8 softmax warps + 4 epilogue warps
+      mbar_init(&ml_full[s], 8);   // 8 softmax warps
     }
-    for (int g = 0; g < 2; ++g) {
-      mbar_init(&s_full[g], 1);
-      mbar_init(&s_free[g], 1);
-      mbar_init(&p_full[g], 4);
-      mbar_init(&o_full[g], 1);
-      mbar_init(&o_free[g], 4);
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 8);          // the 8 softmax warps, once their S loads completed
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&p_free[s], 1);
+      mbar_init(&p_full[s], 8);
+      mbar_init(&o_full[s], 1);
+      mbar_init(&o_free[s], 4);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -174,14 +205,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const WaitCtx wc{abort_flag, args.status};
   const int n_lists = *args.n_lists;
+  // Gathered Q rows are re-read by up to k lists of their wave: keep them in
+  // L2; partial tiles are read once, much later: let them leave first.
+  const uint64_t q_policy = l2_evict_last();
+  const uint64_t part_policy = l2_evict_first();
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer (whole warp)
     // The list's (query, slot) entries are staged in shared memory 256 at a
     // time with coalesced loads, so no TMA issue waits on a dependent global
-    // load; each lane issues the TMA boxes of its own queries.  Gathered Q
-    // rows are re-read by up to k lists of their wave: keep them in L2.
-    const uint64_t q_policy = l2_evict_last();
+    // load; each lane issues the TMA boxes of its own queries.
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
@@ -223,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       ++kvc;
       for (int c0 = 0; c0 < cnt; c0 += QPC) {
-        // Refill the staging buffer every kStageEntries entries.
+        // Refill the staging buffer every kStage entries.
         const int rel = c0 % kStageEntries;
         if (rel == 0) {
           __syncwarp();
@@ -284,12 +317,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    // End markers: one per softmax group (chunks t and t + 1); the MMA
-    // issuers stop at the first.
+    // End marker for the consumers.
     if (lane == 0 && ok && !*abort_flag) {
-      for (int x = 0; x < 2; ++x, ++t) {
-        const int ds = t % kDesc;
-        if (!mbar_wait(&d_empty[ds], ((t / kDesc) & 1) ^ 1, wc)) break;
+      const int ds = t % kDesc;
+      if (mbar_wait(&d_empty[ds], ((t / kDesc) & 1) ^ 1, wc)) {
         desc[ds].end = 1;
         mbar_arrive(&d_full[ds]);
       }
@@ -298,8 +329,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------------- UMMA: S = Q K^T
     // Both issuers run their loops with the whole warp (warp-uniform waits
     // and descriptor math) and issue each MMA predicated on an elected lane:
-    // a divergent single-lane loop loses most issue slots to the busy warps
-    // sharing its SMSP.
+    // a divergent single-lane loop loses most issue slots to the softmax and
+    // epilogue warps sharing its SMSP (measured: 108 against 272 cycles per
+    // MMA with three busy warps).
     constexpr uint32_t idesc_s = idesc_bf16_f32(128, BK, false, false);
     // Descriptors differ only in their start-address field (address >> 4,
     // bits 0-13, never carrying out for shared-memory addresses), so they
@@ -315,30 +347,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&d_empty[ds]);
       if (end) break;
-      const int qs = t % kQStages, g = t & 1;
+      const int qs = t % kQStages;
       if (first) {
         if (!__all_sync(0xffffffffu, mbar_wait(&k_full[kvs], (kvc / kKVStages) & 1, wc))) break;
         ++kvc;
       }
       if (!__all_sync(0xffffffffu, mbar_wait(&q_full[qs], (t / kQStages) & 1, wc))) break;
-      // S(t) reuses S buffer g once PV(t - 2) has read P(t - 2) from it.
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_free[g], ((t >> 1) & 1) ^ 1, wc))) break;
+      // S(t) reuses the single S buffer once the softmax has loaded S(t-1).
+      if (!__all_sync(0xffffffffu, mbar_wait(s_free, (t & 1) ^ 1, wc))) break;
       tc_fence_after();
       const uint64_t qd = q_desc0 + ((qs * Cfg::kQBytes) >> 4);
       const uint64_t kd = k_desc0 + ((kvs * 2 * Cfg::kKVBytes) >> 4);
-      const uint32_t s_tmem = tmem + Cfg::kColS + g * BK;
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks) {
         const uint32_t off = (ks / 4) * (128 * 128) + (ks % 4) * 32;
         const uint32_t koff = (ks / 4) * (BK * 128) + (ks % 4) * 32;
-        umma_ss_elect(s_tmem, qd + (off >> 4), kd + (koff >> 4), idesc_s, ks > 0 ? 1u : 0u);
+        umma_ss_elect(tmem + Cfg::kColS, qd + (off >> 4), kd + (koff >> 4), idesc_s, ks > 0 ? 1u : 0u);
       }
       umma_commit_elect(&q_empty[qs]);
-      umma_commit_elect(&s_full[g]);
+      umma_commit_elect(s_full);
       if (last) umma_commit_elect(&k_empty[kvs]);   // this list's last read of K
       __syncwarp();
     }
-  } else if (warp == 2) {
+  } else if (warp == kPvW) {
     // ---------------------------------------------------------------- UMMA: O = P V
     constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
     const uint64_t v_desc0 = smem_desc(smem_u32(skv) + Cfg::kKVBytes, BK * 128, 1024, kSwizzle128B);
@@ -351,122 +382,93 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&d_empty[ds]);
       if (end) break;
-      const int g = t & 1;
+      const int sb = t & 1;
       if (first) {
         if (!__all_sync(0xffffffffu, mbar_wait(&v_full[kvs], (vc / kKVStages) & 1, wc))) break;
         ++vc;
       }
-      if (!__all_sync(0xffffffffu, mbar_wait(&p_full[g], (t >> 1) & 1, wc))) break;
-      // O buffer g is free once the epilogue of chunk t - 2 has loaded it.
-      if (!__all_sync(0xffffffffu, mbar_wait(&o_free[g], ((t >> 1) & 1) ^ 1, wc))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&p_full[sb], (t >> 1) & 1, wc))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&o_free[sb], ((t >> 1) & 1) ^ 1, wc))) break;
       tc_fence_after();
       const uint64_t vd = v_desc0 + ((kvs * 2 * Cfg::kKVBytes) >> 4);
-      const uint32_t p_tmem = tmem + Cfg::kColS + g * BK;
-      const uint32_t o_tmem = tmem + Cfg::kColO + g * D;
+      const uint32_t p_tmem = tmem + Cfg::kColP + sb * (BK / 2);
+      const uint32_t o_tmem = tmem + Cfg::kColO + sb * D;
 #pragma unroll
       for (int kk = 0; kk < BK / 16; ++kk)
         umma_ts_elect(o_tmem, p_tmem + kk * 8, vd + ((kk * 2048) >> 4), idesc_o, kk > 0 ? 1u : 0u);
-      umma_commit_elect(&o_full[g]);
-      umma_commit_elect(&s_free[g]);
+      umma_commit_elect(&o_full[sb]);
+      umma_commit_elect(&p_free[sb]);
       if (last) umma_commit_elect(&v_empty[kvs]);   // this list's last read of V
       __syncwarp();
     }
-  } else if (warp >= kSoftW0) {
-    // ---------------------------------------------------------------- softmax + epilogue
-    const int g = (warp - kSoftW0) >> 2;   // chunks t with t & 1 == g
+  } else if (warp >= kSoftW0 && warp < kEpiW0) {
+    // ---------------------------------------------------------------- softmax
+    constexpr int HC = BK / 2;                 // columns per thread
     const int quarter = warp & 3;
+    const int half = (warp - kSoftW0) / 4;     // 0: columns [0, HC), 1: [HC, BK)
     const int row = quarter * 32 + lane;
     const int qi = row / G;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    const uint32_t s_tmem = lane_base + Cfg::kColS + g * BK;
-    const uint32_t o_tmem = lane_base + Cfg::kColO + g * D;
     const float c = args.scale_log2;
-    // Partial rows are read once, much later, by the merge: let them leave L2 first.
-    const uint64_t part_policy = l2_evict_first();
-    constexpr float kNegInf = -__builtin_huge_valf();
-    // The epilogue of this group's previous chunk: o = O / l (bf16) and lse2.
-    int pend_chunk = 0;
-    bool pend_valid = false;
-    float pend_m = 0.f, pend_l = 0.f;
-    // O is read 32 columns at a time: PV(t + 2), the next writer of this O
-    // buffer, also waits for P(t + 2), which comes much later, so releasing
-    // the buffer after the last piece costs nothing and keeps registers free.
-    auto epilogue = [&](int jj) -> bool {
-      if (!mbar_wait(&o_full[g], jj & 1, wc)) return false;
-      tc_fence_after();
-      const float inv = pend_l > 0.f ? 1.f / pend_l : 0.f;
-      uint16_t* dst = args.part_o + (static_cast<size_t>(pend_chunk) * (D / 8) * 128 + row) * 8;
-#pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t ov[32];
-        tmem_ld32(o_tmem + cc * 32, ov);
-        tmem_ld_wait();
-        if (pend_valid) {
-#pragma unroll
-          for (int sl = 0; sl < 4; ++sl) {
-            const float* f = reinterpret_cast<const float*>(&ov[sl * 8]);
-            float h[8];
-#pragma unroll
-            for (int x = 0; x < 8; x += 2) fmul2(h[x], h[x + 1], f[x], f[x + 1], inv, inv);
-            st_global_v4_hint(dst + (cc * 4 + sl) * 128 * 8, pack_bf16x2(h[0], h[1]), pack_bf16x2(h[2], h[3]),
-                              pack_bf16x2(h[4], h[5]), pack_bf16x2(h[6], h[7]), part_policy);
-          }
-        }
-      }
-      // O is in registers and stored: PV(t + 2) may overwrite the buffer.
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&o_free[g]);
-      if (pend_valid)
-        args.part_lse[static_cast<size_t>(pend_chunk) * 128 + row] =
-            pend_l > 0.f ? pend_m * c + __log2f(pend_l) : kNegInf;
-      return true;
-    };
-    for (int j = 0;; ++j) {
-      const int t = 2 * j + g;
+    for (int t = 0;; ++t) {
       const int ds = t % kDesc;
       if (!mbar_wait(&d_full[ds], (t / kDesc) & 1, wc)) break;
       const Desc& dd = desc[ds];
-      const int end = dd.end;
-      const int e = (!end && qi < dd.count) ? dd.entry[qi] : -1;
-      const int b = dd.b, chunk = dd.chunk, seq_row0 = dd.seq_row0, seq_len = dd.seq_len;
+      if (dd.end) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&d_empty[ds]);
+        break;
+      }
+      const int e = qi < dd.count ? dd.entry[qi] : -1;
+      const int b = dd.b, seq_row0 = dd.seq_row0, seq_len = dd.seq_len;
       __syncwarp();
       if (lane == 0) mbar_arrive(&d_empty[ds]);
-      // The previous chunk's epilogue runs while the tensor core computes S(t).
-      if (j > 0 && !epilogue(j - 1)) break;
-      if (end) break;
-      int lim = 0;   // visible keys of this block for the row (positions local to its sequence)
-      if (e >= 0) {
+      int lim = 0;   // visible keys of this block for the row, relative to this half
+      if (e >= 0) {   // positions local to the query's sequence
         const int p = (args.cu_seqlens ? 0 : args.q_pos0) + (e >> 5) - seq_row0;
         const int kv_lim = args.causal ? min(p + 1, seq_len) : seq_len;
-        lim = min(BK, kv_lim - b * BK);
+        lim = min(BK, kv_lim - b * BK) - half * HC;
       }
-      if (!mbar_wait(&s_full[g], j & 1, wc)) break;
+      const int sb = t & 1;   // P buffer
+      if (!mbar_wait(s_full, t & 1, wc)) break;
       tc_fence_after();
-      uint32_t sv[BK];
+      const uint32_t s_tmem = lane_base + Cfg::kColS;
+      uint32_t sv[HC];
 #pragma unroll
-      for (int cc = 0; cc < BK / 32; ++cc)
-        tmem_ld32(s_tmem + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[cc * 32]));
+      for (int cc = 0; cc < HC / 32; ++cc)
+        tmem_ld32(s_tmem + half * HC + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[cc * 32]));
       tmem_ld_wait();
-      if (lim < BK) {
+      // S is in registers: hand the S buffer back so the next S MMA can start.
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free);
+      if (lim < HC) {
 #pragma unroll
-        for (int i = 0; i < BK; ++i)
+        for (int i = 0; i < HC; ++i)
           if (i >= lim) sv[i] = 0xff800000u;   // -inf: masked key
       }
-      float mq[4] = {kNegInf, kNegInf, kNegInf, kNegInf};
+      float mq[4] = {__int_as_float(0xff800000), __int_as_float(0xff800000), __int_as_float(0xff800000),
+                     __int_as_float(0xff800000)};
 #pragma unroll
-      for (int i = 0; i < BK; i += 8) {
+      for (int i = 0; i < HC; i += 8) {
         const int k = (i / 8) & 3;
         mq[k] = max3f(mq[k], fmaxf(__uint_as_float(sv[i]), __uint_as_float(sv[i + 1])),
                       max3f(__uint_as_float(sv[i + 2]), __uint_as_float(sv[i + 3]), __uint_as_float(sv[i + 4])));
         mq[k] = max3f(mq[k], __uint_as_float(sv[i + 5]), fmaxf(__uint_as_float(sv[i + 6]), __uint_as_float(sv[i + 7])));
       }
-      const float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
-      const float bias = mx == kNegInf ? 0.f : mx * c;
+      // Exchange the half-row maxima with the partner warp (same lane quarter).
+      // The slot alternates with the chunk parity: a warp rewrites slot
+      // (t & 1) only after the next barrier, which its partner reaches only
+      // after reading this chunk's value.
+      float* xs = smx + (t & 1) * 256;
+      xs[half * 128 + row] = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+      named_bar(2 + quarter, 64);
+      const float mx = fmaxf(xs[row], xs[128 + row]);
+      const float bias = mx == __int_as_float(0xff800000) ? 0.f : mx * c;
       float ls[4] = {0.f, 0.f, 0.f, 0.f};   // two pairs of partial sums
-      uint32_t pk[BK / 2];
+      uint32_t pk[HC / 2];
 #pragma unroll
-      for (int i = 0; i < BK; i += 4) {
+      for (int i = 0; i < HC; i += 4) {
         float x0, x1, x2, x3;
         ffma2(x0, x1, __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]), c, c, -bias, -bias);
         ffma2(x2, x3, __uint_as_float(sv[i + 2]), __uint_as_float(sv[i + 3]), c, c, -bias, -bias);
@@ -478,19 +480,100 @@ __global__ void __launch_bounds__(kThreads, 1)
         pk[i / 2] = pack_bf16x2(p0, p1);
         pk[i / 2 + 1] = pack_bf16x2(p2, p3);
       }
-      // P(t) over S(t): the S values are all in registers.
+      // P(t) goes to P buffer t & 1 once the PV of chunk t - 2 has read it.
+      if (!mbar_wait(&p_free[sb], ((t >> 1) & 1) ^ 1, wc)) break;
+      tc_fence_after();
+      const uint32_t p_tmem = lane_base + Cfg::kColP + sb * (BK / 2);
 #pragma unroll
-      for (int cc = 0; cc < BK / 64; ++cc)
-        tmem_st32(s_tmem + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[cc * 32]));
+      for (int cc = 0; cc < HC / 64; ++cc)
+        tmem_st32(p_tmem + half * (HC / 2) + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[cc * 32]));
+      if (HC / 2 == 16) tmem_st16(p_tmem + half * (HC / 2), *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
+      const float lsum = (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      if (half == 0)
+        ml[ds * 128 + row] = make_float2(mx, lsum);
+      else
+        lhi[ds * 128 + row] = lsum;
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[g]);
-      pend_chunk = chunk;
-      pend_valid = e >= 0;
-      pend_m = mx;
-      pend_l = (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      if (lane == 0) {
+        mbar_arrive(&p_full[sb]);
+        mbar_arrive(&ml_full[ds]);
+      }
     }
+  } else if (warp >= kEpiW0 && warp < kEpiW0 + 4) {
+    // ---------------------------------------------------------------- epilogue
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const int qi = row / G;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const float c = args.scale_log2;
+    for (int t = 0;; ++t) {
+      const int ds = t % kDesc;
+      if (!mbar_wait(&d_full[ds], (t / kDesc) & 1, wc)) break;
+      const Desc& dd = desc[ds];
+      if (dd.end) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&d_empty[ds]);
+        break;
+      }
+      const int e = qi < dd.count ? dd.entry[qi] : -1;
+      const int sb = t & 1;
+      if (!mbar_wait(&o_full[sb], (t >> 1) & 1, wc)) break;
+      if (!mbar_wait(&ml_full[ds], (t / kDesc) & 1, wc)) break;
+      tc_fence_after();
+      const float2 st = ml[ds * 128 + row];
+      const float lsum = st.y + lhi[ds * 128 + row];
+      const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+      const float lse2 = lsum > 0.f ? st.x * c + __log2f(lsum) : __int_as_float(0xff800000);
+      const int chunk = dd.chunk;
+      const int os = t % kOStages;
+      // Stage the bf16 row in the swizzled tile layout (the layout TMA uses),
+      // after the stores that last read this staging buffer have drained.
+      if (warp == kEpiW0 && lane == 0) {
+        if (kOStages == 1)
+          bulk_wait_read0();
+        else
+          bulk_wait_read_le1();
+      }
+      named_bar(1, 128);
+      const uint32_t so_addr = smem_u32(so + os * Cfg::kOBytes);
+#pragma unroll
+      for (int a = 0; a < D / 64; ++a) {
+        uint32_t ov[64];
+        tmem_ld32(lane_base + Cfg::kColO + sb * D + a * 64, *reinterpret_cast<uint32_t(*)[32]>(&ov[0]));
+        tmem_ld32(lane_base + Cfg::kColO + sb * D + a * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&ov[32]));
+        tmem_ld_wait();
+        if (a == D / 64 - 1) {
+          // The O buffer is free once its values are in registers.
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&o_free[sb]);
+        }
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const float* f = reinterpret_cast<const float*>(&ov[ch * 8]);
+          float g[8];
+#pragma unroll
+          for (int j = 0; j < 8; j += 2) fmul2(g[j], g[j + 1], f[j], f[j + 1], inv, inv);
+          st_shared_v4(so_addr + a * 128 * 128 + row * 128 + ((ch ^ (row & 7)) << 4), pack_bf16x2(g[0], g[1]),
+                       pack_bf16x2(g[2], g[3]), pack_bf16x2(g[4], g[5]), pack_bf16x2(g[6], g[7]));
+        }
+      }
+      args.part_lse[static_cast<size_t>(chunk) * 128 + row] = e >= 0 ? lse2 : __int_as_float(0xff800000);
+      fence_proxy_async_smem();
+      named_bar(1, 128);
+      // One thread issues, commits and later waits for the chunk's tile
+      // stores (bulk groups are tracked per thread): one box per d atom.
+      if (warp == kEpiW0 && lane == 0) {
+        for (int a = 0; a < D / 64; ++a)
+          tma_store_2d_hint(&tm_po, so + os * Cfg::kOBytes + a * 128 * 128, a * 64, chunk * 128, part_policy);
+        bulk_commit();
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&d_empty[ds]);   // also releases ml[ds]
+    }
+    if (warp == kEpiW0) bulk_wait0();
   }
 
   tc_fence_before();
@@ -650,13 +733,11 @@ template <int D>
 __global__ void __launch_bounds__(256) merge_partials_kernel(const int* prow_of, const uint16_t* part_o,
                                                              const float* part_lse, uint16_t* o, int h_q, int h_kv,
                                                              int topk) {
-  // One CTA per (query, group); thread = (8-column slice, head within the
-  // group), heads fastest, so a warp reads whole 16 * G-byte runs of the
-  // column-slice layout.  prow_of[(q, r, slot)] is the first partial row
-  // (chunk * 128 + query-in-chunk * G) the block-major kernel wrote for that
-  // selection.  Slots are read 8 at a time with independent loads and folded
-  // in with an online log-sum-exp, so the loads of a group are all in flight
-  // together.
+  // One CTA per (query, group); thread = (head within group, 8-column chunk).
+  // prow_of[(q, r, slot)] is the first partial row (chunk * 128 + query-in-
+  // chunk * G) the block-major kernel wrote for that selection, -1 for none.
+  // Slots are read 8 at a time with independent loads and folded in with an
+  // online log-sum-exp, so the loads of a group are all in flight together.
   constexpr int kGrp = 8;
   const int qr = blockIdx.x;
   const int q = qr / h_kv, r = qr % h_kv;
@@ -664,7 +745,7 @@ __global__ void __launch_bounds__(256) merge_partials_kernel(const int* prow_of,
   constexpr int kChunks = D / 8;
   const int* my_rows = prow_of + static_cast<size_t>(qr) * topk;
   for (int w = threadIdx.x; w < G * kChunks; w += blockDim.x) {
-    const int hh = w % G, ch = w / G;
+    const int hh = w / kChunks, ch = w % kChunks;
     float M = __int_as_float(0xff800000), den = 0.f;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     for (int s0 = 0; s0 < topk; s0 += kGrp) {
@@ -676,9 +757,8 @@ __global__ void __launch_bounds__(256) merge_partials_kernel(const int* prow_of,
         const int pr = s < topk ? my_rows[s] : -1;   // -1: padding or no block of this sequence
         const bool ok = pr >= 0;
         const size_t prow = ok ? static_cast<size_t>(pr) + hh : 0;
-        const size_t at = (((prow >> 7) * kChunks + ch) * 128 + (prow & 127)) * 8;
         ls[j] = ok ? part_lse[prow] : __int_as_float(0xff800000);
-        v[j] = ok ? *reinterpret_cast<const uint4*>(part_o + at) : make_uint4(0, 0, 0, 0);
+        v[j] = ok ? *reinterpret_cast<const uint4*>(part_o + prow * D + ch * 8) : make_uint4(0, 0, 0, 0);
       }
       float gm = M;
 #pragma unroll
@@ -717,7 +797,7 @@ cudaError_t launch_kvo(const CUtensorMap* m, const KvoArgs& a, int grid, cudaStr
   const int smem = KvoCfg<D, BK>::kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, smem, st>>>(m[0], m[1], m[2], a);
+  kern<<<grid, kThreads, smem, st>>>(m[0], m[1], m[2], m[3], a);
   return cudaGetLastError();
 }
 
@@ -826,7 +906,6 @@ int run_sparse_attn_kvouter(const msa_params& p, const void* q, const CUtensorMa
   a.lists = s.lists;
   a.n_lists = s.n_lists;
   a.work_counter = s.work;
-  a.part_o = s.part_o;
   a.part_lse = s.part_lse;
   a.status = status;
   a.n_q = n_q;
@@ -846,7 +925,13 @@ int run_sparse_attn_kvouter(const msa_params& p, const void* q, const CUtensorMa
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = sms;
-  const CUtensorMap maps[3] = {tq, tk, tv};
+  CUtensorMap maps[4] = {tq, tk, tv, tq};
+  {  // chunk-major partial rows [max_chunks * 128][d]: one box = 128 rows x 64 columns
+    const uint64_t dims[2] = {static_cast<uint64_t>(p.d), static_cast<uint64_t>(s.max_chunks) * 128};
+    const uint64_t strides[1] = {static_cast<uint64_t>(p.d) * 2};
+    const uint32_t box[2] = {64, 128};
+    if (!encode_tma_bf16(&maps[3], 2, s.part_o, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MSA_ERR_CUDA;
+  }
   cudaError_t e;
   if (p.d == 64) {
     e = p.block_k == 64 ? launch_kvo_g<64, 64>(G, maps, a, grid, stream)
