@@ -72,6 +72,7 @@ extern "C" {
 #define MSA_OP_DECODE 2
 #define MSA_OP_INDEX_TOPK_VARLEN 3 /* n_q = total rows, batch = sequences */
 #define MSA_OP_PREFILL_VARLEN 4    /* n_q = total rows, batch = sequences */
+#define MSA_OP_INDEX_PROJECT 5     /* n_q = rows */
 
 /* Problem parameters (the pages' notation: H_q, H_kv, d_h, d_idx, B_k, k). */
 typedef struct {
@@ -95,6 +96,24 @@ typedef struct {
  * Returns 0 for invalid arguments.  Host-only; never touches the GPU.
  */
 MSA_API size_t msa_workspace_size(int op, const msa_params* p, int n_q, int n_kv, int batch, int max_kv);
+
+/*
+ * Index projections ahead of the index branch (titansim.online section 4.2:
+ * an index-query projection per GQA group and one index-key projection
+ * shared by all groups):
+ *   Q_idx[i, r, :] = x[i, :] W_q^idx(r)^T,   K_idx[i, 0, :] = x[i, :] W_k^idx^T
+ * computed as one GEMM on the tensor cores with fp32 accumulation, rounded
+ * to bf16 (nearest even).
+ *   x      bf16 [n, d_model]                 hidden states (d_model % 8 == 0)
+ *   w_idx  bf16 [(h_kv + 1) * d_idx, d_model] stacked weights, nn.Linear
+ *          layout: rows r*d_idx .. (r+1)*d_idx - 1 are W_q^idx(r), the last
+ *          d_idx rows W_k^idx
+ *   q_idx  bf16 [n, h_kv, d_idx] output;  k_idx bf16 [n, 1, d_idx] output
+ * Uses p->h_kv and p->d_idx; the workspace is msa_workspace_size
+ * (MSA_OP_INDEX_PROJECT, p, n, 0, 0, 0) bytes (the status word).
+ */
+MSA_API int msa_index_project(const msa_params* p, const void* x, const void* w_idx, int n, int d_model,
+                              void* q_idx, void* k_idx, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Index branch of a (chunked) prefill: eq. (6) scores, causal block

@@ -15,15 +15,15 @@ from typing import Optional
 __all__ = ["MSAError", "Params", "lib", "workspace_size", "index_topk", "sparse_attn_prefill",
            "sparse_attn_decode", "index_topk_varlen", "sparse_attn_prefill_varlen", "device_status",
            "status_string", "OP_INDEX_TOPK", "OP_PREFILL", "OP_DECODE", "OP_INDEX_TOPK_VARLEN",
-           "OP_PREFILL_VARLEN", "POOL_MAX", "POOL_MEAN"]
+           "OP_PREFILL_VARLEN", "OP_INDEX_PROJECT", "index_project", "POOL_MAX", "POOL_MEAN"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmsa.so")
 
-OP_INDEX_TOPK, OP_PREFILL, OP_DECODE, OP_INDEX_TOPK_VARLEN, OP_PREFILL_VARLEN = 0, 1, 2, 3, 4
+OP_INDEX_TOPK, OP_PREFILL, OP_DECODE, OP_INDEX_TOPK_VARLEN, OP_PREFILL_VARLEN, OP_INDEX_PROJECT = 0, 1, 2, 3, 4, 5
 POOL_MAX, POOL_MEAN = 0, 1   # msa_params.pool
 
-SYMBOLS = ("msa_workspace_size", "msa_index_topk", "msa_sparse_attn_prefill", "msa_sparse_attn_decode",
+SYMBOLS = ("msa_workspace_size", "msa_index_project", "msa_index_topk", "msa_sparse_attn_prefill", "msa_sparse_attn_decode",
            "msa_index_topk_varlen", "msa_sparse_attn_prefill_varlen", "msa_sparse_attn_decode_adaptive_k",
            "msa_device_status", "msa_status_string",
            "msa_sparse_attn_decode_noalloc", "msa_test_never_ready_wait")
@@ -69,6 +69,7 @@ def lib():
         L.msa_sparse_attn_decode.argtypes = [P, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, vp, vp, sz, vp]
         L.msa_sparse_attn_decode_adaptive_k.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, vp,
                                                         vp, sz, vp]
+        L.msa_index_project.argtypes = [P, vp, vp, i32, i32, vp, vp, vp, sz, vp]
         L.msa_index_topk_varlen.argtypes = [P, vp, vp, vp, i32, i32, vp, vp, vp, sz, vp]
         L.msa_sparse_attn_prefill_varlen.argtypes = [P, vp, vp, vp, vp, i32, i32, vp, vp, vp, sz, vp]
         L.msa_sparse_attn_decode_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, vp, vp]
@@ -79,7 +80,8 @@ def lib():
         L.msa_status_string.argtypes = [i32]
         L.msa_status_string.restype = C.c_char_p
         for f in ("msa_index_topk", "msa_sparse_attn_prefill", "msa_sparse_attn_decode", "msa_device_status",
-                  "msa_index_topk_varlen", "msa_sparse_attn_prefill_varlen", "msa_sparse_attn_decode_adaptive_k"):
+                  "msa_index_topk_varlen", "msa_sparse_attn_prefill_varlen", "msa_sparse_attn_decode_adaptive_k",
+                  "msa_index_project"):
             getattr(L, f).restype = i32
         _lib = L
     return _lib
@@ -138,6 +140,28 @@ def _workspace(op, p, n_q=0, n_kv=0, batch=0, max_kv=0, ws=None, device=None):
 def _bf16():
     torch = _torch()
     return (torch.bfloat16, torch.uint16, torch.int16)
+
+
+def index_project(p: Params, x, w_idx, q_idx=None, k_idx=None, ws=None, stream=None):
+    """Index projections: (Q_idx [n, h_kv, d_idx], K_idx [n, 1, d_idx]) = x W_idx^T split by rows of the
+    stacked weight w_idx [(h_kv + 1) d_idx, d_model] (group query projections, then the key projection)."""
+    torch = _torch()
+    n, d_model = x.shape
+    _check(x, "x", _bf16(), (n, d_model))
+    _check(w_idx, "w_idx", _bf16(), ((p.h_kv + 1) * p.d_idx, d_model))
+    if q_idx is None:
+        q_idx = torch.empty((n, p.h_kv, p.d_idx), dtype=torch.bfloat16, device=x.device)
+    if k_idx is None:
+        k_idx = torch.empty((n, 1, p.d_idx), dtype=torch.bfloat16, device=x.device)
+    _check(q_idx, "q_idx", _bf16(), (n, p.h_kv, p.d_idx))
+    _check(k_idx, "k_idx", _bf16(), (n, 1, p.d_idx))
+    ws = _workspace(OP_INDEX_PROJECT, p, n, ws=ws, device=x.device)
+    rc = lib().msa_index_project(C.byref(p), _ptr(x), _ptr(w_idx), n, d_model, _ptr(q_idx), _ptr(k_idx), _ptr(ws),
+                                 ws.numel(), _stream(stream))
+    if rc:
+        raise MSAError(rc, "msa_index_project")
+    _after(ws, stream, "msa_index_project")
+    return q_idx, k_idx
 
 
 def index_topk(p: Params, q_idx, k_idx, q_pos0: int = 0, block_ids=None, ws=None, stream=None):

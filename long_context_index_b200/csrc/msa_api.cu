@@ -105,6 +105,9 @@ size_t msa_workspace_size(int op, const msa_params* p, int n_q, int n_kv, int ba
     case MSA_OP_DECODE:
       if (batch <= 0 || max_kv <= 0 || max_kv > kMaxRows) return 0;
       return kWsHeader + align_up(decode_workspace_bytes(*p, batch, max_kv, -1), 256);
+    case MSA_OP_INDEX_PROJECT:
+      if (n_q < 0 || n_q > kMaxRows) return 0;
+      return kWsHeader;
     case MSA_OP_INDEX_TOPK_VARLEN:
     case MSA_OP_PREFILL_VARLEN:
       if (batch <= 0 || check_rows(n_q, n_q > 0 ? n_q : 1, 0) != MSA_OK) return 0;
@@ -112,6 +115,21 @@ size_t msa_workspace_size(int op, const msa_params* p, int n_q, int n_kv, int ba
     default:
       return 0;
   }
+}
+
+int msa_index_project(const msa_params* p, const void* x, const void* w_idx, int n, int d_model, void* q_idx,
+                      void* k_idx, void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_params(p);
+  if (rc) return rc;
+  if (n < 0 || d_model <= 0) return MSA_ERR_INVALID;
+  if (n > kMaxRows || d_model % 8 != 0 || d_model > (1 << 20)) return MSA_ERR_UNSUPPORTED;
+  if ((rc = check_ws(ws, ws_bytes, kWsHeader))) return rc;
+  if (n > 0 && (!x || !w_idx || !q_idx || !k_idx)) return MSA_ERR_INVALID;
+  if (n > 0 && (!aligned16(x) || !aligned16(w_idx) || !aligned16(q_idx) || !aligned16(k_idx)))
+    return MSA_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((rc = clear_status(ws, st))) return rc;
+  return run_index_project(*p, x, w_idx, n, d_model, q_idx, k_idx, static_cast<int*>(ws), st);
 }
 
 int msa_index_topk(const msa_params* p, const void* q_idx, const void* k_idx, int n_q, int n_kv, int q_pos0,

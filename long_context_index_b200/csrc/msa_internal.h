@@ -46,6 +46,12 @@ int run_index_topk_prefill(const msa_params& p, const void* q_idx, const void* k
                            int q_pos0, int32_t* block_ids, int* status, cudaStream_t stream,
                            const Varlen* vl = nullptr);
 
+// Index projections (index_project.cu): q_idx [n, h_kv, d_idx] and
+// k_idx [n, 1, d_idx] from x [n, d_model] and the stacked weight
+// [(h_kv + 1) d_idx, d_model].
+int run_index_project(const msa_params& p, const void* x, const void* w_idx, int n, int d_model, void* q_idx,
+                      void* k_idx, int* status, cudaStream_t stream);
+
 // The varlen entry points (varlen.cu): workspace bytes (header included) and
 // the run of MSA_OP_INDEX_TOPK_VARLEN (a0, a1 = q_idx, k_idx; ids_out) or
 // MSA_OP_PREFILL_VARLEN (a0, a1, a2 = q, k, v; ids_in; o).

@@ -209,3 +209,23 @@ def sparse_attn_varlen(P: Params, q, k, v, ids, cu_seqlens, rows=None) -> np.nda
         else:
             out[pos] = sparse_attn(P, q[lo:hi], k[lo:hi], v[lo:hi], ids[pos], 0, rows=loc)
     return out
+
+
+# ---------------------------------------------------------------------------
+# Index projections (titansim.online section 4.2: an index-query projection
+# per GQA group, one index-key projection shared by all groups).
+# ---------------------------------------------------------------------------
+def _widen(bits) -> np.ndarray:
+    """bf16 bit patterns -> float64, exactly."""
+    b = np.ascontiguousarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def index_project(x, w_idx, h_kv: int, d_idx: int):
+    """Q_idx[i, r, :] = x[i] . W_q^idx(r) and K_idx[i, 0, :] = x[i] . W_k^idx in float64, with the
+    stacked weight w_idx [(h_kv + 1) d_idx, d_model] (rows r*d_idx..: W_q^idx(r); last d_idx rows: W_k^idx)."""
+    xf, wf = _widen(x), _widen(w_idx)
+    assert wf.shape == ((h_kv + 1) * d_idx, xf.shape[1]), wf.shape
+    y = xf @ wf.T
+    n = xf.shape[0]
+    return y[:, :h_kv * d_idx].reshape(n, h_kv, d_idx), y[:, h_kv * d_idx:].reshape(n, 1, d_idx)

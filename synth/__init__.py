@@ -267,3 +267,28 @@ def make_varlen_prefill(w: Workload, lens: Optional[List[int]] = None) -> dict:
     out["cu_seqlens"] = cu
     out["needles"] = needles
     return out
+
+
+def make_index_projection(seed: int, n: int, d_model: int, h_kv: int, d_idx: int, integer: bool = False) -> dict:
+    """Hidden states x [n, d_model] and the stacked index weights
+    w_idx [(h_kv + 1) d_idx, d_model] (uint16 bf16 bits).
+
+    Default: x ~ N(0, 1) and w ~ N(0, 1 / d_model) rounded to bf16.  With
+    ``integer``: every row of x has 8 entries of +-1 at random columns (zeros
+    elsewhere) and w is uniform on {-3..3}, so every projected value is an
+    integer of magnitude <= 24 -- exact in fp32 and bf16, which makes the
+    index ids downstream of the projection reproducible bit for bit.
+    """
+    n_out = (h_kv + 1) * d_idx
+    g = _rng(seed, _T_QIDX, 7)
+    if integer:
+        x = np.zeros((n, d_model), dtype=np.float32)
+        cols = np.argsort(g.random((n, d_model)), axis=1)[:, :8] if d_model <= 4096 else \
+            np.stack([g.choice(d_model, 8, replace=False) for _ in range(n)])
+        signs = g.choice(np.array([-1.0, 1.0], dtype=np.float32), size=(n, 8))
+        np.put_along_axis(x, cols, signs, axis=1)
+        w = g.integers(-3, 4, size=(n_out, d_model)).astype(np.float32)
+    else:
+        x = g.standard_normal((n, d_model), dtype=np.float32)
+        w = g.standard_normal((n_out, d_model), dtype=np.float32) / np.float32(np.sqrt(d_model))
+    return {"x": f32_to_bf16_bits(x), "w_idx": f32_to_bf16_bits(w)}
