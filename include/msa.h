@@ -258,6 +258,21 @@ MSA_API int msa_sparse_attn_decode_noalloc(const msa_params* p, const void* q, c
                                            const int64_t* cu_kv, int batch, int max_kv, int dense,
                                            int32_t* block_ids, void* o, void* stream);
 
+/*
+ * MXFP8 quantisation of a bf16 tensor (the MXFP8 KV cache of the zhichai.net
+ * summary; format: OCP Microscaling formats v1.0, E4M3 elements with an E8M0
+ * scale per 32 consecutive elements of the last dimension).  Per block:
+ * e = floor(log2 max|x|) - 8 clamped to [-127, 127] (-127 for an all-zero
+ * block), elements x / 2^e rounded to the E4M3 grid (nearest even, saturated
+ * at +-448), scale byte e + 127.
+ *   x       bf16  [rows, cols], cols % 32 == 0 (16-byte aligned)
+ *   q       uint8 [rows, cols] E4M3 codes (16-byte aligned), output
+ *   scales  uint8 [rows, cols / 32] E8M0 codes, output
+ * Element i of x dequantises to E4M3(q_i) * 2^(scales[i / 32] - 127).
+ * Asynchronous on `stream`; no workspace.
+ */
+MSA_API int msa_quantize_mxfp8(const void* x, long long rows, int cols, void* q, void* scales, void* stream);
+
 /* Human-readable text of a status code (static storage). */
 MSA_API const char* msa_status_string(int status);
 

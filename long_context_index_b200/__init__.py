@@ -15,7 +15,7 @@ from typing import Optional
 __all__ = ["MSAError", "Params", "lib", "workspace_size", "index_topk", "sparse_attn_prefill",
            "sparse_attn_decode", "index_topk_varlen", "sparse_attn_prefill_varlen", "device_status",
            "status_string", "OP_INDEX_TOPK", "OP_PREFILL", "OP_DECODE", "OP_INDEX_TOPK_VARLEN",
-           "OP_PREFILL_VARLEN", "OP_INDEX_PROJECT", "index_project", "POOL_MAX", "POOL_MEAN"]
+           "OP_PREFILL_VARLEN", "OP_INDEX_PROJECT", "index_project", "quantize_mxfp8", "POOL_MAX", "POOL_MEAN"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmsa.so")
@@ -23,7 +23,7 @@ LIB_PATH = os.path.join(_HERE, "libmsa.so")
 OP_INDEX_TOPK, OP_PREFILL, OP_DECODE, OP_INDEX_TOPK_VARLEN, OP_PREFILL_VARLEN, OP_INDEX_PROJECT = 0, 1, 2, 3, 4, 5
 POOL_MAX, POOL_MEAN = 0, 1   # msa_params.pool
 
-SYMBOLS = ("msa_workspace_size", "msa_index_project", "msa_index_topk", "msa_sparse_attn_prefill", "msa_sparse_attn_decode",
+SYMBOLS = ("msa_workspace_size", "msa_index_project", "msa_quantize_mxfp8", "msa_index_topk", "msa_sparse_attn_prefill", "msa_sparse_attn_decode",
            "msa_index_topk_varlen", "msa_sparse_attn_prefill_varlen", "msa_sparse_attn_decode_adaptive_k",
            "msa_device_status", "msa_status_string",
            "msa_sparse_attn_decode_noalloc", "msa_test_never_ready_wait")
@@ -69,6 +69,8 @@ def lib():
         L.msa_sparse_attn_decode.argtypes = [P, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, vp, vp, sz, vp]
         L.msa_sparse_attn_decode_adaptive_k.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, vp,
                                                         vp, sz, vp]
+        L.msa_quantize_mxfp8.argtypes = [vp, C.c_longlong, i32, vp, vp, vp]
+        L.msa_quantize_mxfp8.restype = i32
         L.msa_index_project.argtypes = [P, vp, vp, i32, i32, vp, vp, vp, sz, vp]
         L.msa_index_topk_varlen.argtypes = [P, vp, vp, vp, i32, i32, vp, vp, vp, sz, vp]
         L.msa_sparse_attn_prefill_varlen.argtypes = [P, vp, vp, vp, vp, i32, i32, vp, vp, vp, sz, vp]
@@ -162,6 +164,24 @@ def index_project(p: Params, x, w_idx, q_idx=None, k_idx=None, ws=None, stream=N
         raise MSAError(rc, "msa_index_project")
     _after(ws, stream, "msa_index_project")
     return q_idx, k_idx
+
+
+def quantize_mxfp8(x, q=None, scales=None, stream=None):
+    """MXFP8 (E4M3 + E8M0 per 32 elements of the last dim) of a bf16 tensor: (q uint8, scales uint8)."""
+    torch = _torch()
+    _check(x, "x", _bf16())
+    cols = x.shape[-1]
+    rows = x.numel() // cols if cols else 0
+    if q is None:
+        q = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(tuple(x.shape[:-1]) + (cols // 32,), dtype=torch.uint8, device=x.device)
+    _check(q, "q", (torch.uint8,), tuple(x.shape))
+    _check(scales, "scales", (torch.uint8,), tuple(x.shape[:-1]) + (cols // 32,))
+    rc = lib().msa_quantize_mxfp8(_ptr(x), rows, cols, _ptr(q), _ptr(scales), _stream(stream))
+    if rc:
+        raise MSAError(rc, "msa_quantize_mxfp8")
+    return q, scales
 
 
 def index_topk(p: Params, q_idx, k_idx, q_pos0: int = 0, block_ids=None, ws=None, stream=None):

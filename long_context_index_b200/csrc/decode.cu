@@ -82,6 +82,31 @@ __device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
                : "l"(p));
   return v;
 }
+__device__ __forceinline__ uint2 ldg_nc_v2(const void* p) {
+  uint2 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+  return v;
+}
+
+// MXFP8 (E4M3 element, E8M0 block scale) -> bf16.  Every E4M3 value is exact
+// in f16, the scale is a power of two, and the product (at most 4 significant
+// bits) is exact in bf16.
+__device__ __forceinline__ float e8m0_scale(uint32_t e) {
+  return e ? __int_as_float(static_cast<int>(e) << 23) : __int_as_float(0x00400000);   // 2^(e - 127)
+}
+__device__ __forceinline__ uint32_t dq_e4m3x2(uint32_t two_bytes, float sc) {
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(static_cast<uint16_t>(two_bytes)));
+  float lo, hi;
+  asm("cvt.f32.f16 %0, %1;" : "=f"(lo) : "h"(static_cast<uint16_t>(h & 0xffffu)));
+  asm("cvt.f32.f16 %0, %1;" : "=f"(hi) : "h"(static_cast<uint16_t>(h >> 16)));
+  return pack_bf16x2(lo * sc, hi * sc);
+}
+// 8 E4M3 codes (one uint2, element 0 in the lowest byte) -> 8 bf16 (one uint4).
+__device__ __forceinline__ uint4 dq_e4m3x8(uint2 v, float sc) {
+  return make_uint4(dq_e4m3x2(v.x & 0xffffu, sc), dq_e4m3x2(v.x >> 16, sc), dq_e4m3x2(v.y & 0xffffu, sc),
+                    dq_e4m3x2(v.y >> 16, sc));
+}
 
 // (score desc, block asc) order used for every selection.
 __device__ __forceinline__ bool better(float s1, int b1, float s2, int b2) {
@@ -106,6 +131,14 @@ struct DecArgs {
   int splits, slots_per_split, dense, head_tiles, pool;
   float scale_log2;
   const int32_t* topk_seq;  // [B] blocks kept per sequence (adaptive k), or null: topk
+  // MXFP8 caches (E4M3 codes + E8M0 scales per 32 elements of the last dim),
+  // or null: the bf16 caches above.
+  const uint8_t* k_idx8;    // [sum L, 1, d_idx] and scales [sum L, 1, d_idx / 32]
+  const uint8_t* k_idx_sc;
+  const uint8_t* k8;        // [sum L, h_kv, d] and scales [sum L, h_kv, d / 32]
+  const uint8_t* k_sc;
+  const uint8_t* v8;
+  const uint8_t* v_sc;
 };
 
 // ---------------------------------------------------------------------------
@@ -126,7 +159,7 @@ template <int BK>
 __device__ void merge_topk_warp(const DecArgs& a, int b, int r, int lane, int* chosen, int c_lo, int nseg,
                                 long long T, int n);
 
-template <int DIDX, int BK, int POOL>
+template <int DIDX, int BK, int POOL, bool F8>
 __global__ void __launch_bounds__(kIdxThreads, kIdxCtasPerSm) decode_index_kernel(const DecArgs a) {
   constexpr int kHalves = DIDX / 32;   // 16-byte vectors per token row per thread
   constexpr int kWarps = kIdxThreads / 32;
@@ -188,6 +221,8 @@ __global__ void __launch_bounds__(kIdxThreads, kIdxCtasPerSm) decode_index_kerne
   // Score: warp w takes blocks w, w + 8, ... of the range.
   int cur = -1, cur_end = 0, cur_p = 0, L = 0;
   const uint16_t* kbase = a.k_idx;
+  const uint8_t* kbase8 = a.k_idx8;       // MXFP8: codes and scales of this sequence
+  const uint8_t* sbase8 = a.k_idx_sc;
   uint4 qv[kHalves];
   for (int i = warp; i < W; i += kWarps) {
     const int gb = G0 + i;
@@ -197,7 +232,12 @@ __global__ void __launch_bounds__(kIdxThreads, kIdxCtasPerSm) decode_index_kerne
       cur_end = pfx[cur + 1];
       const int64_t off = a.cu_kv[cur];
       L = static_cast<int>(a.cu_kv[cur + 1] - off);
-      kbase = a.k_idx + static_cast<size_t>(off) * DIDX;
+      if (F8) {
+        kbase8 = a.k_idx8 + static_cast<size_t>(off) * DIDX;
+        sbase8 = a.k_idx_sc + static_cast<size_t>(off) * (DIDX / 32);
+      } else {
+        kbase = a.k_idx + static_cast<size_t>(off) * DIDX;
+      }
       // Q_idx fragment (B operand): column n = group g, permuted d_idx order.
 #pragma unroll
       for (int h = 0; h < kHalves; ++h) {
@@ -217,8 +257,17 @@ __global__ void __launch_bounds__(kIdxThreads, kIdxCtasPerSm) decode_index_kerne
       uint4 ra[kHalves], rb[kHalves];
 #pragma unroll
       for (int h = 0; h < kHalves; ++h) {
-        ra[h] = ja < L ? ldg_nc_v4(kbase + static_cast<size_t>(ja) * DIDX + 8 * t + 32 * h) : make_uint4(0, 0, 0, 0);
-        rb[h] = jb < L ? ldg_nc_v4(kbase + static_cast<size_t>(jb) * DIDX + 8 * t + 32 * h) : make_uint4(0, 0, 0, 0);
+        if (F8) {   // elements 8t + 32h .. +7 lie in scale block h
+          ra[h] = ja < L ? dq_e4m3x8(ldg_nc_v2(kbase8 + static_cast<size_t>(ja) * DIDX + 8 * t + 32 * h),
+                                     e8m0_scale(sbase8[static_cast<size_t>(ja) * (DIDX / 32) + h]))
+                         : make_uint4(0, 0, 0, 0);
+          rb[h] = jb < L ? dq_e4m3x8(ldg_nc_v2(kbase8 + static_cast<size_t>(jb) * DIDX + 8 * t + 32 * h),
+                                     e8m0_scale(sbase8[static_cast<size_t>(jb) * (DIDX / 32) + h]))
+                         : make_uint4(0, 0, 0, 0);
+        } else {
+          ra[h] = ja < L ? ldg_nc_v4(kbase + static_cast<size_t>(ja) * DIDX + 8 * t + 32 * h) : make_uint4(0, 0, 0, 0);
+          rb[h] = jb < L ? ldg_nc_v4(kbase + static_cast<size_t>(jb) * DIDX + 8 * t + 32 * h) : make_uint4(0, 0, 0, 0);
+        }
       }
       float c[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -724,16 +773,24 @@ constexpr int kStreamThreads = 32 * (kStreamConsumers + 1);
 constexpr int kStreamCtas = 148;       // persistent grid: one CTA per SM
 constexpr int kStreamIdsCap = 1024;    // items per CTA held in shared memory
 
-template <int D, int BK>
+template <int D, int BK, bool F8 = false>
 struct StreamCfg {
   static constexpr int kHalves = D / 64;                  // 128-byte column halves
   static constexpr int kQBytes = 16 * 128 * kHalves;      // 16 head rows x D
-  static constexpr int kKBytes = BK * 128 * kHalves;      // BK keys x D
-  static constexpr int kStageBytes = kQBytes + 2 * kKBytes;
-  static constexpr int kFit = (212 * 1024) / kStageBytes;
+  static constexpr int kKBytes = BK * 128 * kHalves;      // BK keys x D (bf16)
+  // MXFP8 caches: the stage holds E4M3 K and V blocks (BK x D bytes each,
+  // 128B-swizzled rows of D bytes) and their scales (BK x D/32 bytes each);
+  // the consumers dequantise a stage into one bf16 K/V tile pair (kDeqBytes).
+  static constexpr int kK8Bytes = BK * D;
+  static constexpr int kScBytes = BK * (D / 32);
+  static constexpr int kStageBytes =
+      F8 ? ((kQBytes + 2 * kK8Bytes + 2 * kScBytes + 1023) / 1024) * 1024 : kQBytes + 2 * kKBytes;
+  static constexpr int kDeqBytes = F8 ? 2 * kKBytes : 0;
+  static constexpr int kFit = (212 * 1024 - kDeqBytes) / kStageBytes;
   static constexpr int kStages = kFit > 8 ? 8 : kFit;
   static constexpr int kPBytes = 16 * BK * 2;
-  static constexpr int kOffP = kStages * kStageBytes;
+  static constexpr int kOffDeq = kStages * kStageBytes;
+  static constexpr int kOffP = kOffDeq + kDeqBytes;
   static constexpr int kOffRed = kOffP + kPBytes;                       // red_m[4][16], red_l[4][16]
   static constexpr int kOffIds = kOffRed + 2 * kStreamConsumers * 16 * 4;
   static constexpr int kOffMeta = kOffIds + kStreamIdsCap * 4;          // int4 per stage
@@ -754,6 +811,8 @@ struct StreamArgs {
   long long total_items;      // T = U * topk
   int n_cta, h_q, h_kv, topk, head_tiles, group;
   float scale_log2;
+  const uint8_t* k_sc;        // MXFP8 caches: E8M0 scales [sum L, h_kv, d / 32] (null for bf16)
+  const uint8_t* v_sc;
 };
 
 // Byte offset of 16-byte chunk ch of row x in a TMA 128B-swizzled tile of
@@ -766,11 +825,11 @@ __device__ __forceinline__ int cta_of_item(long long g, long long T, int n) {
   return static_cast<int>(((g + 1) * n - 1) / T);
 }
 
-template <int D, int BK>
+template <int D, int BK, bool F8>
 __global__ void __launch_bounds__(kStreamThreads, 1)
     decode_attn_stream_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                               const __grid_constant__ CUtensorMap tm_v, const StreamArgs a) {
-  using C = StreamCfg<D, BK>;
+  using C = StreamCfg<D, BK, F8>;
   constexpr int KPW = BK / kStreamConsumers;   // S keys per warp
   constexpr int NT = KPW / 8;
   constexpr int NCOL = D / kStreamConsumers;   // O columns per warp
@@ -808,7 +867,9 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
   }
   if (tid == 0) {
     for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&full[s], 1);
+      // MXFP8: the TMA bytes, then one cp.async arrival per producer lane
+      // once its share of the block's scales has landed.
+      mbar_init(&full[s], F8 ? 33 : 1);
       mbar_init(&empty[s], kStreamConsumers);
     }
     flags[0] = 0;
@@ -821,10 +882,15 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
 
   if (warp == kStreamConsumers) {
     // ---------------- producer ----------------
-    if (lane != 0) return;
-    tma_prefetch_desc(&tm_q);
-    tma_prefetch_desc(&tm_k);
-    tma_prefetch_desc(&tm_v);
+    // Lane 0 waits for a free stage and issues the TMA loads; with MXFP8
+    // caches the whole warp then gathers the K and V scales of the block into
+    // the stage (a second arrival on its full barrier).
+    if (!F8 && lane != 0) return;
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+    }
     long long cur_u = -1;
     long long off = 0;
     int L = 0, qrow = 0, r = 0;
@@ -843,27 +909,56 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
       }
       const int stage = issued % C::kStages;
       const uint32_t ph = (issued / C::kStages) & 1;
-      if (!mbar_wait(&empty[stage], ph ^ 1, wc)) break;
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(&empty[stage], ph ^ 1, wc);
+      if (F8) ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
       const int j0 = blk * BK;
       // The last (partial) block is fetched as the BK keys ending at L, so no
       // box reaches past this sequence; rows before j0 are masked.
       const int kbase = j0 + BK <= L ? j0 : L - BK;
-      meta[stage] = make_int4(j0, kbase, min(j0 + BK, L), 0);
-      mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
       uint8_t* st = smem + stage * C::kStageBytes;
       const int krow = static_cast<int>(off + kbase);
+      if (lane == 0) {
+        meta[stage] = make_int4(j0, kbase, min(j0 + BK, L), 0);
+        if (F8) {
+          mbar_arrive_expect_tx(&full[stage], C::kQBytes + 2 * C::kK8Bytes);
 #pragma unroll
-      for (int h = 0; h < C::kHalves; ++h) {
-        tma_load_2d(st + h * 16 * 128, &tm_q, &full[stage], h * 64, qrow);
-        tma_load_3d(st + C::kQBytes + h * BK * 128, &tm_k, &full[stage], h * 64, r, krow);
-        tma_load_3d(st + C::kQBytes + C::kKBytes + h * BK * 128, &tm_v, &full[stage], h * 64, r, krow);
+          for (int h = 0; h < C::kHalves; ++h) tma_load_2d(st + h * 16 * 128, &tm_q, &full[stage], h * 64, qrow);
+          tma_load_3d(st + C::kQBytes, &tm_k, &full[stage], 0, r, krow);
+          tma_load_3d(st + C::kQBytes + C::kK8Bytes, &tm_v, &full[stage], 0, r, krow);
+        } else {
+          mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+#pragma unroll
+          for (int h = 0; h < C::kHalves; ++h) {
+            tma_load_2d(st + h * 16 * 128, &tm_q, &full[stage], h * 64, qrow);
+            tma_load_3d(st + C::kQBytes + h * BK * 128, &tm_k, &full[stage], h * 64, r, krow);
+            tma_load_3d(st + C::kQBytes + C::kKBytes + h * BK * 128, &tm_v, &full[stage], h * 64, r, krow);
+          }
+        }
+      }
+      if (F8) {
+        // Scales of keys krow .. krow + BK - 1 of group r (D/32 = 4 bytes per
+        // key), copied asynchronously; each lane's arrival on the stage's full
+        // barrier fires when its copies have landed.
+        static_assert(!F8 || D / 32 == 4, "MXFP8 decode: 4 scale bytes per key row");
+        const uint32_t ssc = smem_u32(st + C::kQBytes + 2 * C::kK8Bytes);
+        for (int x = lane; x < BK; x += 32) {
+          const size_t at = ((static_cast<size_t>(krow) + x) * a.h_kv + r) * 4;
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(ssc + x * 4), "l"(a.k_sc + at) : "memory");
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(ssc + C::kScBytes + x * 4), "l"(a.v_sc + at)
+                       : "memory");
+        }
+        asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&full[stage])) : "memory");
       }
       ++issued;
     }
     // Loads still in flight (only possible after an abort) land before exit.
-    WaitCtx drain{reinterpret_cast<volatile int*>(&flags[2]), a.status};
-    for (int k = issued > C::kStages ? issued - C::kStages : 0; k < issued; ++k)
-      mbar_wait(&full[k % C::kStages], (k / C::kStages) & 1, drain);
+    if (lane == 0) {
+      WaitCtx drain{reinterpret_cast<volatile int*>(&flags[2]), a.status};
+      for (int k = issued > C::kStages ? issued - C::kStages : 0; k < issued; ++k)
+        mbar_wait(&full[k % C::kStages], (k / C::kStages) & 1, drain);
+    }
     return;
   }
 
@@ -887,8 +982,38 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
       const int4 md = meta[stage];
       const int j0 = md.x, kbase = md.y, jend = md.z;
       const uint32_t sQ = sbase + stage * C::kStageBytes;
-      const uint32_t sK = sQ + C::kQBytes;
-      const uint32_t sV = sK + C::kKBytes;
+      uint32_t sK = sQ + C::kQBytes;
+      uint32_t sV = sK + C::kKBytes;
+      if (F8) {
+        // Dequantise the stage's E4M3 K and V blocks into the bf16 tile pair
+        // (the layout the bf16 path reads: 128B-swizzled rows of D/64 column
+        // halves).  The previous item's S and PV have finished with that
+        // pair, and the stage is released as soon as its bytes are converted.
+        sK = sbase + C::kOffDeq;
+        sV = sK + C::kKBytes;
+        named_bar(1, 32 * kStreamConsumers);
+        const uint8_t* s8 = smem + stage * C::kStageBytes + C::kQBytes;
+        const uint8_t* ssc = s8 + 2 * C::kK8Bytes;
+        constexpr int CPR = D / 16;                      // 16-byte chunks per E4M3 row
+        for (int e = tid; e < 2 * BK * CPR; e += 32 * kStreamConsumers) {
+          const int kv = e / (BK * CPR), rem = e - kv * (BK * CPR);
+          const int x = rem / CPR, c = rem - x * CPR;   // row, chunk (16 elements from column 16c)
+          // E4M3 rows of D = 128 bytes, 128B-swizzled by TMA (16-byte chunk c of row x at c ^ (x & 7)).
+          const uint4 raw = *reinterpret_cast<const uint4*>(s8 + kv * C::kK8Bytes + x * D + ((c ^ (x & 7)) << 4));
+          const float sc = e8m0_scale(ssc[kv * C::kScBytes + x * (D / 32) + c / 2]);
+          const uint4 lo = dq_e4m3x8(make_uint2(raw.x, raw.y), sc), hi = dq_e4m3x8(make_uint2(raw.z, raw.w), sc);
+          const uint32_t dst = (kv ? sV : sK);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sw128(dst, BK, x, 2 * c)), "r"(lo.x),
+                       "r"(lo.y), "r"(lo.z), "r"(lo.w)
+                       : "memory");
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sw128(dst, BK, x, 2 * c + 1)), "r"(hi.x),
+                       "r"(hi.y), "r"(hi.z), "r"(hi.w)
+                       : "memory");
+        }
+        named_bar(1, 32 * kStreamConsumers);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[stage]);
+      }
 
       uint32_t qf[D / 16][4];
 #pragma unroll
@@ -1002,9 +1127,11 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
           mma_bf16_16816(oacc[dt + 1], a0, a1, a2, a3, b2, b3);
         }
       }
-      if (zap) fence_proxy_async_smem();   // generic writes before the stage's next TMA fill
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[stage]);
+      if (!F8) {
+        if (zap) fence_proxy_async_smem();   // generic writes before the stage's next TMA fill
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[stage]);
+      }
     }
 
     // End of this CTA's share of unit u: write it out.
@@ -1150,9 +1277,9 @@ int stream_ctas(long long T) {
   return static_cast<int>(n < T ? n : T);
 }
 
-template <int D, int BK>
+template <int D, int BK, bool F8>
 int launch_attn_stream(const DecArgs& a, int max_kv, int* status, cudaStream_t st) {
-  using C = StreamCfg<D, BK>;
+  using C = StreamCfg<D, BK, F8>;
   CUtensorMap tq, tk, tv;
   {
     const uint64_t dims[2] = {static_cast<uint64_t>(D), static_cast<uint64_t>(a.batch) * a.h_q};
@@ -1165,9 +1292,16 @@ int launch_attn_stream(const DecArgs& a, int max_kv, int* status, cudaStream_t s
     const uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(a.h_kv),
                               static_cast<uint64_t>(a.batch) * max_kv};
     const uint64_t strides[2] = {static_cast<uint64_t>(D) * 2, static_cast<uint64_t>(a.h_kv) * D * 2};
-    const uint32_t box[3] = {64, 1, BK};
-    if (!encode_tma_bf16(&tk, 3, a.k_cache, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MSA_ERR_CUDA;
-    if (!encode_tma_bf16(&tv, 3, a.v_cache, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MSA_ERR_CUDA;
+    if (F8) {   // E4M3 codes: one byte per element, a whole D = 128-byte row per box row
+      const uint64_t strides8[2] = {static_cast<uint64_t>(D), static_cast<uint64_t>(a.h_kv) * D};
+      const uint32_t box8[3] = {D, 1, BK};
+      if (!encode_tma_u8(&tk, 3, a.k8, dims, strides8, box8, CU_TENSOR_MAP_SWIZZLE_128B)) return MSA_ERR_CUDA;
+      if (!encode_tma_u8(&tv, 3, a.v8, dims, strides8, box8, CU_TENSOR_MAP_SWIZZLE_128B)) return MSA_ERR_CUDA;
+    } else {
+      const uint32_t box[3] = {64, 1, BK};
+      if (!encode_tma_bf16(&tk, 3, a.k_cache, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MSA_ERR_CUDA;
+      if (!encode_tma_bf16(&tv, 3, a.v_cache, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MSA_ERR_CUDA;
+    }
   }
   StreamArgs s;
   s.block_ids = a.block_ids;
@@ -1184,8 +1318,10 @@ int launch_attn_stream(const DecArgs& a, int max_kv, int* status, cudaStream_t s
   s.head_tiles = a.head_tiles;
   s.group = a.h_q / a.h_kv;
   s.scale_log2 = a.scale_log2;
+  s.k_sc = a.k_sc;
+  s.v_sc = a.v_sc;
   const int smem = C::kSmemBytes + 1024;
-  auto kern = decode_attn_stream_kernel<D, BK>;
+  auto kern = decode_attn_stream_kernel<D, BK, F8>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return MSA_ERR_CUDA;
   kern<<<s.n_cta, kStreamThreads, smem, st>>>(tq, tk, tv, s);
@@ -1195,7 +1331,8 @@ int launch_attn_stream(const DecArgs& a, int max_kv, int* status, cudaStream_t s
 template <int DIDX, int BK>
 int launch_index(const DecArgs& a, size_t smem, cudaStream_t st) {
   if (a.kfree > 0) {
-    auto kern = a.pool ? decode_index_kernel<DIDX, BK, 1> : decode_index_kernel<DIDX, BK, 0>;
+    auto kern = a.k_idx8 ? (a.pool ? decode_index_kernel<DIDX, BK, 1, true> : decode_index_kernel<DIDX, BK, 0, true>)
+                         : (a.pool ? decode_index_kernel<DIDX, BK, 1, false> : decode_index_kernel<DIDX, BK, 0, false>);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
         cudaSuccess)
       return MSA_ERR_CUDA;
@@ -1236,7 +1373,7 @@ size_t decode_workspace_bytes(const msa_params& p, int batch, int max_kv, int de
 int run_sparse_attn_decode(const msa_params& p, const void* q, const void* q_idx, const void* k_cache,
                            const void* v_cache, const void* k_idx_cache, const int64_t* cu_kv, int batch,
                            int max_kv, int dense, int32_t* block_ids, void* o, void* ws, size_t /*ws_bytes*/,
-                           int* status, cudaStream_t stream, const int32_t* topk_seq) {
+                           int* status, cudaStream_t stream, const int32_t* topk_seq, const DecodeMx8* mx8) {
   if (p.h_kv > kDecodeMaxGroups) return MSA_ERR_UNSUPPORTED;
   // TMA row coordinates of the caches are 32-bit.
   if (!dense && static_cast<long long>(batch) * max_kv > 0x7fffffffLL) return MSA_ERR_UNSUPPORTED;
@@ -1260,6 +1397,12 @@ int run_sparse_attn_decode(const msa_params& p, const void* q, const void* q_idx
   a.kfree = p.topk - (p.force_local ? 1 : 0);
   a.pool = p.pool;
   a.topk_seq = topk_seq;
+  a.k8 = mx8 ? static_cast<const uint8_t*>(mx8->k8) : nullptr;
+  a.k_sc = mx8 ? static_cast<const uint8_t*>(mx8->k_sc) : nullptr;
+  a.v8 = mx8 ? static_cast<const uint8_t*>(mx8->v8) : nullptr;
+  a.v_sc = mx8 ? static_cast<const uint8_t*>(mx8->v_sc) : nullptr;
+  a.k_idx8 = mx8 ? static_cast<const uint8_t*>(mx8->k_idx8) : nullptr;
+  a.k_idx_sc = mx8 ? static_cast<const uint8_t*>(mx8->k_idx_sc) : nullptr;
   const IdxPlan ip = plan_index(p, batch, max_kv);
   a.idx_ctas = ip.ctas;
   a.idx_wmax = ip.wmax;
@@ -1292,11 +1435,14 @@ int run_sparse_attn_decode(const msa_params& p, const void* q, const void* q_idx
   }
   if (rc) return rc;
   if (!dense) {
+    if (a.k8)   // MXFP8 caches (d = 128, checked on the host)
+      return p.block_k == 64 ? launch_attn_stream<128, 64, true>(a, max_kv, status, stream)
+                             : launch_attn_stream<128, 128, true>(a, max_kv, status, stream);
     if (p.d == 64)
-      return p.block_k == 64 ? launch_attn_stream<64, 64>(a, max_kv, status, stream)
-                             : launch_attn_stream<64, 128>(a, max_kv, status, stream);
-    return p.block_k == 64 ? launch_attn_stream<128, 64>(a, max_kv, status, stream)
-                           : launch_attn_stream<128, 128>(a, max_kv, status, stream);
+      return p.block_k == 64 ? launch_attn_stream<64, 64, false>(a, max_kv, status, stream)
+                             : launch_attn_stream<64, 128, false>(a, max_kv, status, stream);
+    return p.block_k == 64 ? launch_attn_stream<128, 64, false>(a, max_kv, status, stream)
+                           : launch_attn_stream<128, 128, false>(a, max_kv, status, stream);
   }
   if (p.d == 64) {
     return p.block_k == 64 ? launch_attn_combine<64, 64>(a, stream) : launch_attn_combine<64, 128>(a, stream);

@@ -69,8 +69,8 @@ EncodeTiledFn encode_fn() {
 
 }  // namespace
 
-bool encode_tma_bf16(CUtensorMap* map, int rank, const void* base, const uint64_t* dims, const uint64_t* strides,
-                     const uint32_t* box, CUtensorMapSwizzle swizzle) {
+static bool encode_tma(CUtensorMapDataType type, CUtensorMap* map, int rank, const void* base, const uint64_t* dims,
+                       const uint64_t* strides, const uint32_t* box, CUtensorMapSwizzle swizzle) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t d[5], s[4];
@@ -81,10 +81,20 @@ bool encode_tma_bf16(CUtensorMap* map, int rank, const void* base, const uint64_
     e[i] = 1;
   }
   for (int i = 0; i + 1 < rank; ++i) s[i] = strides[i];
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank), const_cast<void*>(base), d,
+  CUresult r = fn(map, type, static_cast<cuuint32_t>(rank), const_cast<void*>(base), d,
                   s, b, e, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool encode_tma_bf16(CUtensorMap* map, int rank, const void* base, const uint64_t* dims, const uint64_t* strides,
+                     const uint32_t* box, CUtensorMapSwizzle swizzle) {
+  return encode_tma(CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, map, rank, base, dims, strides, box, swizzle);
+}
+
+bool encode_tma_u8(CUtensorMap* map, int rank, const void* base, const uint64_t* dims, const uint64_t* strides,
+                   const uint32_t* box, CUtensorMapSwizzle swizzle) {
+  return encode_tma(CU_TENSOR_MAP_DATA_TYPE_UINT8, map, rank, base, dims, strides, box, swizzle);
 }
 
 }  // namespace msa
@@ -163,10 +173,10 @@ int msa_sparse_attn_prefill(const msa_params* p, const void* q, const void* k, c
                                  static_cast<int*>(ws), st);
 }
 
-int msa_sparse_attn_decode_adaptive_k(const msa_params* p, const void* q, const void* q_idx, const void* k_cache,
-                                      const void* v_cache, const void* k_idx_cache, const int64_t* cu_kv,
-                                      const int32_t* topk_per_seq, int batch, int max_kv, int dense,
-                                      int32_t* block_ids, void* o, void* ws, size_t ws_bytes, void* stream) {
+static int decode_call(const msa_params* p, const void* q, const void* q_idx, const void* k_cache, const void* v_cache,
+                       const void* k_idx_cache, const int64_t* cu_kv, const int32_t* topk_per_seq, int batch,
+                       int max_kv, int dense, int32_t* block_ids, void* o, void* ws, size_t ws_bytes, void* stream,
+                       const DecodeMx8* mx8) {
   int rc = check_params(p);
   if (rc) return rc;
   if (batch <= 0 || max_kv <= 0 || (dense != 0 && dense != 1)) return MSA_ERR_INVALID;
@@ -190,8 +200,35 @@ int msa_sparse_attn_decode_adaptive_k(const msa_params* p, const void* q, const 
   if (cudaMemsetAsync(ws, 0, kWsHeader + decode_counter_bytes(*p, batch), st) != cudaSuccess) return MSA_ERR_CUDA;
   return run_sparse_attn_decode(*p, q, q_idx, k_cache, v_cache, k_idx_cache, cu_kv, batch, max_kv, dense,
                                 block_ids, o, static_cast<uint8_t*>(ws) + kWsHeader, ws_bytes - kWsHeader,
-                                static_cast<int*>(ws), st, dense ? nullptr : topk_per_seq);
+                                static_cast<int*>(ws), st, dense ? nullptr : topk_per_seq, mx8);
 }
+
+int msa_sparse_attn_decode_adaptive_k(const msa_params* p, const void* q, const void* q_idx, const void* k_cache,
+                                      const void* v_cache, const void* k_idx_cache, const int64_t* cu_kv,
+                                      const int32_t* topk_per_seq, int batch, int max_kv, int dense,
+                                      int32_t* block_ids, void* o, void* ws, size_t ws_bytes, void* stream) {
+  return decode_call(p, q, q_idx, k_cache, v_cache, k_idx_cache, cu_kv, topk_per_seq, batch, max_kv, dense,
+                     block_ids, o, ws, ws_bytes, stream, nullptr);
+}
+
+int msa_sparse_attn_decode_mxfp8(const msa_params* p, const void* q, const void* q_idx, const void* k8,
+                                 const void* k_scale, const void* v8, const void* v_scale, const void* k_idx8,
+                                 const void* k_idx_scale, const int64_t* cu_kv, const int32_t* topk_per_seq, int batch,
+                                 int max_kv, int32_t* block_ids, void* o, void* ws, size_t ws_bytes, void* stream) {
+  const int rc = check_params(p);
+  if (rc) return rc;
+  if (p->d != 128) return MSA_ERR_UNSUPPORTED;
+  if (!k8 || !k_scale || !v8 || !v_scale || !k_idx8 || !k_idx_scale) return MSA_ERR_INVALID;
+  if (!aligned16(k8) || !aligned16(v8) || !aligned16(k_idx8)) return MSA_ERR_MISALIGNED;
+  if (((reinterpret_cast<uintptr_t>(k_scale) | reinterpret_cast<uintptr_t>(v_scale)) & 3u) != 0)
+    return MSA_ERR_MISALIGNED;
+  DecodeMx8 mx{k8, k_scale, v8, v_scale, k_idx8, k_idx_scale};
+  // The bf16 cache arguments are unused: the MXFP8 codes stand in for them
+  // (non-null placeholders for the shared validation).
+  return decode_call(p, q, q_idx, k8, v8, k_idx8, cu_kv, topk_per_seq, batch, max_kv, 0, block_ids, o, ws,
+                     ws_bytes, stream, &mx);
+}
+
 
 int msa_sparse_attn_decode(const msa_params* p, const void* q, const void* q_idx, const void* k_cache,
                            const void* v_cache, const void* k_idx_cache, const int64_t* cu_kv, int batch,

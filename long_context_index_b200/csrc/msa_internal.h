@@ -21,6 +21,9 @@ constexpr size_t kWsHeader = 256;
 // dims[0] is innermost; strides[] are the byte strides of dims 1..rank-1.
 bool encode_tma_bf16(CUtensorMap* map, int rank, const void* base, const uint64_t* dims,
                      const uint64_t* strides, const uint32_t* box, CUtensorMapSwizzle swizzle);
+// The same for a uint8 tensor (MXFP8 codes).
+bool encode_tma_u8(CUtensorMap* map, int rank, const void* base, const uint64_t* dims, const uint64_t* strides,
+                   const uint32_t* box, CUtensorMapSwizzle swizzle);
 
 // A packed batch of independent causal prefills (the varlen entry points):
 // sequence s owns rows [cu_seqlens[s], cu_seqlens[s + 1]) of every tensor.
@@ -78,12 +81,19 @@ int run_sparse_attn_kvouter(const msa_params& p, const void* q, const CUtensorMa
 constexpr int kDecodeMaxGroups = 8;     // h_kv: one index-scan warp per group
 constexpr int kDecodeMaxBatch = 4096;   // sparse: the block prefix of every sequence in shared memory
 size_t decode_counter_bytes(const msa_params& p, int batch);
+// MXFP8 decode caches (E4M3 codes with E8M0 scales per 32 elements), or null
+// in run_sparse_attn_decode for the bf16 caches.
+struct DecodeMx8 {
+  const void *k8, *k_sc, *v8, *v_sc;        // [sum L, h_kv, d] codes, [sum L, h_kv, d / 32] scales
+  const void *k_idx8, *k_idx_sc;            // [sum L, 1, d_idx] codes, [sum L, 1, d_idx / 32] scales
+};
 // dense: 1 = the dense run, 0 = the sparse run, -1 = the larger of the two.
 size_t decode_workspace_bytes(const msa_params& p, int batch, int max_kv, int dense);
 int run_sparse_attn_decode(const msa_params& p, const void* q, const void* q_idx, const void* k_cache,
                            const void* v_cache, const void* k_idx_cache, const int64_t* cu_kv, int batch,
                            int max_kv, int dense, int32_t* block_ids, void* o, void* ws, size_t ws_bytes,
-                           int* status, cudaStream_t stream, const int32_t* topk_seq = nullptr);
+                           int* status, cudaStream_t stream, const int32_t* topk_seq = nullptr,
+                           const DecodeMx8* mx8 = nullptr);
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 

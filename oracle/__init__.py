@@ -229,3 +229,74 @@ def index_project(x, w_idx, h_kv: int, d_idx: int):
     y = xf @ wf.T
     n = xf.shape[0]
     return y[:, :h_kv * d_idx].reshape(n, h_kv, d_idx), y[:, h_kv * d_idx:].reshape(n, 1, d_idx)
+
+
+# ---------------------------------------------------------------------------
+# MXFP8 (OCP Microscaling formats v1.0, E4M3 elements, E8M0 block scales):
+# the format of the quantised KV cache (the zhichai.net summary: "MXFP8 KV
+# cache").  Blocks of 32 consecutive elements along the last dimension share
+# one scale 2^e.
+# ---------------------------------------------------------------------------
+MX_BLOCK = 32
+E4M3_MAX = 448.0          # 1.75 * 2^8, the largest E4M3 normal
+E4M3_EMAX = 8             # its exponent
+
+
+def _e4m3_round(s: np.ndarray) -> np.ndarray:
+    """Round float64 values to the E4M3 grid, nearest even, saturating at +-448."""
+    a = np.abs(s)
+    with np.errstate(divide="ignore"):
+        ex = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    quantum = np.where(a >= 2.0 ** -6, 2.0 ** (ex - 3), 2.0 ** -9)
+    r = np.round(a / quantum) * quantum          # numpy rounds halves to even
+    r = np.minimum(r, E4M3_MAX)
+    return np.copysign(r, s)
+
+
+def _e4m3_encode(r: np.ndarray) -> np.ndarray:
+    a = np.abs(r)
+    sign = np.signbit(r).astype(np.uint8) << 7
+    with np.errstate(divide="ignore"):
+        ex = np.floor(np.log2(np.where(a > 0, a, 1.0))).astype(np.int64)
+    normal = a >= 2.0 ** -6
+    mant_n = np.where(normal, a / 2.0 ** ex * 8 - 8, 0).astype(np.int64)
+    code_n = ((ex + 7) << 3) | mant_n
+    code_s = (a / 2.0 ** -9).astype(np.int64)
+    return sign | np.where(normal, code_n, code_s).astype(np.uint8)
+
+
+def e4m3_decode(b: np.ndarray) -> np.ndarray:
+    """E4M3 byte -> float64 (no NaN codes are ever produced by the quantiser)."""
+    b = np.asarray(b, dtype=np.uint8).astype(np.int64)
+    e, m = (b >> 3) & 15, b & 7
+    mag = np.where(e == 0, m * 2.0 ** -9, (1 + m / 8.0) * 2.0 ** (e - 7))
+    return np.where(b & 0x80, -mag, mag)
+
+
+def quantize_mxfp8(x_bits):
+    """bf16 bits [..., C] (C % 32 == 0) -> (E4M3 bytes [..., C], E8M0 bytes [..., C / 32]).
+
+    Per block of 32: e = floor(log2(max |x|)) - 8, clamped to [-127, 127]
+    (a block of zeros takes e = -127); elements are x / 2^e rounded to the
+    E4M3 grid (nearest even, saturating at +-448); the scale byte is e + 127.
+    """
+    x = _widen(x_bits)
+    sh = x.shape
+    assert sh[-1] % MX_BLOCK == 0, sh
+    xb = x.reshape(sh[:-1] + (sh[-1] // MX_BLOCK, MX_BLOCK))
+    amax = np.abs(xb).max(axis=-1)
+    _, ex = np.frexp(amax)                        # amax = m 2^ex, m in [0.5, 1)
+    e = np.where(amax > 0, ex - 1 - E4M3_EMAX, -127)
+    e = np.clip(e, -127, 127).astype(np.int64)
+    scaled = xb / np.ldexp(1.0, e)[..., None]
+    q = _e4m3_encode(_e4m3_round(scaled)).reshape(sh)
+    return q, (e + 127).astype(np.uint8)
+
+
+def dequantize_mxfp8(q, scales) -> np.ndarray:
+    """E4M3 bytes [..., C] and E8M0 bytes [..., C / 32] -> float64 values."""
+    v = e4m3_decode(q)
+    sh = v.shape
+    vb = v.reshape(sh[:-1] + (sh[-1] // MX_BLOCK, MX_BLOCK))
+    sc = np.ldexp(1.0, np.asarray(scales, dtype=np.int64) - 127)
+    return (vb * sc[..., None]).reshape(sh)

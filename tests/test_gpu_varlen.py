@@ -92,9 +92,13 @@ def test_invalid_cu_seqlens_is_reported_not_computed():
     w = wl(seed=506)
     t = make_varlen_prefill(w, lens=[100, 200])
     p, _ = params_pair(w.h_q, w.h_kv, w.d, w.d_idx, w.block_k, w.topk)
-    bad = torch.tensor([0, 250, 300], dtype=torch.int32, device="cuda")   # cu[2] != total rows
+    bad = torch.tensor([0, 200, 150], dtype=torch.int32, device="cuda")   # decreasing: a negative length
     out = torch.full((300, w.h_kv, w.topk), -7, dtype=torch.int32, device="cuda")
     with pytest.raises(msa.MSAError) as err:
         msa.index_topk_varlen(p, dev(t["q_idx"]), dev(t["k_idx"]), bad, block_ids=out)
     assert err.value.code == -1
     assert torch.all(out == -7)           # nothing was written
+    short = torch.tensor([0, 100, 250], dtype=torch.int32, device="cuda")  # cu[batch] != total rows (300)
+    with pytest.raises(msa.MSAError) as err:
+        msa.index_topk_varlen(p, dev(t["q_idx"]), dev(t["k_idx"]), short, block_ids=out)
+    assert err.value.code == -1
