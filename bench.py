@@ -289,6 +289,35 @@ def run_ours(args, rank, world, torch, dist):
             rc = msa.device_status(wsx)
             if rc:
                 raise RuntimeError("device status %d after the dense runs" % rc)
+    # ---- the same decode step over MXFP8 caches (quantised untimed, then
+    # warmed up and timed over as many steps as the bf16 step)
+    t_mx = b_mx = None
+    if not args.no_mxfp8 and wd.d == 128:
+        q8 = {k_: msa.quantize_mxfp8(dd[k_]) for k_ in ("k_cache", "v_cache", "k_idx_cache")}
+        dids8 = torch.empty_like(dids)
+        do8 = torch.empty_like(do)
+
+        def mx_step():
+            msa.sparse_attn_decode_mxfp8(pd, dd["q"], dd["q_idx"], q8["k_cache"][0], q8["k_cache"][1],
+                                         q8["v_cache"][0], q8["v_cache"][1], q8["k_idx_cache"][0],
+                                         q8["k_idx_cache"][1], dd["cu_kv"], max_kv, block_ids=dids8, out=do8,
+                                         ws=ws_d)
+
+        for _ in range(args.warmup):
+            mx_step()
+        mev = [(E(enable_timing=True), E(enable_timing=True)) for _ in range(args.steps)]
+        for a_, b_ in mev:
+            a_.record(stream)
+            mx_step()
+            b_.record(stream)
+        torch.cuda.synchronize()
+        rc = msa.device_status(ws_d)
+        if rc:
+            raise RuntimeError("device status %d after the MXFP8 decode" % rc)
+        t_mx = statistics.median(a_.elapsed_time(b_) for a_, b_ in mev)
+        b_mx = flops.decode_bytes(td["lens"], dids8.cpu().numpy(), wd.h_q, wd.h_kv, wd.d, wd.d_idx, wd.block_k,
+                                  mxfp8=True)
+        del q8
     med_pre = statistics.median(e[0].elapsed_time(e[2]) for e in evs)
     med_dec = statistics.median(e[2].elapsed_time(e[3]) for e in evs)
 
@@ -372,6 +401,10 @@ def run_ours(args, rank, world, torch, dist):
                     "tensor_frac": (f_idx + f_main) / ((t_idx + t_attn) / 1e3) / 1e12 / peaks["bf16_tflops"]},
         "decode": {"ms": t_dec, "tokens_per_s": B * world / (t_dec / 1e3), "bytes": b_dec,
                    "hbm_frac": b_dec / (t_dec / 1e3) / 1e9 / peaks["hbm_gbs"]},
+        "decode_mxfp8": None if t_mx is None else {
+            "ms": t_mx, "tokens_per_s": B * world / (t_mx / 1e3), "bytes": b_mx,
+            "hbm_frac": b_mx / (t_mx / 1e3) / 1e9 / peaks["hbm_gbs"], "stat": "median per step",
+            "note": "the same decode step over MXFP8 (E4M3 + E8M0 per 32) K, V and index-key caches"},
         "dense": None if t_dense_p is None else {
             "prefill_ms": t_dense_p, "decode_ms": t_dense_d, "steps": args.steps, "warmup": args.warmup,
             "stat": "median per step; sparse medians %.3f ms prefill, %.4f ms decode" % (med_pre, med_dec),
@@ -478,6 +511,7 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-mxfp8", action="store_true")
     args = ap.parse_args(argv)
     if args.gpus < 1:
         ap.error("--gpus must be >= 1")

@@ -273,6 +273,28 @@ MSA_API int msa_sparse_attn_decode_noalloc(const msa_params* p, const void* q, c
  */
 MSA_API int msa_quantize_mxfp8(const void* x, long long rows, int cols, void* q, void* scales, void* stream);
 
+/*
+ * One batched decode step over MXFP8 caches (codes and scales as produced by
+ * msa_quantize_mxfp8): K, V and the index keys are stored as E4M3 with an
+ * E8M0 scale per 32 elements, about half the bytes of bf16 caches; the query,
+ * the index query and the output stay bf16.  The kernels dequantise exactly
+ * (E4M3 code * 2^(scale - 127) is exact in bf16), so the result is the bf16
+ * decode step of the dequantised caches: the ids those caches select and
+ * attention over their values.  Sparse run only; d = 128.
+ *   k8, v8         uint8 [sum L_b, h_kv, d]   E4M3 codes (16-byte aligned)
+ *   k_scale,
+ *   v_scale        uint8 [sum L_b, h_kv, d / 32] E8M0 codes (4-byte aligned)
+ *   k_idx8         uint8 [sum L_b, 1, d_idx]  E4M3 codes (16-byte aligned)
+ *   k_idx_scale    uint8 [sum L_b, 1, d_idx / 32]
+ *   topk_per_seq   as for msa_sparse_attn_decode_adaptive_k (NULL: topk)
+ * Other arguments, limits and the workspace as for msa_sparse_attn_decode.
+ */
+MSA_API int msa_sparse_attn_decode_mxfp8(const msa_params* p, const void* q, const void* q_idx, const void* k8,
+                                         const void* k_scale, const void* v8, const void* v_scale,
+                                         const void* k_idx8, const void* k_idx_scale, const int64_t* cu_kv,
+                                         const int32_t* topk_per_seq, int batch, int max_kv, int32_t* block_ids,
+                                         void* o, void* ws, size_t ws_bytes, void* stream);
+
 /* Human-readable text of a status code (static storage). */
 MSA_API const char* msa_status_string(int status);
 

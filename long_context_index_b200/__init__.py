@@ -15,7 +15,8 @@ from typing import Optional
 __all__ = ["MSAError", "Params", "lib", "workspace_size", "index_topk", "sparse_attn_prefill",
            "sparse_attn_decode", "index_topk_varlen", "sparse_attn_prefill_varlen", "device_status",
            "status_string", "OP_INDEX_TOPK", "OP_PREFILL", "OP_DECODE", "OP_INDEX_TOPK_VARLEN",
-           "OP_PREFILL_VARLEN", "OP_INDEX_PROJECT", "index_project", "quantize_mxfp8", "POOL_MAX", "POOL_MEAN"]
+           "OP_PREFILL_VARLEN", "OP_INDEX_PROJECT", "index_project", "quantize_mxfp8", "sparse_attn_decode_mxfp8", "POOL_MAX",
+           "POOL_MEAN"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmsa.so")
@@ -23,7 +24,7 @@ LIB_PATH = os.path.join(_HERE, "libmsa.so")
 OP_INDEX_TOPK, OP_PREFILL, OP_DECODE, OP_INDEX_TOPK_VARLEN, OP_PREFILL_VARLEN, OP_INDEX_PROJECT = 0, 1, 2, 3, 4, 5
 POOL_MAX, POOL_MEAN = 0, 1   # msa_params.pool
 
-SYMBOLS = ("msa_workspace_size", "msa_index_project", "msa_quantize_mxfp8", "msa_index_topk", "msa_sparse_attn_prefill", "msa_sparse_attn_decode",
+SYMBOLS = ("msa_workspace_size", "msa_index_project", "msa_quantize_mxfp8", "msa_sparse_attn_decode_mxfp8", "msa_index_topk", "msa_sparse_attn_prefill", "msa_sparse_attn_decode",
            "msa_index_topk_varlen", "msa_sparse_attn_prefill_varlen", "msa_sparse_attn_decode_adaptive_k",
            "msa_device_status", "msa_status_string",
            "msa_sparse_attn_decode_noalloc", "msa_test_never_ready_wait")
@@ -71,6 +72,9 @@ def lib():
                                                         vp, sz, vp]
         L.msa_quantize_mxfp8.argtypes = [vp, C.c_longlong, i32, vp, vp, vp]
         L.msa_quantize_mxfp8.restype = i32
+        L.msa_sparse_attn_decode_mxfp8.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, vp, vp,
+                                                   vp, sz, vp]
+        L.msa_sparse_attn_decode_mxfp8.restype = i32
         L.msa_index_project.argtypes = [P, vp, vp, i32, i32, vp, vp, vp, sz, vp]
         L.msa_index_topk_varlen.argtypes = [P, vp, vp, vp, i32, i32, vp, vp, vp, sz, vp]
         L.msa_sparse_attn_prefill_varlen.argtypes = [P, vp, vp, vp, vp, i32, i32, vp, vp, vp, sz, vp]
@@ -309,6 +313,39 @@ def sparse_attn_prefill_varlen(p: Params, q, k, v, cu_seqlens, block_ids, out=No
         raise MSAError(rc, "msa_sparse_attn_prefill_varlen")
     _after(ws, stream, "msa_sparse_attn_prefill_varlen")
     return out
+
+
+def sparse_attn_decode_mxfp8(p: Params, q, q_idx, k8, k_scale, v8, v_scale, k_idx8, k_idx_scale, cu_kv,
+                             max_kv: int, block_ids=None, out=None, ws=None, stream=None, topk_per_seq=None):
+    """One decode step over MXFP8 caches (uint8 codes and E8M0 scales from quantize_mxfp8):
+    (block_ids [B, h_kv, topk], O [B, h_q, d])."""
+    torch = _torch()
+    B = q.shape[0]
+    tot = k8.shape[0]
+    _check(q, "q", _bf16(), (B, p.h_q, p.d))
+    _check(q_idx, "q_idx", _bf16(), (B, p.h_kv, p.d_idx))
+    for name, t, shape in (("k8", k8, (tot, p.h_kv, p.d)), ("v8", v8, (tot, p.h_kv, p.d)),
+                           ("k_scale", k_scale, (tot, p.h_kv, p.d // 32)), ("v_scale", v_scale, (tot, p.h_kv, p.d // 32)),
+                           ("k_idx8", k_idx8, (tot, 1, p.d_idx)), ("k_idx_scale", k_idx_scale, (tot, 1, p.d_idx // 32))):
+        _check(t, name, (torch.uint8,), shape)
+    _check(cu_kv, "cu_kv", (torch.int64,), (B + 1,))
+    if topk_per_seq is not None:
+        _check(topk_per_seq, "topk_per_seq", (torch.int32,), (B,))
+    if block_ids is None:
+        block_ids = torch.empty((B, p.h_kv, p.topk), dtype=torch.int32, device=q.device)
+    _check(block_ids, "block_ids", (torch.int32,), (B, p.h_kv, p.topk))
+    if out is None:
+        out = torch.empty((B, p.h_q, p.d), dtype=torch.bfloat16, device=q.device)
+    _check(out, "out", _bf16(), (B, p.h_q, p.d))
+    ws = _workspace(OP_DECODE, p, batch=B, max_kv=max_kv, ws=ws, device=q.device)
+    rc = lib().msa_sparse_attn_decode_mxfp8(C.byref(p), _ptr(q), _ptr(q_idx), _ptr(k8), _ptr(k_scale), _ptr(v8),
+                                            _ptr(v_scale), _ptr(k_idx8), _ptr(k_idx_scale), _ptr(cu_kv),
+                                            _ptr(topk_per_seq), B, int(max_kv), _ptr(block_ids), _ptr(out),
+                                            _ptr(ws), ws.numel(), _stream(stream))
+    if rc:
+        raise MSAError(rc, "msa_sparse_attn_decode_mxfp8")
+    _after(ws, stream, "msa_sparse_attn_decode_mxfp8")
+    return block_ids, out
 
 
 def _after(ws, stream, what):

@@ -59,17 +59,20 @@ def dense_main_flops(n_q: int, n_kv: int, q_pos0: int, h_q: int, d: int, causal:
 
 
 def decode_bytes(lens: np.ndarray, ids: np.ndarray, h_q: int, h_kv: int, d: int, d_idx: int, block_k: int,
-                 dense: bool = False) -> int:
-    """Bytes one decode step must move (bf16 tensors, int32 ids)."""
+                 dense: bool = False, mxfp8: bool = False) -> int:
+    """Bytes one decode step must move (bf16 tensors, int32 ids).  With
+    ``mxfp8`` the caches hold one E4M3 byte per element plus one E8M0 byte per
+    32 elements."""
     lens = np.asarray(lens, dtype=np.int64)
     B = lens.size
+    per = (1.0 + 1.0 / 32) if mxfp8 else 2.0                   # cache bytes per element
     total = 0
     if not dense:
-        total += int(lens.sum()) * d_idx * 2                    # index-key cache, once for all groups
+        total += int(lens.sum() * d_idx * per)                  # index-key cache, once for all groups
         total += B * h_kv * d_idx * 2 + B * h_kv * ids.shape[2] * 4
         for b in range(B):
             sel = selected_keys(ids[b:b + 1], block_k, int(lens[b]), int(lens[b]) - 1)
-            total += sel * d * 2 * 2                             # K and V rows of the selected blocks
+            total += int(sel * d * per * 2)                      # K and V rows of the selected blocks
     else:
         total += int(lens.sum()) * h_kv * d * 2 * 2
     total += B * h_q * d * 2 * 2                                 # Q in, O out
