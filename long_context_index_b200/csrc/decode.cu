@@ -954,6 +954,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
       ++issued;
     }
     // Loads still in flight (only possible after an abort) land before exit.
+    if (F8) asm volatile("cp.async.wait_all;" ::: "memory");
     if (lane == 0) {
       WaitCtx drain{reinterpret_cast<volatile int*>(&flags[2]), a.status};
       for (int k = issued > C::kStages ? issued - C::kStages : 0; k < issued; ++k)
@@ -987,8 +988,9 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
       if (F8) {
         // Dequantise the stage's E4M3 K and V blocks into the bf16 tile pair
         // (the layout the bf16 path reads: 128B-swizzled rows of D/64 column
-        // halves).  The previous item's S and PV have finished with that
-        // pair, and the stage is released as soon as its bytes are converted.
+        // halves).  The previous item's S and PV have finished with that pair
+        // (every consumer warp is past the barrier); the stage itself, which
+        // still holds the Q tile, is released at the end of the item.
         sK = sbase + C::kOffDeq;
         sV = sK + C::kKBytes;
         named_bar(1, 32 * kStreamConsumers);
@@ -1011,8 +1013,6 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
                        : "memory");
         }
         named_bar(1, 32 * kStreamConsumers);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[stage]);
       }
 
       uint32_t qf[D / 16][4];
@@ -1127,11 +1127,9 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
           mma_bf16_16816(oacc[dt + 1], a0, a1, a2, a3, b2, b3);
         }
       }
-      if (!F8) {
-        if (zap) fence_proxy_async_smem();   // generic writes before the stage's next TMA fill
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[stage]);
-      }
+      if (!F8 && zap) fence_proxy_async_smem();   // generic writes before the stage's next TMA fill
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[stage]);
     }
 
     // End of this CTA's share of unit u: write it out.
