@@ -3,8 +3,10 @@
 // For every sequence b the query sits at position p = L_b - 1 of its own
 // contiguous caches.  The step is the prefill math of one row
 // (titansim.online summary of "MiniMax Sparse Attention": eq. (6) and the
-// local-block rule in section 4.2, eq. (8) in section 4.3), as two persistent
-// HBM-streaming launches:
+// local-block rule in section 4.2, eq. (8) in section 4.3), as one fused
+// cooperative launch (below) whenever the step fits one co-resident wave,
+// else as two persistent HBM-streaming launches.  Both forms run the same two
+// parts:
 //
 //   1. decode_index_kernel   The blocks of all sequences, end to end, are cut
 //      into equal ranges, one per CTA.  Streams the index-key cache once for
@@ -21,6 +23,11 @@
 //      TMA-loads the Q tile and the selected K/V block per item; four consumer
 //      warps run QK^T and PV on mma.sync with an fp32 online softmax.  A unit
 //      split between CTAs is merged by the last of them (LSE weights).
+// The fused form (decode_fused_kernel) runs 1 and 2 back to back in every CTA
+// of one cooperative grid; an attention CTA waits only until the ids of its
+// own sequences are published by the CTA that merged them.  With MXFP8 caches
+// (E4M3 + E8M0 per 32 elements) 1 dequantises the index keys in registers and
+// 2 dequantises each K/V block in shared memory before the same math.
 // The dense run (every causal block) skips the index scan and uses
 // decode_attn_kernel: split-KV CTAs staging K/V with cp.async, combined by
 // the last split of each (sequence, group, head tile).
@@ -159,11 +166,13 @@ template <int BK>
 __device__ void merge_topk_warp(const DecArgs& a, int b, int r, int lane, int* chosen, int c_lo, int nseg,
                                 long long T, int n);
 
+// The scan, as run by the persistent index kernel below and by the first
+// phase of the fused decode kernel: ismem is the dynamic shared memory; with
+// seq_ready non-null, the CTA that merges a sequence publishes its ids there.
 template <int DIDX, int BK, int POOL, bool F8>
-__global__ void __launch_bounds__(kIdxThreads, kIdxCtasPerSm) decode_index_kernel(const DecArgs a) {
+__device__ __forceinline__ void decode_index_body(const DecArgs& a, uint8_t* ismem, int* seq_ready) {
   constexpr int kHalves = DIDX / 32;   // 16-byte vectors per token row per thread
   constexpr int kWarps = kIdxThreads / 32;
-  extern __shared__ __align__(16) uint8_t ismem[];
   const int B = a.batch;
   const int wmax = a.idx_wmax;
   int* pfx = reinterpret_cast<int*>(ismem);                                       // [B + 1]
@@ -373,6 +382,18 @@ __global__ void __launch_bounds__(kIdxThreads, kIdxCtasPerSm) decode_index_kerne
     const int c_lo = idx_cta_of(pfx[sb], T, n), c_hi = idx_cta_of(pfx[sb + 1] - 1, T, n);
     merge_topk_warp<BK>(a, sb, r, lane, chosen[warp], c_lo, c_hi - c_lo + 1, T, n);
   }
+  if (seq_ready) {
+    // Every group of the merged sequences is written: publish them.
+    __threadfence();
+    __syncthreads();
+    for (int i = threadIdx.x; i < n_last; i += kIdxThreads) atomicExch(&seq_ready[lastq[i]], 1);
+  }
+}
+
+template <int DIDX, int BK, int POOL, bool F8>
+__global__ void __launch_bounds__(kIdxThreads, kIdxCtasPerSm) decode_index_kernel(const DecArgs a) {
+  extern __shared__ __align__(16) uint8_t ismem[];
+  decode_index_body<DIDX, BK, POOL, F8>(a, ismem, nullptr);
 }
 
 // ---------------------------------------------------------------------------
@@ -825,17 +846,20 @@ __device__ __forceinline__ int cta_of_item(long long g, long long T, int n) {
   return static_cast<int>(((g + 1) * n - 1) / T);
 }
 
+// The attention, as run by the streaming kernel below and by the second
+// phase of the fused decode kernel (smem_raw: the dynamic shared memory;
+// seq_ready non-null: wait until the ids of this CTA's sequences are out).
+// Warps past the producer take no part.
 template <int D, int BK, bool F8>
-__global__ void __launch_bounds__(kStreamThreads, 1)
-    decode_attn_stream_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                              const __grid_constant__ CUtensorMap tm_v, const StreamArgs a) {
+__device__ __forceinline__ void decode_attn_body(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
+                                                 const CUtensorMap* tm_v, const StreamArgs& a, uint8_t* smem_raw,
+                                                 const int* seq_ready) {
   using C = StreamCfg<D, BK, F8>;
   constexpr int KPW = BK / kStreamConsumers;   // S keys per warp
   constexpr int NT = KPW / 8;
   constexpr int NCOL = D / kStreamConsumers;   // O columns per warp
   constexpr int NTO = NCOL / 8;
   constexpr int PST = D + 4;                   // partial row stride (floats)
-  extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* red_m = reinterpret_cast<float*>(smem + C::kOffRed);
   float* red_l = red_m + kStreamConsumers * 16;
@@ -854,15 +878,34 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
   const int n_items = static_cast<int>(g1 - g0);
   const int upb = a.h_kv * a.head_tiles;   // units per sequence
 
+  if (seq_ready) {
+    // Fused step: the ids of this CTA's sequences come from the index phase
+    // of (possibly) other CTAs; wait, bounded, for each to be published.
+    if (tid == 0 && n_items > 0) {
+      const int b_lo = static_cast<int>((g0 / a.topk) / upb), b_hi = static_cast<int>(((g1 - 1) / a.topk) / upb);
+      const unsigned long long t0 = globaltimer();
+      for (int b = b_lo; b <= b_hi; ++b) {
+        while (atomicAdd(const_cast<int*>(&seq_ready[b]), 0) == 0) {
+          if (globaltimer() - t0 > kWaitNs) {
+            if (a.status) atomicExch(a.status, kDevTimeout);
+            break;
+          }
+          __nanosleep(256);
+        }
+      }
+      __threadfence();
+    }
+    __syncthreads();
+  }
   // Block ids of this CTA's items, -1 where the slot is padding or out of range.
-  for (int i = tid; i < n_items; i += kStreamThreads) {
+  for (int i = tid; i < n_items; i += blockDim.x) {
     const long long g = g0 + i;
     const long long u = g / a.topk;
     const int slot = static_cast<int>(g - u * a.topk);
     const int b = static_cast<int>(u / upb), r = static_cast<int>(u % upb) / a.head_tiles;
     const int L = static_cast<int>(a.cu_kv[b + 1] - a.cu_kv[b]);
     const int nb = (L + BK - 1) / BK;
-    const int blk = a.block_ids[(static_cast<size_t>(b) * a.h_kv + r) * a.topk + slot];
+    const int blk = __ldcg(a.block_ids + (static_cast<size_t>(b) * a.h_kv + r) * a.topk + slot);
     s_ids[i] = (blk >= 0 && blk < nb) ? blk : -1;
   }
   if (tid == 0) {
@@ -879,6 +922,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
   }
   __syncthreads();
   WaitCtx wc{reinterpret_cast<volatile int*>(&flags[0]), a.status};
+  if (warp > kStreamConsumers) return;
 
   if (warp == kStreamConsumers) {
     // ---------------- producer ----------------
@@ -887,9 +931,9 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
     // the stage (a second arrival on its full barrier).
     if (!F8 && lane != 0) return;
     if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(tm_q);
+      tma_prefetch_desc(tm_k);
+      tma_prefetch_desc(tm_v);
     }
     long long cur_u = -1;
     long long off = 0;
@@ -924,16 +968,16 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
         if (F8) {
           mbar_arrive_expect_tx(&full[stage], C::kQBytes + 2 * C::kK8Bytes);
 #pragma unroll
-          for (int h = 0; h < C::kHalves; ++h) tma_load_2d(st + h * 16 * 128, &tm_q, &full[stage], h * 64, qrow);
-          tma_load_3d(st + C::kQBytes, &tm_k, &full[stage], 0, r, krow);
-          tma_load_3d(st + C::kQBytes + C::kK8Bytes, &tm_v, &full[stage], 0, r, krow);
+          for (int h = 0; h < C::kHalves; ++h) tma_load_2d(st + h * 16 * 128, tm_q, &full[stage], h * 64, qrow);
+          tma_load_3d(st + C::kQBytes, tm_k, &full[stage], 0, r, krow);
+          tma_load_3d(st + C::kQBytes + C::kK8Bytes, tm_v, &full[stage], 0, r, krow);
         } else {
           mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
 #pragma unroll
           for (int h = 0; h < C::kHalves; ++h) {
-            tma_load_2d(st + h * 16 * 128, &tm_q, &full[stage], h * 64, qrow);
-            tma_load_3d(st + C::kQBytes + h * BK * 128, &tm_k, &full[stage], h * 64, r, krow);
-            tma_load_3d(st + C::kQBytes + C::kKBytes + h * BK * 128, &tm_v, &full[stage], h * 64, r, krow);
+            tma_load_2d(st + h * 16 * 128, tm_q, &full[stage], h * 64, qrow);
+            tma_load_3d(st + C::kQBytes + h * BK * 128, tm_k, &full[stage], h * 64, r, krow);
+            tma_load_3d(st + C::kQBytes + C::kKBytes + h * BK * 128, tm_v, &full[stage], h * 64, r, krow);
           }
         }
       }
@@ -1221,6 +1265,37 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
   }
 }
 
+template <int D, int BK, bool F8>
+__global__ void __launch_bounds__(kStreamThreads, 1)
+    decode_attn_stream_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                              const __grid_constant__ CUtensorMap tm_v, const StreamArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  decode_attn_body<D, BK, F8>(&tm_q, &tm_k, &tm_v, a, smem_raw, nullptr);
+}
+
+// ---------------------------------------------------------------------------
+// 4. fused decode step: one cooperative persistent launch, one CTA per SM.
+//    Phase 1 is the index scan above over this grid (the CTA that completes
+//    a sequence merges its top-k and publishes it in seq_ready); phase 2 is
+//    the streaming attention above, whose CTAs wait (bounded) until the ids
+//    of their own sequences are published -- CTAs whose sequences finish
+//    early start attending while others still scan, and the ids never leave
+//    the L2 between the two.  All CTAs are co-resident (cooperative launch),
+//    and a publishing CTA never waits on anyone, so every wait ends.
+// ---------------------------------------------------------------------------
+constexpr int kFusedThreads = kIdxThreads;   // the scan's 8 warps; the attention uses 5 of them
+
+template <int DIDX, int BK, int POOL, int D, bool F8>
+__global__ void __launch_bounds__(kFusedThreads, 1)
+    decode_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const DecArgs a, const StreamArgs sa,
+                        int* seq_ready) {
+  extern __shared__ __align__(1024) uint8_t fsmem[];
+  decode_index_body<DIDX, BK, POOL, F8>(a, fsmem, seq_ready);
+  __syncthreads();   // the scan's shared memory is reused by the attention
+  decode_attn_body<D, BK, F8>(&tm_q, &tm_k, &tm_v, sa, fsmem, seq_ready);
+}
+
 // Split plan of the dense run, shared by the workspace query and the launch.
 struct SplitPlan {
   int splits, slots_per_split;
@@ -1275,10 +1350,10 @@ int stream_ctas(long long T) {
   return static_cast<int>(n < T ? n : T);
 }
 
+// Tensor maps and arguments of the streaming attention over n_cta CTAs.
 template <int D, int BK, bool F8>
-int launch_attn_stream(const DecArgs& a, int max_kv, int* status, cudaStream_t st) {
-  using C = StreamCfg<D, BK, F8>;
-  CUtensorMap tq, tk, tv;
+int stream_setup(const DecArgs& a, int max_kv, int* status, CUtensorMap& tq, CUtensorMap& tk, CUtensorMap& tv,
+                 StreamArgs& s) {
   {
     const uint64_t dims[2] = {static_cast<uint64_t>(D), static_cast<uint64_t>(a.batch) * a.h_q};
     const uint64_t strides[1] = {static_cast<uint64_t>(D) * 2};
@@ -1301,7 +1376,6 @@ int launch_attn_stream(const DecArgs& a, int max_kv, int* status, cudaStream_t s
       if (!encode_tma_bf16(&tv, 3, a.v_cache, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MSA_ERR_CUDA;
     }
   }
-  StreamArgs s;
   s.block_ids = a.block_ids;
   s.cu_kv = a.cu_kv;
   s.o = a.o;
@@ -1318,12 +1392,81 @@ int launch_attn_stream(const DecArgs& a, int max_kv, int* status, cudaStream_t s
   s.scale_log2 = a.scale_log2;
   s.k_sc = a.k_sc;
   s.v_sc = a.v_sc;
+  return MSA_OK;
+}
+
+template <int D, int BK, bool F8>
+int launch_attn_stream(const DecArgs& a, int max_kv, int* status, cudaStream_t st) {
+  using C = StreamCfg<D, BK, F8>;
+  CUtensorMap tq, tk, tv;
+  StreamArgs s;
+  int rc = stream_setup<D, BK, F8>(a, max_kv, status, tq, tk, tv, s);
+  if (rc) return rc;
   const int smem = C::kSmemBytes + 1024;
   auto kern = decode_attn_stream_kernel<D, BK, F8>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return MSA_ERR_CUDA;
   kern<<<s.n_cta, kStreamThreads, smem, st>>>(tq, tk, tv, s);
   return cudaGetLastError() == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
+}
+
+// The fused step (decode_fused_kernel), when the whole step fits one
+// co-resident wave: every attention CTA holds its items' ids in shared memory
+// (kStreamIdsCap) and every scan CTA its blocks' maxima (kIdxWCap).
+// Returns kNotFused (positive) to ask for the two-launch step instead.
+constexpr int kNotFused = 1;
+
+template <int DIDX, int BK, int D, bool F8>
+int launch_fused(DecArgs a, int max_kv, int* status, int* seq_ready, cudaStream_t st) {
+  using C = StreamCfg<D, BK, F8>;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                cudaSuccess)
+    return MSA_ERR_CUDA;
+  const int grid = sms;
+  CUtensorMap tq, tk, tv;
+  StreamArgs sa;
+  int rc = stream_setup<D, BK, F8>(a, max_kv, status, tq, tk, tv, sa);
+  if (rc) return rc;
+  if (stream_ctas(sa.total_items) > grid) return kNotFused;
+  sa.n_cta = grid;
+  const long long tmax = static_cast<long long>(a.batch) * ((max_kv + BK - 1) / BK);
+  const long long wmax = (tmax + grid - 1) / grid;
+  if (wmax > kIdxWCap) return kNotFused;
+  const size_t idx_smem = align_up(static_cast<size_t>(a.batch + 1) * 4, 16) + static_cast<size_t>(a.h_kv) * wmax * 4 +
+                          static_cast<size_t>(wmax + 1) * 4;
+  if (idx_smem > static_cast<size_t>(C::kSmemBytes)) return kNotFused;
+  a.idx_ctas = grid;
+  a.idx_wmax = static_cast<int>(wmax < 1 ? 1 : wmax);
+  const int smem = C::kSmemBytes + 1024;
+  auto kern = a.pool ? decode_fused_kernel<DIDX, BK, 1, D, F8> : decode_fused_kernel<DIDX, BK, 0, D, F8>;
+  // The scan's static shared memory comes on top of the attention's ring.
+  cudaFuncAttributes fa;
+  int smem_max = 0;
+  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess ||
+      cudaDeviceGetAttribute(&smem_max, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+    return MSA_ERR_CUDA;
+  if (fa.sharedSizeBytes + smem > static_cast<size_t>(smem_max)) return kNotFused;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return MSA_ERR_CUDA;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kFusedThreads, smem) != cudaSuccess || per_sm < 1)
+    return kNotFused;
+  void* args[] = {&tq, &tk, &tv, &a, &sa, &seq_ready};
+  const cudaError_t e =
+      cudaLaunchCooperativeKernel(reinterpret_cast<void*>(kern), grid, kFusedThreads, args, smem, st);
+  if (e == cudaErrorCooperativeLaunchTooLarge) {   // not every CTA can be resident (a shared GPU): two launches
+    cudaGetLastError();
+    return kNotFused;
+  }
+  return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
+}
+
+template <int DIDX, int BK>
+int launch_fused_d(const DecArgs& a, int d, int max_kv, int* status, int* seq_ready, cudaStream_t st) {
+  if (a.k8) return launch_fused<DIDX, BK, 128, true>(a, max_kv, status, seq_ready, st);
+  return d == 64 ? launch_fused<DIDX, BK, 64, false>(a, max_kv, status, seq_ready, st)
+                 : launch_fused<DIDX, BK, 128, false>(a, max_kv, status, seq_ready, st);
 }
 
 template <int DIDX, int BK>
@@ -1343,11 +1486,12 @@ int launch_index(const DecArgs& a, size_t smem, cudaStream_t st) {
 
 }  // namespace
 
-// Completion counters at the front of the decode workspace: [B] index CTAs
-// per sequence, then [B, h_kv, head_tiles] attention CTAs.  The caller zeroes
-// them (with the status word) before every call.
+// Completion counters at the front of the decode workspace.  The caller
+// zeroes them (with the status word) before every call.
 size_t decode_counter_bytes(const msa_params& p, int batch) {
-  const size_t n = static_cast<size_t>(batch) * (1 + p.h_kv * ((p.h_q / p.h_kv + 15) / 16));
+  // [B] index CTAs per sequence, [B, h_kv, head_tiles] attention CTAs per
+  // unit, [B] sequence-ready flags of the fused step.
+  const size_t n = static_cast<size_t>(batch) * (2 + p.h_kv * ((p.h_q / p.h_kv + 15) / 16));
   return align_up(n * 4, 256);
 }
 
@@ -1422,6 +1566,21 @@ int run_sparse_attn_decode(const msa_params& p, const void* q, const void* q_idx
   a.part = reinterpret_cast<float*>(w + 2 * align_up(cand * 4, 256));
 
   int rc = MSA_OK;
+  if (!dense && a.kfree > 0) {
+    // One fused launch when the step fits one co-resident wave.
+    int* seq_ready = a.grp_count + static_cast<size_t>(batch) * p.h_kv * a.head_tiles;
+    if (p.block_k == 64) {
+      rc = p.d_idx == 32 ? launch_fused_d<32, 64>(a, p.d, max_kv, status, seq_ready, stream)
+                         : (p.d_idx == 64 ? launch_fused_d<64, 64>(a, p.d, max_kv, status, seq_ready, stream)
+                                          : launch_fused_d<128, 64>(a, p.d, max_kv, status, seq_ready, stream));
+    } else {
+      rc = p.d_idx == 32 ? launch_fused_d<32, 128>(a, p.d, max_kv, status, seq_ready, stream)
+                         : (p.d_idx == 64 ? launch_fused_d<64, 128>(a, p.d, max_kv, status, seq_ready, stream)
+                                          : launch_fused_d<128, 128>(a, p.d, max_kv, status, seq_ready, stream));
+    }
+    if (rc != kNotFused) return rc;
+    rc = MSA_OK;
+  }
   if (!dense) {
     if (p.block_k == 64) {
       rc = p.d_idx == 32 ? launch_index<32, 64>(a, ip.smem, stream)
