@@ -24,7 +24,11 @@
  *   * Head h of the main branch belongs to group r = h / (h_q / h_kv).
  *   * Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *     default stream).  They are stateless: concurrent calls on different
- *     streams with different workspaces are safe.
+ *     streams with different workspaces are safe.  A sparse prefill of more
+ *     than 4096 query rows forks part of its work onto one auxiliary stream
+ *     per device (created by the library on first use) and joins it back into
+ *     `stream` before returning, so its completion is still ordered on
+ *     `stream` (and the fork/join is captured by CUDA graph capture).
  *   * Return value: MSA_OK, or a negative MSA_ERR_* code.  Argument errors are
  *     detected on the host before anything is launched.  Kernels bound every
  *     wait instead of hanging; a wait that gave up is recorded in the status
@@ -148,11 +152,13 @@ MSA_API int msa_sparse_attn_prefill(const msa_params* p, const void* q, const vo
 /*
  * One batched decode step: for every sequence b the query at position
  * L_b - 1 runs the index branch over its whole index-key cache, then the main
- * branch over the selected blocks.  Both sparse kernels are persistent: the
- * index scan splits the blocks of all sequences into equal ranges per CTA,
- * the attention splits the (sequence, group, slot) list the same way, and
- * partial results of a sequence or group split between CTAs are merged by the
- * last CTA to finish it.
+ * branch over the selected blocks.  The sparse step is persistent: the index
+ * scan splits the blocks of all sequences into equal ranges per CTA, the
+ * attention splits the (sequence, group, slot) list the same way, and partial
+ * results of a sequence or group split between CTAs are merged by the last
+ * CTA to finish it.  When the step fits one co-resident wave of CTAs it runs
+ * as one cooperative launch whose attention CTAs start as soon as the ids of
+ * their own sequences are merged; otherwise as two launches.
  *   q            bf16 [batch, h_q, d]
  *   q_idx        bf16 [batch, h_kv, d_idx]
  *   k_cache,

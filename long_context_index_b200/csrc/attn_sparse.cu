@@ -48,6 +48,7 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <mutex>
 
 #include "msa_internal.h"
 #include "ptx.cuh"
@@ -71,6 +72,7 @@ constexpr int kCtrlBytes = 20480;   // descriptors, softmax stats, staged entrie
 constexpr int kSchedThreads = 256;
 constexpr int kStageEntries = 256;   // list entries staged in shared memory at a time
 constexpr int kWave = 4096;          // query rows per wave (L2-resident Q working set)
+constexpr int kMergeSms = 16;        // SMs the block-major launches leave to the previous wave's merge
 
 template <int D, int BK>
 struct KvoCfg {
@@ -105,8 +107,8 @@ struct KvoArgs {
   const int* chunk_off;  // [n_waves * h_kv * nb] first global chunk id of each list
   const int* entries;    // (query << 5) | slot, grouped by list
   const int* lists;      // non-empty list ids ((wave * h_kv + r) * nb + b)
-  const int* n_lists;
-  int* work_counter;
+  const int* wave_lo;    // this launch's lists: [wave_lo[0], wave_lo[1]) of `lists`
+  int* work_counter;     // this launch's list counter
   float* part_lse;       // [chunks * 128] lse2 of each partial row
   int* status;
   int n_q, n_kv, q_pos0, h_q, h_kv, topk, causal, nb;
@@ -204,7 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const WaitCtx wc{abort_flag, args.status};
-  const int n_lists = *args.n_lists;
+  const int list_lo = args.wave_lo[0], list_hi = args.wave_lo[1];
   // Gathered Q rows are re-read by up to k lists of their wave: keep them in
   // L2; partial tiles are read once, much later: let them leave first.
   const uint64_t q_policy = l2_evict_last();
@@ -225,9 +227,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     while (ok) {
       int li = 0;
-      if (lane == 0) li = atomicAdd(args.work_counter, 1);
+      if (lane == 0) li = list_lo + atomicAdd(args.work_counter, 1);
       li = __shfl_sync(0xffffffffu, li, 0);
-      if (li >= n_lists) break;
+      if (li >= list_hi) break;
       const int rb = args.lists[li];
       const int r = (rb / args.nb) % args.h_kv, gb = rb % args.nb;
       // The block's sequence: its key rows start at seq_row0 + b * BK.
@@ -706,6 +708,22 @@ __global__ void __launch_bounds__(1024) sched_scan_kernel(const int* cnt, int n,
   }
 }
 
+// Start of each query wave's lists in the compacted (ascending) list array:
+// wave_lo[w] = the first position whose list id is in wave w or later.
+__global__ void sched_waves_kernel(const int* lists, const int* n_lists, int n_waves, int lists_per_wave,
+                                   int* wave_lo) {
+  const int w = blockIdx.x * blockDim.x + threadIdx.x;
+  if (w > n_waves) return;
+  const int n = *n_lists;
+  const long long key = static_cast<long long>(w) * lists_per_wave;
+  int lo = 0, hi = n;   // first position with lists[pos] >= key
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (lists[mid] < key) lo = mid + 1; else hi = mid;
+  }
+  wave_lo[w] = lo;
+}
+
 __global__ void sched_fill_kernel(const int32_t* ids, long long total, int h_kv, int topk, int nb, int G,
                                   SchedGeom geo, const int* offs, const int* chunk_off, int* fill, int* entries,
                                   int* prow_of) {
@@ -732,14 +750,14 @@ __global__ void sched_fill_kernel(const int32_t* ids, long long total, int h_kv,
 template <int D>
 __global__ void __launch_bounds__(256) merge_partials_kernel(const int* prow_of, const uint16_t* part_o,
                                                              const float* part_lse, uint16_t* o, int h_q, int h_kv,
-                                                             int topk) {
+                                                             int topk, int q0) {
   // One CTA per (query, group); thread = (head within group, 8-column chunk).
   // prow_of[(q, r, slot)] is the first partial row (chunk * 128 + query-in-
   // chunk * G) the block-major kernel wrote for that selection, -1 for none.
   // Slots are read 8 at a time with independent loads and folded in with an
   // online log-sum-exp, so the loads of a group are all in flight together.
   constexpr int kGrp = 8;
-  const int qr = blockIdx.x;
+  const int qr = q0 * h_kv + static_cast<int>(blockIdx.x);   // this launch: queries from q0
   const int q = qr / h_kv, r = qr % h_kv;
   const int G = h_q / h_kv;
   constexpr int kChunks = D / 8;
@@ -816,7 +834,7 @@ cudaError_t launch_kvo_g(int G, const CUtensorMap* m, const KvoArgs& a, int grid
 }
 
 struct SparseWs {
-  int *cnt, *fill, *offs, *chunk_off, *lists, *n_lists, *work, *entries, *prow_of;
+  int *cnt, *fill, *offs, *chunk_off, *lists, *n_lists, *work, *entries, *prow_of, *wave_lo;
   uint16_t* part_o;
   float* part_lse;
   size_t max_chunks, bytes;
@@ -843,11 +861,13 @@ SparseWs carve(const msa_params& p, int n_q, int n_kv, int batch, void* base) {
     off += align_up(bytes, 256);
     return ptr;
   };
-  // cnt, fill, work counter are contiguous so one memset clears them.
-  s.cnt = reinterpret_cast<int*>(take((2 * nl + 2) * 4));
+  // cnt, fill, the list count and the per-wave work counters are contiguous
+  // so one memset clears them.
+  s.cnt = reinterpret_cast<int*>(take((2 * nl + 1 + n_waves) * 4));
   s.fill = s.cnt ? s.cnt + nl : nullptr;
-  s.work = s.cnt ? s.cnt + 2 * nl : nullptr;
-  s.n_lists = s.cnt ? s.cnt + 2 * nl + 1 : nullptr;
+  s.n_lists = s.cnt ? s.cnt + 2 * nl : nullptr;
+  s.work = s.cnt ? s.cnt + 2 * nl + 1 : nullptr;
+  s.wave_lo = reinterpret_cast<int*>(take((n_waves + 1) * 4));
   s.offs = reinterpret_cast<int*>(take((nl + 1) * 4));
   s.chunk_off = reinterpret_cast<int*>(take(nl * 4));
   s.lists = reinterpret_cast<int*>(take(nl * 4));
@@ -859,6 +879,27 @@ SparseWs carve(const msa_params& p, int n_q, int n_kv, int batch, void* base) {
   s.part_o = reinterpret_cast<uint16_t*>(take(s.max_chunks * 128 * static_cast<size_t>(p.d) * 2));
   s.bytes = off;
   return s;
+}
+
+// One auxiliary stream and event per device for the wave pipeline (created
+// on first use, kept for the life of the process).  Callers hold g_aux_mu
+// while they enqueue on them: the event is re-recorded per wave, and calls
+// from several host threads must not interleave their records and waits.
+constexpr int kMaxDev = 64;
+std::mutex g_aux_mu;
+cudaStream_t g_aux[kMaxDev] = {};
+cudaEvent_t g_aux_ev[kMaxDev] = {};
+
+int aux_stream(cudaStream_t* st, cudaEvent_t* ev) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return MSA_ERR_CUDA;
+  if (!g_aux[dev]) {
+    if (cudaStreamCreateWithFlags(&g_aux[dev], cudaStreamNonBlocking) != cudaSuccess) return MSA_ERR_CUDA;
+    if (cudaEventCreateWithFlags(&g_aux_ev[dev], cudaEventDisableTiming) != cudaSuccess) return MSA_ERR_CUDA;
+  }
+  *st = g_aux[dev];
+  *ev = g_aux_ev[dev];
+  return MSA_OK;
 }
 
 }  // namespace
@@ -891,12 +932,16 @@ int run_sparse_attn_kvouter(const msa_params& p, const void* q, const CUtensorMa
   geo.nb_one = (n_kv + p.block_k - 1) / p.block_k;
   geo.bk = p.block_k;
   geo.nb = nb;
-  if (cudaMemsetAsync(s.cnt, 0, (2 * static_cast<size_t>(nl) + 2) * 4, stream) != cudaSuccess) return MSA_ERR_CUDA;
+  const int n_waves = (n_q + kWave - 1) / kWave;
+  if (cudaMemsetAsync(s.cnt, 0, (2 * static_cast<size_t>(nl) + 1 + n_waves) * 4, stream) != cudaSuccess)
+    return MSA_ERR_CUDA;
   const int gsz = static_cast<int>((total + kSchedThreads - 1) / kSchedThreads);
   sched_count_kernel<<<gsz, kSchedThreads, 0, stream>>>(block_ids, total, p.h_kv, p.topk, nb, geo, s.cnt);
   sched_scan_kernel<<<1, 1024, 0, stream>>>(s.cnt, nl, 128 / G, s.offs, s.chunk_off, s.lists, s.n_lists);
   sched_fill_kernel<<<gsz, kSchedThreads, 0, stream>>>(block_ids, total, p.h_kv, p.topk, nb, G, geo, s.offs,
                                                        s.chunk_off, s.fill, s.entries, s.prow_of);
+  sched_waves_kernel<<<(n_waves + 1 + 255) / 256, 256, 0, stream>>>(s.lists, s.n_lists, n_waves, p.h_kv * nb,
+                                                                    s.wave_lo);
   if (cudaGetLastError() != cudaSuccess) return MSA_ERR_CUDA;
 
   KvoArgs a;
@@ -904,8 +949,6 @@ int run_sparse_attn_kvouter(const msa_params& p, const void* q, const CUtensorMa
   a.chunk_off = s.chunk_off;
   a.entries = s.entries;
   a.lists = s.lists;
-  a.n_lists = s.n_lists;
-  a.work_counter = s.work;
   a.part_lse = s.part_lse;
   a.status = status;
   a.n_q = n_q;
@@ -924,7 +967,6 @@ int run_sparse_attn_kvouter(const msa_params& p, const void* q, const CUtensorMa
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int grid = sms;
   CUtensorMap maps[4] = {tq, tk, tv, tq};
   {  // chunk-major partial rows [max_chunks * 128][d]: one box = 128 rows x 64 columns
     const uint64_t dims[2] = {static_cast<uint64_t>(p.d), static_cast<uint64_t>(s.max_chunks) * 128};
@@ -932,22 +974,53 @@ int run_sparse_attn_kvouter(const msa_params& p, const void* q, const CUtensorMa
     const uint32_t box[2] = {64, 128};
     if (!encode_tma_bf16(&maps[3], 2, s.part_o, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MSA_ERR_CUDA;
   }
-  cudaError_t e;
-  if (p.d == 64) {
-    e = p.block_k == 64 ? launch_kvo_g<64, 64>(G, maps, a, grid, stream)
-                        : launch_kvo_g<64, 128>(G, maps, a, grid, stream);
-  } else {
-    e = p.block_k == 64 ? launch_kvo_g<128, 64>(G, maps, a, grid, stream)
-                        : launch_kvo_g<128, 128>(G, maps, a, grid, stream);
+  auto launch_attn = [&](int w, int grid) -> cudaError_t {
+    a.wave_lo = s.wave_lo + w;
+    a.work_counter = s.work + w;
+    if (p.d == 64)
+      return p.block_k == 64 ? launch_kvo_g<64, 64>(G, maps, a, grid, stream)
+                             : launch_kvo_g<64, 128>(G, maps, a, grid, stream);
+    return p.block_k == 64 ? launch_kvo_g<128, 64>(G, maps, a, grid, stream)
+                           : launch_kvo_g<128, 128>(G, maps, a, grid, stream);
+  };
+  auto launch_merge = [&](int w, cudaStream_t st) {
+    const int q0 = w * kWave, rows = (w + 1 == n_waves ? n_q : q0 + kWave) - q0;
+    if (p.d == 64)
+      merge_partials_kernel<64><<<rows * p.h_kv, 256, 0, st>>>(s.prow_of, s.part_o, s.part_lse,
+                                                               static_cast<uint16_t*>(o), p.h_q, p.h_kv, p.topk, q0);
+    else
+      merge_partials_kernel<128><<<rows * p.h_kv, 256, 0, st>>>(s.prow_of, s.part_o, s.part_lse,
+                                                                static_cast<uint16_t*>(o), p.h_q, p.h_kv, p.topk, q0);
+  };
+  cudaStream_t aux = nullptr;
+  cudaEvent_t ev = nullptr;
+  std::unique_lock<std::mutex> lock(g_aux_mu, std::defer_lock);
+  if (n_waves > 1) {
+    lock.lock();
+    if (aux_stream(&aux, &ev) != MSA_OK) return MSA_ERR_CUDA;
   }
-  if (e != cudaSuccess) return MSA_ERR_CUDA;
-  const int mgrid = n_q * p.h_kv;
-  if (p.d == 64)
-    merge_partials_kernel<64><<<mgrid, 256, 0, stream>>>(s.prow_of, s.part_o, s.part_lse, static_cast<uint16_t*>(o),
-                                                          p.h_q, p.h_kv, p.topk);
-  else
-    merge_partials_kernel<128><<<mgrid, 256, 0, stream>>>(s.prow_of, s.part_o, s.part_lse, static_cast<uint16_t*>(o),
-                                                           p.h_q, p.h_kv, p.topk);
+  if (n_waves == 1 || !aux) {
+    // One wave: the block-major kernel on every SM, then the merge.
+    for (int w = 0; w < n_waves; ++w) {
+      if (launch_attn(w, sms) != cudaSuccess) return MSA_ERR_CUDA;
+      launch_merge(w, stream);
+    }
+  } else {
+    // Wave pipeline: wave w's block-major launch leaves kMergeSms SMs free,
+    // and its merge runs on the auxiliary stream under wave w + 1's launch,
+    // so the partials' HBM round trip overlaps the tensor-core work.  The
+    // auxiliary stream forks from and joins back into the caller's stream.
+    if (cudaEventRecord(ev, stream) != cudaSuccess || cudaStreamWaitEvent(aux, ev, 0) != cudaSuccess)
+      return MSA_ERR_CUDA;
+    for (int w = 0; w < n_waves; ++w) {
+      if (launch_attn(w, sms - kMergeSms) != cudaSuccess) return MSA_ERR_CUDA;
+      if (cudaEventRecord(ev, stream) != cudaSuccess || cudaStreamWaitEvent(aux, ev, 0) != cudaSuccess)
+        return MSA_ERR_CUDA;
+      launch_merge(w, aux);
+    }
+    if (cudaEventRecord(ev, aux) != cudaSuccess || cudaStreamWaitEvent(stream, ev, 0) != cudaSuccess)
+      return MSA_ERR_CUDA;
+  }
   return cudaGetLastError() == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
 }
 
