@@ -874,7 +874,11 @@ __device__ __forceinline__ void decode_attn_body(const CUtensorMap* tm_q, const 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const long long T = a.total_items;
   const int cta = blockIdx.x;
-  const long long g0 = cta * T / a.n_cta, g1 = (cta + 1) * T / a.n_cta;
+  // CTAs past n_cta (the fused grid is one CTA per SM, n_cta <= T) hold no
+  // items: every CTA inside a unit's span then holds at least one of its
+  // items, which the last-arriver count of a split unit relies on.
+  const long long g0 = cta < a.n_cta ? cta * T / a.n_cta : T;
+  const long long g1 = cta < a.n_cta ? (cta + 1) * T / a.n_cta : T;
   const int n_items = static_cast<int>(g1 - g0);
   const int upb = a.h_kv * a.head_tiles;   // units per sequence
 
@@ -1428,8 +1432,7 @@ int launch_fused(DecArgs a, int max_kv, int* status, int* seq_ready, cudaStream_
   StreamArgs sa;
   int rc = stream_setup<D, BK, F8>(a, max_kv, status, tq, tk, tv, sa);
   if (rc) return rc;
-  if (stream_ctas(sa.total_items) > grid) return kNotFused;
-  sa.n_cta = grid;
+  if (sa.n_cta > grid) return kNotFused;   // stream_ctas: at most one CTA per item
   const long long tmax = static_cast<long long>(a.batch) * ((max_kv + BK - 1) / BK);
   const long long wmax = (tmax + grid - 1) / grid;
   if (wmax > kIdxWCap) return kNotFused;
