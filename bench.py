@@ -206,6 +206,8 @@ def run_ours(args, rank, world, torch, dist):
     ws_d = torch.empty(msa.workspace_size(msa.OP_DECODE, pd, batch=B, max_kv=max_kv), dtype=torch.uint8,
                        device=dev)
 
+    decode_form = msa.get_option(msa.OPT_DECODE_FUSED)   # the library's default form
+
     def step():
         msa.index_topk(pp, d_in["q_idx"], d_in["k_idx"], q_pos0, block_ids=ids, ws=ws_i)
         ev[1].record(stream)
@@ -289,9 +291,49 @@ def run_ours(args, rank, world, torch, dist):
             rc = msa.device_status(wsx)
             if rc:
                 raise RuntimeError("device status %d after the dense runs" % rc)
+    def median_ms(fn):
+        """fn warmed up, then the median of as many timed calls as the step."""
+        for _ in range(args.warmup):
+            fn()
+        evp = [(E(enable_timing=True), E(enable_timing=True)) for _ in range(args.steps)]
+        for a_, b_ in evp:
+            a_.record(stream)
+            fn()
+            b_.record(stream)
+        torch.cuda.synchronize()
+        return statistics.median(a_.elapsed_time(b_) for a_, b_ in evp)
+
+    def fused_form(fn):
+        """fn timed with the decode step in its one-launch form."""
+        msa.set_option(msa.OPT_DECODE_FUSED, 1)
+        try:
+            return median_ms(fn)
+        finally:
+            msa.set_option(msa.OPT_DECODE_FUSED, decode_form)
+
+    # ---- the decode step in its other form (one cooperative launch), for
+    # the comparison that picks the library's default
+    t_dec_fused = None
+    if not decode_form:
+        outs = [(torch.empty_like(dids), torch.empty_like(do)) for _ in range(2)]
+
+        def dec_into(i):
+            return lambda: msa.sparse_attn_decode(pd, dd["q"], dd["q_idx"], dd["k_cache"], dd["v_cache"],
+                                                  dd["k_idx_cache"], dd["cu_kv"], max_kv, block_ids=outs[i][0],
+                                                  out=outs[i][1], ws=ws_d)
+        t_dec_fused = fused_form(dec_into(1))
+        dec_into(0)()
+        torch.cuda.synchronize()
+        rc = msa.device_status(ws_d)
+        if rc:
+            raise RuntimeError("device status %d after the fused decode" % rc)
+        if not (torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])):
+            raise RuntimeError("the two decode forms disagree")
+        del outs
+
     # ---- the same decode step over MXFP8 caches (quantised untimed, then
     # warmed up and timed over as many steps as the bf16 step)
-    t_mx = b_mx = None
+    t_mx = b_mx = t_mx_fused = None
     if not args.no_mxfp8 and wd.d == 128:
         q8 = {k_: msa.quantize_mxfp8(dd[k_]) for k_ in ("k_cache", "v_cache", "k_idx_cache")}
         dids8 = torch.empty_like(dids)
@@ -303,18 +345,12 @@ def run_ours(args, rank, world, torch, dist):
                                          q8["k_idx_cache"][1], dd["cu_kv"], max_kv, block_ids=dids8, out=do8,
                                          ws=ws_d)
 
-        for _ in range(args.warmup):
-            mx_step()
-        mev = [(E(enable_timing=True), E(enable_timing=True)) for _ in range(args.steps)]
-        for a_, b_ in mev:
-            a_.record(stream)
-            mx_step()
-            b_.record(stream)
-        torch.cuda.synchronize()
+        t_mx = median_ms(mx_step)
+        if not decode_form:
+            t_mx_fused = fused_form(mx_step)
         rc = msa.device_status(ws_d)
         if rc:
             raise RuntimeError("device status %d after the MXFP8 decode" % rc)
-        t_mx = statistics.median(a_.elapsed_time(b_) for a_, b_ in mev)
         b_mx = flops.decode_bytes(td["lens"], dids8.cpu().numpy(), wd.h_q, wd.h_kv, wd.d, wd.d_idx, wd.block_k,
                                   mxfp8=True)
         del q8
@@ -437,7 +473,9 @@ def run_ours(args, rank, world, torch, dist):
                     "index_ms": t_idx, "attn_ms": t_attn, "useful_tflop": (f_idx + f_main) / 1e12,
                     "tensor_frac": (f_idx + f_main) / ((t_idx + t_attn) / 1e3) / 1e12 / peaks["bf16_tflops"]},
         "decode": {"ms": t_dec, "tokens_per_s": B * world / (t_dec / 1e3), "bytes": b_dec,
-                   "hbm_frac": b_dec / (t_dec / 1e3) / 1e9 / peaks["hbm_gbs"]},
+                   "hbm_frac": b_dec / (t_dec / 1e3) / 1e9 / peaks["hbm_gbs"],
+                   "form": "one fused launch" if decode_form else "index-scan and attention launches",
+                   "fused_form_ms": t_dec_fused, "mxfp8_fused_form_ms": t_mx_fused},
         "decode_mxfp8": None if t_mx is None else {
             "ms": t_mx, "tokens_per_s": B * world / (t_mx / 1e3), "bytes": b_mx,
             "hbm_frac": b_mx / (t_mx / 1e3) / 1e9 / peaks["hbm_gbs"], "stat": "median per step",
@@ -455,11 +493,12 @@ def run_ours(args, rank, world, torch, dist):
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "note": "prefill inputs and outputs cross PCIe every step (double-buffered, uploads and downloads "
                         "on their own streams, overlapping the kernels); decode KV caches stay resident"},
-        # Per step: index top-k (1); sparse prefill: schedule count, scan and
-        # fill (3), block-major attention (1), partial merge (1); decode:
-        # persistent index scan with the merge folded in (1), persistent
-        # attention with the combine folded in (1).
-        "gpu_launches": 8 * args.steps,
+        # Per step: index top-k (1); sparse prefill: schedule count, scan,
+        # fill and list range (4), block-major attention (1), partial merge
+        # (1); decode: persistent index scan with the merge folded in and
+        # persistent attention with the combine folded in (2), or the two
+        # in one fused launch (1).
+        "gpu_launches": (7 + (1 if decode_form else 2)) * args.steps,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.case == "full":

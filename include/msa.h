@@ -24,11 +24,7 @@
  *   * Head h of the main branch belongs to group r = h / (h_q / h_kv).
  *   * Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *     default stream).  They are stateless: concurrent calls on different
- *     streams with different workspaces are safe.  A sparse prefill of more
- *     than 4096 query rows forks part of its work onto one auxiliary stream
- *     per device (created by the library on first use) and joins it back into
- *     `stream` before returning, so its completion is still ordered on
- *     `stream` (and the fork/join is captured by CUDA graph capture).
+ *     streams with different workspaces are safe.
  *   * Return value: MSA_OK, or a negative MSA_ERR_* code.  Argument errors are
  *     detected on the host before anything is launched.  Kernels bound every
  *     wait instead of hanging; a wait that gave up is recorded in the status
@@ -302,6 +298,21 @@ MSA_API int msa_sparse_attn_decode_mxfp8(const msa_params* p, const void* q, con
                                          void* o, void* ws, size_t ws_bytes, void* stream);
 
 /* Human-readable text of a status code (static storage). */
+/*
+ * Process-wide options (host only; take effect at the next call).
+ *   MSA_OPT_DECODE_FUSED  the form of a sparse decode step: 1 = one
+ *       cooperative launch (index scan and attention in every CTA, the ids
+ *       handed over through the L2) whenever the step fits one co-resident
+ *       wave, else the two launches; 0 = always the two persistent launches
+ *       (index scan, then streaming attention).  Both forms compute the same
+ *       ids and outputs bit for bit.
+ * msa_set_option returns MSA_OK, or MSA_ERR_INVALID for an unknown option or
+ * value; msa_get_option returns the value, or MSA_ERR_INVALID.
+ */
+#define MSA_OPT_DECODE_FUSED 0
+MSA_API int msa_set_option(int option, int value);
+MSA_API int msa_get_option(int option);
+
 MSA_API const char* msa_status_string(int status);
 
 #ifdef __cplusplus

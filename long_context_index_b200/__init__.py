@@ -26,7 +26,7 @@ POOL_MAX, POOL_MEAN = 0, 1   # msa_params.pool
 
 SYMBOLS = ("msa_workspace_size", "msa_index_project", "msa_quantize_mxfp8", "msa_sparse_attn_decode_mxfp8", "msa_index_topk", "msa_sparse_attn_prefill", "msa_sparse_attn_decode",
            "msa_index_topk_varlen", "msa_sparse_attn_prefill_varlen", "msa_sparse_attn_decode_adaptive_k",
-           "msa_device_status", "msa_status_string",
+           "msa_device_status", "msa_status_string", "msa_set_option", "msa_get_option",
            "msa_sparse_attn_decode_noalloc", "msa_test_never_ready_wait")
 
 
@@ -84,6 +84,8 @@ def lib():
         L.msa_test_never_ready_wait.restype = i32
         L.msa_device_status.argtypes = [vp, vp]
         L.msa_status_string.argtypes = [i32]
+        L.msa_set_option.argtypes = [i32, i32]
+        L.msa_get_option.argtypes = [i32]
         L.msa_status_string.restype = C.c_char_p
         for f in ("msa_index_topk", "msa_sparse_attn_prefill", "msa_sparse_attn_decode", "msa_device_status",
                   "msa_index_topk_varlen", "msa_sparse_attn_prefill_varlen", "msa_sparse_attn_decode_adaptive_k",
@@ -95,6 +97,25 @@ def lib():
 
 def status_string(code: int) -> str:
     return lib().msa_status_string(int(code)).decode()
+
+
+OPT_DECODE_FUSED = 0
+
+
+def set_option(option: int, value: int) -> None:
+    """Process-wide option (``msa_set_option``): OPT_DECODE_FUSED 1 runs a
+    sparse decode step as one cooperative launch when it fits one wave, 0 as
+    the index-scan and attention launches."""
+    rc = lib().msa_set_option(int(option), int(value))
+    if rc:
+        raise MSAError(rc, "msa_set_option")
+
+
+def get_option(option: int) -> int:
+    rc = lib().msa_get_option(int(option))
+    if rc < 0:
+        raise MSAError(rc, "msa_get_option")
+    return rc
 
 
 def workspace_size(op: int, p: Params, n_q: int = 0, n_kv: int = 0, batch: int = 0, max_kv: int = 0) -> int:

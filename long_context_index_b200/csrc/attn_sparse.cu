@@ -48,7 +48,6 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
-#include <mutex>
 
 #include "msa_internal.h"
 #include "ptx.cuh"
@@ -72,7 +71,6 @@ constexpr int kCtrlBytes = 20480;   // descriptors, softmax stats, staged entrie
 constexpr int kSchedThreads = 256;
 constexpr int kStageEntries = 256;   // list entries staged in shared memory at a time
 constexpr int kWave = 4096;          // query rows per wave (L2-resident Q working set)
-constexpr int kMergeSms = 16;        // SMs the block-major launches leave to the previous wave's merge
 
 template <int D, int BK>
 struct KvoCfg {
@@ -107,8 +105,8 @@ struct KvoArgs {
   const int* chunk_off;  // [n_waves * h_kv * nb] first global chunk id of each list
   const int* entries;    // (query << 5) | slot, grouped by list
   const int* lists;      // non-empty list ids ((wave * h_kv + r) * nb + b)
-  const int* wave_lo;    // this launch's lists: [wave_lo[0], wave_lo[1]) of `lists`
-  int* work_counter;     // this launch's list counter
+  const int* wave_lo;    // the launch's lists: [wave_lo[0], wave_lo[1]) of `lists`
+  int* work_counter;     // the launch's list counter
   float* part_lse;       // [chunks * 128] lse2 of each partial row
   int* status;
   int n_q, n_kv, q_pos0, h_q, h_kv, topk, causal, nb;
@@ -708,20 +706,12 @@ __global__ void __launch_bounds__(1024) sched_scan_kernel(const int* cnt, int n,
   }
 }
 
-// Start of each query wave's lists in the compacted (ascending) list array:
-// wave_lo[w] = the first position whose list id is in wave w or later.
-__global__ void sched_waves_kernel(const int* lists, const int* n_lists, int n_waves, int lists_per_wave,
-                                   int* wave_lo) {
-  const int w = blockIdx.x * blockDim.x + threadIdx.x;
-  if (w > n_waves) return;
-  const int n = *n_lists;
-  const long long key = static_cast<long long>(w) * lists_per_wave;
-  int lo = 0, hi = n;   // first position with lists[pos] >= key
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (lists[mid] < key) lo = mid + 1; else hi = mid;
+// The launch's list range: [0, n_lists).
+__global__ void sched_range_kernel(const int* n_lists, int* range) {
+  if (threadIdx.x == 0) {
+    range[0] = 0;
+    range[1] = *n_lists;
   }
-  wave_lo[w] = lo;
 }
 
 __global__ void sched_fill_kernel(const int32_t* ids, long long total, int h_kv, int topk, int nb, int G,
@@ -861,13 +851,13 @@ SparseWs carve(const msa_params& p, int n_q, int n_kv, int batch, void* base) {
     off += align_up(bytes, 256);
     return ptr;
   };
-  // cnt, fill, the list count and the per-wave work counters are contiguous
-  // so one memset clears them.
-  s.cnt = reinterpret_cast<int*>(take((2 * nl + 1 + n_waves) * 4));
+  // cnt, fill, the list count and the work counter are contiguous so one
+  // memset clears them.
+  s.cnt = reinterpret_cast<int*>(take((2 * nl + 2) * 4));
   s.fill = s.cnt ? s.cnt + nl : nullptr;
   s.n_lists = s.cnt ? s.cnt + 2 * nl : nullptr;
   s.work = s.cnt ? s.cnt + 2 * nl + 1 : nullptr;
-  s.wave_lo = reinterpret_cast<int*>(take((n_waves + 1) * 4));
+  s.wave_lo = reinterpret_cast<int*>(take(2 * 4));
   s.offs = reinterpret_cast<int*>(take((nl + 1) * 4));
   s.chunk_off = reinterpret_cast<int*>(take(nl * 4));
   s.lists = reinterpret_cast<int*>(take(nl * 4));
@@ -879,27 +869,6 @@ SparseWs carve(const msa_params& p, int n_q, int n_kv, int batch, void* base) {
   s.part_o = reinterpret_cast<uint16_t*>(take(s.max_chunks * 128 * static_cast<size_t>(p.d) * 2));
   s.bytes = off;
   return s;
-}
-
-// One auxiliary stream and event per device for the wave pipeline (created
-// on first use, kept for the life of the process).  Callers hold g_aux_mu
-// while they enqueue on them: the event is re-recorded per wave, and calls
-// from several host threads must not interleave their records and waits.
-constexpr int kMaxDev = 64;
-std::mutex g_aux_mu;
-cudaStream_t g_aux[kMaxDev] = {};
-cudaEvent_t g_aux_ev[kMaxDev] = {};
-
-int aux_stream(cudaStream_t* st, cudaEvent_t* ev) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return MSA_ERR_CUDA;
-  if (!g_aux[dev]) {
-    if (cudaStreamCreateWithFlags(&g_aux[dev], cudaStreamNonBlocking) != cudaSuccess) return MSA_ERR_CUDA;
-    if (cudaEventCreateWithFlags(&g_aux_ev[dev], cudaEventDisableTiming) != cudaSuccess) return MSA_ERR_CUDA;
-  }
-  *st = g_aux[dev];
-  *ev = g_aux_ev[dev];
-  return MSA_OK;
 }
 
 }  // namespace
@@ -932,16 +901,13 @@ int run_sparse_attn_kvouter(const msa_params& p, const void* q, const CUtensorMa
   geo.nb_one = (n_kv + p.block_k - 1) / p.block_k;
   geo.bk = p.block_k;
   geo.nb = nb;
-  const int n_waves = (n_q + kWave - 1) / kWave;
-  if (cudaMemsetAsync(s.cnt, 0, (2 * static_cast<size_t>(nl) + 1 + n_waves) * 4, stream) != cudaSuccess)
-    return MSA_ERR_CUDA;
+  if (cudaMemsetAsync(s.cnt, 0, (2 * static_cast<size_t>(nl) + 2) * 4, stream) != cudaSuccess) return MSA_ERR_CUDA;
   const int gsz = static_cast<int>((total + kSchedThreads - 1) / kSchedThreads);
   sched_count_kernel<<<gsz, kSchedThreads, 0, stream>>>(block_ids, total, p.h_kv, p.topk, nb, geo, s.cnt);
   sched_scan_kernel<<<1, 1024, 0, stream>>>(s.cnt, nl, 128 / G, s.offs, s.chunk_off, s.lists, s.n_lists);
   sched_fill_kernel<<<gsz, kSchedThreads, 0, stream>>>(block_ids, total, p.h_kv, p.topk, nb, G, geo, s.offs,
                                                        s.chunk_off, s.fill, s.entries, s.prow_of);
-  sched_waves_kernel<<<(n_waves + 1 + 255) / 256, 256, 0, stream>>>(s.lists, s.n_lists, n_waves, p.h_kv * nb,
-                                                                    s.wave_lo);
+  sched_range_kernel<<<1, 32, 0, stream>>>(s.n_lists, s.wave_lo);
   if (cudaGetLastError() != cudaSuccess) return MSA_ERR_CUDA;
 
   KvoArgs a;
@@ -975,7 +941,7 @@ int run_sparse_attn_kvouter(const msa_params& p, const void* q, const CUtensorMa
     if (!encode_tma_bf16(&maps[3], 2, s.part_o, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MSA_ERR_CUDA;
   }
   auto launch_attn = [&](int w, int grid) -> cudaError_t {
-    a.wave_lo = s.wave_lo + w;
+    a.wave_lo = s.wave_lo + w;   // w = 0 with wave_lo[1] = n_lists: every list
     a.work_counter = s.work + w;
     if (p.d == 64)
       return p.block_k == 64 ? launch_kvo_g<64, 64>(G, maps, a, grid, stream)
@@ -983,44 +949,20 @@ int run_sparse_attn_kvouter(const msa_params& p, const void* q, const CUtensorMa
     return p.block_k == 64 ? launch_kvo_g<128, 64>(G, maps, a, grid, stream)
                            : launch_kvo_g<128, 128>(G, maps, a, grid, stream);
   };
-  auto launch_merge = [&](int w, cudaStream_t st) {
-    const int q0 = w * kWave, rows = (w + 1 == n_waves ? n_q : q0 + kWave) - q0;
+  auto launch_merge = [&](cudaStream_t st) {
     if (p.d == 64)
-      merge_partials_kernel<64><<<rows * p.h_kv, 256, 0, st>>>(s.prow_of, s.part_o, s.part_lse,
-                                                               static_cast<uint16_t*>(o), p.h_q, p.h_kv, p.topk, q0);
+      merge_partials_kernel<64><<<n_q * p.h_kv, 256, 0, st>>>(s.prow_of, s.part_o, s.part_lse,
+                                                              static_cast<uint16_t*>(o), p.h_q, p.h_kv, p.topk, 0);
     else
-      merge_partials_kernel<128><<<rows * p.h_kv, 256, 0, st>>>(s.prow_of, s.part_o, s.part_lse,
-                                                                static_cast<uint16_t*>(o), p.h_q, p.h_kv, p.topk, q0);
+      merge_partials_kernel<128><<<n_q * p.h_kv, 256, 0, st>>>(s.prow_of, s.part_o, s.part_lse,
+                                                               static_cast<uint16_t*>(o), p.h_q, p.h_kv, p.topk, 0);
   };
-  cudaStream_t aux = nullptr;
-  cudaEvent_t ev = nullptr;
-  std::unique_lock<std::mutex> lock(g_aux_mu, std::defer_lock);
-  if (n_waves > 1) {
-    lock.lock();
-    if (aux_stream(&aux, &ev) != MSA_OK) return MSA_ERR_CUDA;
-  }
-  if (n_waves == 1 || !aux) {
-    // One wave: the block-major kernel on every SM, then the merge.
-    for (int w = 0; w < n_waves; ++w) {
-      if (launch_attn(w, sms) != cudaSuccess) return MSA_ERR_CUDA;
-      launch_merge(w, stream);
-    }
-  } else {
-    // Wave pipeline: wave w's block-major launch leaves kMergeSms SMs free,
-    // and its merge runs on the auxiliary stream under wave w + 1's launch,
-    // so the partials' HBM round trip overlaps the tensor-core work.  The
-    // auxiliary stream forks from and joins back into the caller's stream.
-    if (cudaEventRecord(ev, stream) != cudaSuccess || cudaStreamWaitEvent(aux, ev, 0) != cudaSuccess)
-      return MSA_ERR_CUDA;
-    for (int w = 0; w < n_waves; ++w) {
-      if (launch_attn(w, sms - kMergeSms) != cudaSuccess) return MSA_ERR_CUDA;
-      if (cudaEventRecord(ev, stream) != cudaSuccess || cudaStreamWaitEvent(aux, ev, 0) != cudaSuccess)
-        return MSA_ERR_CUDA;
-      launch_merge(w, aux);
-    }
-    if (cudaEventRecord(ev, aux) != cudaSuccess || cudaStreamWaitEvent(stream, ev, 0) != cudaSuccess)
-      return MSA_ERR_CUDA;
-  }
+  // One persistent launch over every wave's lists on every SM, then the
+  // merge.  (Launching each wave separately on fewer SMs, with its merge on a
+  // second stream under the next wave, measured slower: ~0.2 ms of ramp and
+  // tail per wave launch outweighed the overlap.)
+  if (launch_attn(0, sms) != cudaSuccess) return MSA_ERR_CUDA;
+  launch_merge(stream);
   return cudaGetLastError() == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
 }
 

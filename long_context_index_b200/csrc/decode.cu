@@ -169,7 +169,11 @@ __device__ void merge_topk_warp(const DecArgs& a, int b, int r, int lane, int* c
 // The scan, as run by the persistent index kernel below and by the first
 // phase of the fused decode kernel: ismem is the dynamic shared memory; with
 // seq_ready non-null, the CTA that merges a sequence publishes its ids there.
-template <int DIDX, int BK, int POOL, bool F8>
+// UNR: 16-key tiles whose loads a warp keeps in flight.  The index kernel runs
+// three CTAs per SM (24 warps) at 2; the fused kernel has one CTA (8 warps)
+// per SM and the whole register file, so it unrolls further to keep as many
+// bytes in flight per SM.
+template <int DIDX, int BK, int POOL, bool F8, int UNR = 2>
 __device__ __forceinline__ void decode_index_body(const DecArgs& a, uint8_t* ismem, int* seq_ready) {
   constexpr int kHalves = DIDX / 32;   // 16-byte vectors per token row per thread
   constexpr int kWarps = kIdxThreads / 32;
@@ -247,33 +251,54 @@ __device__ __forceinline__ void decode_index_body(const DecArgs& a, uint8_t* ism
       } else {
         kbase = a.k_idx + static_cast<size_t>(off) * DIDX;
       }
-      // Q_idx fragment (B operand): column n = group g, permuted d_idx order.
+      // Q_idx fragment (B operand): column n = group g, permuted d_idx order
+      // (the order of the K_idx fragment below: thread t's h-th 8-vector is
+      // d_idx positions 8t + 32h .. (bf16) or E t + 8h .. (MXFP8, E = d_idx / 4
+      // contiguous codes per thread)).
 #pragma unroll
       for (int h = 0; h < kHalves; ++h) {
         qv[h] = make_uint4(0, 0, 0, 0);
+        const int dpos = F8 ? (DIDX / 4) * t + 8 * h : 8 * t + 32 * h;
         if (g < a.h_kv)
-          qv[h] = *reinterpret_cast<const uint4*>(a.q_idx + (static_cast<size_t>(cur) * a.h_kv + g) * DIDX + 8 * t +
-                                                   32 * h);
+          qv[h] = *reinterpret_cast<const uint4*>(a.q_idx + (static_cast<size_t>(cur) * a.h_kv + g) * DIDX + dpos);
       }
     }
     const int j0 = (gb - cur_p) * BK;
     // Groups 2t, 2t+1: running max (max-pool) or sum (mean-pool; the sum of
     // integer-valued scores is exact in fp32, in any order, below 2^24).
     float m0 = POOL ? 0.f : kNegInf, m1 = POOL ? 0.f : kNegInf;
-#pragma unroll 2
+#pragma unroll UNR
     for (int mt = 0; mt < BK / 16; ++mt) {
       const int ja = j0 + mt * 16 + g, jb = ja + 8;
       uint4 ra[kHalves], rb[kHalves];
+      if (F8) {
+        // Thread t's E = d_idx / 4 contiguous codes of rows ja and jb, all in
+        // scale block (E t) / 32, dequantised into its kHalves 8-vectors.
+        constexpr int E = DIDX / 4;
+        uint32_t ca[E / 4], cb[E / 4];
 #pragma unroll
-      for (int h = 0; h < kHalves; ++h) {
-        if (F8) {   // elements 8t + 32h .. +7 lie in scale block h
-          ra[h] = ja < L ? dq_e4m3x8(ldg_nc_v2(kbase8 + static_cast<size_t>(ja) * DIDX + 8 * t + 32 * h),
-                                     e8m0_scale(sbase8[static_cast<size_t>(ja) * (DIDX / 32) + h]))
-                         : make_uint4(0, 0, 0, 0);
-          rb[h] = jb < L ? dq_e4m3x8(ldg_nc_v2(kbase8 + static_cast<size_t>(jb) * DIDX + 8 * t + 32 * h),
-                                     e8m0_scale(sbase8[static_cast<size_t>(jb) * (DIDX / 32) + h]))
-                         : make_uint4(0, 0, 0, 0);
-        } else {
+        for (int v = 0; v < E / 16; ++v) {
+          const uint4 x = ja < L ? ldg_nc_v4(kbase8 + static_cast<size_t>(ja) * DIDX + E * t + 16 * v) : make_uint4(0, 0, 0, 0);
+          const uint4 y = jb < L ? ldg_nc_v4(kbase8 + static_cast<size_t>(jb) * DIDX + E * t + 16 * v) : make_uint4(0, 0, 0, 0);
+          ca[4 * v] = x.x; ca[4 * v + 1] = x.y; ca[4 * v + 2] = x.z; ca[4 * v + 3] = x.w;
+          cb[4 * v] = y.x; cb[4 * v + 1] = y.y; cb[4 * v + 2] = y.z; cb[4 * v + 3] = y.w;
+        }
+        if (E == 8) {
+          const uint2 x = ja < L ? ldg_nc_v2(kbase8 + static_cast<size_t>(ja) * DIDX + E * t) : make_uint2(0, 0);
+          const uint2 y = jb < L ? ldg_nc_v2(kbase8 + static_cast<size_t>(jb) * DIDX + E * t) : make_uint2(0, 0);
+          ca[0] = x.x; ca[1] = x.y;
+          cb[0] = y.x; cb[1] = y.y;
+        }
+        const float sca = ja < L ? e8m0_scale(sbase8[static_cast<size_t>(ja) * (DIDX / 32) + (E * t) / 32]) : 0.f;
+        const float scb = jb < L ? e8m0_scale(sbase8[static_cast<size_t>(jb) * (DIDX / 32) + (E * t) / 32]) : 0.f;
+#pragma unroll
+        for (int h = 0; h < kHalves; ++h) {
+          ra[h] = dq_e4m3x8(make_uint2(ca[2 * h], ca[2 * h + 1]), sca);
+          rb[h] = dq_e4m3x8(make_uint2(cb[2 * h], cb[2 * h + 1]), scb);
+        }
+      } else {
+#pragma unroll
+        for (int h = 0; h < kHalves; ++h) {
           ra[h] = ja < L ? ldg_nc_v4(kbase + static_cast<size_t>(ja) * DIDX + 8 * t + 32 * h) : make_uint4(0, 0, 0, 0);
           rb[h] = jb < L ? ldg_nc_v4(kbase + static_cast<size_t>(jb) * DIDX + 8 * t + 32 * h) : make_uint4(0, 0, 0, 0);
         }
@@ -1288,6 +1313,9 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
 //    and a publishing CTA never waits on anyone, so every wait ends.
 // ---------------------------------------------------------------------------
 constexpr int kFusedThreads = kIdxThreads;   // the scan's 8 warps; the attention uses 5 of them
+// Tiles in flight per warp in the fused scan: up to 32 16-byte loads a thread.
+template <int DIDX, int BK>
+constexpr int kFusedUnroll = (BK / 16) < 16 / (DIDX / 32) ? (BK / 16) : 16 / (DIDX / 32);
 
 template <int DIDX, int BK, int POOL, int D, bool F8>
 __global__ void __launch_bounds__(kFusedThreads, 1)
@@ -1295,7 +1323,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                         const __grid_constant__ CUtensorMap tm_v, const DecArgs a, const StreamArgs sa,
                         int* seq_ready) {
   extern __shared__ __align__(1024) uint8_t fsmem[];
-  decode_index_body<DIDX, BK, POOL, F8>(a, fsmem, seq_ready);
+  decode_index_body<DIDX, BK, POOL, F8, kFusedUnroll<DIDX, BK>>(a, fsmem, seq_ready);
   __syncthreads();   // the scan's shared memory is reused by the attention
   decode_attn_body<D, BK, F8>(&tm_q, &tm_k, &tm_v, sa, fsmem, seq_ready);
 }
@@ -1569,7 +1597,7 @@ int run_sparse_attn_decode(const msa_params& p, const void* q, const void* q_idx
   a.part = reinterpret_cast<float*>(w + 2 * align_up(cand * 4, 256));
 
   int rc = MSA_OK;
-  if (!dense && a.kfree > 0) {
+  if (!dense && a.kfree > 0 && g_decode_fused.load(std::memory_order_relaxed)) {
     // One fused launch when the step fits one co-resident wave.
     int* seq_ready = a.grp_count + static_cast<size_t>(batch) * p.h_kv * a.head_tiles;
     if (p.block_k == 64) {

@@ -1,5 +1,6 @@
 // msa_internal.h -- declarations shared by the library's translation units.
 #pragma once
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
 #include <cuda.h>
@@ -94,6 +95,9 @@ int run_sparse_attn_decode(const msa_params& p, const void* q, const void* q_idx
                            int max_kv, int dense, int32_t* block_ids, void* o, void* ws, size_t ws_bytes,
                            int* status, cudaStream_t stream, const int32_t* topk_seq = nullptr,
                            const DecodeMx8* mx8 = nullptr);
+
+// MSA_OPT_DECODE_FUSED (msa_set_option).
+extern std::atomic<int> g_decode_fused;
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 

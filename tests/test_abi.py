@@ -34,6 +34,23 @@ def test_status_strings():
     assert msa.status_string(-6) == "kernel wait timed out"
 
 
+def test_options_are_host_only_and_validated():
+    prev = msa.get_option(msa.OPT_DECODE_FUSED)
+    assert prev in (0, 1)
+    try:
+        for v in (1, 0):
+            msa.set_option(msa.OPT_DECODE_FUSED, v)
+            assert msa.get_option(msa.OPT_DECODE_FUSED) == v
+        for opt, v in ((msa.OPT_DECODE_FUSED, 2), (msa.OPT_DECODE_FUSED, -1), (7, 0)):
+            with pytest.raises(msa.MSAError) as err:
+                msa.set_option(opt, v)
+            assert err.value.code == -1
+        with pytest.raises(msa.MSAError):
+            msa.get_option(7)
+    finally:
+        msa.set_option(msa.OPT_DECODE_FUSED, prev)
+
+
 def P(**kw):
     base = dict(h_q=64, h_kv=4, d=128, d_idx=64, block_k=128, topk=16)
     base.update(kw)

@@ -156,3 +156,49 @@ def test_sparse_decode_rejects_batches_beyond_the_index_prefix():
     with pytest.raises(msa.MSAError) as err:
         msa.sparse_attn_decode(p, q, qi, kc, kc, ki, cu, 1)
     assert err.value.code == -2
+
+
+@pytest.fixture
+def fused_form():
+    prev = msa.get_option(msa.OPT_DECODE_FUSED)
+    msa.set_option(msa.OPT_DECODE_FUSED, 1)
+    yield
+    msa.set_option(msa.OPT_DECODE_FUSED, prev)
+
+
+def decode_kernels(fn):
+    """Names of the kernels one call of fn launches (CUPTI via torch.profiler)."""
+    from torch.profiler import ProfilerActivity, profile
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        fn()
+        torch.cuda.synchronize()
+    return [e.name for e in prof.events() if e.device_type.name == "CUDA"]
+
+
+@pytest.mark.parametrize("kw,pool", [
+    (dict(h_q=64, h_kv=4, d=128, d_idx=64, block_k=128, topk=16, batch=3, kv_min=5000, kv_max=20000), 0),
+    (dict(h_q=16, h_kv=4, d=128, d_idx=64, block_k=64, topk=6, batch=4, kv_min=1, kv_max=700), 0),
+    (dict(h_q=64, h_kv=2, d=64, d_idx=128, block_k=128, topk=32, batch=2, kv_min=9000, kv_max=9000), 0),
+    (dict(h_q=4, h_kv=4, d=128, d_idx=32, block_k=128, topk=3, batch=9, kv_min=100, kv_max=3000), 1),
+    (dict(batch=6, kv_min=100, kv_max=3000, seed=43), 1),
+])
+def test_fused_decode_form(fused_form, kw, pool):
+    # The one-launch form: the oracle's ids bit for bit and O within
+    # tolerance, and the same ids and O bit for bit as the two launches.
+    w = small(**kw)
+    run_case(w, pool=pool)
+    t = make_decode(w)
+    p = msa.Params.make(w.h_q, w.h_kv, w.d, w.d_idx, w.block_k, w.topk, pool=pool)
+    args = (p, dev(t["q"]), dev(t["q_idx"]), dev(t["k_cache"]), dev(t["v_cache"]), dev(t["k_idx_cache"]),
+            dev(t["cu_kv"]), int(t["lens"].max()))
+    out = {}
+    names = decode_kernels(lambda: out.setdefault(1, msa.sparse_attn_decode(*args)))
+    assert any("decode_fused_kernel" in n for n in names), names
+    msa.set_option(msa.OPT_DECODE_FUSED, 0)
+    names = decode_kernels(lambda: out.setdefault(0, msa.sparse_attn_decode(*args)))
+    assert not any("decode_fused_kernel" in n for n in names), names
+    assert torch.equal(out[0][0], out[1][0]) and torch.equal(out[0][1], out[1][1])
+
+
+def test_fused_decode_b64_64k_128k(fused_form):
+    run_case(WORKLOADS["decode_b64_64k_128k"])
