@@ -434,6 +434,9 @@ def run_ours(args, rank, world, torch, dist):
         del sets
 
     peaks, peak_src = load_peaks()
+    next_rows = None if args.no_extras else measure_next_rows(
+        msa, torch, args, stream, median_ms, peaks, d_in, dd, wp, wd, td, n, n_kv, q_pos0, max_kv, ids, o, dids,
+        do, ws_d)
     kern = {
         "index_topk_prefill": {"ms": t_idx, "bound": "tensor", "work": f_idx, "unit": "TFLOP/s",
                                "achieved": f_idx / (t_idx / 1e3) / 1e12, "peak": peaks["bf16_tflops"]},
@@ -480,6 +483,7 @@ def run_ours(args, rank, world, torch, dist):
             "ms": t_mx, "tokens_per_s": B * world / (t_mx / 1e3), "bytes": b_mx,
             "hbm_frac": b_mx / (t_mx / 1e3) / 1e9 / peaks["hbm_gbs"], "stat": "median per step",
             "note": "the same decode step over MXFP8 (E4M3 + E8M0 per 32) K, V and index-key caches"},
+        "next_rows": next_rows,
         "dense": None if t_dense_p is None else {
             "prefill_ms": t_dense_p, "decode_ms": t_dense_d, "steps": args.steps, "warmup": args.warmup,
             "stat": "median per step; sparse medians %.3f ms prefill, %.4f ms decode" % (med_pre, med_dec),
@@ -504,6 +508,110 @@ def run_ours(args, rank, world, torch, dist):
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.case == "full":
         line["cpu_baseline"] = cpu_baseline(tp, td, wp, wd)
     return line
+
+
+def measure_next_rows(msa, torch, args, stream, median_ms, peaks, d_in, dd, wp, wd, td, n, n_kv, q_pos0, max_kv,
+                      ids, o, dids, do, ws_d):
+    """The entry points beyond the prefill + decode step, each timed like the
+    step (warm-up, then the median of as many calls) on inputs of the bench's
+    shapes, with its useful work against the measured peak:
+
+    * index_project: Q_idx and K_idx from hidden states x [n, 8192] (the
+      hidden width h_q d of the model shape) and the stacked weight
+      [(h_kv + 1) d_idx, 8192]; x and the weight are seeded normals drawn on
+      the device.
+    * index_topk_mean_pool: the index branch of the prefill with block mean
+      pooling instead of max pooling.
+    * prefill_varlen: index branch + main branch of the prefill's rows cut into
+      a packed batch of independent sequences (seeded lengths in
+      [8192, 24576], the last one cut to fit); the rows are the prefill's own
+      synthetic inputs, so only the sequence boundaries are new.
+    * decode_adaptive_k: the decode step with a seeded per-sequence k in
+      [4, topk]."""
+    from long_context_index_b200 import flops
+    dev = d_in["q"].device
+    out = {}
+
+    def entry(ms, work, bound, note):
+        unit, peak = ("TFLOP/s", peaks["bf16_tflops"]) if bound == "tensor" else ("GB/s", peaks["hbm_gbs"])
+        ach = work / (ms / 1e3) / (1e12 if bound == "tensor" else 1e9)
+        return {"ms": ms, "bound": bound, "achieved": ach, "unit": unit, "peak": peak, "frac": ach / peak,
+                "note": note}
+
+    # index projections
+    d_model = wp.h_q * wp.d
+    pp = msa.Params.make(wp.h_q, wp.h_kv, wp.d, wp.d_idx, wp.block_k, wp.topk)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(6)
+    x = torch.randn((n, d_model), generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    w = (torch.randn(((wp.h_kv + 1) * wp.d_idx, d_model), generator=gen, device=dev, dtype=torch.float32)
+         / d_model ** 0.5).to(torch.bfloat16)
+    qi = torch.empty((n, wp.h_kv, wp.d_idx), dtype=torch.bfloat16, device=dev)
+    ki = torch.empty((n, 1, wp.d_idx), dtype=torch.bfloat16, device=dev)
+    ws_j = torch.empty(max(256, msa.workspace_size(msa.OP_INDEX_PROJECT, pp, n)), dtype=torch.uint8, device=dev)
+    t = median_ms(lambda: msa.index_project(pp, x, w, q_idx=qi, k_idx=ki, ws=ws_j))
+    n_out = (wp.h_kv + 1) * wp.d_idx
+    f = 2.0 * n * d_model * n_out
+    b = (n * d_model + n_out * d_model + n * n_out) * 2
+    # Whichever of the two floors is longer bounds the kernel.
+    bound = "tensor" if f / (peaks["bf16_tflops"] * 1e12) >= b / (peaks["hbm_gbs"] * 1e9) else "hbm"
+    out["index_project"] = entry(t, f if bound == "tensor" else b, bound,
+                                 "x [%d, %d] -> Q_idx, K_idx: %.3f TFLOP, %.2f GB" % (n, d_model, f / 1e12, b / 1e9))
+    out["index_project"]["hbm_frac"] = b / (t / 1e3) / 1e9 / peaks["hbm_gbs"]
+    del x, w, qi, ki, ws_j
+
+    # mean pooling
+    pm = msa.Params.make(wp.h_q, wp.h_kv, wp.d, wp.d_idx, wp.block_k, wp.topk, pool=msa.POOL_MEAN)
+    ws_m = torch.empty(msa.workspace_size(msa.OP_INDEX_TOPK, pm, n, n_kv), dtype=torch.uint8, device=dev)
+    ids_m = torch.empty_like(ids)
+    t = median_ms(lambda: msa.index_topk(pm, d_in["q_idx"], d_in["k_idx"], q_pos0, block_ids=ids_m, ws=ws_m))
+    out["index_topk_mean_pool"] = entry(t, flops.index_flops(n, n_kv, q_pos0, wp.h_kv, wp.d_idx), "tensor",
+                                        "the prefill's index branch, block mean instead of max")
+    del ws_m, ids_m
+
+    # packed batch of independent prefills over the prefill's rows
+    if q_pos0 == 0:
+        g = np.random.default_rng(5)
+        lens = []
+        while sum(lens) < n:
+            lens.append(int(min(g.integers(8192, 24577), n - sum(lens))))
+        cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]).astype(np.int32), device=dev)
+        ws_vi = torch.empty(msa.workspace_size(msa.OP_INDEX_TOPK_VARLEN, pp, n, batch=len(lens)), dtype=torch.uint8,
+                            device=dev)
+        ws_vp = torch.empty(msa.workspace_size(msa.OP_PREFILL_VARLEN, pp, n, batch=len(lens)), dtype=torch.uint8,
+                            device=dev)
+        ids_v = torch.empty_like(ids)
+        o_v = torch.empty_like(o)
+
+        def varlen_step():
+            msa.index_topk_varlen(pp, d_in["q_idx"], d_in["k_idx"], cu, block_ids=ids_v, ws=ws_vi)
+            msa.sparse_attn_prefill_varlen(pp, d_in["q"], d_in["k"], d_in["v"], cu, ids_v, out=o_v, ws=ws_vp)
+        t = median_ms(varlen_step)
+        ids_h = ids_v.cpu().numpy()
+        f_i = f_m = 0.0
+        row = 0
+        for L in lens:
+            f_i += flops.index_flops(L, L, 0, wp.h_kv, wp.d_idx)
+            f_m += flops.main_flops(flops.selected_keys(ids_h[row:row + L], wp.block_k, L, 0), wp.h_q, wp.h_kv,
+                                    wp.d)
+            row += L
+        out["prefill_varlen"] = entry(t, f_i + f_m, "tensor", "%d sequences of %s tokens (%d rows)"
+                                      % (len(lens), "/".join(map(str, lens)), n))
+        out["prefill_varlen"]["tokens_per_s"] = n / (t / 1e3)
+        del ws_vi, ws_vp, ids_v, o_v
+
+    # adaptive k in decode
+    pd = msa.Params.make(wd.h_q, wd.h_kv, wd.d, wd.d_idx, wd.block_k, wd.topk)
+    ks = np.random.default_rng(7).integers(4, wd.topk + 1, size=wd.batch).astype(np.int32)
+    kt = torch.from_numpy(ks).to(dev)
+    dids_a = torch.empty_like(dids)
+    do_a = torch.empty_like(do)
+    t = median_ms(lambda: msa.sparse_attn_decode(pd, dd["q"], dd["q_idx"], dd["k_cache"], dd["v_cache"],
+                                                 dd["k_idx_cache"], dd["cu_kv"], max_kv, block_ids=dids_a, out=do_a,
+                                                 ws=ws_d, topk_per_seq=kt))
+    bts = flops.decode_bytes(td["lens"], dids_a.cpu().numpy(), wd.h_q, wd.h_kv, wd.d, wd.d_idx, wd.block_k)
+    out["decode_adaptive_k"] = entry(t, bts, "hbm", "per-sequence k in [4, %d], mean %.1f" % (wd.topk, ks.mean()))
+    return out
 
 
 # ---------------------------------------------------------------------------
@@ -589,6 +697,8 @@ def main(argv=None):
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-mxfp8", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the projection, mean-pool, packed-batch and adaptive-k measurements")
     args = ap.parse_args(argv)
     if args.gpus < 1:
         ap.error("--gpus must be >= 1")
