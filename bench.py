@@ -46,9 +46,14 @@ def cases(name):
     pair ("long": the last 8192 queries of a 2^20-token chunked prefill and a
     batch of 8 sequences decoding at 2^20), a profiling pair small enough for
     multi-pass ncu captures ("prof": the last 4096 queries of a 65536-token
-    context, about 1 GB of partials, and 8 sequences of 16K-32K tokens), or a
+    context, about 1 GB of partials, and 8 sequences of 16K-32K tokens;
+    "prof_decode": the same prefill and 64 sequences of 16K-32K tokens, whose
+    200 MB of index keys exceed the L2 in 3.3 GB of caches), or a
     tiny pair that runs in seconds ("tiny": the 1K prefill and 4 short decode
     sequences)."""
+    if name == "prof_decode":
+        return (cases("prof")[0],
+                Workload(**{**DECODE.__dict__, "kv_min": 16384, "kv_max": 32768, "name": "decode_b64_16k_32k"}))
     if name == "prof":
         return (Workload(**{**WORKLOADS["prefill_32k"].__dict__, "n_q": 4096, "n_kv": 65536,
                             "name": "chunked_prefill_64k_4k"}),
@@ -66,9 +71,13 @@ def cases(name):
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_BYTES = 126 * 1024 * 1024
 
-# DRAM bytes per call of the dominant unit, measured by ncu on the kernel
-# source with the given digest (a stale digest reports null).
-TRAFFIC = {}
+# DRAM bytes per call of the dominant unit at the bench workload, from ncu's
+# dram__bytes_read.sum + dram__bytes_write.sum of its kernels on the 4096-query
+# chunked prefill at 64K ("prof" case: 2.545 GB), scaled by the query rows
+# (x32; the traffic is the partial rows, one per query, head and selected
+# block), on the kernel source with the given digest (a stale digest reports
+# null).
+TRAFFIC = {"attn_prefill": (2.545e9 * 32, "d9107512a614", "attn_sparse.cu")}
 
 
 def load_peaks():
@@ -692,7 +701,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--case", choices=["full", "small", "long", "prof", "tiny"], default="full")
+    ap.add_argument("--case", choices=["full", "small", "long", "prof", "prof_decode", "tiny"], default="full")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")

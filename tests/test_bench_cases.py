@@ -30,3 +30,12 @@ def test_ranks_get_independent_seeds_of_the_same_shape():
     b_p, b_d = bench.rank_workloads("long", 3)
     assert (a_p.n_q, a_p.n_kv, a_d.batch) == (b_p.n_q, b_p.n_kv, b_d.batch)
     assert b_p.seed - a_p.seed == 3000 and b_d.seed - a_d.seed == 3000
+
+
+def test_profiling_cases_exceed_the_l2_with_few_gb():
+    wp, wd = bench.cases("prof")
+    assert wp.n_q == 4096 and wp.n_kv == 65536 and wd.batch == 8
+    wp2, wd2 = bench.cases("prof_decode")
+    assert wp2 == wp and wd2.batch == 64 and (wd2.kv_min, wd2.kv_max) == (16384, 32768)
+    # index keys: 128 B per token, above the 126 MB L2 even at the shortest lengths
+    assert wd2.batch * wd2.kv_min * wd2.d_idx * 2 > 126 * 2 ** 20
