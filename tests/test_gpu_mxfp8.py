@@ -9,7 +9,7 @@ import torch
 
 import long_context_index_b200 as msa
 import oracle
-from synth import WORKLOADS, Workload, f32_to_bf16_bits, make_decode
+from synth import WORKLOADS, Workload, bf16_bits_to_f32, f32_to_bf16_bits, make_decode
 from tests.gpu_util import assert_close, dev, host_f64, params_pair
 
 pytestmark = pytest.mark.gpu
@@ -34,8 +34,13 @@ def dequant_bits(q, s):
     return f32_to_bf16_bits(oracle.dequantize_mxfp8(q, s).astype(np.float32))
 
 
-def run_case(w, seqs=None, force_local=1):
+def run_case(w, seqs=None, force_local=1, big_qidx=()):
     t = make_decode(w)
+    for b in big_qidx:
+        # Q_idx of sequence b times 2^18: exact in bf16, beyond the f16 range,
+        # so that sequence's index scan takes the bf16-dequantising path
+        # (scores stay exact integers times 2^18).
+        t["q_idx"][b] = f32_to_bf16_bits(bf16_bits_to_f32(t["q_idx"][b]) * np.float32(2.0 ** 18))
     p, po = params_pair(w.h_q, w.h_kv, w.d, w.d_idx, w.block_k, w.topk, 1, force_local)
     q8 = {}
     for name in ("k_cache", "v_cache", "k_idx_cache"):
@@ -79,3 +84,35 @@ def test_mxfp8_decode_model_shape(force_local):
 
 def test_mxfp8_decode_b64_64k_128k_sampled():
     run_case(WORKLOADS["decode_b64_64k_128k"], seqs=[0, 5, 31, 63])
+
+
+def test_mxfp8_decode_q_idx_beyond_f16():
+    # Sequences 1 and 3 take the index scan's bf16 path, the others the f16
+    # path; both give the oracle's ids.
+    run_case(Workload("m8", "decode", h_q=64, h_kv=4, d=128, d_idx=64, block_k=128, topk=16, seed=603, batch=5,
+                      kv_min=3000, kv_max=20000, needles=4), big_qidx=(1, 3))
+
+
+@pytest.mark.parametrize("d_idx", [32, 128])
+def test_mxfp8_decode_index_widths(d_idx):
+    # One and four scale blocks per index key.
+    run_case(Workload("m8", "decode", h_q=32, h_kv=2, d=128, d_idx=d_idx, block_k=64, topk=8, seed=604, batch=4,
+                      kv_min=100, kv_max=5000, needles=2), big_qidx=(2,))
+
+
+def test_mxfp8_fused_form_agrees_with_two_launches():
+    w = Workload("m8", "decode", h_q=64, h_kv=4, d=128, d_idx=64, block_k=128, topk=16, seed=605, batch=6,
+                 kv_min=5000, kv_max=30000, needles=4)
+    prev = msa.get_option(msa.OPT_DECODE_FUSED)
+    try:
+        msa.set_option(msa.OPT_DECODE_FUSED, 1)
+        _, ids1, o1 = run_case(w)
+        msa.set_option(msa.OPT_DECODE_FUSED, 0)
+        _, ids0, o0 = run_case(w)
+    finally:
+        msa.set_option(msa.OPT_DECODE_FUSED, prev)
+    # The same ids; O agrees within rounding (the fused form's attention runs
+    # four consumer warps, the standalone one eight, so row sums are added in
+    # another order) and each matched the oracle above.
+    assert torch.equal(ids0, ids1)
+    assert_close(host_f64(o1), host_f64(o0), what="fused vs two-launch MXFP8 O")
