@@ -287,7 +287,7 @@ MSA_API int msa_quantize_mxfp8(const void* x, long long rows, int cols, void* q,
  *   k_scale,
  *   v_scale        uint8 [sum L_b, h_kv, d / 32] E8M0 codes (4-byte aligned)
  *   k_idx8         uint8 [sum L_b, 1, d_idx]  E4M3 codes (16-byte aligned)
- *   k_idx_scale    uint8 [sum L_b, 1, d_idx / 32] (aligned to d_idx / 32 bytes)
+ *   k_idx_scale    uint8 [sum L_b, 1, d_idx / 32]
  *   topk_per_seq   as for msa_sparse_attn_decode_adaptive_k (NULL: topk)
  * Other arguments, limits and the workspace as for msa_sparse_attn_decode.
  */
@@ -305,9 +305,7 @@ MSA_API int msa_sparse_attn_decode_mxfp8(const msa_params* p, const void* q, con
  *       handed over through the L2) whenever the step fits one co-resident
  *       wave, else the two launches; 0 = always the two persistent launches
  *       (index scan, then streaming attention).  Both forms compute the same
- *       ids, and over bf16 caches the same outputs bit for bit (over MXFP8
- *       caches the outputs agree to rounding: the attention's row sums are
- *       added in another order).
+ *       ids and outputs bit for bit.
  * msa_set_option returns MSA_OK, or MSA_ERR_INVALID for an unknown option or
  * value; msa_get_option returns the value, or MSA_ERR_INVALID.
  */

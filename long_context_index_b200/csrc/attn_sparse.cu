@@ -21,14 +21,12 @@
 //        per chunk in an 8-deep ring; V_b follows the list's first chunk.  K
 //        and V have their own barriers, so the next list's K lands once the
 //        last S has read K while the last PV still reads V.
-//      * warp 1 issues S = Q K_b^T into one of two TMEM S buffers (S of the
-//        next chunk is computed while the softmax works on this one); warp 14
-//        issues O = P V_b (P read from one of two TMEM P buffers) into a TMEM
-//        O buffer (two where TMEM has room).  Both run their loops with the
-//        whole warp and issue from one elected lane with precomputed
-//        descriptors: a tcgen05.mma issuing thread slows with every busy warp
-//        on its SMSP.  An S buffer is released as soon as the softmax has
-//        loaded it.
+//      * warp 1 issues S = Q K_b^T into the TMEM S buffer; warp 14 issues
+//        O = P V_b (P read from one of two TMEM P buffers) into one of two
+//        TMEM O buffers.  Both run their loops with the whole warp and issue
+//        from one elected lane with precomputed descriptors: a tcgen05.mma
+//        issuing thread slows with every busy warp on its SMSP.  S is
+//        released as soon as the softmax has loaded it.
 //      * warps 2..9 (softmax): two threads per row, each owning 64 of the 128
 //        columns; the exact softmax of the row over the block's visible keys
 //        (causal only in the local block); the two halves exchange only their
@@ -82,15 +80,12 @@ struct KvoCfg {
   static constexpr int kOBytes = 128 * D * 2;          // staged bf16 partial tile
   static constexpr int kSmemData = kQStages * kQBytes + kKVStages * 2 * kKVBytes + kOStages * kOBytes;
   static constexpr int kSmemBytes = kSmemData + kCtrlBytes + 1024;
-  // Two S buffers (S(t+1) is computed while the softmax works on S(t)), two
-  // P buffers, and two O buffers where they fit beside them (one at
-  // BK = D = 128: the epilogue frees O as soon as it is in registers).
-  static constexpr int kOBufs = (3 * BK + 2 * D) <= 512 ? 2 : 1;
-  static constexpr int kColS = 0;        // S: [0, BK), [BK, 2BK)
-  static constexpr int kColP = 2 * BK;   // P: [2BK, 2BK + BK/2), [2BK + BK/2, 3BK)
-  static constexpr int kColO = 3 * BK;   // O: kOBufs buffers of D columns
-  static constexpr int kTmemCols = (3 * BK + kOBufs * D) <= 256 ? 256 : 512;
-  static_assert(3 * BK + kOBufs * D <= 512, "TMEM columns");
+  // TMEM: one S buffer (freed as soon as the softmax has loaded it), two P
+  // buffers (bf16 pairs, BK/2 columns each), two O buffers.
+  static constexpr int kColS = 0;        // S: [0, BK)
+  static constexpr int kColP = BK;       // P: [BK, BK + BK/2), [BK + BK/2, 2BK)
+  static constexpr int kColO = 2 * BK;   // O: [2BK, 2BK + D), [2BK + D, 2BK + 2D)
+  static constexpr int kTmemCols = (2 * BK + 2 * D) <= 256 ? 256 : 512;
 };
 
 // One chunk of gathered queries of a (group, block) list.  (Declared before
@@ -161,11 +156,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* v_empty = v_full + kKVStages;
   uint64_t* d_full = v_empty + kKVStages;                    // [kDesc]
   uint64_t* d_empty = d_full + kDesc;
-  uint64_t* s_full = d_empty + kDesc;                        // [2] S ready
-  uint64_t* s_free = s_full + 2;                             // [2] S loaded by the softmax
-  uint64_t* p_free = s_free + 2;                             // [2] P consumed by its PV
+  uint64_t* s_full = d_empty + kDesc;                        // [1] S ready
+  uint64_t* s_free = s_full + 1;                             // [1] S loaded by the softmax
+  uint64_t* p_free = s_free + 1;                             // [2] P consumed by its PV
   uint64_t* p_full = p_free + 2;
-  uint64_t* o_full = p_full + 2;                             // [kOBufs]
+  uint64_t* o_full = p_full + 2;
   uint64_t* o_free = o_full + 2;
   uint64_t* ml_full = o_free + 2;                            // [kDesc]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ml_full + kDesc);
@@ -189,10 +184,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&d_empty[s], 14);  // S and PV issuers + 8 softmax warps + 4 epilogue warps
       mbar_init(&ml_full[s], 8);   // 8 softmax warps
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&s_full[s], 1);
-      mbar_init(&s_free[s], 8);    // the 8 softmax warps, once their S loads completed
-    }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 8);          // the 8 softmax warps, once their S loads completed
     for (int s = 0; s < 2; ++s) {
       mbar_init(&p_free[s], 1);
       mbar_init(&p_full[s], 8);
@@ -360,9 +353,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++kvc;
       }
       if (!__all_sync(0xffffffffu, mbar_wait(&q_full[qs], (t / kQStages) & 1, wc))) break;
-      // S(t) goes to S buffer t & 1 once the softmax has loaded S(t-2).
-      const int sbuf = t & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_free[sbuf], ((t >> 1) & 1) ^ 1, wc))) break;
+      // S(t) reuses the single S buffer once the softmax has loaded S(t-1).
+      if (!__all_sync(0xffffffffu, mbar_wait(s_free, (t & 1) ^ 1, wc))) break;
       tc_fence_after();
       const uint64_t qd = q_desc0 + ((qs * Cfg::kQBytes) >> 4);
       const uint64_t kd = k_desc0 + ((kvs * 2 * Cfg::kKVBytes) >> 4);
@@ -370,10 +362,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int ks = 0; ks < D / 16; ++ks) {
         const uint32_t off = (ks / 4) * (128 * 128) + (ks % 4) * 32;
         const uint32_t koff = (ks / 4) * (BK * 128) + (ks % 4) * 32;
-        umma_ss_elect(tmem + Cfg::kColS + sbuf * BK, qd + (off >> 4), kd + (koff >> 4), idesc_s, ks > 0 ? 1u : 0u);
+        umma_ss_elect(tmem + Cfg::kColS, qd + (off >> 4), kd + (koff >> 4), idesc_s, ks > 0 ? 1u : 0u);
       }
       umma_commit_elect(&q_empty[qs]);
-      umma_commit_elect(&s_full[sbuf]);
+      umma_commit_elect(s_full);
       if (last) umma_commit_elect(&k_empty[kvs]);   // this list's last read of K
       __syncwarp();
     }
@@ -390,22 +382,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&d_empty[ds]);
       if (end) break;
-      const int sb = t & 1;                 // P buffer
-      const int ob = t % Cfg::kOBufs;       // O buffer
+      const int sb = t & 1;
       if (first) {
         if (!__all_sync(0xffffffffu, mbar_wait(&v_full[kvs], (vc / kKVStages) & 1, wc))) break;
         ++vc;
       }
       if (!__all_sync(0xffffffffu, mbar_wait(&p_full[sb], (t >> 1) & 1, wc))) break;
-      if (!__all_sync(0xffffffffu, mbar_wait(&o_free[ob], ((t / Cfg::kOBufs) & 1) ^ 1, wc))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&o_free[sb], ((t >> 1) & 1) ^ 1, wc))) break;
       tc_fence_after();
       const uint64_t vd = v_desc0 + ((kvs * 2 * Cfg::kKVBytes) >> 4);
       const uint32_t p_tmem = tmem + Cfg::kColP + sb * (BK / 2);
-      const uint32_t o_tmem = tmem + Cfg::kColO + ob * D;
+      const uint32_t o_tmem = tmem + Cfg::kColO + sb * D;
 #pragma unroll
       for (int kk = 0; kk < BK / 16; ++kk)
         umma_ts_elect(o_tmem, p_tmem + kk * 8, vd + ((kk * 2048) >> 4), idesc_o, kk > 0 ? 1u : 0u);
-      umma_commit_elect(&o_full[ob]);
+      umma_commit_elect(&o_full[sb]);
       umma_commit_elect(&p_free[sb]);
       if (last) umma_commit_elect(&v_empty[kvs]);   // this list's last read of V
       __syncwarp();
@@ -439,18 +430,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         lim = min(BK, kv_lim - b * BK) - half * HC;
       }
       const int sb = t & 1;   // P buffer
-      if (!mbar_wait(&s_full[t & 1], (t >> 1) & 1, wc)) break;
+      if (!mbar_wait(s_full, t & 1, wc)) break;
       tc_fence_after();
-      const uint32_t s_tmem = lane_base + Cfg::kColS + (t & 1) * BK;
+      const uint32_t s_tmem = lane_base + Cfg::kColS;
       uint32_t sv[HC];
 #pragma unroll
       for (int cc = 0; cc < HC / 32; ++cc)
         tmem_ld32(s_tmem + half * HC + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[cc * 32]));
       tmem_ld_wait();
-      // S is in registers: hand the S buffer back for the S MMA after next.
+      // S is in registers: hand the S buffer back so the next S MMA can start.
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[t & 1]);
+      if (lane == 0) mbar_arrive(s_free);
       if (lim < HC) {
 #pragma unroll
         for (int i = 0; i < HC; ++i)
@@ -527,8 +518,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       const int e = qi < dd.count ? dd.entry[qi] : -1;
-      const int ob = t % Cfg::kOBufs;
-      if (!mbar_wait(&o_full[ob], (t / Cfg::kOBufs) & 1, wc)) break;
+      const int sb = t & 1;
+      if (!mbar_wait(&o_full[sb], (t >> 1) & 1, wc)) break;
       if (!mbar_wait(&ml_full[ds], (t / kDesc) & 1, wc)) break;
       tc_fence_after();
       const float2 st = ml[ds * 128 + row];
@@ -550,14 +541,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int a = 0; a < D / 64; ++a) {
         uint32_t ov[64];
-        tmem_ld32(lane_base + Cfg::kColO + ob * D + a * 64, *reinterpret_cast<uint32_t(*)[32]>(&ov[0]));
-        tmem_ld32(lane_base + Cfg::kColO + ob * D + a * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&ov[32]));
+        tmem_ld32(lane_base + Cfg::kColO + sb * D + a * 64, *reinterpret_cast<uint32_t(*)[32]>(&ov[0]));
+        tmem_ld32(lane_base + Cfg::kColO + sb * D + a * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&ov[32]));
         tmem_ld_wait();
         if (a == D / 64 - 1) {
           // The O buffer is free once its values are in registers.
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&o_free[ob]);
+          if (lane == 0) mbar_arrive(&o_free[sb]);
         }
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {

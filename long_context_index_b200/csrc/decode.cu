@@ -21,16 +21,13 @@
 //   2. decode_attn_stream_kernel  The (sequence, group, head tile, slot)
 //      items are cut into equal ranges, one per CTA.  A producer warp
 //      TMA-loads the Q tile and the selected K/V block per item; four consumer
-//      warps (eight over MXFP8 caches) run QK^T and PV on mma.sync with an
-//      fp32 online softmax.  A unit
+//      warps run QK^T and PV on mma.sync with an fp32 online softmax.  A unit
 //      split between CTAs is merged by the last of them (LSE weights).
 // The fused form (decode_fused_kernel) runs 1 and 2 back to back in every CTA
 // of one cooperative grid; an attention CTA waits only until the ids of its
 // own sequences are published by the CTA that merged them.  With MXFP8 caches
-// (E4M3 + E8M0 per 32 elements) 1 feeds the codes to f16 mma.sync and scales
-// each scale block's sums by its E8M0 factor (when Q_idx is exact in f16;
-// else it dequantises to bf16 in registers), and 2 dequantises each K/V block
-// in shared memory before the same math.
+// (E4M3 + E8M0 per 32 elements) 1 dequantises the index keys in registers and
+// 2 dequantises each K/V block in shared memory before the same math.
 // The dense run (every causal block) skips the index scan and uses
 // decode_attn_kernel: split-KV CTAs staging K/V with cp.async, combined by
 // the last split of each (sequence, group, head tile).
@@ -116,32 +113,6 @@ __device__ __forceinline__ uint32_t dq_e4m3x2(uint32_t two_bytes, float sc) {
 __device__ __forceinline__ uint4 dq_e4m3x8(uint2 v, float sc) {
   return make_uint4(dq_e4m3x2(v.x & 0xffffu, sc), dq_e4m3x2(v.x >> 16, sc), dq_e4m3x2(v.y & 0xffffu, sc),
                     dq_e4m3x2(v.y >> 16, sc));
-}
-
-__device__ __forceinline__ void mma_f16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                              uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-// Two E4M3 codes -> f16x2 (exact).
-__device__ __forceinline__ uint32_t e4m3x2_f16x2(uint32_t two_bytes) {
-  uint32_t h;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(static_cast<uint16_t>(two_bytes)));
-  return h;
-}
-// bf16x2 -> f16x2; ok stays true only if both values convert exactly.
-__device__ __forceinline__ uint32_t bf16x2_f16x2(uint32_t v, bool& ok) {
-  const float lo = __uint_as_float(v << 16), hi = __uint_as_float(v & 0xffff0000u);
-  uint32_t r;
-  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  float blo, bhi;
-  asm("cvt.f32.f16 %0, %1;" : "=f"(blo) : "h"(static_cast<uint16_t>(r & 0xffffu)));
-  asm("cvt.f32.f16 %0, %1;" : "=f"(bhi) : "h"(static_cast<uint16_t>(r >> 16)));
-  ok = ok && blo == lo && bhi == hi;
-  return r;
 }
 
 // (score desc, block asc) order used for every selection.
@@ -266,13 +237,6 @@ __device__ __forceinline__ void decode_index_body(const DecArgs& a, uint8_t* ism
   const uint8_t* kbase8 = a.k_idx8;       // MXFP8: codes and scales of this sequence
   const uint8_t* sbase8 = a.k_idx_sc;
   uint4 qv[kHalves];
-  // MXFP8 with Q_idx exact in f16 (the usual case): the codes feed f16
-  // mma.sync as they are (one conversion per two codes) and each row's E8M0
-  // scales multiply its per-scale-block sums afterwards.  qh is the f16 Q_idx
-  // fragment in the bf16 path's order (thread t's h-th 8-vector is d_idx
-  // positions 8t + 32h .., all inside scale block h).
-  uint32_t qh[F8 ? kHalves : 1][4];
-  bool q16 = false;
   for (int i = warp; i < W; i += kWarps) {
     const int gb = G0 + i;
     if (cur < 0 || gb >= cur_end) {
@@ -298,21 +262,6 @@ __device__ __forceinline__ void decode_index_body(const DecArgs& a, uint8_t* ism
         if (g < a.h_kv)
           qv[h] = *reinterpret_cast<const uint4*>(a.q_idx + (static_cast<size_t>(cur) * a.h_kv + g) * DIDX + dpos);
       }
-      if (F8) {
-        bool ok = true;
-#pragma unroll
-        for (int h = 0; h < kHalves; ++h) {
-          uint4 v = make_uint4(0, 0, 0, 0);
-          if (g < a.h_kv)
-            v = *reinterpret_cast<const uint4*>(a.q_idx + (static_cast<size_t>(cur) * a.h_kv + g) * DIDX + 8 * t +
-                                                32 * h);
-          qh[h][0] = bf16x2_f16x2(v.x, ok);
-          qh[h][1] = bf16x2_f16x2(v.y, ok);
-          qh[h][2] = bf16x2_f16x2(v.z, ok);
-          qh[h][3] = bf16x2_f16x2(v.w, ok);
-        }
-        q16 = __all_sync(0xffffffffu, ok);
-      }
     }
     const int j0 = (gb - cur_p) * BK;
     // Groups 2t, 2t+1: running max (max-pool) or sum (mean-pool; the sum of
@@ -321,43 +270,8 @@ __device__ __forceinline__ void decode_index_body(const DecArgs& a, uint8_t* ism
 #pragma unroll UNR
     for (int mt = 0; mt < BK / 16; ++mt) {
       const int ja = j0 + mt * 16 + g, jb = ja + 8;
-      float c[4] = {0.f, 0.f, 0.f, 0.f};
       uint4 ra[kHalves], rb[kHalves];
-      if (F8 && q16) {
-        // Row ja's / jb's 8 codes of scale block h at d_idx 8t + 32h.
-        uint2 xa[kHalves], xb[kHalves];
-#pragma unroll
-        for (int h = 0; h < kHalves; ++h) {
-          xa[h] = ja < L ? ldg_nc_v2(kbase8 + static_cast<size_t>(ja) * DIDX + 32 * h + 8 * t) : make_uint2(0, 0);
-          xb[h] = jb < L ? ldg_nc_v2(kbase8 + static_cast<size_t>(jb) * DIDX + 32 * h + 8 * t) : make_uint2(0, 0);
-        }
-        // The rows' kHalves scale bytes, contiguous.
-        uint32_t sa = 0, sb = 0;
-        if (kHalves == 1) {
-          sa = ja < L ? sbase8[ja] : 0u;
-          sb = jb < L ? sbase8[jb] : 0u;
-        } else if (kHalves == 2) {
-          sa = ja < L ? *reinterpret_cast<const uint16_t*>(sbase8 + static_cast<size_t>(ja) * 2) : 0u;
-          sb = jb < L ? *reinterpret_cast<const uint16_t*>(sbase8 + static_cast<size_t>(jb) * 2) : 0u;
-        } else {
-          sa = ja < L ? *reinterpret_cast<const uint32_t*>(sbase8 + static_cast<size_t>(ja) * 4) : 0u;
-          sb = jb < L ? *reinterpret_cast<const uint32_t*>(sbase8 + static_cast<size_t>(jb) * 4) : 0u;
-        }
-#pragma unroll
-        for (int h = 0; h < kHalves; ++h) {
-          float cb[4] = {0.f, 0.f, 0.f, 0.f};
-          mma_f16_16816(cb, e4m3x2_f16x2(xa[h].x), e4m3x2_f16x2(xb[h].x), e4m3x2_f16x2(xa[h].x >> 16),
-                        e4m3x2_f16x2(xb[h].x >> 16), qh[h][0], qh[h][1]);
-          mma_f16_16816(cb, e4m3x2_f16x2(xa[h].y), e4m3x2_f16x2(xb[h].y), e4m3x2_f16x2(xa[h].y >> 16),
-                        e4m3x2_f16x2(xb[h].y >> 16), qh[h][2], qh[h][3]);
-          const float sca = ja < L ? e8m0_scale((sa >> (8 * h)) & 0xffu) : 0.f;
-          const float scb = jb < L ? e8m0_scale((sb >> (8 * h)) & 0xffu) : 0.f;
-          c[0] = fmaf(sca, cb[0], c[0]);
-          c[1] = fmaf(sca, cb[1], c[1]);
-          c[2] = fmaf(scb, cb[2], c[2]);
-          c[3] = fmaf(scb, cb[3], c[3]);
-        }
-      } else if (F8) {
+      if (F8) {
         // Thread t's E = d_idx / 4 contiguous codes of rows ja and jb, all in
         // scale block (E t) / 32, dequantised into its kHalves 8-vectors.
         constexpr int E = DIDX / 4;
@@ -389,12 +303,11 @@ __device__ __forceinline__ void decode_index_body(const DecArgs& a, uint8_t* ism
           rb[h] = jb < L ? ldg_nc_v4(kbase + static_cast<size_t>(jb) * DIDX + 8 * t + 32 * h) : make_uint4(0, 0, 0, 0);
         }
       }
-      if (!F8 || !q16) {
+      float c[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int h = 0; h < kHalves; ++h) {
-          mma_bf16_16816(c, ra[h].x, rb[h].x, ra[h].y, rb[h].y, qv[h].x, qv[h].y);
-          mma_bf16_16816(c, ra[h].z, rb[h].z, ra[h].w, rb[h].w, qv[h].z, qv[h].w);
-        }
+      for (int h = 0; h < kHalves; ++h) {
+        mma_bf16_16816(c, ra[h].x, rb[h].x, ra[h].y, rb[h].y, qv[h].x, qv[h].y);
+        mma_bf16_16816(c, ra[h].z, rb[h].z, ra[h].w, rb[h].w, qv[h].z, qv[h].w);
       }
       if (POOL) {   // keys past L loaded zeros, so their scores add 0
         m0 += c[0] + c[2];
@@ -894,23 +807,15 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const DecArgs
 // range [c T / n, (c + 1) T / n), so every SM streams the same number of K/V
 // blocks whatever the batch and selection look like.  Per CTA: one producer
 // warp issues TMA loads (Q tile, K block, V block) into a ring of stages;
-// NC consumer warps (4; 8 over MXFP8 caches) run the online softmax on
-// mma.sync.  Warp w computes S for keys [w BK/NC, (w+1) BK/NC) of the block,
-// the warps agree on the row maxima through shared memory, write P (bf16) to
-// shared memory, and warp w then accumulates O for output columns
-// [w D/NC, (w+1) D/NC) over the whole block, so no cross-warp reduction of O
-// is ever needed.  A unit that lies in
+// four consumer warps run the online softmax on mma.sync.  Warp w computes
+// S for keys [w BK/4, (w+1) BK/4) of the block, the four warps agree on the
+// row maxima through shared memory, write P (bf16) to shared memory, and warp
+// w then accumulates O for output columns [w D/4, (w+1) D/4) over the whole
+// block, so no cross-warp reduction of O is ever needed.  A unit that lies in
 // one CTA is normalised and written directly; a unit split between CTAs
 // leaves an (o, m, l) partial per CTA and the last of them to finish merges.
-constexpr int kStreamConsumers = 4;    // bf16 caches
-// MXFP8 caches: eight consumer warps (each owns BK/8 keys of S and D/8 output
-// columns), so the dequantisation of a block is split twice as wide.
-constexpr int kStreamConsumersF8 = 8;
-constexpr int kStreamMaxConsumers = 8;
-template <bool F8>
-__host__ __device__ constexpr int stream_consumers() { return F8 ? kStreamConsumersF8 : kStreamConsumers; }
-template <bool F8>
-__host__ __device__ constexpr int stream_threads() { return 32 * (stream_consumers<F8>() + 1); }
+constexpr int kStreamConsumers = 4;
+constexpr int kStreamThreads = 32 * (kStreamConsumers + 1);
 constexpr int kStreamCtas = 148;       // persistent grid: one CTA per SM
 constexpr int kStreamIdsCap = 1024;    // items per CTA held in shared memory
 
@@ -933,7 +838,7 @@ struct StreamCfg {
   static constexpr int kOffDeq = kStages * kStageBytes;
   static constexpr int kOffP = kOffDeq + kDeqBytes;
   static constexpr int kOffRed = kOffP + kPBytes;                       // red_m[4][16], red_l[4][16]
-  static constexpr int kOffIds = kOffRed + 2 * kStreamMaxConsumers * 16 * 4;
+  static constexpr int kOffIds = kOffRed + 2 * kStreamConsumers * 16 * 4;
   static constexpr int kOffMeta = kOffIds + kStreamIdsCap * 4;          // int4 per stage
   static constexpr int kOffBar = kOffMeta + kStages * 16;               // full[], empty[]
   static constexpr int kOffFlags = kOffBar + 2 * kStages * 8;
@@ -970,20 +875,19 @@ __device__ __forceinline__ int cta_of_item(long long g, long long T, int n) {
 // phase of the fused decode kernel (smem_raw: the dynamic shared memory;
 // seq_ready non-null: wait until the ids of this CTA's sequences are out).
 // Warps past the producer take no part.
-template <int D, int BK, bool F8, int NC>
+template <int D, int BK, bool F8>
 __device__ __forceinline__ void decode_attn_body(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
                                                  const CUtensorMap* tm_v, const StreamArgs& a, uint8_t* smem_raw,
                                                  const int* seq_ready) {
   using C = StreamCfg<D, BK, F8>;
-  static_assert(NC <= kStreamMaxConsumers && BK / NC >= 8 && (D / NC) % 16 == 0, "consumer split");
-  constexpr int KPW = BK / NC;                 // S keys per warp (NC consumer warps)
+  constexpr int KPW = BK / kStreamConsumers;   // S keys per warp
   constexpr int NT = KPW / 8;
-  constexpr int NCOL = D / NC;                 // O columns per warp
+  constexpr int NCOL = D / kStreamConsumers;   // O columns per warp
   constexpr int NTO = NCOL / 8;
   constexpr int PST = D + 4;                   // partial row stride (floats)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* red_m = reinterpret_cast<float*>(smem + C::kOffRed);
-  float* red_l = red_m + NC * 16;
+  float* red_l = red_m + kStreamConsumers * 16;
   int* s_ids = reinterpret_cast<int*>(smem + C::kOffIds);
   int4* meta = reinterpret_cast<int4*>(smem + C::kOffMeta);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
@@ -1038,7 +942,7 @@ __device__ __forceinline__ void decode_attn_body(const CUtensorMap* tm_q, const 
       // MXFP8: the TMA bytes, then one cp.async arrival per producer lane
       // once its share of the block's scales has landed.
       mbar_init(&full[s], F8 ? 33 : 1);
-      mbar_init(&empty[s], NC);
+      mbar_init(&empty[s], kStreamConsumers);
     }
     flags[0] = 0;
     flags[1] = 0;
@@ -1047,9 +951,9 @@ __device__ __forceinline__ void decode_attn_body(const CUtensorMap* tm_q, const 
   }
   __syncthreads();
   WaitCtx wc{reinterpret_cast<volatile int*>(&flags[0]), a.status};
-  if (warp > NC) return;
+  if (warp > kStreamConsumers) return;
 
-  if (warp == NC) {
+  if (warp == kStreamConsumers) {
     // ---------------- producer ----------------
     // Lane 0 waits for a free stage and issues the TMA loads; with MXFP8
     // caches the whole warp then gathers the K and V scales of the block into
@@ -1132,7 +1036,7 @@ __device__ __forceinline__ void decode_attn_body(const CUtensorMap* tm_q, const 
     return;
   }
 
-  // ---------------- consumers (warps 0 .. NC - 1) ----------------
+  // ---------------- consumers (warps 0..3) ----------------
   const int g = lane >> 2, t = lane & 3;
   const int mi = lane >> 3, rr = lane & 7;
   float oacc[NTO][4];
@@ -1162,11 +1066,11 @@ __device__ __forceinline__ void decode_attn_body(const CUtensorMap* tm_q, const 
         // still holds the Q tile, is released at the end of the item.
         sK = sbase + C::kOffDeq;
         sV = sK + C::kKBytes;
-        named_bar(1, 32 * NC);
+        named_bar(1, 32 * kStreamConsumers);
         const uint8_t* s8 = smem + stage * C::kStageBytes + C::kQBytes;
         const uint8_t* ssc = s8 + 2 * C::kK8Bytes;
         constexpr int CPR = D / 16;                      // 16-byte chunks per E4M3 row
-        for (int e = tid; e < 2 * BK * CPR; e += 32 * NC) {
+        for (int e = tid; e < 2 * BK * CPR; e += 32 * kStreamConsumers) {
           const int kv = e / (BK * CPR), rem = e - kv * (BK * CPR);
           const int x = rem / CPR, c = rem - x * CPR;   // row, chunk (16 elements from column 16c)
           // E4M3 rows of D = 128 bytes, 128B-swizzled by TMA (16-byte chunk c of row x at c ^ (x & 7)).
@@ -1181,7 +1085,7 @@ __device__ __forceinline__ void decode_attn_body(const CUtensorMap* tm_q, const 
                        "r"(hi.y), "r"(hi.z), "r"(hi.w)
                        : "memory");
         }
-        named_bar(1, 32 * NC);
+        named_bar(1, 32 * kStreamConsumers);
       }
 
       uint32_t qf[D / 16][4];
@@ -1222,9 +1126,9 @@ __device__ __forceinline__ void decode_attn_body(const CUtensorMap* tm_q, const 
         red_m[warp * 16 + g] = mx_lo;
         red_m[warp * 16 + g + 8] = mx_hi;
       }
-      named_bar(1, 32 * NC);
+      named_bar(1, 32 * kStreamConsumers);
 #pragma unroll
-      for (int w = 0; w < NC; ++w) {
+      for (int w = 0; w < kStreamConsumers; ++w) {
         mx_lo = fmaxf(mx_lo, red_m[w * 16 + g]);
         mx_hi = fmaxf(mx_hi, red_m[w * 16 + g + 8]);
       }
@@ -1267,10 +1171,10 @@ __device__ __forceinline__ void decode_attn_body(const CUtensorMap* tm_q, const 
                        : "memory");
         }
       }
-      named_bar(1, 32 * NC);
+      named_bar(1, 32 * kStreamConsumers);
       float ls_lo = 0.f, ls_hi = 0.f;
 #pragma unroll
-      for (int w = 0; w < NC; ++w) {
+      for (int w = 0; w < kStreamConsumers; ++w) {
         ls_lo += red_l[w * 16 + g];
         ls_hi += red_l[w * 16 + g + 8];
       }
@@ -1334,12 +1238,12 @@ __device__ __forceinline__ void decode_attn_body(const CUtensorMap* tm_q, const 
         *reinterpret_cast<float2*>(pp + (g + 8) * PST + D) = make_float2(m_hi, l_hi);
       }
       __threadfence();
-      named_bar(1, 32 * NC);
+      named_bar(1, 32 * kStreamConsumers);
       if (tid == 0) {
         flags[1] = atomicAdd(&a.unit_count[u], 1) == c_hi - c_lo;
         __threadfence();
       }
-      named_bar(1, 32 * NC);
+      named_bar(1, 32 * kStreamConsumers);
       if (flags[1]) {
         // Last CTA of the unit: LSE-weighted merge of the c_hi - c_lo + 1 partials.
         float M_lo = kNegInf, M_hi = kNegInf;
@@ -1391,11 +1295,11 @@ __device__ __forceinline__ void decode_attn_body(const CUtensorMap* tm_q, const 
 }
 
 template <int D, int BK, bool F8>
-__global__ void __launch_bounds__(stream_threads<F8>(), 1)
+__global__ void __launch_bounds__(kStreamThreads, 1)
     decode_attn_stream_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                               const __grid_constant__ CUtensorMap tm_v, const StreamArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  decode_attn_body<D, BK, F8, stream_consumers<F8>()>(&tm_q, &tm_k, &tm_v, a, smem_raw, nullptr);
+  decode_attn_body<D, BK, F8>(&tm_q, &tm_k, &tm_v, a, smem_raw, nullptr);
 }
 
 // ---------------------------------------------------------------------------
@@ -1421,8 +1325,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   extern __shared__ __align__(1024) uint8_t fsmem[];
   decode_index_body<DIDX, BK, POOL, F8, kFusedUnroll<DIDX, BK>>(a, fsmem, seq_ready);
   __syncthreads();   // the scan's shared memory is reused by the attention
-  // Four consumer warps here (the grid's 8 warps hold them and the producer).
-  decode_attn_body<D, BK, F8, kStreamConsumers>(&tm_q, &tm_k, &tm_v, sa, fsmem, seq_ready);
+  decode_attn_body<D, BK, F8>(&tm_q, &tm_k, &tm_v, sa, fsmem, seq_ready);
 }
 
 // Split plan of the dense run, shared by the workspace query and the launch.
@@ -1535,7 +1438,7 @@ int launch_attn_stream(const DecArgs& a, int max_kv, int* status, cudaStream_t s
   auto kern = decode_attn_stream_kernel<D, BK, F8>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return MSA_ERR_CUDA;
-  kern<<<s.n_cta, stream_threads<F8>(), smem, st>>>(tq, tk, tv, s);
+  kern<<<s.n_cta, kStreamThreads, smem, st>>>(tq, tk, tv, s);
   return cudaGetLastError() == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
 }
 

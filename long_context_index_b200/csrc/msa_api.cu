@@ -226,9 +226,6 @@ int msa_sparse_attn_decode_mxfp8(const msa_params* p, const void* q, const void*
   if (!aligned16(k8) || !aligned16(v8) || !aligned16(k_idx8)) return MSA_ERR_MISALIGNED;
   if (((reinterpret_cast<uintptr_t>(k_scale) | reinterpret_cast<uintptr_t>(v_scale)) & 3u) != 0)
     return MSA_ERR_MISALIGNED;
-  // The index scan reads a key's d_idx / 32 scale bytes as one word.
-  if ((reinterpret_cast<uintptr_t>(k_idx_scale) & static_cast<uintptr_t>(p->d_idx / 32 - 1)) != 0)
-    return MSA_ERR_MISALIGNED;
   DecodeMx8 mx{k8, k_scale, v8, v_scale, k_idx8, k_idx_scale};
   // The bf16 cache arguments are unused: the MXFP8 codes stand in for them
   // (non-null placeholders for the shared validation).

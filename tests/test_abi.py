@@ -106,13 +106,12 @@ def test_prefill_and_decode_reject_bad_arguments():
     assert L.msa_sparse_attn_decode(C.byref(p), 16, 16, 16, 16, 16, 16, 4, 100, 0, 16, 16, 256, 10, None) == -4
     assert L.msa_sparse_attn_decode(C.byref(p), 16, None, 16, 16, None, 16, 4, 100, 0, None, 16, 256,
                                     1 << 30, None) == -1
-    # MXFP8 decode: code arrays 16-byte aligned, K/V scales 4-byte aligned, the
-    # index-key scales aligned to d_idx / 32 bytes (read as one word per key).
+    # MXFP8 decode: code arrays 16-byte aligned, K/V scales 4-byte aligned.
     mx = L.msa_sparse_attn_decode_mxfp8
-    args = lambda k_idx_sc, k_sc=16: (C.byref(p), 16, 16, 16, k_sc, 16, 16, 16, k_idx_sc, 16, None, 4, 100, 16,
-                                      16, 256, 1 << 40, None)
-    assert mx(*args(17)) == -3
-    assert mx(*args(16, k_sc=18)) == -3
+    args = lambda k8=16, k_sc=16: (C.byref(p), 16, 16, k8, k_sc, 16, 16, 16, 16, 16, None, 4, 100, 16,
+                                   16, 256, 1 << 40, None)
+    assert mx(*args(k8=24)) == -3
+    assert mx(*args(k_sc=18)) == -3
     assert L.msa_sparse_attn_decode_mxfp8(C.byref(P(d=64)), *args(16)[1:]) == -2   # d = 128 only
     # Decode limits, refused on the host before any launch: more than 8 groups;
     # a sparse batch above 4096 or with batch * max_kv >= 2^31 (dense is fine).

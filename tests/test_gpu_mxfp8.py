@@ -37,8 +37,7 @@ def dequant_bits(q, s):
 def run_case(w, seqs=None, force_local=1, big_qidx=()):
     t = make_decode(w)
     for b in big_qidx:
-        # Q_idx of sequence b times 2^18: exact in bf16, beyond the f16 range,
-        # so that sequence's index scan takes the bf16-dequantising path
+        # Q_idx of sequence b times 2^18: exact in bf16, beyond the f16 range
         # (scores stay exact integers times 2^18).
         t["q_idx"][b] = f32_to_bf16_bits(bf16_bits_to_f32(t["q_idx"][b]) * np.float32(2.0 ** 18))
     p, po = params_pair(w.h_q, w.h_kv, w.d, w.d_idx, w.block_k, w.topk, 1, force_local)
@@ -87,8 +86,7 @@ def test_mxfp8_decode_b64_64k_128k_sampled():
 
 
 def test_mxfp8_decode_q_idx_beyond_f16():
-    # Sequences 1 and 3 take the index scan's bf16 path, the others the f16
-    # path; both give the oracle's ids.
+    # Index queries of very different magnitudes in one batch.
     run_case(Workload("m8", "decode", h_q=64, h_kv=4, d=128, d_idx=64, block_k=128, topk=16, seed=603, batch=5,
                       kv_min=3000, kv_max=20000, needles=4), big_qidx=(1, 3))
 
@@ -100,7 +98,7 @@ def test_mxfp8_decode_index_widths(d_idx):
                       kv_min=100, kv_max=5000, needles=2), big_qidx=(2,))
 
 
-def test_mxfp8_fused_form_agrees_with_two_launches():
+def test_mxfp8_fused_form_matches_two_launches():
     w = Workload("m8", "decode", h_q=64, h_kv=4, d=128, d_idx=64, block_k=128, topk=16, seed=605, batch=6,
                  kv_min=5000, kv_max=30000, needles=4)
     prev = msa.get_option(msa.OPT_DECODE_FUSED)
@@ -111,8 +109,4 @@ def test_mxfp8_fused_form_agrees_with_two_launches():
         _, ids0, o0 = run_case(w)
     finally:
         msa.set_option(msa.OPT_DECODE_FUSED, prev)
-    # The same ids; O agrees within rounding (the fused form's attention runs
-    # four consumer warps, the standalone one eight, so row sums are added in
-    # another order) and each matched the oracle above.
-    assert torch.equal(ids0, ids1)
-    assert_close(host_f64(o1), host_f64(o0), what="fused vs two-launch MXFP8 O")
+    assert torch.equal(ids0, ids1) and torch.equal(o0, o1)
