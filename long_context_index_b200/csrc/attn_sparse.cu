@@ -469,17 +469,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                       max3f(__uint_as_float(sv[i + 2]), __uint_as_float(sv[i + 3]), __uint_as_float(sv[i + 4])));
         mq[k] = max3f(mq[k], __uint_as_float(sv[i + 5]), fmaxf(__uint_as_float(sv[i + 6]), __uint_as_float(sv[i + 7])));
       }
-      // Exponentials against this half's own maximum first; the partner's
-      // maximum (same lane quarter) is exchanged meanwhile and the half is
-      // rescaled to the row maximum afterwards: exp2(x - m_h) * exp2(m_h - m).
+      // Exchange the half-row maxima with the partner warp (same lane quarter).
       // The slot alternates with the chunk parity: a warp rewrites slot
       // (t & 1) only after the next barrier, which its partner reaches only
       // after reading this chunk's value.
-      const float mh = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
       float* xs = smx + (t & 1) * 256;
-      xs[half * 128 + row] = mh;
-      const float bias = mh == kNegInfF ? 0.f : mh * c;
+      xs[half * 128 + row] = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+      named_bar(2 + quarter, 64);
+      const float mx = fmaxf(xs[row], xs[128 + row]);
+      const float bias = mx == kNegInfF ? 0.f : mx * c;
       float ls[4] = {0.f, 0.f, 0.f, 0.f};   // two pairs of partial sums
+      uint32_t pk[HC / 2];
 #pragma unroll
       for (int i = 0; i < HC; i += 4) {
         float x0, x1, x2, x3;
@@ -490,23 +490,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         fadd2(s0, s1, p0, p1, p2, p3);
         const int k = ((i / 4) & 1) * 2;
         fadd2(ls[k], ls[k + 1], ls[k], ls[k + 1], s0, s1);
-        sv[i] = __float_as_uint(p0);
-        sv[i + 1] = __float_as_uint(p1);
-        sv[i + 2] = __float_as_uint(p2);
-        sv[i + 3] = __float_as_uint(p3);
+        pk[i / 2] = pack_bf16x2(p0, p1);
+        pk[i / 2 + 1] = pack_bf16x2(p2, p3);
       }
-      named_bar(2 + quarter, 64);
-      const float mx = fmaxf(mh, xs[(1 - half) * 128 + row]);
-      const float f = mh == kNegInfF ? 0.f : ex2_approx((mh - mx) * c);   // mh <= mx
       // The next chunk's descriptor (its loads overlap the P store below).
       const bool have_next = fetch_desc(t + 1);
-      uint32_t pk[HC / 2];
-#pragma unroll
-      for (int i = 0; i < HC; i += 2) {
-        float q0, q1;
-        fmul2(q0, q1, __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]), f, f);
-        pk[i / 2] = pack_bf16x2(q0, q1);
-      }
       // P(t) goes to P buffer t & 1 once the PV of chunk t - 2 has read it.
       if (!mbar_wait(&p_free[sb], ((t >> 1) & 1) ^ 1, wc)) break;
       tc_fence_after();
@@ -515,7 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int cc = 0; cc < HC / 64; ++cc)
         tmem_st32(p_tmem + half * (HC / 2) + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[cc * 32]));
       if (HC / 2 == 16) tmem_st16(p_tmem + half * (HC / 2), *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
-      const float lsum = ((ls[0] + ls[1]) + (ls[2] + ls[3])) * f;
+      const float lsum = (ls[0] + ls[1]) + (ls[2] + ls[3]);
       if (half == 0)
         ml[ds * 128 + row] = make_float2(mx, lsum);
       else
