@@ -410,39 +410,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int qi = row / G;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const float c = args.scale_log2;
-    constexpr float kNegInfF = -__builtin_huge_valf();
-    // The descriptor of chunk t + 1 is read during chunk t (after its
-    // exponentials) and released at the end of chunk t, so no chain of
-    // shared-memory reads separates one chunk's P from the next chunk's S.
-    int n_end = 0, n_e = -1, n_b = 0, n_row0 = 0, n_len = 0;
-    auto fetch_desc = [&](int tt) -> bool {
-      if (!mbar_wait(&d_full[tt % kDesc], (tt / kDesc) & 1, wc)) return false;
-      const Desc& dd = desc[tt % kDesc];
-      n_end = dd.end;
-      n_e = qi < dd.count ? dd.entry[qi] : -1;
-      n_b = dd.b;
-      n_row0 = dd.seq_row0;
-      n_len = dd.seq_len;
-      return true;
-    };
-    auto release_desc = [&](int tt) {
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&d_empty[tt % kDesc]);
-    };
-    // Visible keys of block n_b for the row, relative to this half.
-    auto visible = [&]() -> int {
-      if (n_e < 0) return 0;   // positions local to the query's sequence
-      const int p = (args.cu_seqlens ? 0 : args.q_pos0) + (n_e >> 5) - n_row0;
-      const int kv_lim = args.causal ? min(p + 1, n_len) : n_len;
-      return min(BK, kv_lim - n_b * BK) - half * HC;
-    };
-    bool live = fetch_desc(0);
-    int lim = visible();
-    const bool first_end = n_end;
-    if (live) release_desc(0);
-    if (first_end) live = false;
-    for (int t = 0; live; ++t) {
+    for (int t = 0;; ++t) {
       const int ds = t % kDesc;
+      if (!mbar_wait(&d_full[ds], (t / kDesc) & 1, wc)) break;
+      const Desc& dd = desc[ds];
+      if (dd.end) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&d_empty[ds]);
+        break;
+      }
+      const int e = qi < dd.count ? dd.entry[qi] : -1;
+      const int b = dd.b, seq_row0 = dd.seq_row0, seq_len = dd.seq_len;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&d_empty[ds]);
+      int lim = 0;   // visible keys of this block for the row, relative to this half
+      if (e >= 0) {   // positions local to the query's sequence
+        const int p = (args.cu_seqlens ? 0 : args.q_pos0) + (e >> 5) - seq_row0;
+        const int kv_lim = args.causal ? min(p + 1, seq_len) : seq_len;
+        lim = min(BK, kv_lim - b * BK) - half * HC;
+      }
       const int sb = t & 1;   // P buffer
       if (!mbar_wait(s_full, t & 1, wc)) break;
       tc_fence_after();
@@ -461,7 +447,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < HC; ++i)
           if (i >= lim) sv[i] = 0xff800000u;   // -inf: masked key
       }
-      float mq[4] = {kNegInfF, kNegInfF, kNegInfF, kNegInfF};
+      float mq[4] = {__int_as_float(0xff800000), __int_as_float(0xff800000), __int_as_float(0xff800000),
+                     __int_as_float(0xff800000)};
 #pragma unroll
       for (int i = 0; i < HC; i += 8) {
         const int k = (i / 8) & 3;
@@ -477,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       xs[half * 128 + row] = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
       named_bar(2 + quarter, 64);
       const float mx = fmaxf(xs[row], xs[128 + row]);
-      const float bias = mx == kNegInfF ? 0.f : mx * c;
+      const float bias = mx == __int_as_float(0xff800000) ? 0.f : mx * c;
       float ls[4] = {0.f, 0.f, 0.f, 0.f};   // two pairs of partial sums
       uint32_t pk[HC / 2];
 #pragma unroll
@@ -493,8 +480,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         pk[i / 2] = pack_bf16x2(p0, p1);
         pk[i / 2 + 1] = pack_bf16x2(p2, p3);
       }
-      // The next chunk's descriptor (its loads overlap the P store below).
-      const bool have_next = fetch_desc(t + 1);
       // P(t) goes to P buffer t & 1 once the PV of chunk t - 2 has read it.
       if (!mbar_wait(&p_free[sb], ((t >> 1) & 1) ^ 1, wc)) break;
       tc_fence_after();
@@ -515,10 +500,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&p_full[sb]);
         mbar_arrive(&ml_full[ds]);
       }
-      if (!have_next) break;
-      lim = visible();
-      release_desc(t + 1);
-      if (n_end) break;
     }
   } else if (warp >= kEpiW0 && warp < kEpiW0 + 4) {
     // ---------------------------------------------------------------- epilogue
