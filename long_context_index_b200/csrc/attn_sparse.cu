@@ -55,14 +55,11 @@
 namespace msa {
 namespace {
 
-constexpr int kSoftPer = 4;                     // softmax warps per TMEM lane quarter
-constexpr int kSoftWarps = 4 * kSoftPer;
-constexpr int kSoftW0 = 2;                      // softmax warps 2 .. 17, BK / kSoftPer columns each
-constexpr int kEpiW0 = kSoftW0 + kSoftWarps;    // epilogue warps 18 .. 21
-constexpr int kPvW = kEpiW0 + 4;                // PV issuer (S is issued by warp 1): each SMSP's issue
-                                                // port is shared with the softmax warps, so one thread
-                                                // issuing both would cap the rate
-constexpr int kThreads = 32 * (kPvW + 1);       // 23 warps
+constexpr int kThreads = 480;   // 15 warps
+constexpr int kSoftW0 = 2;      // softmax warps 2..9: two per TMEM lane quarter, 64 columns each
+constexpr int kEpiW0 = 10;      // epilogue warps 10..13
+constexpr int kPvW = 14;        // PV issuer (S is issued by warp 1): each SMSP's issue port is shared
+                                // with two softmax warps, so one thread issuing both would cap the rate
 // One K/V stage suffices because a CTA switches blocks only once per
 // (group, block) list (hundreds of chunks); the partial tile is staged in
 // two shared-memory buffers for the TMA stores.
@@ -70,7 +67,7 @@ constexpr int kQStages = 3;
 constexpr int kKVStages = 1;
 constexpr int kOStages = 1;
 constexpr int kDesc = 8;        // descriptor ring depth (a slot is held until the epilogue is done)
-constexpr int kCtrlBytes = 30720;   // descriptors, softmax stats, staged entries, barriers
+constexpr int kCtrlBytes = 20480;   // descriptors, softmax stats, staged entries, barriers
 constexpr int kSchedThreads = 256;
 constexpr int kStageEntries = 256;   // list entries staged in shared memory at a time
 constexpr int kWave = 4096;          // query rows per wave (L2-resident Q working set)
@@ -100,8 +97,7 @@ struct Desc {
   int seq_row0, seq_len;                     // the block's sequence: first row, length
 };
 
-static_assert(kDesc * (sizeof(Desc) + 128 * (8 + 4 * (kSoftPer - 1))) + 2 * kSoftPer * 128 * 4 + kStageEntries * 4 +
-                      64 * 8 + 16 <= kCtrlBytes,
+static_assert(kDesc * (sizeof(Desc) + 128 * 12) + 4 * 128 * 4 + kStageEntries * 4 + 64 * 8 + 16 <= kCtrlBytes,
               "control block of attn_kvouter_kernel exceeds its shared-memory reservation");
 
 struct KvoArgs {
@@ -144,10 +140,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* skv = smem + kQStages * Cfg::kQBytes;             // [stage][K|V][atoms][BK][128 B]
   uint8_t* so = skv + kKVStages * 2 * Cfg::kKVBytes;         // [stage][atoms][128][128 B] partial tile
   Desc* desc = reinterpret_cast<Desc*>(smem + Cfg::kSmemData);
-  float2* ml = reinterpret_cast<float2*>(desc + kDesc);      // [kDesc][128] (m, l of the first column part)
-  float* lhi = reinterpret_cast<float*>(ml + kDesc * 128);   // [kDesc][kSoftPer - 1][128] l of the others
-  float* smx = lhi + kDesc * (kSoftPer - 1) * 128;           // [2 parity][kSoftPer][128] row-max exchange
-  int* stage = reinterpret_cast<int*>(smx + 2 * kSoftPer * 128);   // [kStageEntries] staged list entries
+  float2* ml = reinterpret_cast<float2*>(desc + kDesc);      // [kDesc][128] (m, l of columns 0..63)
+  float* lhi = reinterpret_cast<float*>(ml + kDesc * 128);   // [kDesc][128] l of columns 64..127
+  float* smx = lhi + kDesc * 128;                            // [2 parity][2 halves][128] row-max exchange
+  int* stage = reinterpret_cast<int*>(smx + 4 * 128);        // [kStageEntries] staged list entries
   uint64_t* bars = reinterpret_cast<uint64_t*>(stage + kStageEntries);
   uint64_t* q_full = bars;                                   // [kQStages]
   uint64_t* q_empty = q_full + kQStages;
@@ -185,14 +181,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < kDesc; ++s) {
       mbar_init(&d_full[s], 1);
-      mbar_init(&d_empty[s], 2 + kSoftWarps + 4);  // S and PV issuers, softmax and epilogue warps
-      mbar_init(&ml_full[s], kSoftWarps);
+      mbar_init(&d_empty[s], 14);  // S and PV issuers + 8 softmax warps + 4 epilogue warps
+      mbar_init(&ml_full[s], 8);   // 8 softmax warps
     }
     mbar_init(s_full, 1);
-    mbar_init(s_free, kSoftWarps);   // the softmax warps, once their S loads completed
+    mbar_init(s_free, 8);          // the 8 softmax warps, once their S loads completed
     for (int s = 0; s < 2; ++s) {
       mbar_init(&p_free[s], 1);
-      mbar_init(&p_full[s], kSoftWarps);
+      mbar_init(&p_full[s], 8);
       mbar_init(&o_full[s], 1);
       mbar_init(&o_free[s], 4);
     }
@@ -407,9 +403,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= kSoftW0 && warp < kEpiW0) {
     // ---------------------------------------------------------------- softmax
-    constexpr int HC = BK / kSoftPer;          // columns per thread
+    constexpr int HC = BK / 2;                 // columns per thread
     const int quarter = warp & 3;
-    const int half = (warp - kSoftW0) / 4;     // column part: [half HC, (half + 1) HC)
+    const int half = (warp - kSoftW0) / 4;     // 0: columns [0, HC), 1: [HC, BK)
     const int row = quarter * 32 + lane;
     const int qi = row / G;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
@@ -438,13 +434,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t s_tmem = lane_base + Cfg::kColS;
       uint32_t sv[HC];
-      if constexpr (HC >= 32) {
 #pragma unroll
-        for (int cc = 0; cc < HC / 32; ++cc)
-          tmem_ld32(s_tmem + half * HC + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[cc * 32]));
-      } else {
-        tmem_ld16(s_tmem + half * HC, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
-      }
+      for (int cc = 0; cc < HC / 32; ++cc)
+        tmem_ld32(s_tmem + half * HC + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[cc * 32]));
       tmem_ld_wait();
       // S is in registers: hand the S buffer back so the next S MMA can start.
       tc_fence_before();
@@ -468,12 +460,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // The slot alternates with the chunk parity: a warp rewrites slot
       // (t & 1) only after the next barrier, which its partner reaches only
       // after reading this chunk's value.
-      float* xs = smx + (t & 1) * (kSoftPer * 128);
+      float* xs = smx + (t & 1) * 256;
       xs[half * 128 + row] = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
-      named_bar(2 + quarter, 32 * kSoftPer);
-      float mx = xs[row];
-#pragma unroll
-      for (int q = 1; q < kSoftPer; ++q) mx = fmaxf(mx, xs[q * 128 + row]);
+      named_bar(2 + quarter, 64);
+      const float mx = fmaxf(xs[row], xs[128 + row]);
       const float bias = mx == __int_as_float(0xff800000) ? 0.f : mx * c;
       float ls[4] = {0.f, 0.f, 0.f, 0.f};   // two pairs of partial sums
       uint32_t pk[HC / 2];
@@ -494,20 +484,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(&p_free[sb], ((t >> 1) & 1) ^ 1, wc)) break;
       tc_fence_after();
       const uint32_t p_tmem = lane_base + Cfg::kColP + sb * (BK / 2);
-      if constexpr (HC / 2 >= 32) {
 #pragma unroll
-        for (int cc = 0; cc < HC / 64; ++cc)
-          tmem_st32(p_tmem + half * (HC / 2) + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[cc * 32]));
-      } else if constexpr (HC / 2 == 16) {
-        tmem_st16(p_tmem + half * (HC / 2), *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
-      } else {
-        tmem_st8(p_tmem + half * (HC / 2), *reinterpret_cast<uint32_t(*)[8]>(&pk[0]));
-      }
+      for (int cc = 0; cc < HC / 64; ++cc)
+        tmem_st32(p_tmem + half * (HC / 2) + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[cc * 32]));
+      if (HC / 2 == 16) tmem_st16(p_tmem + half * (HC / 2), *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
       const float lsum = (ls[0] + ls[1]) + (ls[2] + ls[3]);
       if (half == 0)
         ml[ds * 128 + row] = make_float2(mx, lsum);
       else
-        lhi[(ds * (kSoftPer - 1) + half - 1) * 128 + row] = lsum;
+        lhi[ds * 128 + row] = lsum;
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -538,9 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(&ml_full[ds], (t / kDesc) & 1, wc)) break;
       tc_fence_after();
       const float2 st = ml[ds * 128 + row];
-      float lsum = st.y;
-#pragma unroll
-      for (int q = 0; q < kSoftPer - 1; ++q) lsum += lhi[(ds * (kSoftPer - 1) + q) * 128 + row];
+      const float lsum = st.y + lhi[ds * 128 + row];
       const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
       const float lse2 = lsum > 0.f ? st.x * c + __log2f(lsum) : __int_as_float(0xff800000);
       const int chunk = dd.chunk;
