@@ -21,21 +21,19 @@
 //        per chunk in an 8-deep ring; V_b follows the list's first chunk.  K
 //        and V have their own barriers, so the next list's K lands once the
 //        last S has read K while the last PV still reads V.
-//      * warp 1 issues S = Q K_b^T into S buffer t & 1 of two in TMEM; warp
-//        14 issues O = P V_b (P read from P buffer t & 1) into a TMEM O
-//        buffer (two where TMEM has room).  Both run their loops with the
-//        whole warp and issue from one elected lane with precomputed
-//        descriptors: a tcgen05.mma issuing thread slows with every busy warp
-//        on its SMSP.
-//      * warps 2..9 (softmax): two per TMEM lane quarter, warp (quarter, g)
-//        taking the chunks of parity g, one thread per row: the exact
-//        softmax of the row over the block's visible keys (causal only in
-//        the local block) in two passes over S in TMEM (row maximum, then
-//        exponentials), P (bf16) to P buffer t & 1, (m, l) to the epilogue.
-//        The exponentials are MUFU-bound (16 per clock per SM: one 128x128
-//        tile costs as many cycles as its two MMAs); the two warps of an SMSP
-//        work on consecutive chunks, so one's exponentials overlap the
-//        other's maximum pass and P store.
+//      * warp 1 issues S = Q K_b^T into the TMEM S buffer; warp 14 issues
+//        O = P V_b (P read from one of two TMEM P buffers) into one of two
+//        TMEM O buffers.  Both run their loops with the whole warp and issue
+//        from one elected lane with precomputed descriptors: a tcgen05.mma
+//        issuing thread slows with every busy warp on its SMSP.  S is
+//        released as soon as the softmax has loaded it.
+//      * warps 2..9 (softmax): two threads per row, each owning 64 of the 128
+//        columns; the exact softmax of the row over the block's visible keys
+//        (causal only in the local block); the two halves exchange only their
+//        max through shared memory; P (bf16) goes to a P buffer; (m, l_lo,
+//        l_hi) go to the epilogue.  (The exponentials are MUFU-bound: 16 per
+//        clock per SM, so one 128x128 tile costs as many cycles as its two
+//        MMAs; two warps per SM sub-partition keep the MUFU pipe fed.)
 //      * warps 10..13 (epilogue): o = O / l in bf16 staged in shared memory and
 //        written by TMA (L2 evict-first) as one contiguous 128-row tile per
 //        chunk (chunk-major partials), lse2 = m c + log2 l beside it.
@@ -58,7 +56,7 @@ namespace msa {
 namespace {
 
 constexpr int kThreads = 480;   // 15 warps
-constexpr int kSoftW0 = 2;      // softmax warps 2..9: two per TMEM lane quarter, one per chunk parity
+constexpr int kSoftW0 = 2;      // softmax warps 2..9: two per TMEM lane quarter, 64 columns each
 constexpr int kEpiW0 = 10;      // epilogue warps 10..13
 constexpr int kPvW = 14;        // PV issuer (S is issued by warp 1): each SMSP's issue port is shared
                                 // with two softmax warps, so one thread issuing both would cap the rate
@@ -82,15 +80,12 @@ struct KvoCfg {
   static constexpr int kOBytes = 128 * D * 2;          // staged bf16 partial tile
   static constexpr int kSmemData = kQStages * kQBytes + kKVStages * 2 * kKVBytes + kOStages * kOBytes;
   static constexpr int kSmemBytes = kSmemData + kCtrlBytes + 1024;
-  // Two S buffers (S(t+1) is computed while the softmax works on S(t)), two
-  // P buffers, and two O buffers where they fit beside them (one at
-  // BK = D = 128: the epilogue frees O as soon as it is in registers).
-  static constexpr int kOBufs = (3 * BK + 2 * D) <= 512 ? 2 : 1;
-  static constexpr int kColS = 0;        // S: [0, BK), [BK, 2BK)
-  static constexpr int kColP = 2 * BK;   // P: [2BK, 2BK + BK/2), [2BK + BK/2, 3BK)
-  static constexpr int kColO = 3 * BK;   // O: kOBufs buffers of D columns
-  static constexpr int kTmemCols = (3 * BK + kOBufs * D) <= 256 ? 256 : 512;
-  static_assert(3 * BK + kOBufs * D <= 512, "TMEM columns");
+  // TMEM: one S buffer (freed as soon as the softmax has loaded it), two P
+  // buffers (bf16 pairs, BK/2 columns each), two O buffers.
+  static constexpr int kColS = 0;        // S: [0, BK)
+  static constexpr int kColP = BK;       // P: [BK, BK + BK/2), [BK + BK/2, 2BK)
+  static constexpr int kColO = 2 * BK;   // O: [2BK, 2BK + D), [2BK + D, 2BK + 2D)
+  static constexpr int kTmemCols = (2 * BK + 2 * D) <= 256 ? 256 : 512;
 };
 
 // One chunk of gathered queries of a (group, block) list.  (Declared before
@@ -102,7 +97,7 @@ struct Desc {
   int seq_row0, seq_len;                     // the block's sequence: first row, length
 };
 
-static_assert(kDesc * (sizeof(Desc) + 128 * 8) + kStageEntries * 4 + 64 * 8 + 16 <= kCtrlBytes,
+static_assert(kDesc * (sizeof(Desc) + 128 * 12) + 4 * 128 * 4 + kStageEntries * 4 + 64 * 8 + 16 <= kCtrlBytes,
               "control block of attn_kvouter_kernel exceeds its shared-memory reservation");
 
 struct KvoArgs {
@@ -145,8 +140,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* skv = smem + kQStages * Cfg::kQBytes;             // [stage][K|V][atoms][BK][128 B]
   uint8_t* so = skv + kKVStages * 2 * Cfg::kKVBytes;         // [stage][atoms][128][128 B] partial tile
   Desc* desc = reinterpret_cast<Desc*>(smem + Cfg::kSmemData);
-  float2* ml = reinterpret_cast<float2*>(desc + kDesc);      // [kDesc][128] (m, l) of each row
-  int* stage = reinterpret_cast<int*>(ml + kDesc * 128);     // [kStageEntries] staged list entries
+  float2* ml = reinterpret_cast<float2*>(desc + kDesc);      // [kDesc][128] (m, l of columns 0..63)
+  float* lhi = reinterpret_cast<float*>(ml + kDesc * 128);   // [kDesc][128] l of columns 64..127
+  float* smx = lhi + kDesc * 128;                            // [2 parity][2 halves][128] row-max exchange
+  int* stage = reinterpret_cast<int*>(smx + 4 * 128);        // [kStageEntries] staged list entries
   uint64_t* bars = reinterpret_cast<uint64_t*>(stage + kStageEntries);
   uint64_t* q_full = bars;                                   // [kQStages]
   uint64_t* q_empty = q_full + kQStages;
@@ -159,11 +156,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* v_empty = v_full + kKVStages;
   uint64_t* d_full = v_empty + kKVStages;                    // [kDesc]
   uint64_t* d_empty = d_full + kDesc;
-  uint64_t* s_full = d_empty + kDesc;                        // [2] S ready
-  uint64_t* s_free = s_full + 2;                             // [2] S loaded by the softmax
-  uint64_t* p_free = s_free + 2;                             // [2] P consumed by its PV
+  uint64_t* s_full = d_empty + kDesc;                        // [1] S ready
+  uint64_t* s_free = s_full + 1;                             // [1] S loaded by the softmax
+  uint64_t* p_free = s_free + 1;                             // [2] P consumed by its PV
   uint64_t* p_full = p_free + 2;
-  uint64_t* o_full = p_full + 2;                             // [kOBufs]
+  uint64_t* o_full = p_full + 2;
   uint64_t* o_free = o_full + 2;
   uint64_t* ml_full = o_free + 2;                            // [kDesc]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ml_full + kDesc);
@@ -184,16 +181,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < kDesc; ++s) {
       mbar_init(&d_full[s], 1);
-      mbar_init(&d_empty[s], 10);  // S and PV issuers + the chunk's 4 softmax warps + 4 epilogue warps
-      mbar_init(&ml_full[s], 4);   // the chunk's 4 softmax warps
+      mbar_init(&d_empty[s], 14);  // S and PV issuers + 8 softmax warps + 4 epilogue warps
+      mbar_init(&ml_full[s], 8);   // 8 softmax warps
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&s_full[s], 1);
-      mbar_init(&s_free[s], 4);    // the 4 softmax warps of the buffer's chunks, done reading S
-    }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 8);          // the 8 softmax warps, once their S loads completed
     for (int s = 0; s < 2; ++s) {
       mbar_init(&p_free[s], 1);
-      mbar_init(&p_full[s], 4);
+      mbar_init(&p_full[s], 8);
       mbar_init(&o_full[s], 1);
       mbar_init(&o_free[s], 4);
     }
@@ -322,12 +317,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    // End markers for the consumers: two, since each softmax warp reads
-    // only the descriptors of its chunk parity.
+    // End marker for the consumers.
     if (lane == 0 && ok && !*abort_flag) {
-      for (int k = 0; k < 2; ++k, ++t) {
-        const int ds = t % kDesc;
-        if (!mbar_wait(&d_empty[ds], ((t / kDesc) & 1) ^ 1, wc)) break;
+      const int ds = t % kDesc;
+      if (mbar_wait(&d_empty[ds], ((t / kDesc) & 1) ^ 1, wc)) {
         desc[ds].end = 1;
         mbar_arrive(&d_full[ds]);
       }
@@ -360,9 +353,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++kvc;
       }
       if (!__all_sync(0xffffffffu, mbar_wait(&q_full[qs], (t / kQStages) & 1, wc))) break;
-      // S(t) goes to S buffer t & 1 once the softmax has loaded S(t-2).
-      const int sbuf = t & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_free[sbuf], ((t >> 1) & 1) ^ 1, wc))) break;
+      // S(t) reuses the single S buffer once the softmax has loaded S(t-1).
+      if (!__all_sync(0xffffffffu, mbar_wait(s_free, (t & 1) ^ 1, wc))) break;
       tc_fence_after();
       const uint64_t qd = q_desc0 + ((qs * Cfg::kQBytes) >> 4);
       const uint64_t kd = k_desc0 + ((kvs * 2 * Cfg::kKVBytes) >> 4);
@@ -370,10 +362,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int ks = 0; ks < D / 16; ++ks) {
         const uint32_t off = (ks / 4) * (128 * 128) + (ks % 4) * 32;
         const uint32_t koff = (ks / 4) * (BK * 128) + (ks % 4) * 32;
-        umma_ss_elect(tmem + Cfg::kColS + sbuf * BK, qd + (off >> 4), kd + (koff >> 4), idesc_s, ks > 0 ? 1u : 0u);
+        umma_ss_elect(tmem + Cfg::kColS, qd + (off >> 4), kd + (koff >> 4), idesc_s, ks > 0 ? 1u : 0u);
       }
       umma_commit_elect(&q_empty[qs]);
-      umma_commit_elect(&s_full[sbuf]);
+      umma_commit_elect(s_full);
       if (last) umma_commit_elect(&k_empty[kvs]);   // this list's last read of K
       __syncwarp();
     }
@@ -390,43 +382,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&d_empty[ds]);
       if (end) break;
-      const int sb = t & 1;                 // P buffer
-      const int ob = t % Cfg::kOBufs;       // O buffer
+      const int sb = t & 1;
       if (first) {
         if (!__all_sync(0xffffffffu, mbar_wait(&v_full[kvs], (vc / kKVStages) & 1, wc))) break;
         ++vc;
       }
       if (!__all_sync(0xffffffffu, mbar_wait(&p_full[sb], (t >> 1) & 1, wc))) break;
-      if (!__all_sync(0xffffffffu, mbar_wait(&o_free[ob], ((t / Cfg::kOBufs) & 1) ^ 1, wc))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&o_free[sb], ((t >> 1) & 1) ^ 1, wc))) break;
       tc_fence_after();
       const uint64_t vd = v_desc0 + ((kvs * 2 * Cfg::kKVBytes) >> 4);
       const uint32_t p_tmem = tmem + Cfg::kColP + sb * (BK / 2);
-      const uint32_t o_tmem = tmem + Cfg::kColO + ob * D;
+      const uint32_t o_tmem = tmem + Cfg::kColO + sb * D;
 #pragma unroll
       for (int kk = 0; kk < BK / 16; ++kk)
         umma_ts_elect(o_tmem, p_tmem + kk * 8, vd + ((kk * 2048) >> 4), idesc_o, kk > 0 ? 1u : 0u);
-      umma_commit_elect(&o_full[ob]);
+      umma_commit_elect(&o_full[sb]);
       umma_commit_elect(&p_free[sb]);
       if (last) umma_commit_elect(&v_empty[kvs]);   // this list's last read of V
       __syncwarp();
     }
   } else if (warp >= kSoftW0 && warp < kEpiW0) {
     // ---------------------------------------------------------------- softmax
-    // Warp (quarter, g) takes the chunks t with t & 1 == g, whole rows: the
-    // two softmax warps sharing an SMSP work on consecutive chunks, so one's
-    // exponentials overlap the other's maximum and P store.  S (buffer t & 1)
-    // is read from TMEM twice, for the row maximum and for the exponentials,
-    // 64 columns at a time, and released after the second pass.
-    constexpr int HC = 64;                     // columns per pass
-    constexpr int NP = BK / HC;                // passes
+    constexpr int HC = BK / 2;                 // columns per thread
     const int quarter = warp & 3;
-    const int grp = (warp - kSoftW0) / 4;      // chunk parity
+    const int half = (warp - kSoftW0) / 4;     // 0: columns [0, HC), 1: [HC, BK)
     const int row = quarter * 32 + lane;
     const int qi = row / G;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const float c = args.scale_log2;
-    constexpr float kNegInfF = -__builtin_huge_valf();
-    for (int t = grp;; t += 2) {
+    for (int t = 0;; ++t) {
       const int ds = t % kDesc;
       if (!mbar_wait(&d_full[ds], (t / kDesc) & 1, wc)) break;
       const Desc& dd = desc[ds];
@@ -439,81 +423,76 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int b = dd.b, seq_row0 = dd.seq_row0, seq_len = dd.seq_len;
       __syncwarp();
       if (lane == 0) mbar_arrive(&d_empty[ds]);
-      int lim = 0;   // visible keys of this block for the row
+      int lim = 0;   // visible keys of this block for the row, relative to this half
       if (e >= 0) {   // positions local to the query's sequence
         const int p = (args.cu_seqlens ? 0 : args.q_pos0) + (e >> 5) - seq_row0;
         const int kv_lim = args.causal ? min(p + 1, seq_len) : seq_len;
-        lim = min(BK, kv_lim - b * BK);
+        lim = min(BK, kv_lim - b * BK) - half * HC;
       }
-      const int sb = t & 1;   // S and P buffer
-      if (!mbar_wait(&s_full[sb], (t >> 1) & 1, wc)) break;
+      const int sb = t & 1;   // P buffer
+      if (!mbar_wait(s_full, t & 1, wc)) break;
       tc_fence_after();
-      const uint32_t s_tmem = lane_base + Cfg::kColS + sb * BK;
+      const uint32_t s_tmem = lane_base + Cfg::kColS;
       uint32_t sv[HC];
-      // Pass 1: the row maximum.
-      float mq[4] = {kNegInfF, kNegInfF, kNegInfF, kNegInfF};
 #pragma unroll
-      for (int h = 0; h < NP; ++h) {
-        tmem_ld32(s_tmem + h * HC, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        tmem_ld32(s_tmem + h * HC + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-        tmem_ld_wait();
-        const int hl = lim - h * HC;
-        if (hl < HC) {
+      for (int cc = 0; cc < HC / 32; ++cc)
+        tmem_ld32(s_tmem + half * HC + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[cc * 32]));
+      tmem_ld_wait();
+      // S is in registers: hand the S buffer back so the next S MMA can start.
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free);
+      if (lim < HC) {
 #pragma unroll
-          for (int i = 0; i < HC; ++i)
-            if (i >= hl) sv[i] = 0xff800000u;   // -inf: masked key
-        }
-#pragma unroll
-        for (int i = 0; i < HC; i += 8) {
-          const int k = (i / 8) & 3;
-          mq[k] = max3f(mq[k], fmaxf(__uint_as_float(sv[i]), __uint_as_float(sv[i + 1])),
-                        max3f(__uint_as_float(sv[i + 2]), __uint_as_float(sv[i + 3]), __uint_as_float(sv[i + 4])));
-          mq[k] = max3f(mq[k], __uint_as_float(sv[i + 5]), fmaxf(__uint_as_float(sv[i + 6]), __uint_as_float(sv[i + 7])));
-        }
+        for (int i = 0; i < HC; ++i)
+          if (i >= lim) sv[i] = 0xff800000u;   // -inf: masked key
       }
-      const float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
-      const float bias = mx == kNegInfF ? 0.f : mx * c;
+      float mq[4] = {__int_as_float(0xff800000), __int_as_float(0xff800000), __int_as_float(0xff800000),
+                     __int_as_float(0xff800000)};
+#pragma unroll
+      for (int i = 0; i < HC; i += 8) {
+        const int k = (i / 8) & 3;
+        mq[k] = max3f(mq[k], fmaxf(__uint_as_float(sv[i]), __uint_as_float(sv[i + 1])),
+                      max3f(__uint_as_float(sv[i + 2]), __uint_as_float(sv[i + 3]), __uint_as_float(sv[i + 4])));
+        mq[k] = max3f(mq[k], __uint_as_float(sv[i + 5]), fmaxf(__uint_as_float(sv[i + 6]), __uint_as_float(sv[i + 7])));
+      }
+      // Exchange the half-row maxima with the partner warp (same lane quarter).
+      // The slot alternates with the chunk parity: a warp rewrites slot
+      // (t & 1) only after the next barrier, which its partner reaches only
+      // after reading this chunk's value.
+      float* xs = smx + (t & 1) * 256;
+      xs[half * 128 + row] = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+      named_bar(2 + quarter, 64);
+      const float mx = fmaxf(xs[row], xs[128 + row]);
+      const float bias = mx == __int_as_float(0xff800000) ? 0.f : mx * c;
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};   // two pairs of partial sums
+      uint32_t pk[HC / 2];
+#pragma unroll
+      for (int i = 0; i < HC; i += 4) {
+        float x0, x1, x2, x3;
+        ffma2(x0, x1, __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]), c, c, -bias, -bias);
+        ffma2(x2, x3, __uint_as_float(sv[i + 2]), __uint_as_float(sv[i + 3]), c, c, -bias, -bias);
+        const float p0 = ex2_approx(x0), p1 = ex2_approx(x1), p2 = ex2_approx(x2), p3 = ex2_approx(x3);
+        float s0, s1;
+        fadd2(s0, s1, p0, p1, p2, p3);
+        const int k = ((i / 4) & 1) * 2;
+        fadd2(ls[k], ls[k + 1], ls[k], ls[k + 1], s0, s1);
+        pk[i / 2] = pack_bf16x2(p0, p1);
+        pk[i / 2 + 1] = pack_bf16x2(p2, p3);
+      }
       // P(t) goes to P buffer t & 1 once the PV of chunk t - 2 has read it.
       if (!mbar_wait(&p_free[sb], ((t >> 1) & 1) ^ 1, wc)) break;
       tc_fence_after();
       const uint32_t p_tmem = lane_base + Cfg::kColP + sb * (BK / 2);
-      // Pass 2: exponentials, row sum, P (bf16 pairs) to TMEM.
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};   // two pairs of partial sums
 #pragma unroll
-      for (int h = 0; h < NP; ++h) {
-        tmem_ld32(s_tmem + h * HC, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        tmem_ld32(s_tmem + h * HC + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-        tmem_ld_wait();
-        if (h == NP - 1) {
-          // S is no longer needed: hand the buffer back for S(t + 2).
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&s_free[sb]);
-        }
-        const int hl = lim - h * HC;
-        if (hl < HC) {
-#pragma unroll
-          for (int i = 0; i < HC; ++i)
-            if (i >= hl) sv[i] = 0xff800000u;
-        }
-        uint32_t pk[HC / 2];
-#pragma unroll
-        for (int i = 0; i < HC; i += 4) {
-          float x0, x1, x2, x3;
-          ffma2(x0, x1, __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]), c, c, -bias, -bias);
-          ffma2(x2, x3, __uint_as_float(sv[i + 2]), __uint_as_float(sv[i + 3]), c, c, -bias, -bias);
-          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1), p2 = ex2_approx(x2), p3 = ex2_approx(x3);
-          float s0, s1;
-          fadd2(s0, s1, p0, p1, p2, p3);
-          const int k = ((i / 4) & 1) * 2;
-          fadd2(ls[k], ls[k + 1], ls[k], ls[k + 1], s0, s1);
-          pk[i / 2] = pack_bf16x2(p0, p1);
-          pk[i / 2 + 1] = pack_bf16x2(p2, p3);
-        }
-        tmem_st32(p_tmem + h * (HC / 2), pk);
-      }
+      for (int cc = 0; cc < HC / 64; ++cc)
+        tmem_st32(p_tmem + half * (HC / 2) + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[cc * 32]));
+      if (HC / 2 == 16) tmem_st16(p_tmem + half * (HC / 2), *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
       const float lsum = (ls[0] + ls[1]) + (ls[2] + ls[3]);
-      ml[ds * 128 + row] = make_float2(mx, lsum);
+      if (half == 0)
+        ml[ds * 128 + row] = make_float2(mx, lsum);
+      else
+        lhi[ds * 128 + row] = lsum;
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -539,12 +518,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       const int e = qi < dd.count ? dd.entry[qi] : -1;
-      const int ob = t % Cfg::kOBufs;
-      if (!mbar_wait(&o_full[ob], (t / Cfg::kOBufs) & 1, wc)) break;
+      const int sb = t & 1;
+      if (!mbar_wait(&o_full[sb], (t >> 1) & 1, wc)) break;
       if (!mbar_wait(&ml_full[ds], (t / kDesc) & 1, wc)) break;
       tc_fence_after();
       const float2 st = ml[ds * 128 + row];
-      const float lsum = st.y;
+      const float lsum = st.y + lhi[ds * 128 + row];
       const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
       const float lse2 = lsum > 0.f ? st.x * c + __log2f(lsum) : __int_as_float(0xff800000);
       const int chunk = dd.chunk;
@@ -562,14 +541,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int a = 0; a < D / 64; ++a) {
         uint32_t ov[64];
-        tmem_ld32(lane_base + Cfg::kColO + ob * D + a * 64, *reinterpret_cast<uint32_t(*)[32]>(&ov[0]));
-        tmem_ld32(lane_base + Cfg::kColO + ob * D + a * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&ov[32]));
+        tmem_ld32(lane_base + Cfg::kColO + sb * D + a * 64, *reinterpret_cast<uint32_t(*)[32]>(&ov[0]));
+        tmem_ld32(lane_base + Cfg::kColO + sb * D + a * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&ov[32]));
         tmem_ld_wait();
         if (a == D / 64 - 1) {
           // The O buffer is free once its values are in registers.
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&o_free[ob]);
+          if (lane == 0) mbar_arrive(&o_free[sb]);
         }
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
