@@ -445,10 +445,13 @@ __device__ void merge_topk_warp(const DecArgs& a, int b, int r, int lane, int* c
     return ((cc + b) * a.h_kv + r) * a.kfree + slot;
   };
   // Streaming merge: candidates arrive in chunks of 32 * kMergeRegCand (one
-  // coalesced load per lane and slot); each chunk is merged with the running
-  // top-kfree list, lane k holding its k-th entry, by kfree rounds of warp
-  // argmax whose winner is retired by its owner (block ids are unique across
-  // shares).
+  // coalesced load per lane and slot) into a running top-kfree list, lane k
+  // holding its k-th entry (block ids are unique across shares, so the order
+  // (score desc, block asc) is strict).  The first chunk is selected by kfree
+  // rounds of warp argmax; a later chunk only contributes the candidates that
+  // beat the list's last entry -- few, since every share is itself sorted and
+  // the list's threshold rises as it fills -- each inserted at its place by
+  // one ballot and one shift.
   float run_s = kNegInf;
   int run_b = -1;
   for (int c0 = 0; c0 < ncand; c0 += 32 * kMergeRegCand) {
@@ -464,6 +467,37 @@ __device__ void merge_topk_warp(const DecArgs& a, int b, int r, int lane, int* c
         cb[i] = __ldcg(a.cand_b + idx);
         cs[i] = __ldcg(a.cand_s + idx);
       }
+    }
+    if (c0 > 0) {
+      if (kfree_b <= 0) break;
+#pragma unroll
+      for (int i = 0; i < kMergeRegCand; ++i) {
+        const float ks = __shfl_sync(0xffffffffu, run_s, kfree_b - 1);
+        const int kbl = __shfl_sync(0xffffffffu, run_b, kfree_b - 1);
+        unsigned m = __ballot_sync(0xffffffffu, cb[i] >= 0 && (kbl < 0 || better(cs[i], cb[i], ks, kbl)));
+        while (m) {
+          const int src = __ffs(m) - 1;
+          m &= m - 1;
+          const float xs = __shfl_sync(0xffffffffu, cs[i], src);
+          const int xb = __shfl_sync(0xffffffffu, cb[i], src);
+          // Entries are sorted and empty ones come last, so the entries x
+          // beats are a suffix; x goes to its first position.
+          const unsigned bm =
+              __ballot_sync(0xffffffffu, lane < kfree_b && (run_b < 0 || better(xs, xb, run_s, run_b)));
+          if (bm == 0) continue;
+          const int pos = __ffs(bm) - 1;
+          const float up_s = __shfl_up_sync(0xffffffffu, run_s, 1);
+          const int up_b = __shfl_up_sync(0xffffffffu, run_b, 1);
+          if (lane == pos) {
+            run_s = xs;
+            run_b = xb;
+          } else if (lane > pos && lane < kfree_b) {
+            run_s = up_s;
+            run_b = up_b;
+          }
+        }
+      }
+      continue;
     }
     float new_s = kNegInf;
     int new_b = -1;

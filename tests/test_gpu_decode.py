@@ -92,6 +92,16 @@ def test_decode_b8_1m_dense():
     run_case(WORKLOADS["decode_b8_1m"], dense=True)
 
 
+@pytest.mark.parametrize("kw", [
+    dict(batch=1, kv_min=200000, kv_max=200000, topk=8),          # one sequence over every index CTA
+    dict(batch=3, kv_min=500, kv_max=150000, topk=16, seed=81),   # one long, two short
+])
+def test_top_k_merge_over_many_shares(kw):
+    # A sequence whose blocks span hundreds of index CTAs: its top-k merge
+    # takes many candidate chunks (the later ones by insertion).
+    run_case(small(**kw))
+
+
 def test_many_items_per_cta():
     # 2048 x 8 x 16 = 262144 (sequence, group, slot) items: more than 1024 per
     # CTA at 148 CTAs, so the persistent attention grid grows; sampled rows.
