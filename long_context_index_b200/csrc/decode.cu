@@ -438,10 +438,12 @@ __device__ void merge_topk_warp(const DecArgs& a, int b, int r, int lane, int* c
   // kept its top kfree >= kfree_b, so the global top kfree_b is among them.
   const int kb = a.topk_seq ? min(max(static_cast<int>(a.topk_seq[b]), 1), a.topk) : a.topk;
   const int kfree_b = min(a.kfree, kb - (a.force_local ? 1 : 0));
+  // Ranges are empty only when the grid has more CTAs than blocks.
+  const bool some_empty = T < n;
   auto cand_index = [&](int c) -> long long {   // -1: share of an empty range
     const int sg = c / a.kfree, slot = c - sg * a.kfree;
     const long long cc = c_lo + sg;
-    if ((cc + 1) * T / n == cc * T / n) return -1;
+    if (some_empty && (cc + 1) * T / n == cc * T / n) return -1;
     return ((cc + b) * a.h_kv + r) * a.kfree + slot;
   };
   // Streaming merge: candidates arrive in chunks of 32 * kMergeRegCand (one
@@ -526,23 +528,18 @@ __device__ void merge_topk_warp(const DecArgs& a, int b, int r, int lane, int* c
     run_s = new_s;
     run_b = new_b;
   }
-  const int nsel0 = __popc(__ballot_sync(0xffffffffu, run_b >= 0));   // lanes 0 .. nsel0 - 1
-  if (run_b >= 0) chosen[lane] = run_b;
-  __syncwarp();
-  int nsel = nsel0;
-  if (lane == 0) {
-    if (a.force_local) chosen[nsel++] = b_loc;
-    // insertion sort (<= 32 entries)
-    for (int i = 1; i < nsel; ++i) {
-      const int v = chosen[i];
-      int j = i - 1;
-      while (j >= 0 && chosen[j] > v) { chosen[j + 1] = chosen[j]; --j; }
-      chosen[j + 1] = v;
-    }
-    int32_t* out = a.block_ids + (static_cast<size_t>(b) * a.h_kv + r) * a.topk;
-    for (int i = 0; i < a.topk; ++i) out[i] = i < nsel ? chosen[i] : -1;
-  }
-  __syncwarp();
+  // The selected blocks (lanes 0 .. nsel0 - 1) plus the local block, written
+  // ascending: each lane's place is the number of smaller ids (all distinct).
+  const int nsel0 = __popc(__ballot_sync(0xffffffffu, run_b >= 0));
+  const int nsel = nsel0 + (a.force_local ? 1 : 0);
+  int v = run_b >= 0 ? run_b : 0x7fffffff;
+  if (a.force_local && lane == nsel0) v = b_loc;
+  int place = 0;
+  for (int j = 0; j < nsel; ++j) place += __shfl_sync(0xffffffffu, v, j) < v;
+  int32_t* out = a.block_ids + (static_cast<size_t>(b) * a.h_kv + r) * a.topk;
+  if (lane < nsel) out[place] = v;
+  for (int i = nsel + lane; i < a.topk; i += 32) out[i] = -1;
+  (void)chosen;
 }
 
 // topk == 1 with the forced local block: no scan, every sequence's ids are
