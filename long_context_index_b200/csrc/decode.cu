@@ -456,9 +456,8 @@ __device__ void merge_topk_warp(const DecArgs& a, int b, int r, int lane, int* c
   // one ballot and one shift.
   float run_s = kNegInf;
   int run_b = -1;
-  for (int c0 = 0; c0 < ncand; c0 += 32 * kMergeRegCand) {
-    float cs[kMergeRegCand];
-    int cb[kMergeRegCand];
+  // The next chunk's loads are issued before the current chunk is merged.
+  auto load_chunk = [&](int c0, float (&cs)[kMergeRegCand], int (&cb)[kMergeRegCand]) {
 #pragma unroll
     for (int i = 0; i < kMergeRegCand; ++i) {
       const int c = c0 + lane + 32 * i;
@@ -470,6 +469,19 @@ __device__ void merge_topk_warp(const DecArgs& a, int b, int r, int lane, int* c
         cs[i] = __ldcg(a.cand_s + idx);
       }
     }
+  };
+  float nx_s[kMergeRegCand];
+  int nx_b[kMergeRegCand];
+  if (ncand > 0) load_chunk(0, nx_s, nx_b);
+  for (int c0 = 0; c0 < ncand; c0 += 32 * kMergeRegCand) {
+    float cs[kMergeRegCand];
+    int cb[kMergeRegCand];
+#pragma unroll
+    for (int i = 0; i < kMergeRegCand; ++i) {
+      cs[i] = nx_s[i];
+      cb[i] = nx_b[i];
+    }
+    if (c0 + 32 * kMergeRegCand < ncand) load_chunk(c0 + 32 * kMergeRegCand, nx_s, nx_b);
     if (c0 > 0) {
       if (kfree_b <= 0) break;
 #pragma unroll
