@@ -1113,6 +1113,9 @@ __device__ __forceinline__ void decode_attn_body(const CUtensorMap* tm_q, const 
         const uint8_t* s8 = smem + stage * C::kStageBytes + C::kQBytes;
         const uint8_t* ssc = s8 + 2 * C::kK8Bytes;
         constexpr int CPR = D / 16;                      // 16-byte chunks per E4M3 row
+        // Four chunks in flight per thread: the loop is bound by the latency of
+        // its shared-memory loads, not by the conversions.
+#pragma unroll 4
         for (int e = tid; e < 2 * BK * CPR; e += 32 * kStreamConsumers) {
           const int kv = e / (BK * CPR), rem = e - kv * (BK * CPR);
           const int x = rem / CPR, c = rem - x * CPR;   // row, chunk (16 elements from column 16c)
