@@ -152,9 +152,10 @@ MSA_API int msa_sparse_attn_prefill(const msa_params* p, const void* q, const vo
  * scan splits the blocks of all sequences into equal ranges per CTA, the
  * attention splits the (sequence, group, slot) list the same way, and partial
  * results of a sequence or group split between CTAs are merged by the last
- * CTA to finish it.  When the step fits one co-resident wave of CTAs it runs
- * as one cooperative launch whose attention CTAs start as soon as the ids of
- * their own sequences are merged; otherwise as two launches.
+ * CTA to finish it.  The step runs as two launches (index scan, then
+ * attention); with MSA_OPT_DECODE_FUSED set (msa_set_option) a step that fits
+ * one co-resident wave of CTAs runs as one cooperative launch whose attention
+ * CTAs start as soon as the ids of their own sequences are merged.
  *   q            bf16 [batch, h_q, d]
  *   q_idx        bf16 [batch, h_kv, d_idx]
  *   k_cache,

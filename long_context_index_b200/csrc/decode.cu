@@ -3,10 +3,10 @@
 // For every sequence b the query sits at position p = L_b - 1 of its own
 // contiguous caches.  The step is the prefill math of one row
 // (titansim.online summary of "MiniMax Sparse Attention": eq. (6) and the
-// local-block rule in section 4.2, eq. (8) in section 4.3), as one fused
-// cooperative launch (below) whenever the step fits one co-resident wave,
-// else as two persistent HBM-streaming launches.  Both forms run the same two
-// parts:
+// local-block rule in section 4.2, eq. (8) in section 4.3), as two
+// persistent HBM-streaming launches, or (process option MSA_OPT_DECODE_FUSED)
+// as one fused cooperative launch when the step fits one co-resident wave.
+// Both forms run the same two parts:
 //
 //   1. decode_index_kernel   The blocks of all sequences, end to end, are cut
 //      into equal ranges, one per CTA.  Streams the index-key cache once for
