@@ -506,8 +506,8 @@ def run_ours(args, rank, world, torch, dist):
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "note": "prefill inputs and outputs cross PCIe every step (double-buffered, uploads and downloads "
                         "on their own streams, overlapping the kernels); decode KV caches stay resident"},
-        # Per step: index top-k (1); sparse prefill: schedule count, scan,
-        # fill and list range (4), block-major attention (1), partial merge
+        # Per step: index top-k (1); sparse prefill: schedule count, tile
+        # sums, tile scans and fill (4), block-major attention (1), partial merge
         # (1); decode: persistent index scan with the merge folded in and
         # persistent attention with the combine folded in (2), or the two
         # in one fused launch (1).

@@ -7,8 +7,9 @@
 // the per-block results are merged afterwards (the pages' "two-stage merge",
 // with no atomics on the outputs).
 //
-//   1. sched_count / sched_scan / sched_fill: invert block_ids [n_q, h_kv, k]
-//      into one list per (query wave, group r, block b) of the (query, slot)
+//   1. sched_count / sched_tile_sums + sched_scan_tiles / sched_fill: invert
+//      block_ids [n_q, h_kv, k] into one list per (query wave, group r,
+//      block b) of the (query, slot)
 //      pairs that selected it (counting sort; slot = position of b in the
 //      query's ids).  Lists are handed out in (wave, group, block) order, so
 //      at any moment the CTAs gather the queries of one wave of kWave rows,
@@ -618,99 +619,129 @@ __global__ void sched_count_kernel(const int32_t* ids, long long total, int h_kv
   atomicAdd(&cnt[((q / kWave) * h_kv + r) * nb + gb], 1);
 }
 
-// One CTA: exclusive scans of cnt -> offs and of ceil(cnt / qpc) -> chunk_off,
-// and the compacted list of non-empty lists.  Each thread owns 8 consecutive
-// entries per pass; the per-thread totals are scanned with warp shuffles and
-// one cross-warp step, carrying the running totals between passes.
-__global__ void __launch_bounds__(1024) sched_scan_kernel(const int* cnt, int n, int qpc, int* offs, int* chunk_off,
-                                                          int* lists, int* n_lists) {
-  constexpr int kPer = 8;
-  __shared__ int wsum[3][32];
-  __shared__ int carry[3];
+// The schedule's exclusive prefixes over the lists (entries, non-empty lists,
+// chunks of 128 / G queries), in two multi-CTA passes over tiles of
+// kScanTile lists: the tile totals, then each tile's scan on top of the sum of
+// the tiles before it.  The second pass also compacts the non-empty lists
+// (ascending) and, in its last thread, writes the totals and the launch's
+// list range [0, n_lists).
+constexpr int kScanThreads = 256;
+constexpr int kScanPer = 8;
+constexpr int kScanTile = kScanThreads * kScanPer;
+
+__device__ __forceinline__ void list_totals(int v, int qpc, int& a, int& b, int& c) {
+  a += v;
+  b += v > 0;
+  c += (v + qpc - 1) / qpc;
+}
+
+__global__ void __launch_bounds__(kScanThreads) sched_tile_sums_kernel(const int* cnt, int n, int qpc, int* tsum) {
+  __shared__ int ws[3][kScanThreads / 32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (threadIdx.x < 3) carry[threadIdx.x] = 0;
-  __syncthreads();
-  for (int base = 0; base < n; base += 1024 * kPer) {
-    const int i0 = base + threadIdx.x * kPer;
-    int v[kPer];
-    int ta = 0, tb = 0, tc = 0;
+  const int i0 = blockIdx.x * kScanTile + threadIdx.x * kScanPer;
+  int a = 0, b = 0, c = 0;
 #pragma unroll
-    for (int k = 0; k < kPer; ++k) {
-      v[k] = i0 + k < n ? cnt[i0 + k] : 0;
-      ta += v[k];
-      tb += v[k] > 0;
-      tc += (v[k] + qpc - 1) / qpc;
-    }
-    // Inclusive warp scan of the thread totals.
-    int ia = ta, ib = tb, ic = tc;
+  for (int k = 0; k < kScanPer; ++k) list_totals(i0 + k < n ? cnt[i0 + k] : 0, qpc, a, b, c);
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int xa = __shfl_up_sync(0xffffffffu, ia, off);
-      const int xb = __shfl_up_sync(0xffffffffu, ib, off);
-      const int xc = __shfl_up_sync(0xffffffffu, ic, off);
-      if (lane >= off) {
-        ia += xa;
-        ib += xb;
-        ic += xc;
-      }
-    }
-    if (lane == 31) {
-      wsum[0][warp] = ia;
-      wsum[1][warp] = ib;
-      wsum[2][warp] = ic;
-    }
-    __syncthreads();
-    if (warp == 0) {
-      int a = wsum[0][lane], b = wsum[1][lane], c = wsum[2][lane];
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int xa = __shfl_up_sync(0xffffffffu, a, off);
-        const int xb = __shfl_up_sync(0xffffffffu, b, off);
-        const int xc = __shfl_up_sync(0xffffffffu, c, off);
-        if (lane >= off) {
-          a += xa;
-          b += xb;
-          c += xc;
-        }
-      }
-      wsum[0][lane] = a;   // inclusive over warps
-      wsum[1][lane] = b;
-      wsum[2][lane] = c;
-    }
-    __syncthreads();
-    int pa = carry[0] + (warp ? wsum[0][warp - 1] : 0) + ia - ta;
-    int pb = carry[1] + (warp ? wsum[1][warp - 1] : 0) + ib - tb;
-    int pc = carry[2] + (warp ? wsum[2][warp - 1] : 0) + ic - tc;
-#pragma unroll
-    for (int k = 0; k < kPer; ++k) {
-      const int i = i0 + k;
-      if (i < n) {
-        offs[i] = pa;
-        chunk_off[i] = pc;
-        if (v[k] > 0) lists[pb++] = i;
-      }
-      pa += v[k];
-      pc += (v[k] + qpc - 1) / qpc;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      carry[0] += wsum[0][31];
-      carry[1] += wsum[1][31];
-      carry[2] += wsum[2][31];
-    }
-    __syncthreads();
+  for (int x = 16; x > 0; x >>= 1) {
+    a += __shfl_xor_sync(0xffffffffu, a, x);
+    b += __shfl_xor_sync(0xffffffffu, b, x);
+    c += __shfl_xor_sync(0xffffffffu, c, x);
   }
-  if (threadIdx.x == 0) {
-    offs[n] = carry[0];
-    *n_lists = carry[1];
+  if (lane == 0) {
+    ws[0][warp] = a;
+    ws[1][warp] = b;
+    ws[2][warp] = c;
+  }
+  __syncthreads();
+  if (threadIdx.x < 3) {
+    int t = 0;
+#pragma unroll
+    for (int w = 0; w < kScanThreads / 32; ++w) t += ws[threadIdx.x][w];
+    tsum[3 * blockIdx.x + threadIdx.x] = t;
   }
 }
 
-// The launch's list range: [0, n_lists).
-__global__ void sched_range_kernel(const int* n_lists, int* range) {
-  if (threadIdx.x == 0) {
+__global__ void __launch_bounds__(kScanThreads) sched_scan_tiles_kernel(const int* cnt, int n, int qpc,
+                                                                        const int* tsum, int* offs, int* chunk_off,
+                                                                        int* lists, int* n_lists, int* range) {
+  constexpr int kW = kScanThreads / 32;
+  __shared__ int ws[3][kW];
+  __shared__ int tile_base[3];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (warp == 0) {
+    // Sum of the totals of the tiles before this one.
+    int a = 0, b = 0, c = 0;
+    for (int t = lane; t < static_cast<int>(blockIdx.x); t += 32) {
+      a += tsum[3 * t];
+      b += tsum[3 * t + 1];
+      c += tsum[3 * t + 2];
+    }
+#pragma unroll
+    for (int x = 16; x > 0; x >>= 1) {
+      a += __shfl_xor_sync(0xffffffffu, a, x);
+      b += __shfl_xor_sync(0xffffffffu, b, x);
+      c += __shfl_xor_sync(0xffffffffu, c, x);
+    }
+    if (lane == 0) {
+      tile_base[0] = a;
+      tile_base[1] = b;
+      tile_base[2] = c;
+    }
+  }
+  const int i0 = blockIdx.x * kScanTile + threadIdx.x * kScanPer;
+  int v[kScanPer];
+  int ta = 0, tb = 0, tc = 0;
+#pragma unroll
+  for (int k = 0; k < kScanPer; ++k) {
+    v[k] = i0 + k < n ? cnt[i0 + k] : 0;
+    list_totals(v[k], qpc, ta, tb, tc);
+  }
+  // Inclusive warp scan of the thread totals, then over the warps.
+  int ia = ta, ib = tb, ic = tc;
+#pragma unroll
+  for (int x = 1; x < 32; x <<= 1) {
+    const int xa = __shfl_up_sync(0xffffffffu, ia, x);
+    const int xb = __shfl_up_sync(0xffffffffu, ib, x);
+    const int xc = __shfl_up_sync(0xffffffffu, ic, x);
+    if (lane >= x) {
+      ia += xa;
+      ib += xb;
+      ic += xc;
+    }
+  }
+  if (lane == 31) {
+    ws[0][warp] = ia;
+    ws[1][warp] = ib;
+    ws[2][warp] = ic;
+  }
+  __syncthreads();
+  int pa = tile_base[0] + ia - ta, pb = tile_base[1] + ib - tb, pc = tile_base[2] + ic - tc;
+#pragma unroll
+  for (int w = 0; w < kW; ++w) {
+    if (w < warp) {
+      pa += ws[0][w];
+      pb += ws[1][w];
+      pc += ws[2][w];
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < kScanPer; ++k) {
+    const int i = i0 + k;
+    if (i < n) {
+      offs[i] = pa;
+      chunk_off[i] = pc;
+      if (v[k] > 0) lists[pb++] = i;
+    }
+    pa += v[k];
+    pc += (v[k] + qpc - 1) / qpc;
+  }
+  if (blockIdx.x == gridDim.x - 1 && threadIdx.x == kScanThreads - 1) {
+    // Lists past n add nothing, so this thread's running sums are the totals.
+    offs[n] = pa;
+    *n_lists = pb;
     range[0] = 0;
-    range[1] = *n_lists;
+    range[1] = pb;
   }
 }
 
@@ -824,7 +855,7 @@ cudaError_t launch_kvo_g(int G, const CUtensorMap* m, const KvoArgs& a, int grid
 }
 
 struct SparseWs {
-  int *cnt, *fill, *offs, *chunk_off, *lists, *n_lists, *work, *entries, *prow_of, *wave_lo;
+  int *cnt, *fill, *offs, *chunk_off, *lists, *n_lists, *work, *entries, *prow_of, *wave_lo, *tsum;
   uint16_t* part_o;
   float* part_lse;
   size_t max_chunks, bytes;
@@ -858,6 +889,7 @@ SparseWs carve(const msa_params& p, int n_q, int n_kv, int batch, void* base) {
   s.n_lists = s.cnt ? s.cnt + 2 * nl : nullptr;
   s.work = s.cnt ? s.cnt + 2 * nl + 1 : nullptr;
   s.wave_lo = reinterpret_cast<int*>(take(2 * 4));
+  s.tsum = reinterpret_cast<int*>(take(static_cast<size_t>((nl + kScanTile - 1) / kScanTile) * 3 * 4));
   s.offs = reinterpret_cast<int*>(take((nl + 1) * 4));
   s.chunk_off = reinterpret_cast<int*>(take(nl * 4));
   s.lists = reinterpret_cast<int*>(take(nl * 4));
@@ -904,10 +936,12 @@ int run_sparse_attn_kvouter(const msa_params& p, const void* q, const CUtensorMa
   if (cudaMemsetAsync(s.cnt, 0, (2 * static_cast<size_t>(nl) + 2) * 4, stream) != cudaSuccess) return MSA_ERR_CUDA;
   const int gsz = static_cast<int>((total + kSchedThreads - 1) / kSchedThreads);
   sched_count_kernel<<<gsz, kSchedThreads, 0, stream>>>(block_ids, total, p.h_kv, p.topk, nb, geo, s.cnt);
-  sched_scan_kernel<<<1, 1024, 0, stream>>>(s.cnt, nl, 128 / G, s.offs, s.chunk_off, s.lists, s.n_lists);
+  const int n_tiles = (nl + kScanTile - 1) / kScanTile;
+  sched_tile_sums_kernel<<<n_tiles, kScanThreads, 0, stream>>>(s.cnt, nl, 128 / G, s.tsum);
+  sched_scan_tiles_kernel<<<n_tiles, kScanThreads, 0, stream>>>(s.cnt, nl, 128 / G, s.tsum, s.offs, s.chunk_off,
+                                                                 s.lists, s.n_lists, s.wave_lo);
   sched_fill_kernel<<<gsz, kSchedThreads, 0, stream>>>(block_ids, total, p.h_kv, p.topk, nb, G, geo, s.offs,
                                                        s.chunk_off, s.fill, s.entries, s.prow_of);
-  sched_range_kernel<<<1, 32, 0, stream>>>(s.n_lists, s.wave_lo);
   if (cudaGetLastError() != cudaSuccess) return MSA_ERR_CUDA;
 
   KvoArgs a;
