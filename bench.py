@@ -73,11 +73,11 @@ L2_BYTES = 126 * 1024 * 1024
 
 # DRAM bytes per call of the dominant unit at the bench workload, from ncu's
 # dram__bytes_read.sum + dram__bytes_write.sum of its kernels on the 4096-query
-# chunked prefill at 64K ("prof" case: 2.545 GB), scaled by the query rows
+# chunked prefill at 64K ("prof" case: 2.5436 GB), scaled by the query rows
 # (x32; the traffic is the partial rows, one per query, head and selected
 # block), on the kernel source with the given digest (a stale digest reports
 # null).
-TRAFFIC = {"attn_prefill": (2.545e9 * 32, "d9107512a614", "attn_sparse.cu")}
+TRAFFIC = {"attn_prefill": (2.5436e9 * 32, "61f508beef40", "attn_sparse.cu")}
 
 
 def load_peaks():
