@@ -140,6 +140,11 @@ MSA_API int msa_index_topk(const msa_params* p, const void* q_idx, const void* k
  * Ids must be valid: each -1 or a block holding a visible key of the row,
  * and the non-negative ids of a (row, group) pairwise distinct (a repeated id
  * would be attended twice; msa_index_topk never emits one).
+ * The sparse run indexes its schedule with 32-bit integers: n_q * h_kv * topk,
+ * the (query wave of 4096 rows, group, block) lists, and the partial rows
+ * (about 128 * n_q * h_kv * topk * h_kv / h_q) must each stay below 2^31
+ * (MSA_ERR_UNSUPPORTED otherwise; far beyond what one GPU's memory holds at
+ * the model shapes).
  */
 MSA_API int msa_sparse_attn_prefill(const msa_params* p, const void* q, const void* k, const void* v,
                             const int32_t* block_ids, int n_q, int n_kv, int q_pos0, void* o, void* ws,

@@ -905,6 +905,18 @@ SparseWs carve(const msa_params& p, int n_q, int n_kv, int batch, void* base) {
 
 }  // namespace
 
+// The schedule indexes lists, entries and partial rows with 32-bit integers
+// (list ids, prefix sums, TMA row coordinates of the partial tiles).
+bool sparse_sizes_supported(const msa_params& p, int n_q, int n_kv, int batch) {
+  const long long kMax = 0x7fffffffLL;
+  const long long nb = sched_blocks(p, n_kv, batch);
+  const long long nl = static_cast<long long>((n_q + kWave - 1) / kWave) * p.h_kv * nb;
+  const long long nnz = static_cast<long long>(n_q) * p.h_kv * p.topk;
+  const long long qpc = 128 / (p.h_q / p.h_kv);
+  const long long rows = ((nnz + qpc - 1) / qpc + nl) * 128;
+  return nl <= kMax && nnz <= kMax && rows <= kMax;
+}
+
 size_t sparse_prefill_workspace_bytes(const msa_params& p, int n_q, int n_kv, int batch) {
   return carve(p, n_q, n_kv, batch, nullptr).bytes;
 }
@@ -913,6 +925,7 @@ int run_sparse_attn_kvouter(const msa_params& p, const void* q, const CUtensorMa
                             const int32_t* block_ids, int n_q, int n_kv, int q_pos0, void* o, void* ws,
                             size_t ws_bytes, int* status, cudaStream_t stream, const Varlen* vl) {
   const int batch = vl ? vl->batch : 0;
+  if (!sparse_sizes_supported(p, n_q, n_kv, batch)) return MSA_ERR_UNSUPPORTED;
   SparseWs s = carve(p, n_q, n_kv, batch, ws);
   if (ws_bytes < s.bytes) return MSA_ERR_WORKSPACE;
   const int G = p.h_q / p.h_kv;

@@ -170,6 +170,7 @@ int msa_sparse_attn_prefill(const msa_params* p, const void* q, const void* k, c
   if (n_q > 0 && (!q || !k || !v || !o)) return MSA_ERR_INVALID;
   if (n_q > 0 && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))) return MSA_ERR_MISALIGNED;
   if (block_ids && !aligned16(block_ids)) return MSA_ERR_MISALIGNED;
+  if (block_ids && n_q > 0 && !sparse_sizes_supported(*p, n_q, n_kv, 0)) return MSA_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if ((rc = clear_status(ws, st))) return rc;
   return run_sparse_attn_prefill(*p, q, k, v, block_ids, n_q, n_kv, q_pos0, o,
@@ -250,6 +251,8 @@ int varlen_call(int op, const msa_params* p, const void* a0, const void* a1, con
   if (rc) return rc;
   if (batch <= 0 || total < 0 || !cu) return MSA_ERR_INVALID;
   if (total > kMaxRows || batch > kMaxRows) return MSA_ERR_UNSUPPORTED;
+  if (op == MSA_OP_PREFILL_VARLEN && total > 0 && !sparse_sizes_supported(*p, total, total, batch))
+    return MSA_ERR_UNSUPPORTED;
   if ((rc = check_ws(ws, ws_bytes, varlen_workspace_bytes(op, *p, batch, total)))) return rc;
   if ((reinterpret_cast<uintptr_t>(cu) & 3u) != 0) return MSA_ERR_MISALIGNED;
   if (topk_seq && (reinterpret_cast<uintptr_t>(topk_seq) & 3u) != 0) return MSA_ERR_MISALIGNED;

@@ -73,6 +73,9 @@ int run_sparse_attn_prefill(const msa_params& p, const void* q, const void* k, c
 
 // Block-major sparse prefill (attn_sparse.cu).
 size_t sparse_prefill_workspace_bytes(const msa_params& p, int n_q, int n_kv, int batch);
+// False when the block-major schedule's 32-bit list, entry or partial-row
+// indices would overflow (huge n_q * h_kv * topk or lists).
+bool sparse_sizes_supported(const msa_params& p, int n_q, int n_kv, int batch);
 int run_sparse_attn_kvouter(const msa_params& p, const void* q, const CUtensorMap& tk, const CUtensorMap& tv,
                             const int32_t* block_ids, int n_q, int n_kv, int q_pos0, void* o, void* ws,
                             size_t ws_bytes, int* status, cudaStream_t stream, const Varlen* vl);

@@ -106,6 +106,13 @@ def test_prefill_and_decode_reject_bad_arguments():
     assert L.msa_sparse_attn_decode(C.byref(p), 16, 16, 16, 16, 16, 16, 4, 100, 0, 16, 16, 256, 10, None) == -4
     assert L.msa_sparse_attn_decode(C.byref(p), 16, None, 16, 16, None, 16, 4, 100, 0, None, 16, 256,
                                     1 << 30, None) == -1
+    # Sparse prefill sizes whose schedule would overflow its 32-bit indices:
+    # 2^24 rows x 128 groups x 32 slots, refused before any launch.
+    big = P(h_q=128, h_kv=128, d=64, d_idx=32, block_k=64, topk=32)
+    n = 1 << 24
+    assert L.msa_sparse_attn_prefill(C.byref(big), 16, 16, 16, 16, n, n, 0, 16, 256, 1 << 62, None) == -2
+    assert L.msa_sparse_attn_prefill_varlen(C.byref(big), 16, 16, 16, 16, 1, n, 16, 16, 256, 1 << 62,
+                                            None) == -2
     # MXFP8 decode: code arrays 16-byte aligned, K/V scales 4-byte aligned.
     mx = L.msa_sparse_attn_decode_mxfp8
     args = lambda k8=16, k_sc=16: (C.byref(p), 16, 16, k8, k_sc, 16, 16, 16, 16, 16, None, 4, 100, 16,
